@@ -1,0 +1,184 @@
+/*
+ * fp4.h -- C ABI of libfp4: the 4-bit linear layer of FP4 LLM pre-training on B200
+ * (sm_100a).
+ *
+ *   x (bf16) --rotate(H16/H32, along the contraction axis)--> fp32
+ *            --microscale (MXFP4 | NVFP4)--> packed E2M1 codes + block scales
+ *   A, B (FP4) --block-scaled tcgen05 GEMM, fp32 accumulate--> C (fp32 | bf16)
+ *
+ * Pages this follows (cited by title and section):
+ *   gist.science, "기술 요약: MXFP4 를 활용한 대규모 언어 모델 사전 학습" (summary of
+ *   arXiv 2605.09825): "방법론" (Methodology) item 2 (Fprop, Dgrad and Wgrad each in
+ *   MXFP4), item 3 (deterministic 16x16 / 32x32 Hadamard rotations); "주요 기여 및
+ *   발견" (Findings) sections 1-2 (Wgrad dominates the instability; deterministic
+ *   H16 restores it).
+ *   molayo1419.me, "Blackwell의 NVIDIA NVFP4, MaxText에서 JAX 학습 속도 1.8배 향상":
+ *   "주요 사실" (Key facts) bullets 2 and 5 (two 4-bit values per byte; FP4 tensor
+ *   cores on Blackwell).
+ *
+ * Conventions for every entry point
+ *   - All data pointers are DEVICE pointers owned by the caller, 16-byte aligned.
+ *     The library never allocates, frees or retains device memory.
+ *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream). Arguments are validated on the host before anything is
+ *     launched: a call that returns an error launched nothing.
+ *   - Device-side failures (a pipeline wait that exceeded its time limit) do not
+ *     trap: the kernel records them in a device status word and returns; read it
+ *     with fp4_check_status().
+ *   - Results are deterministic: the same inputs give bit-identical outputs on every
+ *     run (fixed butterfly order, order-independent max reductions, no split-K).
+ *
+ * Data formats
+ *   codes  : uint8 [R][C/2]; element 2i in the low nibble of byte i, 2i+1 in the high
+ *            nibble; nibble = sign << 3 | E2M1 magnitude index
+ *            (0, 0.5, 1, 1.5, 2, 3, 4, 6).
+ *   scales : one byte per block of bs elements along C (bs = 32 MXFP4, 16 NVFP4):
+ *            MXFP4 E8M0 (value 2^(byte-127)), NVFP4 UE4M3 (OCP E4M3, sign 0).
+ *            Scale (r, kb), KB = C/bs, is stored at byte
+ *              ((r/128)*KB4 + kb/4)*512 + (r%32)*16 + ((r%128)/32)*4 + kb%4,
+ *            KB4 = ceil(KB/4): 128-row x 4-block atoms of 512 bytes, the order the
+ *            tensor cores read them in. Padding bytes are written as zero.
+ *   NVFP4 tensor scale : fp32 S = amax / (6*448) of the rotated tensor (S = 1 when
+ *            amax is 0). Element value = e2m1 * ue4m3(scale byte) * S.
+ */
+#ifndef FP4_H_
+#define FP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream, declared here without CUDA headers. */
+typedef struct CUstream_st *fp4_stream_t;
+
+typedef enum {
+    FP4_OK = 0,
+    FP4_ERR_INVALID_ARG = 1,        /* bad enum value, NULL pointer, or a pointer that must be NULL */
+    FP4_ERR_SHAPE = 2,              /* a size the kernels do not tile (see each call) */
+    FP4_ERR_ALIGN = 3,              /* a data pointer not 16-byte aligned */
+    FP4_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not compute capability 10.x */
+    FP4_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed */
+    FP4_ERR_TIMEOUT = 6,            /* a device-side pipeline wait gave up (fp4_check_status) */
+    FP4_ERR_WORKSPACE = 7           /* workspace NULL or smaller than required */
+} fp4_status;
+
+typedef enum { FP4_MXFP4 = 0, FP4_NVFP4 = 1 } fp4_format;
+typedef enum { FP4_AXIS_ROW = 0, FP4_AXIS_COL = 1 } fp4_axis;
+typedef enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 } fp4_out_dtype;
+typedef enum { FP4_PASS_FPROP = 0, FP4_PASS_DGRAD = 1, FP4_PASS_WGRAD = 2 } fp4_pass;
+
+/* Version of this ABI; bumped on any incompatible change. */
+int fp4_abi_version(void);
+
+/* Bytes of a packed code matrix with R rows of C elements: R*C/2. */
+size_t fp4_codes_bytes(int64_t rows, int64_t cols);
+
+/* Bytes of the scale matrix of an [R][C] code matrix in the atom layout above:
+ * ceil(R/128)*128 * ceil(C/bs/4)*4. */
+size_t fp4_scales_bytes(int64_t rows, int64_t cols, fp4_format fmt);
+
+/*
+ * fp4_quantize -- rotate and quantise one bf16 matrix x[rows][cols] (row-major).
+ *   Rotation: every aligned group of hadamard_n (0 = none, 16, 32) elements along the
+ *   contraction axis is replaced by H*v/sqrt(n) (Sylvester H, fp32 butterfly with
+ *   strides 1, 2, 4, ... in that order; the factor 1/sqrt(n) is RN_fp32(1/sqrt(n))).
+ *   [MXFP4 pre-training summary, Methodology item 3.]
+ *   axis = FP4_AXIS_ROW : groups and blocks run along each row;
+ *                         codes [rows][cols/2], scales for an [rows][cols] matrix.
+ *   axis = FP4_AXIS_COL : groups and blocks run down each column, output transposed;
+ *                         codes [cols][rows/2], scales for a [cols][rows] matrix.
+ *   MXFP4: per 32-block, e = floor(log2 amax) - 2 clamped to [-127,127] (amax 0 -> -127),
+ *          scale byte e+127, code = E2M1_RNE_satfinite(v * 2^-e).
+ *   NVFP4: S = amax_tensor/2688; per 16-block sb = E4M3_RNE_satfinite(bmax/(6*S)),
+ *          code = E2M1_RNE_satfinite(v / (ue4m3(sb)*S)).
+ *   tensor_scale: NVFP4 -> device float[2], written {S, amax}; slot [1] is also the
+ *                 reduction cell of the amax pass. MXFP4 -> must be NULL.
+ *   Shape: rows % 32 == 0 and cols % 32 == 0 (rows or cols 0: nothing is done).
+ *   Launches: MXFP4 one kernel; NVFP4 a 4-byte memset, an amax kernel, a quantise kernel.
+ */
+fp4_status fp4_quantize(const void *x_bf16, void *codes, void *scales, float *tensor_scale,
+                        int64_t rows, int64_t cols, fp4_format fmt, int hadamard_n,
+                        fp4_axis axis, fp4_stream_t stream);
+
+/*
+ * fp4_quantize_dual -- both layouts of fp4_quantize from ONE read of x: the row-wise
+ * result (row_codes, row_scales) and the column-wise transposed one (col_codes,
+ * col_scales), bit-identical to two separate fp4_quantize calls.
+ *   tensor_scale: NVFP4 -> device float[4], written {S_row, S_col, amax_row, amax_col}
+ *                 (each layout is scaled by the amax of its own rotation).
+ *                 MXFP4 -> must be NULL.
+ *   Shape: as fp4_quantize.
+ */
+fp4_status fp4_quantize_dual(const void *x_bf16, void *row_codes, void *row_scales,
+                             void *col_codes, void *col_scales, float *tensor_scale,
+                             int64_t rows, int64_t cols, fp4_format fmt, int hadamard_n,
+                             fp4_stream_t stream);
+
+/*
+ * fp4_gemm -- C[M][N] = deq(A)[M][K] * deq(B)[N][K]^T with fp32 accumulation on the
+ * sm_100a block-scaled tensor cores (tcgen05.mma kind::mxf4 / kind::mxf4nvf4).
+ * [MXFP4 pre-training summary, Methodology item 2; NVFP4/MaxText page, Key facts 5.]
+ *   A_codes [M][K/2], A_scales (layout above, M rows); B likewise with N rows; both
+ *   quantised along K (fp4_quantize ROW of an [M][K] / [N][K] matrix, or COL of the
+ *   transposed one).
+ *   A_tensor_scale, B_tensor_scale: NVFP4 -> device float* to S of each operand; the
+ *   epilogue multiplies by S_A*S_B (fp32). MXFP4 -> must be NULL.
+ *   C: row-major [M][N], fp32 or bf16 (round-to-nearest-even of the fp32 result).
+ *   Shape: M, N, K multiples of 32 (0 -> nothing is done).
+ */
+fp4_status fp4_gemm(const void *A_codes, const void *A_scales, const float *A_tensor_scale,
+                    const void *B_codes, const void *B_scales, const float *B_tensor_scale,
+                    void *C, int64_t M, int64_t N, int64_t K, fp4_format fmt,
+                    fp4_out_dtype out_dtype, fp4_stream_t stream);
+
+/*
+ * The three passes of a linear layer Y = X W^T with X [M][K], W [N][K], dY [M][N],
+ * each quantising its operands along its own contraction axis and multiplying them.
+ * [MXFP4 pre-training summary, Methodology item 2: Fprop, Dgrad, Wgrad.]
+ *   fprop: Y [M][N]  = Q_row(X) . Q_row(W)^T                  (contraction over K)
+ *   dgrad: dX [M][K] = Q_row(dY) . Q_col(W)^T  (W along N)    (contraction over N)
+ *   wgrad: dW [N][K] = Q_col(dY) . Q_col(X)^T  (along tokens) (contraction over M)
+ * ws / ws_bytes: caller-owned device scratch of at least fp4_linear_workspace_size()
+ * bytes; it receives the quantised operands (and NVFP4 tensor scales) in an
+ * unspecified layout. Shape: M, N, K multiples of 32.
+ */
+size_t fp4_linear_workspace_size(fp4_pass pass, int64_t M, int64_t N, int64_t K, fp4_format fmt);
+
+fp4_status fp4_linear_fprop(const void *X, const void *W, void *Y, int64_t M, int64_t N, int64_t K,
+                            fp4_format fmt, int hadamard_n, fp4_out_dtype out_dtype, void *ws,
+                            size_t ws_bytes, fp4_stream_t stream);
+fp4_status fp4_linear_dgrad(const void *dY, const void *W, void *dX, int64_t M, int64_t N,
+                            int64_t K, fp4_format fmt, int hadamard_n, fp4_out_dtype out_dtype,
+                            void *ws, size_t ws_bytes, fp4_stream_t stream);
+fp4_status fp4_linear_wgrad(const void *dY, const void *X, void *dW, int64_t M, int64_t N,
+                            int64_t K, fp4_format fmt, int hadamard_n, fp4_out_dtype out_dtype,
+                            void *ws, size_t ws_bytes, fp4_stream_t stream);
+
+/*
+ * fp4_check_status -- synchronises `stream`, then returns and clears the device
+ * status word of the current device: FP4_ERR_TIMEOUT if any kernel's bounded wait
+ * gave up since the last check, FP4_ERR_CUDA if the synchronisation failed, else
+ * FP4_OK.
+ */
+fp4_status fp4_check_status(fp4_stream_t stream);
+
+/*
+ * fp4_selftest_timeout -- launches one tiny kernel that waits on a pipeline barrier
+ * nobody arrives at, using the same bounded wait as the GEMM and quantise kernels,
+ * with a limit of timeout_ns nanoseconds. It gives up, records FP4_ERR_TIMEOUT in
+ * the status word and returns normally; no fault, no trap. Used to test the
+ * failure-reporting path.
+ */
+fp4_status fp4_selftest_timeout(uint64_t timeout_ns, fp4_stream_t stream);
+
+/* Static English text for a status code. */
+const char *fp4_status_string(fp4_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP4_H_ */

@@ -1,0 +1,247 @@
+"""CPU oracle for the rotate -> FP4-quantise -> block-scaled GEMM path.
+
+TEST INFRASTRUCTURE. Only the test suite, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package. It shares no code with
+the CUDA library (``fp4_block_scaled_deterministic_b200``) and never imports it.
+
+The arithmetic lives in ``fp4_oracle.c`` (plain scalar C, fp32 where the method
+computes in fp32, fp64 for the GEMM reference); this module only compiles it with
+gcc and marshals numpy arrays. See the header of ``fp4_oracle.c`` for the pages
+each step follows and for every reading taken where the pages are silent.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+MXFP4, NVFP4 = 0, 1
+ROW, COL = 0, 1
+BLOCK = {MXFP4: 32, NVFP4: 16}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fp4_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile fp4_oracle.c with gcc. No fast-math and no FP contraction, so every
+    fp32 operation rounds once, as IEEE 754 prescribes."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
+               "-shared", _SRC, "-o", _LIB + ".tmp", "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+def _L():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        i64 = ctypes.c_int64
+        lib.fp4o_e2m1_decode.restype = ctypes.c_double
+        lib.fp4o_e2m1_decode.argtypes = [ctypes.c_uint8]
+        lib.fp4o_e2m1_encode.restype = ctypes.c_uint8
+        lib.fp4o_e2m1_encode.argtypes = [ctypes.c_float]
+        lib.fp4o_mx_scale_exponent.restype = ctypes.c_int
+        lib.fp4o_mx_scale_exponent.argtypes = [ctypes.c_float]
+        lib.fp4o_e4m3_decode.restype = ctypes.c_double
+        lib.fp4o_e4m3_decode.argtypes = [ctypes.c_uint8]
+        lib.fp4o_e4m3_encode.restype = ctypes.c_uint8
+        lib.fp4o_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.fp4o_hadamard_scale.restype = ctypes.c_float
+        lib.fp4o_hadamard_scale.argtypes = [ctypes.c_int]
+        lib.fp4o_fwht_f32.restype = None
+        lib.fp4o_fwht_f32.argtypes = [P, ctypes.c_int]
+        lib.fp4o_rotate.restype = ctypes.c_int
+        lib.fp4o_rotate.argtypes = [P, i64, i64, ctypes.c_int, ctypes.c_int, P]
+        lib.fp4o_scale_layout_bytes.restype = i64
+        lib.fp4o_scale_layout_bytes.argtypes = [i64, i64]
+        lib.fp4o_scale_offset.restype = i64
+        lib.fp4o_scale_offset.argtypes = [i64, i64, i64]
+        lib.fp4o_quantize_block_mx.restype = None
+        lib.fp4o_quantize_block_mx.argtypes = [P, ctypes.c_int, P, P]
+        lib.fp4o_quantize_block_nv.restype = None
+        lib.fp4o_quantize_block_nv.argtypes = [P, ctypes.c_int, ctypes.c_float, P, P]
+        lib.fp4o_nv_tensor_scale.restype = ctypes.c_float
+        lib.fp4o_nv_tensor_scale.argtypes = [ctypes.c_float]
+        lib.fp4o_quantize.restype = ctypes.c_int
+        lib.fp4o_quantize.argtypes = [P, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                      P, P, P, P]
+        lib.fp4o_dequantize.restype = None
+        lib.fp4o_dequantize.argtypes = [P, P, ctypes.c_float, i64, i64, ctypes.c_int, P]
+        lib.fp4o_gemm_f64.restype = None
+        lib.fp4o_gemm_f64.argtypes = [P, P, P, i64, i64, i64]
+        lib.fp4o_gemm_entries.restype = None
+        lib.fp4o_gemm_entries.argtypes = [P, P, ctypes.c_float, P, P, ctypes.c_float, i64,
+                                          ctypes.c_int, P, P, i64, P]
+        for name, t_in, t_out in (("fp4o_e2m1_encode_array", P, P),
+                                  ("fp4o_e4m3_encode_array", P, P),
+                                  ("fp4o_mx_scale_exponent_array", P, P)):
+            f = getattr(lib, name)
+            f.restype = None
+            f.argtypes = [t_in, t_out, i64]
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+# ----------------------------------------------------------------- scalar codecs
+
+def e2m1_decode(nibble: int) -> float:
+    return _L().fp4o_e2m1_decode(nibble)
+
+
+def e2m1_encode(q) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.float32)
+    out = np.empty(q.shape, np.uint8)
+    _L().fp4o_e2m1_encode_array(_ptr(q), _ptr(out), q.size)
+    return out
+
+
+def e4m3_decode(code: int) -> float:
+    return _L().fp4o_e4m3_decode(code)
+
+
+def e4m3_encode(t) -> np.ndarray:
+    t = np.ascontiguousarray(t, dtype=np.float32)
+    out = np.empty(t.shape, np.uint8)
+    _L().fp4o_e4m3_encode_array(_ptr(t), _ptr(out), t.size)
+    return out
+
+
+def mx_scale_exponent(amax) -> np.ndarray:
+    a = np.ascontiguousarray(amax, dtype=np.float32)
+    out = np.empty(a.shape, np.int32)
+    _L().fp4o_mx_scale_exponent_array(_ptr(a), _ptr(out), a.size)
+    return out
+
+
+def hadamard_scale(n: int) -> float:
+    return _L().fp4o_hadamard_scale(n)
+
+
+def fwht(v) -> np.ndarray:
+    """Normalised in-place FWHT of one fp32 group (length a power of two)."""
+    v = np.array(v, dtype=np.float32, copy=True)
+    _L().fp4o_fwht_f32(_ptr(v), v.size)
+    return v
+
+
+def scale_offset(r: int, kb: int, kblocks: int) -> int:
+    return _L().fp4o_scale_offset(r, kb, kblocks)
+
+
+def scale_layout_bytes(rows: int, kblocks: int) -> int:
+    return _L().fp4o_scale_layout_bytes(rows, kblocks)
+
+
+def quantize_block_mx(v, bs=None):
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    bs = v.size if bs is None else bs
+    codes = np.empty(bs, np.uint8)
+    sb = np.zeros(1, np.uint8)
+    _L().fp4o_quantize_block_mx(_ptr(v), bs, _ptr(codes), _ptr(sb))
+    return codes, int(sb[0])
+
+
+def quantize_block_nv(v, S: float, bs=None):
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    bs = v.size if bs is None else bs
+    codes = np.empty(bs, np.uint8)
+    sb = np.zeros(1, np.uint8)
+    _L().fp4o_quantize_block_nv(_ptr(v), bs, S, _ptr(codes), _ptr(sb))
+    return codes, int(sb[0])
+
+
+def nv_tensor_scale(amax: float) -> float:
+    return _L().fp4o_nv_tensor_scale(amax)
+
+
+# ----------------------------------------------------------------- tensors
+
+def _bf16_bits(x) -> np.ndarray:
+    """Accept a uint16 array of bf16 bit patterns or a torch bf16 CPU tensor."""
+    if isinstance(x, np.ndarray):
+        assert x.dtype == np.uint16
+        return np.ascontiguousarray(x)
+    import torch  # plumbing only: reinterpret bits
+    assert x.dtype == torch.bfloat16 and x.device.type == "cpu"
+    return np.ascontiguousarray(x.contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+def rotate(x, hn: int, axis: int = ROW) -> np.ndarray:
+    xb = _bf16_bits(x)
+    rows, cols = xb.shape
+    R, C = (rows, cols) if axis == ROW else (cols, rows)
+    out = np.empty((R, C), np.float32)
+    if _L().fp4o_rotate(_ptr(xb), rows, cols, hn, axis, _ptr(out)) != 0:
+        raise ValueError("rotation group does not divide the axis")
+    return out
+
+
+def quantize(x, fmt: int, hn: int, axis: int = ROW):
+    """Returns (codes [R][C/2] uint8, scales (layout R7) uint8, S, amax) where
+    (R, C) = x.shape for ROW and x.shape[::-1] for COL. S and amax are None for MXFP4."""
+    xb = _bf16_bits(x)
+    rows, cols = xb.shape
+    R, C = (rows, cols) if axis == ROW else (cols, rows)
+    bs = BLOCK[fmt]
+    codes = np.zeros((R, C // 2), np.uint8)
+    scales = np.zeros(scale_layout_bytes(R, C // bs), np.uint8)
+    s = np.zeros(1, np.float32)
+    t = np.zeros(1, np.float32)
+    rc = _L().fp4o_quantize(_ptr(xb), rows, cols, fmt, hn, axis, _ptr(codes), _ptr(scales),
+                            _ptr(s), _ptr(t))
+    if rc != 0:
+        raise ValueError(f"oracle quantize rejected shape {xb.shape} fmt={fmt} hn={hn} axis={axis}")
+    if fmt == NVFP4:
+        return codes, scales, float(s[0]), float(t[0])
+    return codes, scales, None, None
+
+
+def dequantize(codes: np.ndarray, scales: np.ndarray, tensor_scale, fmt: int) -> np.ndarray:
+    R, C2 = codes.shape
+    out = np.empty((R, 2 * C2), np.float64)
+    ts = 1.0 if tensor_scale is None else float(tensor_scale)
+    _L().fp4o_dequantize(_ptr(np.ascontiguousarray(codes)), _ptr(np.ascontiguousarray(scales)),
+                         ts, R, 2 * C2, fmt, _ptr(out))
+    return out
+
+
+def gemm_f64(A: np.ndarray, B: np.ndarray) -> np.ndarray:
+    """C = A @ B.T in fp64 by the plain triple loop (A [M][K], B [N][K])."""
+    A = np.ascontiguousarray(A, dtype=np.float64)
+    B = np.ascontiguousarray(B, dtype=np.float64)
+    M, K = A.shape
+    N = B.shape[0]
+    C = np.empty((M, N), np.float64)
+    _L().fp4o_gemm_f64(_ptr(A), _ptr(B), _ptr(C), M, N, K)
+    return C
+
+
+def gemm_entries(a_q, b_q, fmt: int, ms, ns) -> np.ndarray:
+    """Entries (ms[i], ns[i]) of deq(A) @ deq(B).T from quantised operands
+    a_q = (codes, scales, S) of A [M][K] and b_q likewise of B [N][K]."""
+    ac, asc, ats = a_q
+    bc, bsc, bts = b_q
+    K = ac.shape[1] * 2
+    ms = np.ascontiguousarray(ms, dtype=np.int64)
+    ns = np.ascontiguousarray(ns, dtype=np.int64)
+    out = np.empty(ms.size, np.float64)
+    _L().fp4o_gemm_entries(_ptr(np.ascontiguousarray(ac)), _ptr(np.ascontiguousarray(asc)),
+                           1.0 if ats is None else float(ats),
+                           _ptr(np.ascontiguousarray(bc)), _ptr(np.ascontiguousarray(bsc)),
+                           1.0 if bts is None else float(bts), K, fmt, _ptr(ms), _ptr(ns),
+                           ms.size, _ptr(out))
+    return out

@@ -1,0 +1,350 @@
+/*
+ * fp4_oracle.c -- plain, slow, scalar CPU oracle for the 4-bit linear-layer path:
+ *   deterministic block Hadamard rotation (H16 / H32) along the contraction axis
+ *   -> microscaled FP4 quantisation (MXFP4 or NVFP4, E2M1 codes, two per byte)
+ *   -> block-scaled FP4 GEMM, evaluated here in fp64 on the dequantised operands.
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the smoke check and the benchmark's
+ * CPU-baseline leg may load this file. It shares no code, header, table or
+ * constant with the CUDA library: every encoder below is written from the
+ * format definitions, not from the kernels.
+ *
+ * Sources (web pages; cited by title and section):
+ *   [MXFP4-PT]  gist.science, "기술 요약: MXFP4 를 활용한 대규모 언어 모델 사전 학습"
+ *               (summary of arXiv 2605.09825).
+ *               - "방법론" (Methodology), item 2: Fprop, Dgrad and Wgrad are each run
+ *                 in MXFP4.
+ *               - "방법론", item 3: deterministic Hadamard rotations with 16x16 (H16)
+ *                 and 32x32 (H32) matrices.
+ *               - "주요 기여 및 발견" (Findings) section 2: deterministic H16 restores
+ *                 stability of the full MXFP4 pipeline.
+ *   [NVFP4-MT]  molayo1419.me, "Blackwell의 NVIDIA NVFP4, MaxText에서 JAX 학습 속도 1.8배
+ *               향상": "주요 사실" (Key facts), 2nd bullet: two 4-bit values are packed
+ *               into one 8-bit register; body, first paragraph: a shared exponent keeps
+ *               the dynamic range.
+ *   The pages name the formats but do not spell out their numerics. The format
+ *   definitions used here are: MXFP4 = 32-element blocks sharing one power-of-two
+ *   E8M0 scale taken from the block amax, E2M1 elements {0, +-0.5, +-1, +-1.5, +-2,
+ *   +-3, +-4, +-6} with round-to-nearest-even; NVFP4 = 16-element blocks with an
+ *   E4M3 block scale under an fp32 per-tensor scale amax / (6 * 448).
+ *
+ * Readings where the pages are silent (each is a choice, listed with the others
+ * in the design notes of the repository):
+ *   R1  Rotation: Sylvester Hadamard, applied to each aligned group of hn elements
+ *       along the contraction axis as an in-place butterfly with strides
+ *       h = 1, 2, 4, ..., hn/2 in that order, each sum and difference rounded to
+ *       fp32, then every element multiplied by c_hn = RN_fp32(1/sqrt(hn)).
+ *       The rotated values stay fp32.
+ *   R2  MX scale exponent e = floor(log2(amax)) - 2 (2 = largest E2M1 exponent),
+ *       clamped to [-127, 127]; amax == 0 gives e = -127. Scale byte = e + 127.
+ *   R3  MX element: q = v * 2^-e (fp32), code = E2M1_RNE_satfinite(q).
+ *   R4  E2M1 rounding: nearest of the 8 magnitudes, ties to the even code,
+ *       magnitudes above 6 saturate to 6, the sign bit of q is kept even when
+ *       the magnitude rounds to zero.
+ *   R5  NVFP4: T = max|v| over the whole rotated tensor, S = T / 2688 (fp32; S = 1
+ *       when T == 0); per 16-block t = B / (6 * S) (two fp32 roundings),
+ *       sb = E4M3_RNE_satfinite(t); d = decode(sb) * S (fp32); q = v / d (fp32
+ *       division); sb == 0 gives signed zero codes.
+ *   R6  Packing: element 2i in the low nibble of byte i, element 2i+1 in the high
+ *       nibble; nibble = sign << 3 | magnitude index.
+ *   R7  Scale layout: scale (r, kb) of a matrix with KB = cols / bs blocks per row
+ *       lives at byte ((r/128) * KB4 + kb/4) * 512 + (r%32) * 16 + ((r%128)/32) * 4
+ *       + kb%4, KB4 = ceil(KB/4); rows are padded to a multiple of 128 and KB to a
+ *       multiple of 4; padding bytes are zero.
+ *   R8  Column-wise ("COL") quantisation of x[R][C] quantises x^T: codes [C][R/2],
+ *       scales laid out for a [C][R/bs] scale matrix.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define FP4O_MXFP4 0
+#define FP4O_NVFP4 1
+#define FP4O_ROW 0
+#define FP4O_COL 1
+
+/* ---------------------------------------------------------------- bit helpers */
+
+static float bits_to_f32(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
+static uint32_t f32_to_bits(float f) { uint32_t u; memcpy(&u, &f, 4); return u; }
+
+/* bf16 -> fp32 is exact: the bf16 pattern is the upper half of the fp32 pattern. */
+float fp4o_bf16_to_f32(uint16_t b) { return bits_to_f32((uint32_t)b << 16); }
+
+/* ---------------------------------------------------------------- E2M1 */
+
+/* The eight E2M1 magnitudes indexed by the 3-bit magnitude field (exponent bias 1,
+ * one mantissa bit, subnormal 0.5). */
+static const double E2M1_MAG[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+double fp4o_e2m1_decode(uint8_t nibble) {
+    double m = E2M1_MAG[nibble & 7];
+    return (nibble & 8) ? -m : m;
+}
+
+/* R4. The thresholds are the midpoints between neighbouring magnitudes; a value
+ * exactly on a midpoint goes to the neighbour with the even magnitude index
+ * (index parity = mantissa bit), so "<=" is used where the lower neighbour is
+ * even and "<" where the upper one is. */
+uint8_t fp4o_e2m1_encode(float q) {
+    uint8_t sign = (f32_to_bits(q) >> 31) ? 8 : 0;
+    float a = fabsf(q);
+    uint8_t idx;
+    if (a <= 0.25f)      idx = 0;  /* midpoint 0.25 between 0 (idx 0) and 0.5 (idx 1) */
+    else if (a < 0.75f)  idx = 1;  /* midpoint 0.75 between 0.5 (idx 1) and 1 (idx 2) */
+    else if (a <= 1.25f) idx = 2;  /* midpoint 1.25 between 1 (idx 2) and 1.5 (idx 3) */
+    else if (a < 1.75f)  idx = 3;  /* midpoint 1.75 between 1.5 (idx 3) and 2 (idx 4) */
+    else if (a <= 2.5f)  idx = 4;  /* midpoint 2.5 between 2 (idx 4) and 3 (idx 5) */
+    else if (a < 3.5f)   idx = 5;  /* midpoint 3.5 between 3 (idx 5) and 4 (idx 6) */
+    else if (a <= 5.0f)  idx = 6;  /* midpoint 5 between 4 (idx 6) and 6 (idx 7) */
+    else                 idx = 7;  /* everything above saturates to 6 */
+    return (uint8_t)(sign | idx);
+}
+
+/* ---------------------------------------------------------------- E8M0 */
+
+/* R2. floor(log2(amax)) is read exactly with frexp: amax = f * 2^ex, f in [0.5, 1),
+ * so floor(log2(amax)) = ex - 1, also for subnormal amax. */
+int fp4o_mx_scale_exponent(float amax) {
+    if (!(amax > 0.0f)) return -127;
+    int ex;
+    (void)frexpf(amax, &ex);
+    int e = (ex - 1) - 2;
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+    return e;
+}
+
+double fp4o_e8m0_decode(uint8_t b) { return ldexp(1.0, (int)b - 127); }
+
+/* ---------------------------------------------------------------- E4M3 (OCP FP8) */
+
+/* E4M3: exponent bias 7, 3 mantissa bits, subnormals k * 2^-9 (k = 1..7), largest
+ * finite 448 (code 0x7E), code 0x7F is NaN, no infinity. */
+double fp4o_e4m3_decode(uint8_t c) {
+    int s = (c >> 7) & 1, E = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (E == 15 && m == 7) return NAN;
+    if (E == 0) v = ldexp((double)m, -9);
+    else v = ldexp(1.0 + m / 8.0, E - 7);
+    return s ? -v : v;
+}
+
+/* Round to nearest even with saturation to +-448. The code of a finite magnitude
+ * is 8 * (E + 7) + m for normal values and k for subnormal ones, which is one
+ * monotone integer scale, so rounding the mantissa step count with nearbyint
+ * (round-half-even in the default rounding mode) and letting a carry flow into
+ * the exponent gives the RNE code directly; an even step count is an even code. */
+uint8_t fp4o_e4m3_encode(float t) {
+    uint8_t sign = (f32_to_bits(t) >> 31) ? 0x80 : 0;
+    double a = fabs((double)t);
+    if (isnan(t)) return 0x7F;
+    if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+    long code;
+    if (a < ldexp(1.0, -6)) {
+        code = (long)nearbyint(a * 512.0);                 /* steps of 2^-9 */
+    } else {
+        int ex;
+        double f = frexp(a, &ex);                          /* a = f * 2^ex, f in [0.5,1) */
+        int E = ex - 1;                                    /* a in [2^E, 2^(E+1)) */
+        long m = (long)nearbyint((ldexp(f, 1) - 1.0) * 8.0); /* 0..8 */
+        code = 8L * (E + 7) + m;
+    }
+    if (code > 0x7E) code = 0x7E;
+    return (uint8_t)(sign | (uint8_t)code);
+}
+
+/* ---------------------------------------------------------------- rotation (R1) */
+
+#define FP4O_C32_BITS 0x3E3504F3u /* RN_fp32(1/sqrt(32)) */
+
+float fp4o_hadamard_scale(int n) {
+    if (n == 16) return 0.25f;
+    if (n == 32) return bits_to_f32(FP4O_C32_BITS);
+    return (float)(1.0 / sqrt((double)n));
+}
+
+/* In-place normalised fast Walsh-Hadamard transform of one group of n (a power of
+ * two) fp32 values, Sylvester (natural) order, strides 1, 2, 4, ... in that order. */
+void fp4o_fwht_f32(float *v, int n) {
+    for (int h = 1; h < n; h <<= 1) {
+        for (int i = 0; i < n; i++) {
+            if ((i & h) == 0) {
+                float a = v[i], b = v[i + h];
+                v[i] = a + b;
+                v[i + h] = a - b;
+            }
+        }
+    }
+    float c = fp4o_hadamard_scale(n);
+    for (int i = 0; i < n; i++) v[i] = v[i] * c;
+}
+
+/* Rotate a bf16 matrix along its contraction axis. For axis ROW the groups run along
+ * each row of x[rows][cols] and out is [rows][cols]; for axis COL they run down each
+ * column and out is the transpose, [cols][rows] (R8). hn == 0 only widens. */
+int fp4o_rotate(const uint16_t *x, int64_t rows, int64_t cols, int hn, int axis, float *out) {
+    int64_t R = axis == FP4O_ROW ? rows : cols, C = axis == FP4O_ROW ? cols : rows;
+    if (hn != 0 && (C % hn) != 0) return -1;
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t c = 0; c < C; c++)
+            out[r * C + c] = fp4o_bf16_to_f32(axis == FP4O_ROW ? x[r * cols + c] : x[c * cols + r]);
+    if (hn != 0)
+        for (int64_t r = 0; r < R; r++)
+            for (int64_t g = 0; g < C; g += hn) fp4o_fwht_f32(out + r * C + g, hn);
+    return 0;
+}
+
+/* ---------------------------------------------------------------- scale layout (R7) */
+
+int64_t fp4o_scale_layout_bytes(int64_t rows, int64_t kblocks) {
+    int64_t rp = (rows + 127) / 128 * 128, kp = (kblocks + 3) / 4 * 4;
+    return rp * kp;
+}
+
+int64_t fp4o_scale_offset(int64_t r, int64_t kb, int64_t kblocks) {
+    int64_t kb4 = (kblocks + 3) / 4;
+    return ((r / 128) * kb4 + kb / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + (kb % 4);
+}
+
+/* ---------------------------------------------------------------- block quantisers */
+
+/* MX block (R2, R3): bs values -> bs codes (one per byte, unpacked) and one E8M0 byte. */
+void fp4o_quantize_block_mx(const float *v, int bs, uint8_t *codes, uint8_t *scale_byte) {
+    float amax = 0.0f;
+    for (int i = 0; i < bs; i++) amax = fmaxf(amax, fabsf(v[i]));
+    int e = fp4o_mx_scale_exponent(amax);
+    float inv = (float)ldexp(1.0, -e); /* 2^-e, exact in fp32 for e in [-127, 127] */
+    for (int i = 0; i < bs; i++) codes[i] = fp4o_e2m1_encode(v[i] * inv);
+    *scale_byte = (uint8_t)(e + 127);
+}
+
+/* NV tensor scale (R5). */
+float fp4o_nv_tensor_scale(float tensor_amax) {
+    if (!(tensor_amax > 0.0f)) return 1.0f;
+    return tensor_amax / 2688.0f;
+}
+
+/* NV block (R5): bs values -> bs codes and one UE4M3 byte, under tensor scale S. */
+void fp4o_quantize_block_nv(const float *v, int bs, float S, uint8_t *codes, uint8_t *scale_byte) {
+    float bmax = 0.0f;
+    for (int i = 0; i < bs; i++) bmax = fmaxf(bmax, fabsf(v[i]));
+    float six_s = 6.0f * S;
+    float t = bmax / six_s;
+    uint8_t sb = fp4o_e4m3_encode(t);
+    float d = (float)fp4o_e4m3_decode(sb) * S; /* decode is exact in fp32; one rounding */
+    for (int i = 0; i < bs; i++) {
+        if (sb == 0) codes[i] = (f32_to_bits(v[i]) >> 31) ? 8 : 0;
+        else codes[i] = fp4o_e2m1_encode(v[i] / d);
+    }
+    *scale_byte = sb;
+}
+
+/* ---------------------------------------------------------------- tensor quantiser */
+
+/* Quantise x[rows][cols] (bf16 bit patterns) along `axis`.
+ *   codes:  [R][C/2] bytes, R x C = rows x cols (ROW) or cols x rows (COL)
+ *   scales: fp4o_scale_layout_bytes(R, C/bs) bytes, written in layout R7
+ *   nv_scale_out / nv_amax_out: NVFP4 only (may be NULL otherwise)
+ * Returns 0, or -1 on a shape the format cannot block. */
+int fp4o_quantize(const uint16_t *x, int64_t rows, int64_t cols, int fmt, int hn, int axis,
+                  uint8_t *codes, uint8_t *scales, float *nv_scale_out, float *nv_amax_out) {
+    int bs = fmt == FP4O_MXFP4 ? 32 : 16;
+    int64_t R = axis == FP4O_ROW ? rows : cols, C = axis == FP4O_ROW ? cols : rows;
+    if (C % bs != 0 || (hn != 0 && C % hn != 0) || C % 2 != 0) return -1;
+    int64_t KB = C / bs;
+    float *v = (float *)malloc(sizeof(float) * (size_t)(R * C > 0 ? R * C : 1));
+    if (!v) return -2;
+    /* steps 1-2: widen, rotate */
+    fp4o_rotate(x, rows, cols, hn, axis, v);
+    /* step 3 (NVFP4 only): tensor amax of the rotated values and the tensor scale */
+    float S = 1.0f;
+    if (fmt == FP4O_NVFP4) {
+        float T = 0.0f;
+        for (int64_t i = 0; i < R * C; i++) T = fmaxf(T, fabsf(v[i]));
+        S = fp4o_nv_tensor_scale(T);
+        if (nv_scale_out) *nv_scale_out = S;
+        if (nv_amax_out) *nv_amax_out = T;
+    }
+    /* steps 4-5: block scales and codes; step 6: pack */
+    memset(scales, 0, (size_t)fp4o_scale_layout_bytes(R, KB));
+    uint8_t blk[32];
+    for (int64_t r = 0; r < R; r++) {
+        for (int64_t kb = 0; kb < KB; kb++) {
+            const float *bv = v + r * C + kb * bs;
+            uint8_t sb;
+            if (fmt == FP4O_MXFP4) fp4o_quantize_block_mx(bv, bs, blk, &sb);
+            else fp4o_quantize_block_nv(bv, bs, S, blk, &sb);
+            scales[fp4o_scale_offset(r, kb, KB)] = sb;
+            for (int i = 0; i < bs; i += 2)
+                codes[r * (C / 2) + (kb * bs + i) / 2] = (uint8_t)(blk[i] | (blk[i + 1] << 4));
+        }
+    }
+    free(v);
+    return 0;
+}
+
+/* ---------------------------------------------------------------- dequantisation */
+
+/* Value of element (r, c) of a quantised [R][C] matrix, exactly, in fp64. */
+static double deq_elem(const uint8_t *codes, const uint8_t *scales, double S, int64_t C, int fmt,
+                       int64_t r, int64_t c) {
+    int bs = fmt == FP4O_MXFP4 ? 32 : 16;
+    int64_t KB = C / bs;
+    uint8_t byte = codes[r * (C / 2) + c / 2];
+    uint8_t nib = (c & 1) ? (byte >> 4) : (byte & 15);
+    uint8_t sb = scales[fp4o_scale_offset(r, c / bs, KB)];
+    double q = fp4o_e2m1_decode(nib);
+    if (fmt == FP4O_MXFP4) return q * fp4o_e8m0_decode(sb);
+    return q * fp4o_e4m3_decode(sb) * S;
+}
+
+void fp4o_dequantize(const uint8_t *codes, const uint8_t *scales, float tensor_scale, int64_t R,
+                     int64_t C, int fmt, double *out) {
+    double S = fmt == FP4O_NVFP4 ? (double)tensor_scale : 1.0;
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t c = 0; c < C; c++) out[r * C + c] = deq_elem(codes, scales, S, C, fmt, r, c);
+}
+
+/* ---------------------------------------------------------------- GEMM */
+
+/* C[m][n] = sum_k A[m][k] * B[n][k] in fp64 (both operands K-major). */
+void fp4o_gemm_f64(const double *A, const double *B, double *Cm, int64_t M, int64_t N, int64_t K) {
+    for (int64_t m = 0; m < M; m++)
+        for (int64_t n = 0; n < N; n++) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; k++) acc += A[m * K + k] * B[n * K + k];
+            Cm[m * N + n] = acc;
+        }
+}
+
+/* Selected entries of the block-scaled GEMM C = deq(A) * deq(B)^T, computed from the
+ * quantised operands directly (A is [M][K], B is [N][K], both quantised along K). */
+void fp4o_gemm_entries(const uint8_t *a_codes, const uint8_t *a_scales, float a_ts,
+                       const uint8_t *b_codes, const uint8_t *b_scales, float b_ts, int64_t K,
+                       int fmt, const int64_t *ms, const int64_t *ns, int64_t count, double *out) {
+    double SA = fmt == FP4O_NVFP4 ? (double)a_ts : 1.0;
+    double SB = fmt == FP4O_NVFP4 ? (double)b_ts : 1.0;
+    for (int64_t i = 0; i < count; i++) {
+        double acc = 0.0;
+        for (int64_t k = 0; k < K; k++)
+            acc += deq_elem(a_codes, a_scales, SA, K, fmt, ms[i], k) *
+                   deq_elem(b_codes, b_scales, SB, K, fmt, ns[i], k);
+        out[i] = acc;
+    }
+}
+
+/* ---------------------------------------------------------------- array helpers */
+
+void fp4o_e2m1_encode_array(const float *q, uint8_t *out, int64_t n) {
+    for (int64_t i = 0; i < n; i++) out[i] = fp4o_e2m1_encode(q[i]);
+}
+
+void fp4o_e4m3_encode_array(const float *t, uint8_t *out, int64_t n) {
+    for (int64_t i = 0; i < n; i++) out[i] = fp4o_e4m3_encode(t[i]);
+}
+
+void fp4o_mx_scale_exponent_array(const float *a, int32_t *out, int64_t n) {
+    for (int64_t i = 0; i < n; i++) out[i] = fp4o_mx_scale_exponent(a[i]);
+}
