@@ -1,0 +1,466 @@
+"""Benchmark of the 4-bit linear layer on B200: one step = the forward and backward
+passes of every projection of a Llama-3.1-8B transformer layer (QKV, O, gate, up,
+down) on 8192 tokens, each pass rotated (H16), quantised (MXFP4) and multiplied on
+the FP4 tensor cores:
+
+    per projection: dual-layout quantise of X, W and dY (3 kernels),
+                    Fprop Y = X W^T (bf16 out), Dgrad dX = dY W (bf16 out),
+                    Wgrad dW = dY^T X (fp32 out)  -> 3 GEMM kernels
+    with N > 1 ranks: data parallel over tokens (8192 per rank), dW all-reduced
+    (NCCL) per projection, overlapped with the next projection.
+
+Prints ONE JSON line (rank 0). `value` is the step's GEMM FLOPs divided by the step
+time (quantisation included), summed over ranks. Inputs are synthetic, seeded, and
+resident in HBM before the timed region; the step's working set (~4 GB) is far
+larger than L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fp4|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "FP4 GEMM TFLOPS (fprop/dgrad/wgrad) + H16-quantize GB/s, % of B200 roofline"
+FP4_OVER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput (9 : 2.25 PFLOP/s)
+PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+WORKLOAD = ("llama3.1-8b layer fwd+bwd: qkv 6144x4096, o 4096x4096, gate/up 14336x4096, "
+            "down 4096x14336; 8192 tokens/rank; MXFP4 + H16")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["fp4", "reference"], default="fp4")
+    ap.add_argument("--format", choices=["mxfp4", "nvfp4"], default="mxfp4")
+    ap.add_argument("--hadamard", type=int, default=16, choices=[0, 16, 32])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    a = ap.parse_args()
+    a.warmup = max(3, a.warmup)
+    return a
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d, "measured"
+    return dict(PEAK_FALLBACK), "fallback"
+
+
+# ---------------------------------------------------------------- clocks sampler
+class Clocks:
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.sw_power_cap,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown")
+
+    def __init__(self, dev: int):
+        self.dev, self.proc, self.lines = dev, None, []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ("sw_power_cap", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+        for ln in self.lines:
+            p = [x.strip() for x in ln.split(",")]
+            if len(p) < 6:
+                continue
+            try:
+                sm.append(float(p[0]))
+                mx.append(float(p[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, p[2:6]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- workload
+class LlamaLayer:
+    """Inputs, quantised operands and outputs of every projection, all on the device."""
+
+    def __init__(self, device, fmt, hn, tokens=8192, seed=0):
+        import fp4_block_scaled_deterministic_b200 as fp4
+        from fp4_block_scaled_deterministic_b200 import synthetic
+        self.fp4, self.fmt, self.hn, self.M = fp4, fmt, hn, tokens
+        self.projs = []
+        g = torch.Generator(device=device)
+        for i, (name, N, K) in enumerate(synthetic.LLAMA_LAYERS):
+            X = synthetic.normal(tokens, K, 1.0, seed=seed + i, outlier_frac=0.001,
+                                 outlier_mult=50.0, device=device)
+            W = synthetic.normal(N, K, 0.02, seed=seed + 100 + i, device=device)
+            dY = synthetic.heavy_tailed_grad(tokens, N, 1e-3, seed=seed + 200 + i, device=device)
+            p = {"name": name, "N": N, "K": K, "X": X, "W": W, "dY": dY}
+            for key, (r, c) in (("X", (tokens, K)), ("W", (N, K)), ("dY", (tokens, N))):
+                p[key + "_row"] = self._qbuf(r, c, device)
+                p[key + "_col"] = self._qbuf(c, r, device)
+                p[key + "_ts"] = torch.zeros(4, dtype=torch.float32, device=device)
+            p["Y"] = torch.empty(tokens, N, dtype=torch.bfloat16, device=device)
+            p["dX"] = torch.empty(tokens, K, dtype=torch.bfloat16, device=device)
+            p["dW"] = torch.empty(N, K, dtype=torch.float32, device=device)
+            self.projs.append(p)
+        del g
+
+    def _qbuf(self, r, c, device):
+        f = self.fp4
+        return (torch.empty(r, c // 2, dtype=torch.uint8, device=device),
+                torch.empty(f.fp4_scales_bytes(r, c, self.fmt), dtype=torch.uint8, device=device))
+
+    def flops(self):
+        return sum(3 * 2.0 * self.M * p["N"] * p["K"] for p in self.projs)
+
+    def quant_elems(self):
+        return sum(self.M * p["K"] + p["N"] * p["K"] + self.M * p["N"] for p in self.projs)
+
+    def bytes_in(self):
+        return sum(t.numel() * t.element_size() for p in self.projs for t in (p["X"], p["W"], p["dY"]))
+
+    def bytes_out(self):
+        return sum(t.numel() * t.element_size() for p in self.projs for t in (p["Y"], p["dX"], p["dW"]))
+
+    def launches_per_step(self):
+        per_q = 1 if self.fmt == 0 else 2  # NVFP4 adds the amax pass (plus a memset)
+        return len(self.projs) * (3 * per_q + 3)
+
+    def step(self, stream, timers=None, allreduce=None):
+        """One fwd+bwd pass over every projection. timers: dict kind -> list of event
+        pairs to record around each quantise / GEMM launch."""
+        f, fmt, hn = self.fp4, self.fmt, self.hn
+        s = stream.cuda_stream
+        pending = []
+
+        def timed(kind, fn):
+            if timers is None:
+                return fn()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            r = fn()
+            e1.record(stream)
+            timers[kind].append((e0, e1))
+            return r
+
+        for p in self.projs:
+            for key, (r, c) in (("X", (self.M, p["K"])), ("W", (p["N"], p["K"])),
+                                ("dY", (self.M, p["N"]))):
+                row, col, ts = p[key + "_row"], p[key + "_col"], p[key + "_ts"]
+                st = timed("quant", lambda: f.fp4_quantize_dual(
+                    p[key], row[0], row[1], col[0], col[1], ts if fmt == 1 else None, r, c, fmt,
+                    hn, s))
+                assert st == 0, f.status_string(st)
+            tsx, tsw, tsy = p["X_ts"], p["W_ts"], p["dY_ts"]
+            nv = fmt == 1
+            M, N, K = self.M, p["N"], p["K"]
+            # Fprop: Y[M][N] = X_row . W_row^T
+            st = timed("gemm", lambda: f.fp4_gemm(
+                p["X_row"][0], p["X_row"][1], tsx[0:1] if nv else None, p["W_row"][0],
+                p["W_row"][1], tsw[0:1] if nv else None, p["Y"], M, N, K, fmt, 1, s))
+            assert st == 0
+            # Dgrad: dX[M][K] = dY_row . W_col^T  (contraction over N)
+            st = timed("gemm", lambda: f.fp4_gemm(
+                p["dY_row"][0], p["dY_row"][1], tsy[0:1] if nv else None, p["W_col"][0],
+                p["W_col"][1], tsw[1:2] if nv else None, p["dX"], M, K, N, fmt, 1, s))
+            assert st == 0
+            # Wgrad: dW[N][K] = dY_col . X_col^T  (contraction over the tokens)
+            st = timed("gemm", lambda: f.fp4_gemm(
+                p["dY_col"][0], p["dY_col"][1], tsy[1:2] if nv else None, p["X_col"][0],
+                p["X_col"][1], tsx[1:2] if nv else None, p["dW"], N, K, M, fmt, 0, s))
+            assert st == 0
+            if allreduce is not None:
+                pending.append(allreduce(p["dW"]))
+        for w in pending:
+            w.wait()
+
+
+def gemm_flops_of(layer):
+    per = []
+    for p in layer.projs:
+        per += [2.0 * layer.M * p["N"] * p["K"]] * 3
+    return per
+
+
+# ---------------------------------------------------------------- CPU baseline
+def cpu_oracle_rate(seconds_budget: float, fmt: int, hn: int):
+    """Time the oracle on a bounded sample of the same step: dual quantisation of a
+    row slice of every operand and a sample of GEMM outputs of every pass. Returns
+    (extrapolated seconds per full step, description, cores used)."""
+    import numpy as np
+    import oracle
+    from fp4_block_scaled_deterministic_b200 import synthetic
+    oracle.build()
+    M = 8192
+    rows = 64
+    q_time, q_elems, g_time, g_macs = 0.0, 0, 0.0, 0
+    t_start = time.perf_counter()
+    for i, (name, N, K) in enumerate(synthetic.LLAMA_LAYERS):
+        X = synthetic.normal(rows * 2, K, 1.0, seed=i, outlier_frac=0.001, outlier_mult=50.0)
+        W = synthetic.normal(rows * 2, K, 0.02, seed=100 + i)
+        t0 = time.perf_counter()
+        xq = oracle.quantize(X, fmt, hn, oracle.ROW)
+        oracle.quantize(X, fmt, hn, oracle.COL)
+        wq = oracle.quantize(W, fmt, hn, oracle.ROW)
+        oracle.quantize(W, fmt, hn, oracle.COL)
+        q_time += time.perf_counter() - t0
+        q_elems += 2 * X.numel() + 2 * W.numel()
+        rng = np.random.default_rng(2)
+        n_ent = 48
+        ms, ns = rng.integers(0, rows * 2, n_ent), rng.integers(0, rows * 2, n_ent)
+        t0 = time.perf_counter()
+        oracle.gemm_entries(xq[:3], wq[:3], fmt, ms, ns)
+        g_time += time.perf_counter() - t0
+        g_macs += n_ent * K
+        if time.perf_counter() - t_start > seconds_budget:
+            break
+    # full step: dual quantisation of X, W, dY of each projection, and 3 GEMMs
+    step_elems, step_macs = 0, 0
+    for name, N, K in synthetic.LLAMA_LAYERS:
+        step_elems += 2 * (M * K + N * K + M * N)
+        step_macs += 3 * M * N * K
+    t_step = q_time / q_elems * step_elems + g_time / g_macs * step_macs
+    desc = (f"oracle (scalar C, 1 thread): dual quantise of {rows * 2}-row slices of X and W "
+            f"of each projection and {48} GEMM outputs per projection "
+            f"({q_elems} elements, {g_macs} MACs, {q_time + g_time:.1f} s), extrapolated "
+            f"linearly to the full step")
+    return t_step, desc, 1
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    fmt = 0 if a.format == "mxfp4" else 1
+    from fp4_block_scaled_deterministic_b200 import synthetic
+    flops = sum(3 * 2.0 * 8192 * N * K for _, N, K in synthetic.LLAMA_LAYERS)
+    budget = max(2.0, 150.0 / (a.steps + a.warmup))
+    for _ in range(a.warmup):
+        cpu_oracle_rate(min(budget, 2.0), fmt, a.hadamard)
+    ts = []
+    desc = ""
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        t_step, desc, cores = cpu_oracle_rate(budget, fmt, a.hadamard)
+        ts.append(t_step)
+    wall = time.perf_counter() - t0
+    t_med = statistics.median(ts)
+    value = flops / t_med / 1e12
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": a.gpus,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": t_med * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD, "format": a.format, "hadamard_n": a.hadamard,
+                       "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                             "sample": desc, "wall_s": wall},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- traffic record
+def recorded_traffic(kernel_key: str):
+    """dram bytes per launch of the dominant kernel from the committed ncu summary,
+    valid only while the kernel sources hash to the value recorded with it."""
+    path = os.path.join(ROOT, "profiles", "gemm_llama_traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        rec = json.load(open(path))
+    except ValueError:
+        return None
+    if rec.get("source_sha1") != kernel_source_hash():
+        return None
+    return rec.get("per_launch_bytes", {}).get(kernel_key)
+
+
+def kernel_source_hash():
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "fp4_block_scaled_deterministic_b200", "csrc")
+    for f in ("common.cuh", "gemm.cuh"):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()
+
+
+# ---------------------------------------------------------------- main
+def main():
+    a = parse()
+    if a.impl == "reference":
+        return run_reference(a)
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    import fp4_block_scaled_deterministic_b200 as fp4
+    fp4.lib()  # fails loudly if the library is missing
+    fmt = 0 if a.format == "mxfp4" else 1
+    layer = LlamaLayer(dev, fmt, a.hadamard, seed=1000 * rank)
+    stream = torch.cuda.current_stream(dev)
+    allreduce = None
+    if world > 1:
+        allreduce = lambda t: dist.all_reduce(t, op=dist.ReduceOp.SUM, async_op=True)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize(dev)
+
+    for _ in range(a.warmup):
+        layer.step(stream, None, allreduce)
+    barrier()
+    assert fp4.fp4_check_status() == 0
+
+    timers = {"quant": [], "gemm": []}
+    clocks = Clocks(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(a.steps):
+        layer.step(stream, timers, allreduce)
+    e1.record(stream)
+    barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    status = fp4.fp4_check_status()
+    if status != 0:
+        raise RuntimeError(f"device status {fp4.status_string(status)}")
+
+    flops_step = layer.flops()
+    value = flops_step * world / (ms / a.steps * 1e-3) / 1e12
+    gemm_ms = [x.elapsed_time(y) for x, y in timers["gemm"]]
+    quant_ms = [x.elapsed_time(y) for x, y in timers["quant"]]
+    per_launch_flops = gemm_flops_of(layer) * a.steps
+    gemm_tflops = sum(per_launch_flops) / (sum(gemm_ms) * 1e-3) / 1e12
+    bpe = 2.0 + 2 * (0.5 + (1 / 32 if fmt == 0 else 1 / 16)) + (2.0 if fmt == 1 else 0.0)
+    q_bytes = layer.quant_elems() * bpe * a.steps
+    quant_gbs = q_bytes / (sum(quant_ms) * 1e-3) / 1e9
+
+    pk, pk_kind = peaks()
+    peak_fp4 = pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) * FP4_OVER_BF16
+    avg_launch_ms = sum(gemm_ms) / len(gemm_ms)
+    avg_flops = sum(per_launch_flops) / len(per_launch_flops)
+    traffic = recorded_traffic("gemm_fp4_kernel<mx,*>" if fmt == 0 else "gemm_fp4_kernel<nv,*>")
+    roof = {"bound": "tensor", "achieved": gemm_tflops, "peak": peak_fp4, "unit": "TFLOP/s",
+            "frac": gemm_tflops / peak_fp4, "traffic": traffic,
+            "kernel": "gemm_fp4_kernel (tcgen05 block-scaled FP4)",
+            "per_launch": {"avg_flops": avg_flops, "avg_ms": avg_launch_ms,
+                           "launches": len(gemm_ms)},
+            "peak_source": f"{pk_kind}: bf16_tflops_sustained x {FP4_OVER_BF16} (nominal FP4:BF16)"}
+    qroof = {"bound": "hbm", "achieved": quant_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+             "frac": quant_gbs / pk["hbm_gbs"], "bytes_per_elem": bpe,
+             "kernel": "quantize_kernel dual layout", "launches": len(quant_ms),
+             "avg_ms": sum(quant_ms) / len(quant_ms), "peak_source": f"{pk_kind}: hbm_gbs"}
+
+    out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+           "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms / a.steps,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp4_e2m1",
+           "data": "synthetic",
+           "config": {"workload": WORKLOAD, "format": a.format, "hadamard_n": a.hadamard,
+                      "tokens_per_rank": layer.M,
+                      "l2": f"inputs larger than L2 ({(layer.bytes_in() + layer.bytes_out()) / 1e9:.1f} GB per step)",
+                      "parallelism": f"dp{world}"},
+           "gemm_tflops": gemm_tflops, "quantize_gbs": quant_gbs,
+           "roofline": roof, "roofline_quantize": qroof, "clocks": clk,
+           "gpu_launches": layer.launches_per_step() * a.steps}
+
+    # end to end through the C ABI from pinned host buffers (inputs H2D, outputs D2H)
+    if not a.no_e2e:
+        host_in = [[t.cpu().pin_memory() for t in (p["X"], p["W"], p["dY"])] for p in layer.projs]
+        host_out = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                     for t in (p["Y"], p["dX"], p["dW"])] for p in layer.projs]
+        barrier()
+
+        def e2e_step():
+            for p, hin in zip(layer.projs, host_in):
+                p["X"].copy_(hin[0], non_blocking=True)
+                p["W"].copy_(hin[1], non_blocking=True)
+                p["dY"].copy_(hin[2], non_blocking=True)
+            layer.step(stream, None, allreduce)
+            for p, hout in zip(layer.projs, host_out):
+                hout[0].copy_(p["Y"], non_blocking=True)
+                hout[1].copy_(p["dX"], non_blocking=True)
+                hout[2].copy_(p["dW"], non_blocking=True)
+
+        e2e_step()
+        barrier()
+        e0.record(stream)
+        for _ in range(a.steps):
+            e2e_step()
+        e1.record(stream)
+        barrier()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        out["e2e"] = {"value": flops_step * world / (ems / a.steps * 1e-3) / 1e12,
+                      "unit": "TFLOP/s", "h2d_bytes_per_step": layer.bytes_in(),
+                      "d2h_bytes_per_step": layer.bytes_out(), "ms_per_step": ems / a.steps}
+    else:
+        out["e2e"] = None
+
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        t_step, desc, cores = cpu_oracle_rate(a.cpu_seconds, fmt, a.hadamard)
+        out["cpu_baseline"] = {"value": flops_step / t_step / 1e12, "unit": "TFLOP/s",
+                               "cores": cores, "kind": "oracle", "sample": desc}
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

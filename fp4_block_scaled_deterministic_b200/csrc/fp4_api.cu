@@ -1,0 +1,505 @@
+// fp4_api.cu -- the C ABI of libfp4 (declared in include/fp4.h): host-side argument
+// validation, TMA descriptor construction and kernel launches on the caller's stream.
+// The library allocates no device memory; all buffers belong to the caller.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fp4.h"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "quantize.cuh"
+
+using namespace fp4k;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultWaitLimitNs = 1000000000ull;  // 1 s per pipeline wait
+
+// ---------------------------------------------------------------- device facts (cached)
+struct DeviceInfo {
+  int sm_count = 0;
+  int cc_major = 0;
+  bool ok = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::once_flag g_dev_once[kMaxDevices];
+
+fp4_status current_device(int* dev_out, const DeviceInfo** info) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FP4_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FP4_ERR_UNSUPPORTED_DEVICE;
+  std::call_once(g_dev_once[dev], [dev] {
+    DeviceInfo d;
+    if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) ==
+            cudaSuccess)
+      d.ok = true;
+    g_dev[dev] = d;
+  });
+  const DeviceInfo& d = g_dev[dev];
+  if (!d.ok) return FP4_ERR_CUDA;
+  if (d.cc_major != 10) return FP4_ERR_UNSUPPORTED_DEVICE;
+  *dev_out = dev;
+  *info = &d;
+  return FP4_OK;
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+EncodeTiledFn encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  return g_encode;
+}
+
+// 2-D row-major tensor [outer][inner] of `elem_bytes` elements.
+bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* base,
+                 uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer,
+                 CUtensorMapSwizzle sw) {
+  EncodeTiledFn enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * static_cast<uint64_t>(elem_bytes)};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Raise a kernel's dynamic shared-memory limit once per device.
+template <typename K>
+cudaError_t ensure_smem(K kernel, int bytes, int dev, std::atomic<uint64_t>& done) {
+  const uint64_t bit = 1ull << dev;
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int block_of(fp4_format f) { return f == FP4_MXFP4 ? 32 : 16; }
+
+// ---------------------------------------------------------------- quantise launch
+template <int FMT, int HN, int MODE, bool AMAX>
+cudaError_t launch_q(const CUtensorMap& ti, const CUtensorMap& tr, const CUtensorMap& tc,
+                     const QuantArgs& a, int grid, int dev, cudaStream_t s) {
+  static std::atomic<uint64_t> done{0};
+  auto k = quantize_kernel<FMT, HN, MODE, AMAX>;
+  cudaError_t e = ensure_smem(k, kQSmemBytes, dev, done);
+  if (e != cudaSuccess) return e;
+  k<<<grid, kQThreads, kQSmemBytes, s>>>(ti, tr, tc, a);
+  return cudaGetLastError();
+}
+
+template <int FMT, int HN, bool AMAX>
+cudaError_t dispatch_mode(int mode, const CUtensorMap& ti, const CUtensorMap& tr,
+                          const CUtensorMap& tc, const QuantArgs& a, int grid, int dev,
+                          cudaStream_t s) {
+  switch (mode) {
+    case kModeRow: return launch_q<FMT, HN, kModeRow, AMAX>(ti, tr, tc, a, grid, dev, s);
+    case kModeCol: return launch_q<FMT, HN, kModeCol, AMAX>(ti, tr, tc, a, grid, dev, s);
+    default: return launch_q<FMT, HN, kModeDual, AMAX>(ti, tr, tc, a, grid, dev, s);
+  }
+}
+
+template <int FMT, bool AMAX>
+cudaError_t dispatch_hn(int hn, int mode, const CUtensorMap& ti, const CUtensorMap& tr,
+                        const CUtensorMap& tc, const QuantArgs& a, int grid, int dev,
+                        cudaStream_t s) {
+  switch (hn) {
+    case 0: return dispatch_mode<FMT, 0, AMAX>(mode, ti, tr, tc, a, grid, dev, s);
+    case 16: return dispatch_mode<FMT, 16, AMAX>(mode, ti, tr, tc, a, grid, dev, s);
+    default: return dispatch_mode<FMT, 32, AMAX>(mode, ti, tr, tc, a, grid, dev, s);
+  }
+}
+
+fp4_status validate_quant_common(const void* x, int64_t rows, int64_t cols, fp4_format fmt,
+                                 int hn) {
+  if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
+  if (hn != 0 && hn != 16 && hn != 32) return FP4_ERR_INVALID_ARG;
+  if (rows < 0 || cols < 0) return FP4_ERR_SHAPE;
+  if (rows % 32 != 0 || cols % 32 != 0) return FP4_ERR_SHAPE;
+  if (rows > (int64_t(1) << 31) - 128 || cols > (int64_t(1) << 31) - 128) return FP4_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return FP4_OK;
+  if (!x) return FP4_ERR_INVALID_ARG;
+  if (!aligned16(x)) return FP4_ERR_ALIGN;
+  return FP4_OK;
+}
+
+fp4_status quantize_impl(const void* x, void* rcodes, void* rscales, void* ccodes, void* cscales,
+                         float* ts, int64_t rows, int64_t cols, fp4_format fmt, int hn, int mode,
+                         cudaStream_t stream) {
+  fp4_status st = validate_quant_common(x, rows, cols, fmt, hn);
+  if (st != FP4_OK) return st;
+  const bool do_row = mode & kModeRow, do_col = mode & kModeCol;
+  if (fmt == FP4_MXFP4 && ts) return FP4_ERR_INVALID_ARG;
+  if (fmt == FP4_NVFP4 && !ts) return FP4_ERR_INVALID_ARG;
+  if (rows == 0 || cols == 0) return FP4_OK;
+  if ((do_row && (!rcodes || !rscales)) || (do_col && (!ccodes || !cscales)))
+    return FP4_ERR_INVALID_ARG;
+  if ((do_row && (!aligned16(rcodes) || !aligned16(rscales))) ||
+      (do_col && (!aligned16(ccodes) || !aligned16(cscales))) ||
+      (ts && (reinterpret_cast<uintptr_t>(ts) & 3u)))
+    return FP4_ERR_ALIGN;
+  int dev;
+  const DeviceInfo* info;
+  st = current_device(&dev, &info);
+  if (st != FP4_OK) return st;
+
+  CUtensorMap tm_in, tm_r, tm_c;
+  std::memset(&tm_r, 0, sizeof(tm_r));
+  std::memset(&tm_c, 0, sizeof(tm_c));
+  if (!make_map_2d(&tm_in, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, cols, rows, 64, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return FP4_ERR_CUDA;
+  if (do_row && !make_map_2d(&tm_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rcodes, cols / 2, rows, 64,
+                             128, CU_TENSOR_MAP_SWIZZLE_64B))
+    return FP4_ERR_CUDA;
+  if (do_col && !make_map_2d(&tm_c, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ccodes, rows / 2, cols, 64,
+                             128, CU_TENSOR_MAP_SWIZZLE_64B))
+    return FP4_ERR_CUDA;
+
+  const int bs = block_of(fmt);
+  QuantArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.rows = rows;
+  a.cols = cols;
+  a.tiles_c = static_cast<int>(ceil_div(cols, 128));
+  const int64_t tiles = ceil_div(rows, 128) * a.tiles_c;
+  if (tiles > INT32_MAX) return FP4_ERR_SHAPE;
+  a.num_tiles = static_cast<int>(tiles);
+  a.row_scales = static_cast<uint8_t*>(rscales);
+  a.col_scales = static_cast<uint8_t*>(cscales);
+  a.row_kb4 = static_cast<int>(ceil_div(cols / bs, 4));
+  a.col_kb4 = static_cast<int>(ceil_div(rows / bs, 4));
+  a.wait_limit_ns = kDefaultWaitLimitNs;
+  const int grid = static_cast<int>(a.num_tiles < info->sm_count ? a.num_tiles : info->sm_count);
+
+  cudaError_t e = cudaSuccess;
+  if (fmt == FP4_MXFP4) {
+    e = dispatch_hn<kFmtMX, false>(hn, mode, tm_in, tm_r, tm_c, a, grid, dev, stream);
+  } else {
+    // ts layout: single -> {S, amax}; dual -> {S_row, S_col, amax_row, amax_col}
+    float* amax_r = nullptr;
+    float* amax_c = nullptr;
+    if (mode == kModeDual) {
+      a.s_row_out = ts;
+      a.s_col_out = ts + 1;
+      amax_r = ts + 2;
+      amax_c = ts + 3;
+    } else if (mode == kModeRow) {
+      a.s_row_out = ts;
+      amax_r = ts + 1;
+    } else {
+      a.s_col_out = ts;
+      amax_c = ts + 1;
+    }
+    a.amax_row = amax_r;
+    a.amax_col = amax_c;
+    a.amax_row_acc = reinterpret_cast<unsigned*>(amax_r);
+    a.amax_col_acc = reinterpret_cast<unsigned*>(amax_c);
+    float* first = amax_r ? amax_r : amax_c;
+    const size_t nbytes = (amax_r && amax_c) ? 2 * sizeof(float) : sizeof(float);
+    e = cudaMemsetAsync(first, 0, nbytes, stream);
+    if (e == cudaSuccess)
+      e = dispatch_hn<kFmtNV, true>(hn, mode, tm_in, tm_r, tm_c, a, grid, dev, stream);
+    if (e == cudaSuccess)
+      e = dispatch_hn<kFmtNV, false>(hn, mode, tm_in, tm_r, tm_c, a, grid, dev, stream);
+  }
+  return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- GEMM launch
+template <int FMT, int OUT>
+cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& sa,
+                        const CUtensorMap& sb, const GemmArgs& g, int grid, int dev,
+                        cudaStream_t s) {
+  static std::atomic<uint64_t> done{0};
+  auto k = gemm_fp4_kernel<FMT, OUT>;
+  cudaError_t e = ensure_smem(k, GemmCfg<FMT>::kSmemBytes, dev, done);
+  if (e != cudaSuccess) return e;
+  k<<<grid, kGThreads, GemmCfg<FMT>::kSmemBytes, s>>>(a, b, sa, sb, g);
+  return cudaGetLastError();
+}
+
+fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void* B,
+                     const void* Bs, const float* Bts, void* C, int64_t M, int64_t N, int64_t K,
+                     fp4_format fmt, fp4_out_dtype od, cudaStream_t stream) {
+  if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
+  if (od != FP4_OUT_F32 && od != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K < 0 || M % 32 || N % 32 || K % 32) return FP4_ERR_SHAPE;
+  if (M > (int64_t(1) << 31) - 256 || N > (int64_t(1) << 31) - 256 ||
+      K > (int64_t(1) << 31) - 256)
+    return FP4_ERR_SHAPE;
+  if (fmt == FP4_MXFP4 && (Ats || Bts)) return FP4_ERR_INVALID_ARG;
+  if (fmt == FP4_NVFP4 && (!Ats || !Bts)) return FP4_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return FP4_OK;
+  if (!C) return FP4_ERR_INVALID_ARG;
+  if (K == 0) return FP4_ERR_SHAPE;  // an empty contraction is not a launch the tiles express
+  if (!A || !As || !B || !Bs) return FP4_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(As) || !aligned16(B) || !aligned16(Bs) || !aligned16(C))
+    return FP4_ERR_ALIGN;
+  int dev;
+  const DeviceInfo* info;
+  fp4_status st = current_device(&dev, &info);
+  if (st != FP4_OK) return st;
+
+  const int bs = block_of(fmt);
+  const int64_t kb4 = ceil_div(K / bs, 4);
+  const int atoms = kGBK / (4 * bs);
+  CUtensorMap ta, tb, tsa, tsb;
+  if (!make_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K / 2, M, kGBK / 2, kGBM,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K / 2, N, kGBK / 2, kGBN,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tsa, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, As, kb4 * 64, ceil_div(M, 128),
+                   atoms * 64, 1, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map_2d(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, Bs, kb4 * 64, ceil_div(N, 128),
+                   atoms * 64, 2, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return FP4_ERR_CUDA;
+
+  GemmArgs g;
+  g.M = static_cast<int>(M);
+  g.N = static_cast<int>(N);
+  g.K = static_cast<int>(K);
+  g.tiles_m = static_cast<int>(ceil_div(M, kGBM));
+  g.tiles_n = static_cast<int>(ceil_div(N, kGBN));
+  const int64_t tiles = int64_t(g.tiles_m) * g.tiles_n;
+  if (tiles > INT32_MAX) return FP4_ERR_SHAPE;
+  g.num_tiles = static_cast<int>(tiles);
+  g.k_tiles = static_cast<int>(ceil_div(K, kGBK));
+  g.C = C;
+  g.sa = Ats;
+  g.sb = Bts;
+  g.wait_limit_ns = kDefaultWaitLimitNs;
+  const int grid = g.num_tiles < info->sm_count ? g.num_tiles : info->sm_count;
+
+  cudaError_t e;
+  if (fmt == FP4_MXFP4)
+    e = od == FP4_OUT_F32 ? launch_gemm<kFmtMX, 0>(ta, tb, tsa, tsb, g, grid, dev, stream)
+                          : launch_gemm<kFmtMX, 1>(ta, tb, tsa, tsb, g, grid, dev, stream);
+  else
+    e = od == FP4_OUT_F32 ? launch_gemm<kFmtNV, 0>(ta, tb, tsa, tsb, g, grid, dev, stream)
+                          : launch_gemm<kFmtNV, 1>(ta, tb, tsa, tsb, g, grid, dev, stream);
+  return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- linear-layer passes
+inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
+
+// Workspace of one pass: operand A (R_a x K') and operand B (R_b x K') quantised
+// along the contraction K', plus 16 floats of NVFP4 tensor-scale cells.
+struct WsPlan {
+  size_t a_codes, a_scales, b_codes, b_scales, ts, total;
+};
+
+WsPlan plan_ws(int64_t ra, int64_t rb, int64_t kc, fp4_format fmt) {
+  WsPlan p;
+  size_t off = 0;
+  p.a_codes = off;  off += align256(fp4_codes_bytes(ra, kc));
+  p.a_scales = off; off += align256(fp4_scales_bytes(ra, kc, fmt));
+  p.b_codes = off;  off += align256(fp4_codes_bytes(rb, kc));
+  p.b_scales = off; off += align256(fp4_scales_bytes(rb, kc, fmt));
+  p.ts = off;       off += 256;
+  p.total = off;
+  return p;
+}
+
+void pass_dims(fp4_pass pass, int64_t M, int64_t N, int64_t K, int64_t* ra, int64_t* rb,
+               int64_t* kc) {
+  switch (pass) {
+    case FP4_PASS_FPROP: *ra = M; *rb = N; *kc = K; break;  // Y = X W^T
+    case FP4_PASS_DGRAD: *ra = M; *rb = K; *kc = N; break;  // dX = dY W
+    default: *ra = N; *rb = K; *kc = M; break;              // dW = dY^T X
+  }
+}
+
+fp4_status linear_impl(fp4_pass pass, const void* P, const void* Q, void* out, int64_t M,
+                       int64_t N, int64_t K, fp4_format fmt, int hn, fp4_out_dtype od, void* ws,
+                       size_t ws_bytes, cudaStream_t stream) {
+  if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
+  if (hn != 0 && hn != 16 && hn != 32) return FP4_ERR_INVALID_ARG;
+  if (od != FP4_OUT_F32 && od != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K < 0 || M % 32 || N % 32 || K % 32) return FP4_ERR_SHAPE;
+  int64_t ra, rb, kc;
+  pass_dims(pass, M, N, K, &ra, &rb, &kc);
+  if (ra == 0 || rb == 0) return FP4_OK;
+  if (kc == 0) return FP4_ERR_SHAPE;
+  if (!P || !Q || !out) return FP4_ERR_INVALID_ARG;
+  const WsPlan p = plan_ws(ra, rb, kc, fmt);
+  if (!ws || ws_bytes < p.total) return FP4_ERR_WORKSPACE;
+  if (!aligned16(ws)) return FP4_ERR_ALIGN;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  float* ts = fmt == FP4_NVFP4 ? reinterpret_cast<float*>(w + p.ts) : nullptr;
+  float* tsa = ts;
+  float* tsb = ts ? ts + 4 : nullptr;
+  fp4_status st;
+  switch (pass) {
+    case FP4_PASS_FPROP:  // A = X [M][K] rows, B = W [N][K] rows
+      st = quantize_impl(P, w + p.a_codes, w + p.a_scales, nullptr, nullptr, tsa, M, K, fmt, hn,
+                         kModeRow, stream);
+      if (st == FP4_OK)
+        st = quantize_impl(Q, w + p.b_codes, w + p.b_scales, nullptr, nullptr, tsb, N, K, fmt, hn,
+                           kModeRow, stream);
+      break;
+    case FP4_PASS_DGRAD:  // A = dY [M][N] rows, B = W [N][K] along N -> [K][N]
+      st = quantize_impl(P, w + p.a_codes, w + p.a_scales, nullptr, nullptr, tsa, M, N, fmt, hn,
+                         kModeRow, stream);
+      if (st == FP4_OK)
+        st = quantize_impl(Q, nullptr, nullptr, w + p.b_codes, w + p.b_scales, tsb, N, K, fmt, hn,
+                           kModeCol, stream);
+      break;
+    default:  // A = dY [M][N] along M -> [N][M], B = X [M][K] along M -> [K][M]
+      st = quantize_impl(P, nullptr, nullptr, w + p.a_codes, w + p.a_scales, tsa, M, N, fmt, hn,
+                         kModeCol, stream);
+      if (st == FP4_OK)
+        st = quantize_impl(Q, nullptr, nullptr, w + p.b_codes, w + p.b_scales, tsb, M, K, fmt, hn,
+                           kModeCol, stream);
+      break;
+  }
+  if (st != FP4_OK) return st;
+  return gemm_impl(w + p.a_codes, w + p.a_scales, tsa, w + p.b_codes, w + p.b_scales, tsb, out, ra,
+                   rb, kc, fmt, od, stream);
+}
+
+// ---------------------------------------------------------------- failure-path self test
+__global__ void wait_selftest_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  // Nobody arrives: the bounded wait must give up and record the timeout.
+  (void)mbar_wait(&bar, 0u, limit_ns);
+}
+
+}  // namespace
+
+// ==================================================================== C ABI
+extern "C" {
+
+int fp4_abi_version(void) { return 1; }
+
+size_t fp4_codes_bytes(int64_t rows, int64_t cols) {
+  if (rows <= 0 || cols <= 0) return 0;
+  return static_cast<size_t>(rows) * static_cast<size_t>(cols) / 2;
+}
+
+size_t fp4_scales_bytes(int64_t rows, int64_t cols, fp4_format fmt) {
+  if (rows <= 0 || cols <= 0) return 0;
+  const int64_t kb = cols / block_of(fmt);
+  return static_cast<size_t>(ceil_div(rows, 128) * 128) * static_cast<size_t>(ceil_div(kb, 4) * 4);
+}
+
+fp4_status fp4_quantize(const void* x, void* codes, void* scales, float* ts, int64_t rows,
+                        int64_t cols, fp4_format fmt, int hn, fp4_axis axis, fp4_stream_t stream) {
+  if (axis != FP4_AXIS_ROW && axis != FP4_AXIS_COL) return FP4_ERR_INVALID_ARG;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (axis == FP4_AXIS_ROW)
+    return quantize_impl(x, codes, scales, nullptr, nullptr, ts, rows, cols, fmt, hn, kModeRow, s);
+  return quantize_impl(x, nullptr, nullptr, codes, scales, ts, rows, cols, fmt, hn, kModeCol, s);
+}
+
+fp4_status fp4_quantize_dual(const void* x, void* row_codes, void* row_scales, void* col_codes,
+                             void* col_scales, float* ts, int64_t rows, int64_t cols,
+                             fp4_format fmt, int hn, fp4_stream_t stream) {
+  return quantize_impl(x, row_codes, row_scales, col_codes, col_scales, ts, rows, cols, fmt, hn,
+                       kModeDual, reinterpret_cast<cudaStream_t>(stream));
+}
+
+fp4_status fp4_gemm(const void* A, const void* As, const float* Ats, const void* B, const void* Bs,
+                    const float* Bts, void* C, int64_t M, int64_t N, int64_t K, fp4_format fmt,
+                    fp4_out_dtype od, fp4_stream_t stream) {
+  return gemm_impl(A, As, Ats, B, Bs, Bts, C, M, N, K, fmt, od,
+                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t fp4_linear_workspace_size(fp4_pass pass, int64_t M, int64_t N, int64_t K, fp4_format fmt) {
+  if (pass != FP4_PASS_FPROP && pass != FP4_PASS_DGRAD && pass != FP4_PASS_WGRAD) return 0;
+  if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return 0;
+  if (M < 0 || N < 0 || K < 0) return 0;
+  int64_t ra, rb, kc;
+  pass_dims(pass, M, N, K, &ra, &rb, &kc);
+  return plan_ws(ra, rb, kc, fmt).total;
+}
+
+fp4_status fp4_linear_fprop(const void* X, const void* W, void* Y, int64_t M, int64_t N, int64_t K,
+                            fp4_format fmt, int hn, fp4_out_dtype od, void* ws, size_t ws_bytes,
+                            fp4_stream_t stream) {
+  return linear_impl(FP4_PASS_FPROP, X, W, Y, M, N, K, fmt, hn, od, ws, ws_bytes,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+fp4_status fp4_linear_dgrad(const void* dY, const void* W, void* dX, int64_t M, int64_t N,
+                            int64_t K, fp4_format fmt, int hn, fp4_out_dtype od, void* ws,
+                            size_t ws_bytes, fp4_stream_t stream) {
+  return linear_impl(FP4_PASS_DGRAD, dY, W, dX, M, N, K, fmt, hn, od, ws, ws_bytes,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+fp4_status fp4_linear_wgrad(const void* dY, const void* X, void* dW, int64_t M, int64_t N,
+                            int64_t K, fp4_format fmt, int hn, fp4_out_dtype od, void* ws,
+                            size_t ws_bytes, fp4_stream_t stream) {
+  return linear_impl(FP4_PASS_WGRAD, dY, X, dW, M, N, K, fmt, hn, od, ws, ws_bytes,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+fp4_status fp4_check_status(fp4_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return FP4_ERR_CUDA;
+  unsigned word = 0;
+  const unsigned zero = 0;
+  if (cudaMemcpyFromSymbol(&word, g_status_word, sizeof(word)) != cudaSuccess) return FP4_ERR_CUDA;
+  if (word != 0 && cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero)) != cudaSuccess)
+    return FP4_ERR_CUDA;
+  return (word & kDevErrTimeout) ? FP4_ERR_TIMEOUT : FP4_OK;
+}
+
+fp4_status fp4_selftest_timeout(uint64_t timeout_ns, fp4_stream_t stream) {
+  int dev;
+  const DeviceInfo* info;
+  fp4_status st = current_device(&dev, &info);
+  if (st != FP4_OK) return st;
+  wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(timeout_ns);
+  return cudaGetLastError() == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+}
+
+const char* fp4_status_string(fp4_status s) {
+  switch (s) {
+    case FP4_OK: return "ok";
+    case FP4_ERR_INVALID_ARG: return "invalid argument";
+    case FP4_ERR_SHAPE: return "unsupported shape";
+    case FP4_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case FP4_ERR_UNSUPPORTED_DEVICE: return "device is not sm_100 (B200)";
+    case FP4_ERR_CUDA: return "CUDA error";
+    case FP4_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case FP4_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

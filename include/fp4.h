@@ -47,6 +47,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define FP4_API __attribute__((visibility("default")))
+#else
+#define FP4_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -71,14 +77,14 @@ typedef enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 } fp4_out_dtype;
 typedef enum { FP4_PASS_FPROP = 0, FP4_PASS_DGRAD = 1, FP4_PASS_WGRAD = 2 } fp4_pass;
 
 /* Version of this ABI; bumped on any incompatible change. */
-int fp4_abi_version(void);
+FP4_API int fp4_abi_version(void);
 
 /* Bytes of a packed code matrix with R rows of C elements: R*C/2. */
-size_t fp4_codes_bytes(int64_t rows, int64_t cols);
+FP4_API size_t fp4_codes_bytes(int64_t rows, int64_t cols);
 
 /* Bytes of the scale matrix of an [R][C] code matrix in the atom layout above:
  * ceil(R/128)*128 * ceil(C/bs/4)*4. */
-size_t fp4_scales_bytes(int64_t rows, int64_t cols, fp4_format fmt);
+FP4_API size_t fp4_scales_bytes(int64_t rows, int64_t cols, fp4_format fmt);
 
 /*
  * fp4_quantize -- rotate and quantise one bf16 matrix x[rows][cols] (row-major).
@@ -99,7 +105,7 @@ size_t fp4_scales_bytes(int64_t rows, int64_t cols, fp4_format fmt);
  *   Shape: rows % 32 == 0 and cols % 32 == 0 (rows or cols 0: nothing is done).
  *   Launches: MXFP4 one kernel; NVFP4 a 4-byte memset, an amax kernel, a quantise kernel.
  */
-fp4_status fp4_quantize(const void *x_bf16, void *codes, void *scales, float *tensor_scale,
+FP4_API fp4_status fp4_quantize(const void *x_bf16, void *codes, void *scales, float *tensor_scale,
                         int64_t rows, int64_t cols, fp4_format fmt, int hadamard_n,
                         fp4_axis axis, fp4_stream_t stream);
 
@@ -112,7 +118,7 @@ fp4_status fp4_quantize(const void *x_bf16, void *codes, void *scales, float *te
  *                 MXFP4 -> must be NULL.
  *   Shape: as fp4_quantize.
  */
-fp4_status fp4_quantize_dual(const void *x_bf16, void *row_codes, void *row_scales,
+FP4_API fp4_status fp4_quantize_dual(const void *x_bf16, void *row_codes, void *row_scales,
                              void *col_codes, void *col_scales, float *tensor_scale,
                              int64_t rows, int64_t cols, fp4_format fmt, int hadamard_n,
                              fp4_stream_t stream);
@@ -129,7 +135,7 @@ fp4_status fp4_quantize_dual(const void *x_bf16, void *row_codes, void *row_scal
  *   C: row-major [M][N], fp32 or bf16 (round-to-nearest-even of the fp32 result).
  *   Shape: M, N, K multiples of 32 (0 -> nothing is done).
  */
-fp4_status fp4_gemm(const void *A_codes, const void *A_scales, const float *A_tensor_scale,
+FP4_API fp4_status fp4_gemm(const void *A_codes, const void *A_scales, const float *A_tensor_scale,
                     const void *B_codes, const void *B_scales, const float *B_tensor_scale,
                     void *C, int64_t M, int64_t N, int64_t K, fp4_format fmt,
                     fp4_out_dtype out_dtype, fp4_stream_t stream);
@@ -145,15 +151,15 @@ fp4_status fp4_gemm(const void *A_codes, const void *A_scales, const float *A_te
  * bytes; it receives the quantised operands (and NVFP4 tensor scales) in an
  * unspecified layout. Shape: M, N, K multiples of 32.
  */
-size_t fp4_linear_workspace_size(fp4_pass pass, int64_t M, int64_t N, int64_t K, fp4_format fmt);
+FP4_API size_t fp4_linear_workspace_size(fp4_pass pass, int64_t M, int64_t N, int64_t K, fp4_format fmt);
 
-fp4_status fp4_linear_fprop(const void *X, const void *W, void *Y, int64_t M, int64_t N, int64_t K,
+FP4_API fp4_status fp4_linear_fprop(const void *X, const void *W, void *Y, int64_t M, int64_t N, int64_t K,
                             fp4_format fmt, int hadamard_n, fp4_out_dtype out_dtype, void *ws,
                             size_t ws_bytes, fp4_stream_t stream);
-fp4_status fp4_linear_dgrad(const void *dY, const void *W, void *dX, int64_t M, int64_t N,
+FP4_API fp4_status fp4_linear_dgrad(const void *dY, const void *W, void *dX, int64_t M, int64_t N,
                             int64_t K, fp4_format fmt, int hadamard_n, fp4_out_dtype out_dtype,
                             void *ws, size_t ws_bytes, fp4_stream_t stream);
-fp4_status fp4_linear_wgrad(const void *dY, const void *X, void *dW, int64_t M, int64_t N,
+FP4_API fp4_status fp4_linear_wgrad(const void *dY, const void *X, void *dW, int64_t M, int64_t N,
                             int64_t K, fp4_format fmt, int hadamard_n, fp4_out_dtype out_dtype,
                             void *ws, size_t ws_bytes, fp4_stream_t stream);
 
@@ -163,7 +169,7 @@ fp4_status fp4_linear_wgrad(const void *dY, const void *X, void *dW, int64_t M, 
  * gave up since the last check, FP4_ERR_CUDA if the synchronisation failed, else
  * FP4_OK.
  */
-fp4_status fp4_check_status(fp4_stream_t stream);
+FP4_API fp4_status fp4_check_status(fp4_stream_t stream);
 
 /*
  * fp4_selftest_timeout -- launches one tiny kernel that waits on a pipeline barrier
@@ -172,10 +178,10 @@ fp4_status fp4_check_status(fp4_stream_t stream);
  * the status word and returns normally; no fault, no trap. Used to test the
  * failure-reporting path.
  */
-fp4_status fp4_selftest_timeout(uint64_t timeout_ns, fp4_stream_t stream);
+FP4_API fp4_status fp4_selftest_timeout(uint64_t timeout_ns, fp4_stream_t stream);
 
 /* Static English text for a status code. */
-const char *fp4_status_string(fp4_status s);
+FP4_API const char *fp4_status_string(fp4_status s);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,110 @@
+"""The C-ABI library loads, exports every entry point include/fp4.h declares, and
+rejects bad arguments on the host before touching a device (no GPU needed: every
+call below fails validation, so nothing is launched)."""
+import ctypes
+
+import numpy as np
+import pytest
+
+import fp4_block_scaled_deterministic_b200 as fp4
+
+OK, INVALID, SHAPE, ALIGN, CUDA, WORKSPACE = 0, 1, 2, 3, 5, 7
+A16 = 1 << 20          # a 16-byte aligned fake pointer value (never dereferenced)
+MIS = A16 + 8          # misaligned
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from fp4_block_scaled_deterministic_b200 import build
+    build.build()
+
+
+def test_every_header_symbol_is_exported():
+    syms = fp4.header_symbols()
+    assert len(syms) >= 13
+    L = ctypes.CDLL(fp4.LIB_PATH)
+    for s in syms:
+        assert hasattr(L, s), s
+    assert fp4.lib().fp4_abi_version() == 1
+
+
+def test_status_strings():
+    for code in range(8):
+        assert fp4.status_string(code)
+    assert fp4.status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("rows,cols", [(32, 32), (160, 224), (128, 4096), (8192, 14336)])
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_size_queries_match_layout(orc, rows, cols, fmt):
+    assert fp4.fp4_codes_bytes(rows, cols) == rows * cols // 2
+    assert fp4.fp4_scales_bytes(rows, cols, fmt) == orc.scale_layout_bytes(rows, cols // orc.BLOCK[fmt])
+
+
+def test_workspace_size_covers_operands():
+    for p, (ra, rb, kc) in {0: (64, 96, 128), 1: (64, 128, 96), 2: (96, 128, 64)}.items():
+        need = fp4.fp4_linear_workspace_size(p, 64, 96, 128, 0)
+        assert need >= ra * kc // 2 + rb * kc // 2
+    assert fp4.fp4_linear_workspace_size(7, 64, 96, 128, 0) == 0
+
+
+def q(x=A16, codes=A16, scales=A16, ts=None, rows=64, cols=64, fmt=0, hn=16, axis=0):
+    return fp4.lib().fp4_quantize(x, codes, scales, ts, rows, cols, fmt, hn, axis, None)
+
+
+def test_quantize_validation():
+    assert q(fmt=2) == INVALID
+    assert q(hn=8) == INVALID
+    assert q(axis=3) == INVALID
+    assert q(rows=48) == SHAPE
+    assert q(cols=40) == SHAPE
+    assert q(rows=-32) == SHAPE
+    assert q(x=MIS) == ALIGN
+    assert q(codes=MIS) == ALIGN
+    assert q(x=None) == INVALID
+    assert q(scales=None) == INVALID
+    assert q(ts=A16) == INVALID            # MXFP4 takes no tensor scale
+    assert q(fmt=1, ts=None) == INVALID    # NVFP4 needs one
+    assert q(rows=0) == OK and q(cols=0) == OK  # empty: nothing to do
+
+
+def test_quantize_dual_validation():
+    L = fp4.lib()
+    assert L.fp4_quantize_dual(A16, A16, A16, None, A16, None, 64, 64, 0, 16, None) == INVALID
+    assert L.fp4_quantize_dual(A16, A16, A16, A16, MIS, None, 64, 64, 0, 16, None) == ALIGN
+    assert L.fp4_quantize_dual(A16, A16, A16, A16, A16, None, 64, 80, 0, 16, None) == SHAPE
+
+
+def g(A=A16, As=A16, Ats=None, B=A16, Bs=A16, Bts=None, C=A16, M=128, N=128, K=128, fmt=0, od=0):
+    return fp4.lib().fp4_gemm(A, As, Ats, B, Bs, Bts, C, M, N, K, fmt, od, None)
+
+
+def test_gemm_validation():
+    assert g(fmt=5) == INVALID
+    assert g(od=2) == INVALID
+    assert g(M=100) == SHAPE
+    assert g(K=48) == SHAPE
+    assert g(Ats=A16) == INVALID
+    assert g(fmt=1) == INVALID
+    assert g(C=None) == INVALID
+    assert g(B=MIS) == ALIGN
+    assert g(K=0) == SHAPE
+    assert g(M=0) == OK
+
+
+def test_linear_validation():
+    L = fp4.lib()
+    need = fp4.fp4_linear_workspace_size(0, 64, 64, 64, 0)
+    assert L.fp4_linear_fprop(A16, A16, A16, 64, 64, 64, 0, 16, 1, A16, need - 1, None) == WORKSPACE
+    assert L.fp4_linear_fprop(A16, A16, A16, 64, 64, 64, 0, 16, 1, None, need, None) == WORKSPACE
+    assert L.fp4_linear_dgrad(A16, A16, A16, 64, 64, 64, 0, 12, 1, A16, need, None) == INVALID
+    assert L.fp4_linear_wgrad(A16, A16, A16, 64, 40, 64, 0, 16, 1, A16, need, None) == SHAPE
+    assert L.fp4_linear_wgrad(A16, A16, A16, 64, 64, 64, 0, 16, 1, MIS, need, None) == ALIGN
+
+
+def test_valid_call_without_gpu_reports_cuda_or_device_error():
+    """With valid arguments and no usable device the call fails cleanly (no crash)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert q() in (CUDA, 4)
