@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--proj", default="qkv,o,gate,up,down",
+                    help="comma-separated subset of the layer's projections (profiling cases)")
     a = ap.parse_args()
     a.warmup = max(3, a.warmup)
     return a
@@ -120,13 +122,15 @@ class Clocks:
 class LlamaLayer:
     """Inputs, quantised operands and outputs of every projection, all on the device."""
 
-    def __init__(self, device, fmt, hn, tokens=8192, seed=0):
+    def __init__(self, device, fmt, hn, tokens=8192, seed=0, names=None):
         import fp4_block_scaled_deterministic_b200 as fp4
         from fp4_block_scaled_deterministic_b200 import synthetic
         self.fp4, self.fmt, self.hn, self.M = fp4, fmt, hn, tokens
         self.projs = []
         g = torch.Generator(device=device)
         for i, (name, N, K) in enumerate(synthetic.LLAMA_LAYERS):
+            if names is not None and name not in names:
+                continue
             X = synthetic.normal(tokens, K, 1.0, seed=seed + i, outlier_frac=0.001,
                                  outlier_mult=50.0, device=device)
             W = synthetic.normal(N, K, 0.02, seed=seed + 100 + i, device=device)
@@ -339,11 +343,11 @@ def main():
     import fp4_block_scaled_deterministic_b200 as fp4
     fp4.lib()  # fails loudly if the library is missing
     fmt = 0 if a.format == "mxfp4" else 1
-    layer = LlamaLayer(dev, fmt, a.hadamard, seed=1000 * rank)
+    names = [n.strip() for n in a.proj.split(",") if n.strip()]
+    layer = LlamaLayer(dev, fmt, a.hadamard, seed=1000 * rank, names=names)
     stream = torch.cuda.current_stream(dev)
-    allreduce = None
-    if world > 1:
-        allreduce = lambda t: dist.all_reduce(t, op=dist.ReduceOp.SUM, async_op=True)
+    from fp4_block_scaled_deterministic_b200 import dp
+    allreduce = dp.allreduce_wgrad if world > 1 else None
 
     def barrier():
         if world > 1:
@@ -368,11 +372,7 @@ def main():
     e1.record(stream)
     barrier()
     clk = clocks.stop()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = dp.max_over_ranks(e0.elapsed_time(e1), dev)
     status = fp4.fp4_check_status()
     if status != 0:
         raise RuntimeError(f"device status {fp4.status_string(status)}")
@@ -407,8 +407,9 @@ def main():
            "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms / a.steps,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp4_e2m1",
            "data": "synthetic",
-           "config": {"workload": WORKLOAD, "format": a.format, "hadamard_n": a.hadamard,
-                      "tokens_per_rank": layer.M,
+           "config": {"workload": WORKLOAD if len(names) == 5 else
+                      f"subset {','.join(names)} of: {WORKLOAD}",
+                      "format": a.format, "hadamard_n": a.hadamard, "tokens_per_rank": layer.M,
                       "l2": f"inputs larger than L2 ({(layer.bytes_in() + layer.bytes_out()) / 1e9:.1f} GB per step)",
                       "parallelism": f"dp{world}"},
            "gemm_tflops": gemm_tflops, "quantize_gbs": quant_gbs,
@@ -440,18 +441,14 @@ def main():
             e2e_step()
         e1.record(stream)
         barrier()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ems], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = dp.max_over_ranks(e0.elapsed_time(e1), dev)
         out["e2e"] = {"value": flops_step * world / (ems / a.steps * 1e-3) / 1e12,
                       "unit": "TFLOP/s", "h2d_bytes_per_step": layer.bytes_in(),
                       "d2h_bytes_per_step": layer.bytes_out(), "ms_per_step": ems / a.steps}
     else:
         out["e2e"] = None
 
-    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+    if rank == 0 and world == 1 and not a.no_cpu_baseline and len(names) == 5:
         t_step, desc, cores = cpu_oracle_rate(a.cpu_seconds, fmt, a.hadamard)
         out["cpu_baseline"] = {"value": flops_step / t_step / 1e12, "unit": "TFLOP/s",
                                "cores": cores, "kind": "oracle", "sample": desc}
