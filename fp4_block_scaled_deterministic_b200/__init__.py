@@ -64,6 +64,7 @@ def lib() -> ctypes.CDLL:
             "fp4_linear_fprop": (I32, [P, P, P, I64, I64, I64, I32, I32, I32, P, SZ, P]),
             "fp4_linear_dgrad": (I32, [P, P, P, I64, I64, I64, I32, I32, I32, P, SZ, P]),
             "fp4_linear_wgrad": (I32, [P, P, P, I64, I64, I64, I32, I32, I32, P, SZ, P]),
+            "fp4_linear_fprop_noalloc": (I32, [P, P, P, I64, I64, I64, I32, I32, I32, P]),
             "fp4_check_status": (I32, [P]),
             "fp4_selftest_timeout": (I32, [ctypes.c_uint64, P]),
             "fp4_status_string": (ctypes.c_char_p, [I32]),
@@ -149,6 +150,13 @@ def fp4_linear_dgrad(dY, W, dX, M, N, K, fmt, hn, out_dtype, ws, ws_bytes, strea
 def fp4_linear_wgrad(dY, X, dW, M, N, K, fmt, hn, out_dtype, ws, ws_bytes, stream=None):
     return lib().fp4_linear_wgrad(_ptr(dY), _ptr(X), _ptr(dW), M, N, K, fmt, hn, out_dtype,
                                   _ptr(ws), ws_bytes, _stream(stream))
+
+
+def fp4_linear_fprop_noalloc(X, W, Y, M, N, K, fmt, hn, out_dtype, stream=None):
+    """fp4_linear_fprop on the library's static scratch (no workspace argument), for
+    callers that cannot allocate device memory; see include/fp4.h for its limit."""
+    return lib().fp4_linear_fprop_noalloc(_ptr(X), _ptr(W), _ptr(Y), M, N, K, fmt, hn, out_dtype,
+                                          _stream(stream))
 
 
 def fp4_check_status(stream=None) -> int:

@@ -399,6 +399,33 @@ __global__ void wait_selftest_kernel(uint64_t limit_ns) {
 
 }  // namespace
 
+// ---------------------------------------------------------------- no-allocation scratch
+// Scratch of fp4_linear_fprop_noalloc: a file-scope device array, so callers that
+// cannot allocate still get the workspace the fprop pass needs. Host code must not
+// pass g_noalloc_scratch itself to a kernel (on the host that name is only a
+// stand-in); it passes the device address looked up once per device below.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[FP4_NOALLOC_SCRATCH_BYTES];
+
+void* g_noalloc_ptr[kMaxDevices];
+cudaError_t g_noalloc_err[kMaxDevices];
+std::once_flag g_noalloc_once[kMaxDevices];
+
+// Device address of the scratch array on the current device (looked up on the first
+// call for that device, with that device current).
+fp4_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FP4_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FP4_ERR_UNSUPPORTED_DEVICE;
+  std::call_once(g_noalloc_once[dev], [dev] {
+    void* p = nullptr;
+    g_noalloc_err[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    g_noalloc_ptr[dev] = g_noalloc_err[dev] == cudaSuccess ? p : nullptr;
+  });
+  if (g_noalloc_err[dev] != cudaSuccess || !g_noalloc_ptr[dev]) return FP4_ERR_CUDA;
+  *out = g_noalloc_ptr[dev];
+  return FP4_OK;
+}
+
 // ==================================================================== C ABI
 extern "C" {
 
@@ -465,6 +492,22 @@ fp4_status fp4_linear_wgrad(const void* dY, const void* X, void* dW, int64_t M, 
                             int64_t K, fp4_format fmt, int hn, fp4_out_dtype od, void* ws,
                             size_t ws_bytes, fp4_stream_t stream) {
   return linear_impl(FP4_PASS_WGRAD, dY, X, dW, M, N, K, fmt, hn, od, ws, ws_bytes,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+fp4_status fp4_linear_fprop_noalloc(const void* X, const void* W, void* Y, int64_t M, int64_t N,
+                                    int64_t K, fp4_format fmt, int hn, fp4_out_dtype od,
+                                    fp4_stream_t stream) {
+  if (fp4_linear_workspace_size(FP4_PASS_FPROP, M, N, K, fmt) > FP4_NOALLOC_SCRATCH_BYTES)
+    return FP4_ERR_WORKSPACE;
+  int dev;
+  const DeviceInfo* info;
+  fp4_status st = current_device(&dev, &info);
+  if (st != FP4_OK) return st;
+  void* ws = nullptr;
+  st = noalloc_scratch(&ws);
+  if (st != FP4_OK) return st;
+  return linear_impl(FP4_PASS_FPROP, X, W, Y, M, N, K, fmt, hn, od, ws, FP4_NOALLOC_SCRATCH_BYTES,
                      reinterpret_cast<cudaStream_t>(stream));
 }
 

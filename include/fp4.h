@@ -164,6 +164,32 @@ FP4_API fp4_status fp4_linear_wgrad(const void *dY, const void *X, void *dW, int
                             void *ws, size_t ws_bytes, fp4_stream_t stream);
 
 /*
+ * fp4_linear_fprop_noalloc -- fp4_linear_fprop with library-owned scratch instead
+ * of a caller workspace. The pages have no counterpart to this call; it exists for
+ * callers that cannot allocate device memory: code running inside a host framework
+ * that has already reserved the GPU's memory for its own allocator, plug-ins and
+ * callbacks that are handed tensors but no allocator, and latency-critical loops
+ * that must not call cudaMalloc (which can synchronise the whole device).
+ *   Scratch: one static device array of FP4_NOALLOC_SCRATCH_BYTES (32 MiB) per GPU,
+ *   reserved when the library's device code is loaded on that GPU and held until the
+ *   process exits. The call allocates and frees nothing.
+ *   Limit: if fp4_linear_workspace_size(FP4_PASS_FPROP, M, N, K, fmt) exceeds
+ *   FP4_NOALLOC_SCRATCH_BYTES the call returns FP4_ERR_WORKSPACE and launches nothing.
+ *   Set-up: the first call on each device looks the array's device address up (with
+ *   that device current) and caches it; make that first call before any stream
+ *   capture begins.
+ *   Sharing: every call on a device uses the same array, which keeps the previous
+ *   call's contents; each call re-zeroes what must start at zero. Calls whose GPU work
+ *   can overlap (for example on two streams with no ordering between them) race on
+ *   the array: order them on one stream or with events.
+ *   Arguments, shapes, outputs and the other errors are those of fp4_linear_fprop.
+ */
+#define FP4_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+FP4_API fp4_status fp4_linear_fprop_noalloc(const void *X, const void *W, void *Y, int64_t M,
+                                            int64_t N, int64_t K, fp4_format fmt, int hadamard_n,
+                                            fp4_out_dtype out_dtype, fp4_stream_t stream);
+
+/*
  * fp4_check_status -- synchronises `stream`, then returns and clears the device
  * status word of the current device: FP4_ERR_TIMEOUT if any kernel's bounded wait
  * gave up since the last check, FP4_ERR_CUDA if the synchronisation failed, else

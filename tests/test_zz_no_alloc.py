@@ -1,0 +1,53 @@
+"""fp4_linear_fprop_noalloc: the Fprop pass on the library's static scratch, for
+callers that cannot allocate device memory (a host framework that has reserved the
+GPU's memory for its own allocator, plug-ins handed tensors but no allocator, loops
+that must not call cudaMalloc because it can synchronise the device).
+
+Its output must match fp4_linear_fprop with a caller-allocated workspace, within the
+tolerance of the other GEMM tests, on consecutive calls that share the scratch (the
+second NVFP4 call has a smaller tensor amax than the first, so a scratch cell left
+over from the first call would change its result). This file is collected last."""
+import pytest
+import torch
+
+import fp4_block_scaled_deterministic_b200 as fp4
+from fp4_block_scaled_deterministic_b200 import synthetic
+from gpu_util import need_gpu, rel_fro
+
+pytestmark = pytest.mark.gpu
+TOL = 1e-4
+
+
+def _noalloc(X, W, fmt, hn, out_dtype):
+    (M, K), N = X.shape, W.shape[0]
+    dt = torch.float32 if out_dtype == fp4.OUT_F32 else torch.bfloat16
+    Y = torch.empty(M, N, dtype=dt, device="cuda")
+    st = fp4.fp4_linear_fprop_noalloc(X, W, Y, M, N, K, fmt, hn, out_dtype)
+    assert st == 0, fp4.status_string(st)
+    return Y
+
+
+def test_noalloc_fprop_matches_workspace_fprop():
+    need_gpu()
+    calls = [  # (M, N, K, fmt, outlier multiplier): consecutive calls share the scratch
+        (256, 384, 512, fp4.NVFP4, 50.0),
+        (160, 96, 224, fp4.NVFP4, 1.0),
+        (512, 256, 1024, fp4.MXFP4, 50.0),
+    ]
+    for i, (M, N, K, fmt, mult) in enumerate(calls):
+        X = synthetic.normal(M, K, 1.0, seed=40 + i, outlier_frac=0.01, outlier_mult=mult).cuda()
+        W = synthetic.normal(N, K, 0.02, seed=50 + i).cuda()
+        Y = _noalloc(X, W, fmt, 16, fp4.OUT_F32)
+        Y_ref = fp4.linear_fprop(X, W, fmt, 16, fp4.OUT_F32)
+        torch.cuda.synchronize()
+        assert fp4.fp4_check_status() == 0
+        err = rel_fro(Y.cpu().numpy(), Y_ref.cpu().numpy())
+        assert err <= TOL, (i, err)
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch():
+    need_gpu()
+    M = N = K = 8192  # needs ~66 MB of scratch, more than the 32 MiB array
+    assert fp4.fp4_linear_workspace_size(fp4.FPROP, M, N, K, fp4.MXFP4) > 32 << 20
+    st = fp4.fp4_linear_fprop_noalloc(None, None, None, M, N, K, fp4.MXFP4, 16, fp4.OUT_BF16)
+    assert st == 7  # FP4_ERR_WORKSPACE, nothing launched
