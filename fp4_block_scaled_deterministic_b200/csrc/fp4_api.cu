@@ -196,7 +196,8 @@ fp4_status quantize_impl(const void* x, void* rcodes, void* rscales, void* ccode
   a.row_kb4 = static_cast<int>(ceil_div(cols / bs, 4));
   a.col_kb4 = static_cast<int>(ceil_div(rows / bs, 4));
   a.wait_limit_ns = kDefaultWaitLimitNs;
-  const int grid = static_cast<int>(a.num_tiles < info->sm_count ? a.num_tiles : info->sm_count);
+  const int resident = kQCtasPerSM * info->sm_count;
+  const int grid = a.num_tiles < resident ? a.num_tiles : resident;
 
   cudaError_t e = cudaSuccess;
   if (fmt == FP4_MXFP4) {
@@ -245,6 +246,42 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtens
   return cudaGetLastError();
 }
 
+// CTA-pair kernel: the grid is two CTAs per pair tile, capped at the number of CTA pairs
+// the device can hold at once (queried once per device), so the persistent loop never
+// waits for a pair that is not resident.
+template <int FMT, int OUT>
+cudaError_t launch_gemm_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& sa,
+                             const CUtensorMap& sb, const GemmArgs& g, int dev, cudaStream_t s) {
+  static std::atomic<uint64_t> done{0};
+  static int max_pairs[kMaxDevices];
+  static std::once_flag once[kMaxDevices];
+  auto k = gemm_fp4_pair_kernel<FMT, OUT>;
+  cudaError_t e = ensure_smem(k, PairCfg<FMT>::kSmemBytes, dev, done);
+  if (e != cudaSuccess) return e;
+  std::call_once(once[dev], [&] {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * g_dev[dev].sm_count / 2, 1, 1);
+    cfg.blockDim = dim3(kGThreads, 1, 1);
+    cfg.dynamicSmemBytes = PairCfg<FMT>::kSmemBytes;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k, &cfg) != cudaSuccess || n <= 0) {
+      (void)cudaGetLastError();
+      n = g_dev[dev].sm_count / 2;
+    }
+    max_pairs[dev] = n;
+  });
+  const int pairs = g.num_tiles < max_pairs[dev] ? g.num_tiles : max_pairs[dev];
+  k<<<2 * pairs, kGThreads, PairCfg<FMT>::kSmemBytes, s>>>(a, b, sa, sb, g);
+  return cudaGetLastError();
+}
+
 fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void* B,
                      const void* Bs, const float* Bts, void* C, int64_t M, int64_t N, int64_t K,
                      fp4_format fmt, fp4_out_dtype od, cudaStream_t stream) {
@@ -269,11 +306,17 @@ fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void
 
   const int bs = block_of(fmt);
   const int64_t kb4 = ceil_div(K / bs, 4);
-  const int atoms = kGBK / (4 * bs);
+  // Rows of 256 (M > 128) go to the CTA-pair kernel; a single 128-row band of M to the
+  // one-CTA kernel. Each kernel has its own K per pipeline stage.
+  const bool pair = M > 128;
+  const int slab_k = !pair ? kGBK : (fmt == FP4_MXFP4 ? PairCfg<kFmtMX>::kSlabK
+                                                      : PairCfg<kFmtNV>::kSlabK);
+  const int atoms = slab_k / (4 * bs);
+  const uint32_t b_box_rows = pair ? 128 : kGBN;
   CUtensorMap ta, tb, tsa, tsb;
   if (!make_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K / 2, M, kGBK / 2, kGBM,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K / 2, N, kGBK / 2, kGBN,
+      !make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K / 2, N, kGBK / 2, b_box_rows,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&tsa, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, As, kb4 * 64, ceil_div(M, 128),
                    atoms * 64, 1, CU_TENSOR_MAP_SWIZZLE_NONE) ||
@@ -285,12 +328,12 @@ fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void
   g.M = static_cast<int>(M);
   g.N = static_cast<int>(N);
   g.K = static_cast<int>(K);
-  g.tiles_m = static_cast<int>(ceil_div(M, kGBM));
+  g.tiles_m = static_cast<int>(ceil_div(M, pair ? 256 : kGBM));
   g.tiles_n = static_cast<int>(ceil_div(N, kGBN));
   const int64_t tiles = int64_t(g.tiles_m) * g.tiles_n;
   if (tiles > INT32_MAX) return FP4_ERR_SHAPE;
   g.num_tiles = static_cast<int>(tiles);
-  g.k_tiles = static_cast<int>(ceil_div(K, kGBK));
+  g.k_tiles = static_cast<int>(ceil_div(K, slab_k));
   g.C = C;
   g.sa = Ats;
   g.sb = Bts;
@@ -298,12 +341,20 @@ fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void
   const int grid = g.num_tiles < info->sm_count ? g.num_tiles : info->sm_count;
 
   cudaError_t e;
-  if (fmt == FP4_MXFP4)
+  if (pair) {
+    if (fmt == FP4_MXFP4)
+      e = od == FP4_OUT_F32 ? launch_gemm_pair<kFmtMX, 0>(ta, tb, tsa, tsb, g, dev, stream)
+                            : launch_gemm_pair<kFmtMX, 1>(ta, tb, tsa, tsb, g, dev, stream);
+    else
+      e = od == FP4_OUT_F32 ? launch_gemm_pair<kFmtNV, 0>(ta, tb, tsa, tsb, g, dev, stream)
+                            : launch_gemm_pair<kFmtNV, 1>(ta, tb, tsa, tsb, g, dev, stream);
+  } else if (fmt == FP4_MXFP4) {
     e = od == FP4_OUT_F32 ? launch_gemm<kFmtMX, 0>(ta, tb, tsa, tsb, g, grid, dev, stream)
                           : launch_gemm<kFmtMX, 1>(ta, tb, tsa, tsb, g, grid, dev, stream);
-  else
+  } else {
     e = od == FP4_OUT_F32 ? launch_gemm<kFmtNV, 0>(ta, tb, tsa, tsb, g, grid, dev, stream)
                           : launch_gemm<kFmtNV, 1>(ta, tb, tsa, tsb, g, grid, dev, stream);
+  }
   return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }
 

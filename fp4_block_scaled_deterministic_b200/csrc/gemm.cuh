@@ -20,7 +20,8 @@
 //              the 256 columns: it pulls its 32x128 fp32 block into registers,
 //              releases the accumulator (so the next tile's MMAs start), then scales
 //              and stores fp32 or bf16 rows to global memory.
-// TMEM columns: [0,256) accumulator, then the scale factors of the current slab.
+// TMEM columns: [0,256) accumulator, then a ring of 4 scale-factor regions (one per
+// slab in flight, so a slab's scale copies never wait for the previous slab's MMAs).
 // No cluster multicast anywhere. Every wait is bounded (status word on expiry).
 #pragma once
 
@@ -41,8 +42,11 @@ struct GemmCfg {
   static constexpr int kSFABytes = kAtoms * 512;
   static constexpr int kSFBBytes = 2 * kAtoms * 512;
   static constexpr int kStageBytes = kGABytes + kGBBytes + kSFABytes + kSFBBytes;
-  static constexpr int kTmemSFA = 256;
-  static constexpr int kTmemSFB = 256 + 4 * kAtoms;
+  // Scale factors of consecutive slabs go to a ring of kSFBufs TMEM regions so that a
+  // slab's smem->TMEM copies never overwrite columns the previous slab's MMAs still read.
+  static constexpr int kSFCols = 12 * kAtoms;  // 4*kAtoms (A) + 8*kAtoms (B) per slab
+  static constexpr int kSFBufs = 4;
+  static constexpr int kTmemSF = 256;
   static constexpr int kSmemBytes = 1024 + kGStages * kStageBytes + 256;
 };
 
@@ -80,6 +84,107 @@ template <int FMT>
 __device__ __forceinline__ constexpr uint32_t idesc_fp4() {
   return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kGBN >> 3) << 17) |
          ((FMT == kFmtMX ? 1u : 0u) << 23) | (static_cast<uint32_t>(kGBM >> 4) << 24);
+}
+
+
+// Instruction descriptor of the pair MMA: as idesc_fp4 with M = 256.
+template <int FMT>
+__device__ __forceinline__ constexpr uint32_t idesc_fp4_pair() {
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(256 >> 3) << 17) |
+         ((FMT == kFmtMX ? 1u : 0u) << 23) | (static_cast<uint32_t>(256 >> 4) << 24);
+}
+
+// Issue one K slab: copy its scale atoms into TMEM ring slot (t_sfa, t_sfb = t_sfa +
+// 4*atoms) and run the 4 MMAs of K = 64 each. dA/dB/dSFA/dSFB are the slab's shared
+// memory descriptors; stepping inside the slab only adds to their start-address field
+// (+2 per 32 bytes of K, +32 per 512-byte atom), which never carries out of the field.
+template <int FMT, bool PAIR, int SLAB_K = kGBK>
+__device__ __forceinline__ void issue_slab(uint32_t tmem_acc, uint32_t t_sfa, uint64_t dA,
+                                           uint64_t dB, uint64_t dSFA, uint64_t dSFB,
+                                           uint32_t first_slab) {
+  // A slab wider than 256 elements is staged as SLAB_K/256 sub-tiles of 128-byte rows,
+  // each its own 128B-swizzle block of (rows x 128 B); MMA j reads sub-tile j/4.
+  constexpr int kAtoms = SLAB_K / (4 * (FMT == kFmtMX ? 32 : 16));
+  const uint32_t t_sfb = t_sfa + 4 * kAtoms;
+#pragma unroll
+  for (int at = 0; at < kAtoms; ++at) {
+    if constexpr (PAIR) tc_cp_32x128b_warpx4_pair(t_sfa + 4 * at, dSFA + 32 * at);
+    else tc_cp_32x128b_warpx4(t_sfa + 4 * at, dSFA + 32 * at);
+  }
+#pragma unroll
+  for (int rb = 0; rb < 2; ++rb)
+#pragma unroll
+    for (int at = 0; at < kAtoms; ++at) {
+      const uint64_t d = dSFB + rb * (kAtoms * 32) + 32 * at;
+      if constexpr (PAIR) tc_cp_32x128b_warpx4_pair(t_sfb + 8 * at + 4 * rb, d);
+      else tc_cp_32x128b_warpx4(t_sfb + 8 * at + 4 * rb, d);
+    }
+  constexpr uint32_t kIdesc = PAIR ? idesc_fp4_pair<FMT>() : idesc_fp4<FMT>();
+#pragma unroll
+  for (int j = 0; j < SLAB_K / 64; ++j) {
+    // MXFP4: two MMAs share one atom column, bytes {0,1} then {2,3} (scale id 0 / 2);
+    // NVFP4: one atom column per MMA, all four bytes (scale id 0).
+    const int at = FMT == kFmtMX ? (j >> 1) : j;
+    const uint32_t id = FMT == kFmtMX ? static_cast<uint32_t>((j & 1) * 2) : 0u;
+    const uint32_t tsfa = (t_sfa + 4 * at) | (id << 30);
+    const uint32_t tsfb = (t_sfb + 8 * at) | (id << 30);
+    const uint32_t idesc = kIdesc | (id << 29) | (id << 4);
+    const uint32_t acc = (j > 0 || !first_slab) ? 1u : 0u;
+    const uint64_t koff = (j >> 2) * (PAIR ? (128 * 128 >> 4) : 0) + 2 * (j & 3);
+    if constexpr (PAIR)
+      tc_mma_fp4_pair<FMT == kFmtMX>(tmem_acc, dA + koff, dB + koff, idesc, tsfa, tsfb, acc);
+    else
+      tc_mma_fp4<FMT == kFmtMX>(tmem_acc, dA + koff, dB + koff, idesc, tsfa, tsfb, acc);
+  }
+}
+
+// Scale (NVFP4) and store one thread's row segment of 128 accumulator columns:
+// output row m, columns [n0, n0 + 128), skipping rows >= M and 32-column chunks >= N.
+template <int FMT, int OUT_BF16>
+__device__ __forceinline__ void store_row_segment(const uint32_t (&r)[128], int m, int n0,
+                                                  const GemmArgs& g, float alpha) {
+  if (m >= g.M) return;
+  if constexpr (OUT_BF16) {
+    __nv_bfloat16* crow = static_cast<__nv_bfloat16*>(g.C) + static_cast<int64_t>(m) * g.N + n0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (n0 + 32 * c < g.N) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          uint32_t w[4];
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            float x0 = __uint_as_float(r[32 * c + 8 * i + 2 * p]);
+            float x1 = __uint_as_float(r[32 * c + 8 * i + 2 * p + 1]);
+            if constexpr (FMT == kFmtNV) { x0 = __fmul_rn(x0, alpha); x1 = __fmul_rn(x1, alpha); }
+            const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+            w[p] = *reinterpret_cast<const uint32_t*>(&h);
+          }
+          *reinterpret_cast<uint4*>(crow + 32 * c + 8 * i) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+  } else {
+    float* crow = static_cast<float*>(g.C) + static_cast<int64_t>(m) * g.N + n0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (n0 + 32 * c < g.N) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float4 o;
+          o.x = __uint_as_float(r[32 * c + 4 * i + 0]);
+          o.y = __uint_as_float(r[32 * c + 4 * i + 1]);
+          o.z = __uint_as_float(r[32 * c + 4 * i + 2]);
+          o.w = __uint_as_float(r[32 * c + 4 * i + 3]);
+          if constexpr (FMT == kFmtNV) {
+            o.x = __fmul_rn(o.x, alpha); o.y = __fmul_rn(o.y, alpha);
+            o.z = __fmul_rn(o.z, alpha); o.w = __fmul_rn(o.w, alpha);
+          }
+          *reinterpret_cast<float4*>(crow + 32 * c + 4 * i) = o;
+        }
+      }
+    }
+  }
 }
 
 template <int FMT, int OUT_BF16>
@@ -136,7 +241,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
       for (int tile = blockIdx.x; tile < g.num_tiles && !*abort_flag; tile += gridDim.x) {
         const int tm = tile % g.tiles_m, tn = tile / g.tiles_m;
         for (int kt = 0; kt < g.k_tiles; ++kt) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, g.wait_limit_ns) || *abort_flag) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, g.wait_limit_ns)) {
             *abort_flag = 1;
             break;
           }
@@ -154,6 +259,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
+      const uint64_t dA0 = desc_kmajor_sw128(smem_u32(sA)), dB0 = desc_kmajor_sw128(smem_u32(sB));
+      const uint64_t dSA0 = desc_sf_atom(smem_u32(sSFA)), dSB0 = desc_sf_atom(smem_u32(sSFB));
+      const uint32_t t_sf0 = tmem + Cfg::kTmemSF;
+      uint64_t dA = dA0, dB = dB0, dSA = dSA0, dSB = dSB0;
+      uint32_t t_sf = t_sf0, sf_slot = 0;
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       for (int tile = blockIdx.x; tile < g.num_tiles && !*abort_flag; tile += gridDim.x) {
@@ -164,40 +274,22 @@ __global__ void __launch_bounds__(kGThreads, 1)
         tc_fence_after();
         bool ok = true;
         for (int kt = 0; kt < g.k_tiles; ++kt) {
-          if (!mbar_wait(&full[stage], phase, g.wait_limit_ns) || *abort_flag) {
+          if (!mbar_wait(&full[stage], phase, g.wait_limit_ns)) {
             *abort_flag = 1;
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t a_base = smem_u32(sA + stage * kGABytes);
-          const uint32_t b_base = smem_u32(sB + stage * kGBBytes);
-          const uint32_t sfa = smem_u32(sSFA + stage * Cfg::kSFABytes);
-          const uint32_t sfb = smem_u32(sSFB + stage * Cfg::kSFBBytes);
-#pragma unroll
-          for (int at = 0; at < Cfg::kAtoms; ++at)
-            tc_cp_32x128b_warpx4(tmem + Cfg::kTmemSFA + 4 * at, desc_sf_atom(sfa + 512 * at));
-#pragma unroll
-          for (int rb = 0; rb < 2; ++rb)
-#pragma unroll
-            for (int at = 0; at < Cfg::kAtoms; ++at)
-              tc_cp_32x128b_warpx4(tmem + Cfg::kTmemSFB + 8 * at + 4 * rb,
-                                   desc_sf_atom(sfb + rb * Cfg::kSFABytes + 512 * at));
-#pragma unroll
-          for (int j = 0; j < kGBK / 64; ++j) {
-            // MXFP4: two MMAs share one atom column, bytes {0,1} then {2,3} (scale id 0/2);
-            // NVFP4: one atom column per MMA, all four bytes (scale id 0).
-            const int at = FMT == kFmtMX ? (j >> 1) : j;
-            const uint32_t id = FMT == kFmtMX ? static_cast<uint32_t>((j & 1) * 2) : 0u;
-            const uint32_t tsfa = (tmem + Cfg::kTmemSFA + 4 * at) | (id << 30);
-            const uint32_t tsfb = (tmem + Cfg::kTmemSFB + 8 * at) | (id << 30);
-            const uint32_t idesc = idesc_fp4<FMT>() | (id << 29) | (id << 4);
-            tc_mma_fp4<FMT == kFmtMX>(tmem, desc_kmajor_sw128(a_base + 32 * j),
-                                      desc_kmajor_sw128(b_base + 32 * j), idesc, tsfa, tsfb,
-                                      (kt | j) != 0 ? 1u : 0u);
-          }
+          issue_slab<FMT, false>(tmem, t_sf, dA, dB, dSA, dSB, kt == 0);
           tc_commit(&empty[stage]);
-          if (++stage == kGStages) { stage = 0; phase ^= 1u; }
+          if (++sf_slot == Cfg::kSFBufs) { sf_slot = 0; t_sf = t_sf0; } else { t_sf += Cfg::kSFCols; }
+          if (++stage == kGStages) {
+            stage = 0;
+            phase ^= 1u;
+            dA = dA0; dB = dB0; dSA = dSA0; dSB = dSB0;
+          } else {
+            dA += kGABytes >> 4; dB += kGBBytes >> 4;
+            dSA += Cfg::kSFABytes >> 4; dSB += Cfg::kSFBBytes >> 4;
+          }
         }
         if (!ok) break;
         tc_commit(acc_full);
@@ -219,61 +311,16 @@ __global__ void __launch_bounds__(kGThreads, 1)
         break;
       }
       tc_fence_after();
-      uint32_t r[4][32];
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * quarter) << 16) + 128 * half;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(taddr + 32 * c, r[c]);
+      uint32_t r[128];
+      tmem_ld_32x32b_x128(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + 128 * half, r);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);
       acc_phase ^= 1u;
 
-      const int m = tm * kGBM + 32 * quarter + lane;
-      const int n0 = tn * kGBN + 128 * half;
-      if (m < g.M) {
-        if constexpr (OUT_BF16) {
-          __nv_bfloat16* crow = static_cast<__nv_bfloat16*>(g.C) + static_cast<int64_t>(m) * g.N + n0;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            if (n0 + 32 * c < g.N) {
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                uint32_t w[4];
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                  float x0 = __uint_as_float(r[c][8 * i + 2 * p]);
-                  float x1 = __uint_as_float(r[c][8 * i + 2 * p + 1]);
-                  if constexpr (FMT == kFmtNV) { x0 = __fmul_rn(x0, alpha); x1 = __fmul_rn(x1, alpha); }
-                  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
-                  w[p] = *reinterpret_cast<const uint32_t*>(&h);
-                }
-                *reinterpret_cast<uint4*>(crow + 32 * c + 8 * i) = make_uint4(w[0], w[1], w[2], w[3]);
-              }
-            }
-          }
-        } else {
-          float* crow = static_cast<float*>(g.C) + static_cast<int64_t>(m) * g.N + n0;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            if (n0 + 32 * c < g.N) {
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                float4 o;
-                o.x = __uint_as_float(r[c][4 * i + 0]);
-                o.y = __uint_as_float(r[c][4 * i + 1]);
-                o.z = __uint_as_float(r[c][4 * i + 2]);
-                o.w = __uint_as_float(r[c][4 * i + 3]);
-                if constexpr (FMT == kFmtNV) {
-                  o.x = __fmul_rn(o.x, alpha); o.y = __fmul_rn(o.y, alpha);
-                  o.z = __fmul_rn(o.z, alpha); o.w = __fmul_rn(o.w, alpha);
-                }
-                *reinterpret_cast<float4*>(crow + 32 * c + 4 * i) = o;
-              }
-            }
-          }
-        }
-      }
+      store_row_segment<FMT, OUT_BF16>(r, tm * kGBM + 32 * quarter + lane, tn * kGBN + 128 * half,
+                                       g, alpha);
     }
   }
   __syncwarp();
@@ -282,6 +329,197 @@ __global__ void __launch_bounds__(kGThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+
+// ====================================================================================
+// CTA-pair variant (cta_group::2): a cluster of two CTAs on two SMs computes a 256x256
+// output tile. Each CTA stages its own 128 rows of A and its own 128-row half of B
+// (plus the scales of all 256 B rows, which both tensor cores need), so each SM pulls
+// a third less operand data per flop from L2 than the single-CTA kernel, and the
+// smaller stages allow a deeper ring. CTA rank 0 of the pair (the leader) issues the
+// pair-wide MMAs; both CTAs load through TMA into their own shared memory with the
+// transfers counted on the leader's barrier, and both drain their own half of the
+// accumulator (rows 128*rank ... +128, all 256 columns) from their own TMEM.
+// The loads carry no multicast; only the tcgen05.commit arrivals are multicast to the
+// two CTAs of the pair.
+template <int FMT>
+struct PairCfg {
+  static constexpr int kBlock = FMT == kFmtMX ? 32 : 16;
+  // K per stage: 512 for MXFP4 (8 MMAs per barrier wait and commit, 3 stages), 256 for
+  // NVFP4 (whose scale copies are twice as many per K; 5 stages).
+  static constexpr int kSlabK = FMT == kFmtMX ? 512 : 256;
+  static constexpr int kSub = kSlabK / 256;          // 128-byte-wide swizzled sub-tiles
+  static constexpr int kAtoms = kSlabK / (4 * kBlock);
+  static constexpr int kABytes = 128 * kSlabK / 2;   // this CTA's 128 rows of A
+  static constexpr int kBBytes = 128 * kSlabK / 2;   // this CTA's 128-row half of B
+  static constexpr int kSFABytes = kAtoms * 512;     // scales of this CTA's A rows
+  static constexpr int kSFBBytes = 2 * kAtoms * 512; // scales of all 256 B rows
+  static constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
+  static constexpr int kStages = FMT == kFmtMX ? 3 : 5;
+  static constexpr int kSFCols = 12 * kAtoms;
+  static constexpr int kSFBufs = 4;
+  static constexpr int kTmemSF = 256;
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 256;
+};
+
+
+template <int FMT, int OUT_BF16>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
+    gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                         const __grid_constant__ CUtensorMap tmB,
+                         const __grid_constant__ CUtensorMap tmSFA,
+                         const __grid_constant__ CUtensorMap tmSFB, const GemmArgs g) {
+  using Cfg = PairCfg<FMT>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + S * Cfg::kABytes;
+  uint8_t* sSFA = sB + S * Cfg::kBBytes;
+  uint8_t* sSFB = sSFA + S * Cfg::kSFABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sSFB + S * Cfg::kSFBBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* acc_full = bars + 2 * S;
+  uint64_t* acc_empty = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmSFA);
+    tma_prefetch_desc(&tmSFB);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 16);  // 8 epilogue warps in each CTA of the pair
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t leader_full = mapa_shared(smem_u32(full), 0);
+  const uint32_t leader_acc_empty = mapa_shared(smem_u32(acc_empty), 0);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer (both CTAs)
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = pair; tile < g.num_tiles && !*abort_flag; tile += npairs) {
+        const int tm = tile % g.tiles_m, tn = tile / g.tiles_m;
+        for (int kt = 0; kt < g.k_tiles; ++kt) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, g.wait_limit_ns)) {
+            *abort_flag = 1;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kStageBytes);
+          const uint32_t bar = leader_full + 8u * stage;
+#pragma unroll
+          for (int sub = 0; sub < Cfg::kSub; ++sub) {
+            const int kx = kt * (Cfg::kSlabK / 2) + 128 * sub;
+            tma_load_2d_pair(sA + stage * Cfg::kABytes + sub * 16384, &tmA, bar, kx,
+                             tm * 256 + 128 * static_cast<int>(rank));
+            tma_load_2d_pair(sB + stage * Cfg::kBBytes + sub * 16384, &tmB, bar, kx,
+                             tn * 256 + 128 * static_cast<int>(rank));
+          }
+          tma_load_2d_pair(sSFA + stage * Cfg::kSFABytes, &tmSFA, bar, kt * Cfg::kAtoms * 64,
+                           2 * tm + static_cast<int>(rank));
+          tma_load_2d_pair(sSFB + stage * Cfg::kSFBBytes, &tmSFB, bar, kt * Cfg::kAtoms * 64,
+                           2 * tn);
+          if (++stage == S) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ------------------------------------------------------------ MMA issuer (leader)
+      const uint64_t dA0 = desc_kmajor_sw128(smem_u32(sA)), dB0 = desc_kmajor_sw128(smem_u32(sB));
+      const uint64_t dSA0 = desc_sf_atom(smem_u32(sSFA)), dSB0 = desc_sf_atom(smem_u32(sSFB));
+      const uint32_t t_sf0 = tmem + Cfg::kTmemSF;
+      uint64_t dA = dA0, dB = dB0, dSA = dSA0, dSB = dSB0;
+      uint32_t t_sf = t_sf0, sf_slot = 0;
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      for (int tile = pair; tile < g.num_tiles && !*abort_flag; tile += npairs) {
+        if (!mbar_wait(acc_empty, acc_phase ^ 1u, g.wait_limit_ns)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        bool ok = true;
+        for (int kt = 0; kt < g.k_tiles; ++kt) {
+          if (!mbar_wait(&full[stage], phase, g.wait_limit_ns)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          issue_slab<FMT, true, Cfg::kSlabK>(tmem, t_sf, dA, dB, dSA, dSB, kt == 0);
+          tc_commit_pair_mc(&empty[stage], 0x3);
+          if (++sf_slot == Cfg::kSFBufs) { sf_slot = 0; t_sf = t_sf0; } else { t_sf += Cfg::kSFCols; }
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+            dA = dA0; dB = dB0; dSA = dSA0; dSB = dSB0;
+          } else {
+            dA += Cfg::kABytes >> 4; dB += Cfg::kBBytes >> 4;
+            dSA += Cfg::kSFABytes >> 4; dSB += Cfg::kSFBBytes >> 4;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(acc_full, 0x3);
+        acc_phase ^= 1u;
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue (both CTAs)
+    const int ew = warp - 2;
+    const int quarter = warp & 3;
+    const int half = ew >> 2;
+    float alpha = 1.0f;
+    if constexpr (FMT == kFmtNV) alpha = __fmul_rn(*g.sa, *g.sb);
+    uint32_t acc_phase = 0;
+    for (int tile = pair; tile < g.num_tiles && !*abort_flag; tile += npairs) {
+      const int tm = tile % g.tiles_m, tn = tile / g.tiles_m;
+      if (!mbar_wait(acc_full, acc_phase, g.wait_limit_ns)) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      uint32_t r[128];
+      tmem_ld_32x32b_x128(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + 128 * half, r);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(leader_acc_empty);
+      acc_phase ^= 1u;
+      store_row_segment<FMT, OUT_BF16>(r, tm * 256 + 128 * static_cast<int>(rank) + 32 * quarter +
+                                              lane,
+                                       tn * kGBN + 128 * half, g, alpha);
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
   }
 }
 

@@ -11,15 +11,16 @@
 //   output is transposed, codes [C][R/2] (the token-axis layout Wgrad needs).
 //   DUAL: both from one read of x.
 //
-// Structure (one CTA per SM, persistent): the input is cut into 128x128 bf16 tiles;
-// a 3-stage TMA pipeline brings each tile into shared memory as two 128B-swizzled
-// boxes of 128 rows x 64 columns. 256 threads then work from shared memory:
-//   ROW job  = one row, 32 consecutive columns (4 x 16-byte conflict-free reads);
-//   COL job  = two adjacent columns, 32 consecutive rows (32 x 4-byte reads);
-// the rotation runs entirely in registers, codes are staged in a 64B-swizzled
-// [128][64 B] tile and written by a TMA store, scale atoms are assembled in shared
-// memory and written by bulk copies. Staging is double-buffered so stores overlap
-// the next tile.
+// Structure (two CTAs per SM, persistent): the input is cut into 128x128 bf16 tiles;
+// a 2-stage TMA pipeline per CTA brings each tile into shared memory as two
+// 128B-swizzled boxes of 128 rows x 64 columns. 256 threads then work from shared
+// memory in jobs of two 32-element vectors held lane-wise in float2 registers:
+//   ROW job = one row, 64 consecutive columns (two segments; 8 conflict-free 16-B reads);
+//   COL job = two adjacent columns, 32 consecutive rows (32 conflict-free 4-B reads);
+// the rotation runs in registers with packed fp32x2 arithmetic, codes are staged in a
+// 64B-swizzled [128][64 B] tile and written by a TMA store, scale atoms are assembled
+// in shared memory (2- and 4-byte stores) and written by bulk copies. Staging is
+// double-buffered so stores overlap the next tile.
 #pragma once
 
 #include "common.cuh"
@@ -29,7 +30,8 @@ namespace fp4k {
 enum { kModeRow = 1, kModeCol = 2, kModeDual = 3 };
 
 constexpr int kQThreads = 256;
-constexpr int kQStages = 3;
+constexpr int kQCtasPerSM = 2;
+constexpr int kQStages = 2;
 constexpr int kQBoxBytes = 128 * 64 * 2;    // 128 rows x 64 bf16
 constexpr int kQInBytes = 2 * kQBoxBytes;   // a 128 x 128 bf16 tile
 constexpr int kQCodeBytes = 128 * 64;       // 128 rows x 64 code bytes
@@ -52,103 +54,200 @@ struct QuantArgs {
   uint64_t wait_limit_ns;
 };
 
-// Normalised block FWHT of 32 registers holding 32/HN independent groups.
+// Every unit of work ("job") is two independent 32-element vectors held lane-wise in
+// float2 registers (.x = first vector, .y = second), so the butterflies, scalings and
+// quotients use the packed fp32x2 instructions; each lane is rounded exactly as the
+// scalar operation would be.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  return __fadd2_rn(a, make_float2(-b.x, -b.y));  // a - b == a + (-b), same rounding
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+
+// Normalised block FWHT of both lanes: groups of HN along the 32 elements, butterfly
+// strides 1, 2, 4, ... in that order, then x RN(1/sqrt(HN)).
 template <int HN>
-__device__ __forceinline__ void fwht32(float (&v)[32]) {
+__device__ __forceinline__ void fwht_x2(float2 (&p)[32]) {
   if constexpr (HN > 0) {
 #pragma unroll
     for (int h = 1; h < HN; h <<= 1) {
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         if ((i & h) == 0) {
-          const float a = v[i], b = v[i + h];
-          v[i] = __fadd_rn(a, b);
-          v[i + h] = __fsub_rn(a, b);
+          const float2 a = p[i], b = p[i + h];
+          p[i] = add2(a, b);
+          p[i + h] = sub2(a, b);
         }
       }
     }
     // 0.25 = 1/sqrt(16) exactly; 0x3E3504F3 = fp32 nearest to 1/sqrt(32)
     const float c = (HN == 16) ? 0.25f : __uint_as_float(0x3E3504F3u);
+    const float2 c2 = make_float2(c, c);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], c);
+    for (int i = 0; i < 32; ++i) p[i] = mul2(p[i], c2);
   }
 }
 
-__device__ __forceinline__ float amax_of(const float* v, int n) {
-  float m = 0.0f;
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// max |x| over elements [b, b+n) of each lane.
+__device__ __forceinline__ float2 amax_x2(const float2 (&p)[32], int b, int n) {
+  float m0 = 0.0f, m1 = 0.0f;
 #pragma unroll
-  for (int i = 0; i < n; ++i) m = fmaxf(m, fabsf(v[i]));
-  return m;
+  for (int i = 0; i < n; i += 2) {
+    m0 = max3f(m0, fabsf(p[b + i].x), fabsf(p[b + i + 1].x));
+    m1 = max3f(m1, fabsf(p[b + i].y), fabsf(p[b + i + 1].y));
+  }
+  return make_float2(m0, m1);
 }
 
-// MXFP4 block of 32: E8M0 byte = max(biased exponent of amax - 2, 0), i.e. the byte of
+__device__ __forceinline__ uint32_t cvt8x(const float2 (&p)[32], int b) {
+  const float v[8] = {p[b].x, p[b + 1].x, p[b + 2].x, p[b + 3].x,
+                      p[b + 4].x, p[b + 5].x, p[b + 6].x, p[b + 7].x};
+  return cvt_e2m1x8(v);
+}
+__device__ __forceinline__ uint32_t cvt8y(const float2 (&p)[32], int b) {
+  const float v[8] = {p[b].y, p[b + 1].y, p[b + 2].y, p[b + 3].y,
+                      p[b + 4].y, p[b + 5].y, p[b + 6].y, p[b + 7].y};
+  return cvt_e2m1x8(v);
+}
+
+// Encoded job: 16 code bytes per lane and its scale bytes (MXFP4: byte 0; NVFP4: bytes
+// 0 and 1 for the two 16-element blocks).
+struct Enc {
+  uint4 cx, cy;
+  uint32_t sx, sy;  // scale bytes, lowest byte first
+};
+
+// MXFP4 block of 32 per lane: byte = max(biased exponent of amax - 2, 0), i.e. the byte of
 // e = floor(log2 amax) - 2 clamped at -127 (zero and subnormal amax give 0); codes of
-// v * 2^-e. 2^-e = 2^(127 - byte) is built from its bit pattern (byte <= 252).
-__device__ __forceinline__ uint32_t mx_encode32(float (&v)[32], uint4& codes) {
-  const float amax = amax_of(v, 32);
-  const uint32_t ex = (__float_as_uint(amax) >> 23) & 0xFFu;
-  const uint32_t sb = ex > 2u ? ex - 2u : 0u;
-  const float inv = __uint_as_float((254u - sb) << 23);
+// v * 2^-e, 2^-e = 2^(127 - byte) built from its bit pattern (byte <= 252).
+__device__ __forceinline__ Enc mx_encode_x2(float2 (&p)[32]) {
+  const float2 am = amax_x2(p, 0, 32);
+  const uint32_t ex = (__float_as_uint(am.x) >> 23) & 0xFFu;
+  const uint32_t ey = (__float_as_uint(am.y) >> 23) & 0xFFu;
+  const uint32_t bx = ex > 2u ? ex - 2u : 0u, by = ey > 2u ? ey - 2u : 0u;
+  const float2 inv = make_float2(__uint_as_float((254u - bx) << 23), __uint_as_float((254u - by) << 23));
 #pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], inv);
-  codes.x = cvt_e2m1x8(v + 0);
-  codes.y = cvt_e2m1x8(v + 8);
-  codes.z = cvt_e2m1x8(v + 16);
-  codes.w = cvt_e2m1x8(v + 24);
-  return sb;
+  for (int i = 0; i < 32; ++i) p[i] = mul2(p[i], inv);
+  Enc e;
+  e.cx = make_uint4(cvt8x(p, 0), cvt8x(p, 8), cvt8x(p, 16), cvt8x(p, 24));
+  e.cy = make_uint4(cvt8y(p, 0), cvt8y(p, 8), cvt8y(p, 16), cvt8y(p, 24));
+  e.sx = bx;
+  e.sy = by;
+  return e;
 }
 
-// NVFP4 block of 16 under tensor scale S (six_s = 6*S, rounded once):
-// byte = UE4M3_RNE_satfinite(bmax / six_s), d = ue4m3(byte) * S, codes of v / d;
-// a zero byte gives signed zeros.
-__device__ __forceinline__ uint32_t nv_encode16(float* v, float S, float six_s, uint32_t& c0,
-                                                uint32_t& c1) {
-  const float bmax = amax_of(v, 16);
-  const uint32_t sb = cvt_e4m3(__fdiv_rn(bmax, six_s));
-  if (sb == 0u) {
+// True when q lies within 4 units in the last place of a number with at most two
+// fraction bits; every E2M1 rounding threshold (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5) is
+// such a number.
+__device__ __forceinline__ bool near_e2m1_threshold(float q) {
+  return ((__float_as_uint(q) + 4u) & 0x1FFFFFu) < 9u;
+}
+
+// NVFP4 block of 16 per lane under tensor scale S (six_s = 6*S, rounded once):
+// byte = UE4M3_RNE_satfinite(bmax / six_s), d = ue4m3(byte) * S, codes of the fp32
+// quotient v / d; a zero byte gives signed zeros.
+// The quotient is formed as v * y with y = RN(1/d): then |v*y - v/d| < 2 ulps, so v*y and
+// RN(v/d) fall on the same side of every E2M1 threshold unless v*y is within 4 ulps of
+// one; those (rare) blocks, and blocks whose 1/d overflows, are divided exactly.
+__device__ __forceinline__ void nv_block_x2(float2 (&p)[32], int b, float S, float six_s,
+                                            uint32_t& sbx, uint32_t& sby) {
+  const float2 bm = amax_x2(p, b, 16);
+  sbx = cvt_e4m3(__fdiv_rn(bm.x, six_s));
+  sby = cvt_e4m3(__fdiv_rn(bm.y, six_s));
+  const float dx = __fmul_rn(e4m3_to_f32(sbx), S), dy = __fmul_rn(e4m3_to_f32(sby), S);
+  const float yx = __frcp_rn(dx), yy = __frcp_rn(dy);
+  const float2 y2 = make_float2(yx, yy);
+  float2 q[16];
+  bool exact = !(yx <= 3.0e38f) || !(yy <= 3.0e38f);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(__float_as_uint(v[i]) & 0x80000000u);
-  } else {
-    const float d = __fmul_rn(e4m3_to_f32(sb), S);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __fdiv_rn(v[i], d);
+  for (int i = 0; i < 16; ++i) {
+    q[i] = mul2(p[b + i], y2);
+    exact |= near_e2m1_threshold(q[i].x) | near_e2m1_threshold(q[i].y);
   }
-  c0 = cvt_e2m1x8(v);
-  c1 = cvt_e2m1x8(v + 8);
-  return sb;
+  if (exact) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) q[i] = make_float2(__fdiv_rn(p[b + i].x, dx), __fdiv_rn(p[b + i].y, dy));
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    p[b + i].x = sbx == 0u ? __uint_as_float(__float_as_uint(p[b + i].x) & 0x80000000u) : q[i].x;
+    p[b + i].y = sby == 0u ? __uint_as_float(__float_as_uint(p[b + i].y) & 0x80000000u) : q[i].y;
+  }
 }
 
-// Offset of scale (row-in-atom-block r, block kb within the tile's atoms) in a staged
-// scale tile holding one or two atoms: atom = kb/4, then (r%32)*16 + (r/32)*4 + kb%4.
+__device__ __forceinline__ Enc nv_encode_x2(float2 (&p)[32], float S, float six_s) {
+  uint32_t x0, y0, x1, y1;
+  nv_block_x2(p, 0, S, six_s, x0, y0);
+  nv_block_x2(p, 16, S, six_s, x1, y1);
+  Enc e;
+  e.cx = make_uint4(cvt8x(p, 0), cvt8x(p, 8), cvt8x(p, 16), cvt8x(p, 24));
+  e.cy = make_uint4(cvt8y(p, 0), cvt8y(p, 8), cvt8y(p, 16), cvt8y(p, 24));
+  e.sx = x0 | (x1 << 8);
+  e.sy = y0 | (y1 << 8);
+  return e;
+}
+
+template <int FMT>
+__device__ __forceinline__ Enc encode_x2(float2 (&p)[32], float S, float six_s) {
+  if constexpr (FMT == kFmtMX) return mx_encode_x2(p);
+  else return nv_encode_x2(p, S, six_s);
+}
+
+// Offset of scale (row r of the 128-row atom block, block kb of the tile) in a staged
+// scale tile of one or two atoms: atom kb/4, then (r%32)*16 + (r/32)*4 + kb%4.
 __device__ __forceinline__ int atom_off(int r, int kb) {
   return (kb >> 2) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (kb & 3);
 }
+// Staged code tile [128 rows][64 B], 64-byte swizzle: 16-byte chunk q of row r.
+__device__ __forceinline__ uint8_t* code_chunk(uint8_t* tile, int r, int q) {
+  return tile + r * 64 + ((q ^ ((r >> 1) & 3)) << 4);
+}
 
-// Encode 32 rotated values (one ROW segment or one COL column segment) into 16 code
-// bytes at code_dst and their scale byte(s) into the staged atom(s).
-template <int FMT>
-__device__ __forceinline__ void encode32(float (&v)[32], uint8_t* code_dst, uint8_t* sc_tile,
-                                         int r, int seg, float S, float six_s) {
-  uint4 codes;
-  if constexpr (FMT == kFmtMX) {
-    const uint32_t sb = mx_encode32(v, codes);
-    sc_tile[atom_off(r, seg)] = static_cast<uint8_t>(sb);
-  } else {
-    const uint32_t s0 = nv_encode16(v, S, six_s, codes.x, codes.y);
-    const uint32_t s1 = nv_encode16(v + 16, S, six_s, codes.z, codes.w);
-    sc_tile[atom_off(r, 2 * seg)] = static_cast<uint8_t>(s0);
-    sc_tile[atom_off(r, 2 * seg + 1)] = static_cast<uint8_t>(s1);
+// ROW job: tile row r, box b (columns 64b .. 64b+63) = segments 2b (lane x) and 2b+1
+// (lane y); 8 conflict-free 16-byte reads of the 128B-swizzled box row.
+__device__ __forceinline__ void load_row_job(const uint8_t* in, int r, int b, float2 (&p)[32]) {
+  const uint8_t* rowp = in + b * kQBoxBytes + r * 128;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 wx = *reinterpret_cast<const uint4*>(rowp + ((i ^ (r & 7)) << 4));
+    const uint4 wy = *reinterpret_cast<const uint4*>(rowp + (((4 + i) ^ (r & 7)) << 4));
+    p[8 * i + 0] = make_float2(bf16lo(wx.x), bf16lo(wy.x));
+    p[8 * i + 1] = make_float2(bf16hi(wx.x), bf16hi(wy.x));
+    p[8 * i + 2] = make_float2(bf16lo(wx.y), bf16lo(wy.y));
+    p[8 * i + 3] = make_float2(bf16hi(wx.y), bf16hi(wy.y));
+    p[8 * i + 4] = make_float2(bf16lo(wx.z), bf16lo(wy.z));
+    p[8 * i + 5] = make_float2(bf16hi(wx.z), bf16hi(wy.z));
+    p[8 * i + 6] = make_float2(bf16lo(wx.w), bf16lo(wy.w));
+    p[8 * i + 7] = make_float2(bf16hi(wx.w), bf16hi(wy.w));
   }
-  *reinterpret_cast<uint4*>(code_dst) = codes;
+}
+// COL job: tile columns c = 64b + 2w (lane x) and c + 1 (lane y), rows 32s .. 32s+31;
+// 32 conflict-free 4-byte reads.
+__device__ __forceinline__ void load_col_job(const uint8_t* in, int b, int w, int s,
+                                             float2 (&p)[32]) {
+  const uint8_t* boxp = in + b * kQBoxBytes;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int r = 32 * s + i;
+    const uint32_t v = *reinterpret_cast<const uint32_t*>(boxp + r * 128 +
+                                                          (((w >> 2) ^ (r & 7)) << 4) + ((w & 3) << 2));
+    p[i] = make_float2(bf16lo(v), bf16hi(v));
+  }
 }
 
 template <int FMT, int HN, int MODE, bool AMAX>
-__global__ void __launch_bounds__(kQThreads, 1)
+__global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
     quantize_kernel(const __grid_constant__ CUtensorMap tm_in,
                     const __grid_constant__ CUtensorMap tm_rcodes,
                     const __grid_constant__ CUtensorMap tm_ccodes, const QuantArgs a) {
   constexpr bool kRow = (MODE & kModeRow) != 0;
   constexpr bool kCol = (MODE & kModeCol) != 0;
+  constexpr bool kDual = kRow && kCol;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -201,6 +300,17 @@ __global__ void __launch_bounds__(kQThreads, 1)
     for (int s = 0; s < pro; ++s) issue_load(s, bid + s * nctas);
   }
 
+  // Work split of one 128x128 tile over the 256 threads:
+  //   ROW only : thread -> row tid%128, box tid/128                 (1 ROW job)
+  //   COL only : thread -> column pair tid%64, segment tid/64        (1 COL job)
+  //   DUAL     : threads 0-127 -> row tid, boxes 0 and 1              (2 ROW jobs)
+  //              threads 128-255 -> pair t%64, segments 2(t/64)+{0,1} (2 COL jobs)
+  const bool row_thread = kRow && (!kDual || tid < 128);
+  const int ct = kDual ? tid - 128 : tid;
+  const int row_r = tid & 127;
+  const int col_pair = ct & 63, col_b = col_pair >> 5, col_w = col_pair & 31;
+  const int col_c = 64 * col_b + 2 * col_w;
+
   float amax_r = 0.0f, amax_c = 0.0f;
   for (int it = 0; it < my_tiles; ++it) {
     const int tile = bid + it * nctas;
@@ -209,59 +319,69 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const bool ok = mbar_wait(&full[st], static_cast<uint32_t>((it / kQStages) & 1), a.wait_limit_ns);
     if (__syncthreads_or(!ok)) break;  // give up together; the status word says why
     const uint8_t* in = s_in + st * kQInBytes;
+    uint8_t* rcode = s_rcode + ob * kQCodeBytes;
+    uint8_t* ccode = s_ccode + ob * kQCodeBytes;
+    uint8_t* rsc = s_rsc + ob * kQScaleBytes;
+    uint8_t* csc = s_csc + ob * kQScaleBytes;
 
-    if constexpr (kRow) {
-      // ROW jobs: row r of the tile, 32-column segments seg = 2*(warp/4) + j
-      const int r = 32 * (warp & 3) + lane;
+    if (row_thread) {
+      const int b0 = kDual ? 0 : (tid >> 7), nb = kDual ? 2 : 1;
 #pragma unroll 1
-      for (int j = 0; j < 2; ++j) {
-        const int seg = 2 * (warp >> 2) + j;
-        const uint8_t* rowp = in + (seg >> 1) * kQBoxBytes + r * 128;
-        float v[32];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int chunk = (seg & 1) * 4 + i;
-          const uint4 w = *reinterpret_cast<const uint4*>(rowp + ((chunk ^ (r & 7)) << 4));
-          v[8 * i + 0] = bf16lo(w.x); v[8 * i + 1] = bf16hi(w.x);
-          v[8 * i + 2] = bf16lo(w.y); v[8 * i + 3] = bf16hi(w.y);
-          v[8 * i + 4] = bf16lo(w.z); v[8 * i + 5] = bf16hi(w.z);
-          v[8 * i + 6] = bf16lo(w.w); v[8 * i + 7] = bf16hi(w.w);
-        }
-        fwht32<HN>(v);
+      for (int b = b0; b < b0 + nb; ++b) {
+        float2 p[32];
+        load_row_job(in, row_r, b, p);
+        fwht_x2<HN>(p);
         if constexpr (AMAX) {
-          amax_r = fmaxf(amax_r, amax_of(v, 32));
+          const float2 m = amax_x2(p, 0, 32);
+          amax_r = max3f(amax_r, m.x, m.y);
         } else {
-          uint8_t* cdst = s_rcode + ob * kQCodeBytes + r * 64 + ((seg ^ ((r >> 1) & 3)) << 4);
-          encode32<FMT>(v, cdst, s_rsc + ob * kQScaleBytes, r, seg, S_r, six_r);
+          const Enc e = encode_x2<FMT>(p, S_r, six_r);
+          *reinterpret_cast<uint4*>(code_chunk(rcode, row_r, 2 * b)) = e.cx;
+          *reinterpret_cast<uint4*>(code_chunk(rcode, row_r, 2 * b + 1)) = e.cy;
+          if constexpr (FMT == kFmtMX)  // blocks 2b, 2b+1 of this row: adjacent bytes
+            *reinterpret_cast<uint16_t*>(rsc + atom_off(row_r, 2 * b)) =
+                static_cast<uint16_t>(e.sx | (e.sy << 8));
+          else  // blocks 4b .. 4b+3: one 4-byte group of atom b
+            *reinterpret_cast<uint32_t*>(rsc + atom_off(row_r, 4 * b)) = e.sx | (e.sy << 16);
         }
       }
     }
-    if constexpr (kCol) {
-      // COL jobs: box b = warp%2 (tile columns 64b..64b+63), rows 32*seg..32*seg+31,
-      // lane -> tile columns c = 64b + 2*lane and c + 1
-      const int b = warp & 1, seg = warp >> 1;
-      const uint8_t* boxp = in + b * kQBoxBytes;
-      float v0[32], v1[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int r = 32 * seg + i;
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(
-            boxp + r * 128 + ((((lane >> 2) ^ (r & 7))) << 4) + ((lane & 3) << 2));
-        v0[i] = bf16lo(w);
-        v1[i] = bf16hi(w);
+    if (kCol && !row_thread) {
+      const int s0 = kDual ? 2 * (ct >> 6) : (ct >> 6), ns = kDual ? 2 : 1;
+      uint32_t scx = 0, scy = 0;  // scale bytes of columns c and c+1, segment s0 first
+#pragma unroll 1
+      for (int s = s0; s < s0 + ns; ++s) {
+        float2 p[32];
+        load_col_job(in, col_b, col_w, s, p);
+        fwht_x2<HN>(p);
+        if constexpr (AMAX) {
+          const float2 m = amax_x2(p, 0, 32);
+          amax_c = max3f(amax_c, m.x, m.y);
+        } else {
+          const Enc e = encode_x2<FMT>(p, S_c, six_c);
+          *reinterpret_cast<uint4*>(code_chunk(ccode, col_c, s)) = e.cx;
+          *reinterpret_cast<uint4*>(code_chunk(ccode, col_c + 1, s)) = e.cy;
+          constexpr int kBytes = FMT == kFmtMX ? 1 : 2;
+          scx |= e.sx << (8 * kBytes * (s - s0));
+          scy |= e.sy << (8 * kBytes * (s - s0));
+        }
       }
-      fwht32<HN>(v0);
-      fwht32<HN>(v1);
-      if constexpr (AMAX) {
-        amax_c = fmaxf(amax_c, fmaxf(amax_of(v0, 32), amax_of(v1, 32)));
-      } else {
-        const int c = 64 * b + 2 * lane;
-        uint8_t* ctile = s_ccode + ob * kQCodeBytes;
-        uint8_t* stile = s_csc + ob * kQScaleBytes;
-        encode32<FMT>(v0, ctile + c * 64 + ((seg ^ ((c >> 1) & 3)) << 4), stile, c, seg, S_c,
-                      six_c);
-        encode32<FMT>(v1, ctile + (c + 1) * 64 + ((seg ^ (((c + 1) >> 1) & 3)) << 4), stile,
-                      c + 1, seg, S_c, six_c);
+      if constexpr (!AMAX) {
+        // kb of segment s0: s0 (MXFP4) or 2*s0 (NVFP4); ns*kBytes consecutive bytes
+        const int kb0 = FMT == kFmtMX ? s0 : 2 * s0;
+        constexpr int kBytes = FMT == kFmtMX ? 1 : 2;
+        if (kDual || kBytes == 2) {
+          if (ns * kBytes == 4) {
+            *reinterpret_cast<uint32_t*>(csc + atom_off(col_c, kb0)) = scx;
+            *reinterpret_cast<uint32_t*>(csc + atom_off(col_c + 1, kb0)) = scy;
+          } else {
+            *reinterpret_cast<uint16_t*>(csc + atom_off(col_c, kb0)) = static_cast<uint16_t>(scx);
+            *reinterpret_cast<uint16_t*>(csc + atom_off(col_c + 1, kb0)) = static_cast<uint16_t>(scy);
+          }
+        } else {
+          csc[atom_off(col_c, kb0)] = static_cast<uint8_t>(scx);
+          csc[atom_off(col_c + 1, kb0)] = static_cast<uint8_t>(scy);
+        }
       }
     }
 
@@ -271,18 +391,18 @@ __global__ void __launch_bounds__(kQThreads, 1)
       if constexpr (!AMAX) {
         constexpr int kAtomsPerTile = (FMT == kFmtMX) ? 1 : 2;
         if constexpr (kRow) {
-          tma_store_2d(&tm_rcodes, s_rcode + ob * kQCodeBytes, tc * 64, tr * 128);
+          tma_store_2d(&tm_rcodes, rcode, tc * 64, tr * 128);
           const int first = tc * kAtomsPerTile;
           const int n = (a.row_kb4 - first) < kAtomsPerTile ? (a.row_kb4 - first) : kAtomsPerTile;
-          bulk_store(a.row_scales + (static_cast<int64_t>(tr) * a.row_kb4 + first) * 512,
-                     s_rsc + ob * kQScaleBytes, static_cast<uint32_t>(n * 512));
+          bulk_store(a.row_scales + (static_cast<int64_t>(tr) * a.row_kb4 + first) * 512, rsc,
+                     static_cast<uint32_t>(n * 512));
         }
         if constexpr (kCol) {
-          tma_store_2d(&tm_ccodes, s_ccode + ob * kQCodeBytes, tr * 64, tc * 128);
+          tma_store_2d(&tm_ccodes, ccode, tr * 64, tc * 128);
           const int first = tr * kAtomsPerTile;
           const int n = (a.col_kb4 - first) < kAtomsPerTile ? (a.col_kb4 - first) : kAtomsPerTile;
-          bulk_store(a.col_scales + (static_cast<int64_t>(tc) * a.col_kb4 + first) * 512,
-                     s_csc + ob * kQScaleBytes, static_cast<uint32_t>(n * 512));
+          bulk_store(a.col_scales + (static_cast<int64_t>(tc) * a.col_kb4 + first) * 512, csc,
+                     static_cast<uint32_t>(n * 512));
         }
         bulk_commit();
       }
