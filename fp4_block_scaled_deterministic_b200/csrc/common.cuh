@@ -61,6 +61,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking check whether the phase of `bar` with the given parity has completed.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Wait for the phase of `bar` with the given parity to complete, for at most
 // limit_ns nanoseconds. On expiry the status word records a timeout and the call
 // returns false; the caller then unwinds instead of hanging the GPU.
@@ -69,6 +81,39 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      atomicOr(&g_status_word, kDevErrTimeout);
+      return false;
+    }
+  }
+}
+
+// Waits on barriers that the peer CTA of a pair completes (remote arrivals, remote
+// transaction bytes). kWaitCluster: try_wait with cluster-scope acquire. kWaitPoll:
+// non-suspending test_wait loop. Both bounded like mbar_wait.
+enum { kWaitCluster = 1, kWaitPoll = 2 };
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+template <int KIND>
+__device__ __forceinline__ bool mbar_wait_remote(uint64_t* bar, uint32_t parity,
+                                                 uint64_t limit_ns) {
+  auto probe = [&]() {
+    if constexpr (KIND == kWaitCluster) return mbar_try_wait_cluster(bar, parity);
+    else return mbar_test_wait(bar, parity);
+  };
+  if (probe()) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (probe()) return true;
     if (globaltimer_ns() - t0 > limit_ns) {
       atomicOr(&g_status_word, kDevErrTimeout);
       return false;
@@ -261,6 +306,12 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
 // Arrive on an mbarrier given by its cluster-shared address (possibly in the peer CTA).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+// Same with CTA-scope release semantics (orders only this thread's prior operations at
+// CTA scope before the arrival).
+__device__ __forceinline__ void mbar_arrive_cluster_cta_release(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
 }
 // TMA load into this CTA's shared memory whose completion is counted on an mbarrier of

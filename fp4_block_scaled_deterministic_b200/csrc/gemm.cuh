@@ -94,49 +94,128 @@ __device__ __forceinline__ constexpr uint32_t idesc_fp4_pair() {
          ((FMT == kFmtMX ? 1u : 0u) << 23) | (static_cast<uint32_t>(256 >> 4) << 24);
 }
 
-// Issue one K slab: copy its scale atoms into TMEM ring slot (t_sfa, t_sfb = t_sfa +
-// 4*atoms) and run the 4 MMAs of K = 64 each. dA/dB/dSFA/dSFB are the slab's shared
-// memory descriptors; stepping inside the slab only adds to their start-address field
-// (+2 per 32 bytes of K, +32 per 512-byte atom), which never carries out of the field.
-template <int FMT, bool PAIR, int SLAB_K = kGBK>
-__device__ __forceinline__ void issue_slab(uint32_t tmem_acc, uint32_t t_sfa, uint64_t dA,
-                                           uint64_t dB, uint64_t dSFA, uint64_t dSFB,
-                                           uint32_t first_slab) {
-  // A slab wider than 256 elements is staged as SLAB_K/256 sub-tiles of 128-byte rows,
-  // each its own 128B-swizzle block of (rows x 128 B); MMA j reads sub-tile j/4.
-  constexpr int kAtoms = SLAB_K / (4 * (FMT == kFmtMX ? 32 : 16));
-  const uint32_t t_sfb = t_sfa + 4 * kAtoms;
-#pragma unroll
-  for (int at = 0; at < kAtoms; ++at) {
-    if constexpr (PAIR) tc_cp_32x128b_warpx4_pair(t_sfa + 4 * at, dSFA + 32 * at);
-    else tc_cp_32x128b_warpx4(t_sfa + 4 * at, dSFA + 32 * at);
-  }
-#pragma unroll
-  for (int rb = 0; rb < 2; ++rb)
-#pragma unroll
-    for (int at = 0; at < kAtoms; ++at) {
-      const uint64_t d = dSFB + rb * (kAtoms * 32) + 32 * at;
-      if constexpr (PAIR) tc_cp_32x128b_warpx4_pair(t_sfb + 8 * at + 4 * rb, d);
-      else tc_cp_32x128b_warpx4(t_sfb + 8 * at + 4 * rb, d);
+// ---------------------------------------------------------------- MMA issuer
+// The issuing thread walks the K slabs of its tiles with a cursor: the slab's pipeline
+// stage and phase, the shared-memory descriptors of its A, B and scale tiles, and the
+// TMEM ring slot of its scale factors. Stepping the descriptors only adds to their
+// start-address field (+2 per 32 bytes of K inside a 128-byte row, +1024 per 16 KB
+// sub-tile, +32 per 512-byte scale atom), which never carries out of the field.
+struct SlabCursor {
+  int stage;
+  uint32_t phase;
+  uint64_t dA, dB, dSA, dSB;
+  uint32_t t_sf, slot;
+};
+
+template <int FMT, bool PAIR, int SLAB_K, int STAGES, int A_BYTES, int B_BYTES, int SFA_BYTES,
+          int SFB_BYTES, int SF_COLS, int SF_BUFS>
+struct Issuer {
+  static constexpr int kAtoms = SLAB_K / (4 * (FMT == kFmtMX ? 32 : 16));
+  static constexpr int kMMAs = SLAB_K / 64;
+  static constexpr int kCopies = 3 * kAtoms;  // A atoms, then B atoms of row blocks 0 and 1
+
+  __device__ __forceinline__ static void step(SlabCursor& c, const SlabCursor& base) {
+    if (++c.stage == STAGES) {
+      c.stage = 0;
+      c.phase ^= 1u;
+      c.dA = base.dA; c.dB = base.dB; c.dSA = base.dSA; c.dSB = base.dSB;
+    } else {
+      c.dA += A_BYTES >> 4; c.dB += B_BYTES >> 4;
+      c.dSA += SFA_BYTES >> 4; c.dSB += SFB_BYTES >> 4;
     }
-  constexpr uint32_t kIdesc = PAIR ? idesc_fp4_pair<FMT>() : idesc_fp4<FMT>();
+    if (++c.slot == SF_BUFS) { c.slot = 0; c.t_sf = base.t_sf; } else { c.t_sf += SF_COLS; }
+  }
+  // Scale-factor copies [lo, hi) of a slab into its TMEM ring slot (t_sfb = t_sfa + 4*atoms).
+  template <int LO, int HI>
+  __device__ __forceinline__ static void copies(const SlabCursor& c) {
 #pragma unroll
-  for (int j = 0; j < SLAB_K / 64; ++j) {
+    for (int i = LO; i < HI; ++i) {
+      uint32_t t;
+      uint64_t d;
+      if (i < kAtoms) {
+        t = c.t_sf + 4 * i;
+        d = c.dSA + 32 * i;
+      } else {
+        const int rb = (i - kAtoms) / kAtoms, at = (i - kAtoms) % kAtoms;
+        t = c.t_sf + 4 * kAtoms + 8 * at + 4 * rb;
+        d = c.dSB + rb * (kAtoms * 32) + 32 * at;
+      }
+      if constexpr (PAIR) tc_cp_32x128b_warpx4_pair(t, d);
+      else tc_cp_32x128b_warpx4(t, d);
+    }
+  }
+  // MMA j of a slab: K elements [64j, 64j+64).
+  __device__ __forceinline__ static void mma(const SlabCursor& c, uint32_t tmem_acc, int j,
+                                             bool first) {
     // MXFP4: two MMAs share one atom column, bytes {0,1} then {2,3} (scale id 0 / 2);
     // NVFP4: one atom column per MMA, all four bytes (scale id 0).
     const int at = FMT == kFmtMX ? (j >> 1) : j;
     const uint32_t id = FMT == kFmtMX ? static_cast<uint32_t>((j & 1) * 2) : 0u;
-    const uint32_t tsfa = (t_sfa + 4 * at) | (id << 30);
-    const uint32_t tsfb = (t_sfb + 8 * at) | (id << 30);
+    const uint32_t tsfa = (c.t_sf + 4 * at) | (id << 30);
+    const uint32_t tsfb = (c.t_sf + 4 * kAtoms + 8 * at) | (id << 30);
+    constexpr uint32_t kIdesc = PAIR ? idesc_fp4_pair<FMT>() : idesc_fp4<FMT>();
     const uint32_t idesc = kIdesc | (id << 29) | (id << 4);
-    const uint32_t acc = (j > 0 || !first_slab) ? 1u : 0u;
-    const uint64_t koff = (j >> 2) * (PAIR ? (128 * 128 >> 4) : 0) + 2 * (j & 3);
+    const uint64_t koff = (j >> 2) * (128 * 128 >> 4) + 2 * (j & 3);
+    const uint32_t acc = first ? 0u : 1u;
     if constexpr (PAIR)
-      tc_mma_fp4_pair<FMT == kFmtMX>(tmem_acc, dA + koff, dB + koff, idesc, tsfa, tsfb, acc);
+      tc_mma_fp4_pair<FMT == kFmtMX>(tmem_acc, c.dA + koff, c.dB + koff, idesc, tsfa, tsfb, acc);
     else
-      tc_mma_fp4<FMT == kFmtMX>(tmem_acc, dA + koff, dB + koff, idesc, tsfa, tsfb, acc);
+      tc_mma_fp4<FMT == kFmtMX>(tmem_acc, c.dA + koff, c.dB + koff, idesc, tsfa, tsfb, acc);
   }
-}
+  template <int J>
+  __device__ __forceinline__ static void slab_mmas(const SlabCursor& c, uint32_t tmem_acc,
+                                                   bool first_slab) {
+    if constexpr (J < kMMAs) {
+      mma(c, tmem_acc, J, first_slab && J == 0);
+      slab_mmas<J + 1>(c, tmem_acc, first_slab);
+    }
+  }
+  __device__ __forceinline__ static void commit(uint64_t* bar) {
+    if constexpr (PAIR) tc_commit_pair_mc(bar, 0x3);
+    else tc_commit(bar);
+  }
+
+  // Runs all tiles of this CTA (or CTA pair): tiles first, first+stride, ... < num_tiles.
+  __device__ static void run(uint32_t tmem, uint8_t* sA, uint8_t* sB, uint8_t* sSFA,
+                             uint8_t* sSFB, uint64_t* full, uint64_t* empty, uint64_t* acc_full,
+                             uint64_t* acc_empty, volatile int* abort_flag, int first,
+                             int stride, const GemmArgs& g) {
+    SlabCursor base;
+    base.stage = 0;
+    base.phase = 0;
+    base.dA = desc_kmajor_sw128(smem_u32(sA));
+    base.dB = desc_kmajor_sw128(smem_u32(sB));
+    base.dSA = desc_sf_atom(smem_u32(sSFA));
+    base.dSB = desc_sf_atom(smem_u32(sSFB));
+    base.t_sf = tmem + 256;
+    base.slot = 0;
+    SlabCursor cur = base;
+    const int my_tiles = first < g.num_tiles ? (g.num_tiles - first + stride - 1) / stride : 0;
+    uint32_t acc_phase = 0;
+    for (int t = 0; t < my_tiles; ++t) {
+      if (!mbar_wait(acc_empty, acc_phase ^ 1u, g.wait_limit_ns) || *abort_flag) {
+        *abort_flag = 1;
+        return;
+      }
+      tc_fence_after();
+      for (int kt = 0; kt < g.k_tiles; ++kt) {
+        // Each slab: wait for its stage, copy its scales into its TMEM ring slot, issue its
+        // MMAs back to back, then release the stage. (Spreading the next slab's copies
+        // between this slab's MMAs was measured to be slower.)
+        if (!mbar_wait(&full[cur.stage], cur.phase, g.wait_limit_ns)) {
+          *abort_flag = 1;
+          return;
+        }
+        copies<0, kCopies>(cur);
+        slab_mmas<0>(cur, tmem, kt == 0);
+        commit(&empty[cur.stage]);
+        step(cur, base);
+      }
+      commit(acc_full);
+      acc_phase ^= 1u;
+    }
+  }
+};
 
 // Scale (NVFP4) and store one thread's row segment of 128 accumulator columns:
 // output row m, columns [n0, n0 + 128), skipping rows >= M and 32-column chunks >= N.
@@ -259,42 +338,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
-      const uint64_t dA0 = desc_kmajor_sw128(smem_u32(sA)), dB0 = desc_kmajor_sw128(smem_u32(sB));
-      const uint64_t dSA0 = desc_sf_atom(smem_u32(sSFA)), dSB0 = desc_sf_atom(smem_u32(sSFB));
-      const uint32_t t_sf0 = tmem + Cfg::kTmemSF;
-      uint64_t dA = dA0, dB = dB0, dSA = dSA0, dSB = dSB0;
-      uint32_t t_sf = t_sf0, sf_slot = 0;
-      int stage = 0;
-      uint32_t phase = 0, acc_phase = 0;
-      for (int tile = blockIdx.x; tile < g.num_tiles && !*abort_flag; tile += gridDim.x) {
-        if (!mbar_wait(acc_empty, acc_phase ^ 1u, g.wait_limit_ns)) {
-          *abort_flag = 1;
-          break;
-        }
-        tc_fence_after();
-        bool ok = true;
-        for (int kt = 0; kt < g.k_tiles; ++kt) {
-          if (!mbar_wait(&full[stage], phase, g.wait_limit_ns)) {
-            *abort_flag = 1;
-            ok = false;
-            break;
-          }
-          issue_slab<FMT, false>(tmem, t_sf, dA, dB, dSA, dSB, kt == 0);
-          tc_commit(&empty[stage]);
-          if (++sf_slot == Cfg::kSFBufs) { sf_slot = 0; t_sf = t_sf0; } else { t_sf += Cfg::kSFCols; }
-          if (++stage == kGStages) {
-            stage = 0;
-            phase ^= 1u;
-            dA = dA0; dB = dB0; dSA = dSA0; dSB = dSB0;
-          } else {
-            dA += kGABytes >> 4; dB += kGBBytes >> 4;
-            dSA += Cfg::kSFABytes >> 4; dSB += Cfg::kSFBBytes >> 4;
-          }
-        }
-        if (!ok) break;
-        tc_commit(acc_full);
-        acc_phase ^= 1u;
-      }
+      Issuer<FMT, false, kGBK, kGStages, kGABytes, kGBBytes, Cfg::kSFABytes, Cfg::kSFBBytes,
+             Cfg::kSFCols, Cfg::kSFBufs>::run(tmem, sA, sB, sSFA, sSFB, full, empty, acc_full,
+                                              acc_empty, abort_flag, blockIdx.x, gridDim.x, g);
     }
   } else {
     // -------------------------------------------------------------- epilogue
@@ -450,42 +496,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
       // ------------------------------------------------------------ MMA issuer (leader)
-      const uint64_t dA0 = desc_kmajor_sw128(smem_u32(sA)), dB0 = desc_kmajor_sw128(smem_u32(sB));
-      const uint64_t dSA0 = desc_sf_atom(smem_u32(sSFA)), dSB0 = desc_sf_atom(smem_u32(sSFB));
-      const uint32_t t_sf0 = tmem + Cfg::kTmemSF;
-      uint64_t dA = dA0, dB = dB0, dSA = dSA0, dSB = dSB0;
-      uint32_t t_sf = t_sf0, sf_slot = 0;
-      int stage = 0;
-      uint32_t phase = 0, acc_phase = 0;
-      for (int tile = pair; tile < g.num_tiles && !*abort_flag; tile += npairs) {
-        if (!mbar_wait(acc_empty, acc_phase ^ 1u, g.wait_limit_ns)) {
-          *abort_flag = 1;
-          break;
-        }
-        tc_fence_after();
-        bool ok = true;
-        for (int kt = 0; kt < g.k_tiles; ++kt) {
-          if (!mbar_wait(&full[stage], phase, g.wait_limit_ns)) {
-            *abort_flag = 1;
-            ok = false;
-            break;
-          }
-          issue_slab<FMT, true, Cfg::kSlabK>(tmem, t_sf, dA, dB, dSA, dSB, kt == 0);
-          tc_commit_pair_mc(&empty[stage], 0x3);
-          if (++sf_slot == Cfg::kSFBufs) { sf_slot = 0; t_sf = t_sf0; } else { t_sf += Cfg::kSFCols; }
-          if (++stage == S) {
-            stage = 0;
-            phase ^= 1u;
-            dA = dA0; dB = dB0; dSA = dSA0; dSB = dSB0;
-          } else {
-            dA += Cfg::kABytes >> 4; dB += Cfg::kBBytes >> 4;
-            dSA += Cfg::kSFABytes >> 4; dSB += Cfg::kSFBBytes >> 4;
-          }
-        }
-        if (!ok) break;
-        tc_commit_pair_mc(acc_full, 0x3);
-        acc_phase ^= 1u;
-      }
+      Issuer<FMT, true, Cfg::kSlabK, S, Cfg::kABytes, Cfg::kBBytes, Cfg::kSFABytes,
+             Cfg::kSFBBytes, Cfg::kSFCols, Cfg::kSFBufs>::run(tmem, sA, sB, sSFA, sSFB, full,
+                                                              empty, acc_full, acc_empty,
+                                                              abort_flag, pair, npairs, g);
     }
   } else {
     // -------------------------------------------------------------- epilogue (both CTAs)
@@ -507,7 +521,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(leader_acc_empty);
+      // CTA-scope release: a cluster-scope release here would first wait for this thread's
+      // earlier global stores (the previous tile's output) and stall the leader's MMAs by
+      // about a microsecond per tile.
+      if (lane == 0) mbar_arrive_cluster_cta_release(leader_acc_empty);
       acc_phase ^= 1u;
       store_row_segment<FMT, OUT_BF16>(r, tm * 256 + 128 * static_cast<int>(rank) + 32 * quarter +
                                               lane,
