@@ -76,8 +76,11 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 // Wait for the phase of `bar` with the given parity to complete, for at most
 // limit_ns nanoseconds. On expiry the status word records a timeout and the call
 // returns false; the caller then unwinds instead of hanging the GPU.
+// The first check is a non-blocking test_wait: a try_wait that succeeds at once still
+// costs the issuing thread ~200 cycles, enough to drain the tensor-core queue when the
+// MMA thread checks a stage that has already landed.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;

@@ -94,6 +94,7 @@ __device__ __forceinline__ constexpr uint32_t idesc_fp4_pair() {
          ((FMT == kFmtMX ? 1u : 0u) << 23) | (static_cast<uint32_t>(256 >> 4) << 24);
 }
 
+
 // ---------------------------------------------------------------- MMA issuer
 // The issuing thread walks the K slabs of its tiles with a cursor: the slab's pipeline
 // stage and phase, the shared-memory descriptors of its A, B and scale tiles, and the

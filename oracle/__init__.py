@@ -74,6 +74,11 @@ def _L():
         lib.fp4o_quantize.restype = ctypes.c_int
         lib.fp4o_quantize.argtypes = [P, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                       P, P, P, P]
+        lib.fp4o_quantize_ex.restype = ctypes.c_int
+        lib.fp4o_quantize_ex.argtypes = [P, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         P, P, P, P, P]
+        lib.fp4o_rotated_amax.restype = ctypes.c_float
+        lib.fp4o_rotated_amax.argtypes = [P, i64, i64, ctypes.c_int, ctypes.c_int]
         lib.fp4o_dequantize.restype = None
         lib.fp4o_dequantize.argtypes = [P, P, ctypes.c_float, i64, i64, ctypes.c_int, P]
         lib.fp4o_gemm_f64.restype = None
@@ -190,9 +195,18 @@ def rotate(x, hn: int, axis: int = ROW) -> np.ndarray:
     return out
 
 
-def quantize(x, fmt: int, hn: int, axis: int = ROW):
+def rotated_amax(x, hn: int, axis: int = ROW) -> float:
+    """max |v| over the rotated matrix (NVFP4 tensor amax), computed row by row."""
+    xb = _bf16_bits(x)
+    rows, cols = xb.shape
+    return float(_L().fp4o_rotated_amax(_ptr(xb), rows, cols, hn, axis))
+
+
+def quantize(x, fmt: int, hn: int, axis: int = ROW, amax: float | None = None):
     """Returns (codes [R][C/2] uint8, scales (layout R7) uint8, S, amax) where
-    (R, C) = x.shape for ROW and x.shape[::-1] for COL. S and amax are None for MXFP4."""
+    (R, C) = x.shape for ROW and x.shape[::-1] for COL. S and amax are None for MXFP4.
+    For NVFP4, `amax` supplies the tensor amax when x is a slice of the tensor (rows of a
+    ROW quantisation or columns of a COL one)."""
     xb = _bf16_bits(x)
     rows, cols = xb.shape
     R, C = (rows, cols) if axis == ROW else (cols, rows)
@@ -201,8 +215,10 @@ def quantize(x, fmt: int, hn: int, axis: int = ROW):
     scales = np.zeros(scale_layout_bytes(R, C // bs), np.uint8)
     s = np.zeros(1, np.float32)
     t = np.zeros(1, np.float32)
-    rc = _L().fp4o_quantize(_ptr(xb), rows, cols, fmt, hn, axis, _ptr(codes), _ptr(scales),
-                            _ptr(s), _ptr(t))
+    a_in = None if amax is None else np.array([amax], np.float32)
+    rc = _L().fp4o_quantize_ex(_ptr(xb), rows, cols, fmt, hn, axis,
+                               None if a_in is None else _ptr(a_in), _ptr(codes), _ptr(scales),
+                               _ptr(s), _ptr(t))
     if rc != 0:
         raise ValueError(f"oracle quantize rejected shape {xb.shape} fmt={fmt} hn={hn} axis={axis}")
     if fmt == NVFP4:

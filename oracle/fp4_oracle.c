@@ -196,6 +196,23 @@ int fp4o_rotate(const uint16_t *x, int64_t rows, int64_t cols, int hn, int axis,
     return 0;
 }
 
+/* max |v| over the rotated matrix (the NVFP4 tensor amax of step 3), one row of the
+ * rotated matrix at a time. */
+float fp4o_rotated_amax(const uint16_t *x, int64_t rows, int64_t cols, int hn, int axis) {
+    int64_t R = axis == FP4O_ROW ? rows : cols, C = axis == FP4O_ROW ? cols : rows;
+    float *v = (float *)malloc(sizeof(float) * (size_t)(C > 0 ? C : 1));
+    float T = 0.0f;
+    for (int64_t r = 0; r < R; r++) {
+        for (int64_t c = 0; c < C; c++)
+            v[c] = fp4o_bf16_to_f32(axis == FP4O_ROW ? x[r * cols + c] : x[c * cols + r]);
+        if (hn != 0)
+            for (int64_t g = 0; g < C; g += hn) fp4o_fwht_f32(v + g, hn);
+        for (int64_t c = 0; c < C; c++) T = fmaxf(T, fabsf(v[c]));
+    }
+    free(v);
+    return T;
+}
+
 /* ---------------------------------------------------------------- scale layout (R7) */
 
 int64_t fp4o_scale_layout_bytes(int64_t rows, int64_t kblocks) {
@@ -248,8 +265,22 @@ void fp4o_quantize_block_nv(const float *v, int bs, float S, uint8_t *codes, uin
  *   scales: fp4o_scale_layout_bytes(R, C/bs) bytes, written in layout R7
  *   nv_scale_out / nv_amax_out: NVFP4 only (may be NULL otherwise)
  * Returns 0, or -1 on a shape the format cannot block. */
+int fp4o_quantize_ex(const uint16_t *x, int64_t rows, int64_t cols, int fmt, int hn, int axis,
+                     const float *amax_in, uint8_t *codes, uint8_t *scales, float *nv_scale_out,
+                     float *nv_amax_out);
+
 int fp4o_quantize(const uint16_t *x, int64_t rows, int64_t cols, int fmt, int hn, int axis,
                   uint8_t *codes, uint8_t *scales, float *nv_scale_out, float *nv_amax_out) {
+    return fp4o_quantize_ex(x, rows, cols, fmt, hn, axis, NULL, codes, scales, nv_scale_out,
+                            nv_amax_out);
+}
+
+/* As fp4o_quantize; for NVFP4 a non-NULL amax_in supplies the tensor amax T of step 3
+ * (the amax of the whole rotated tensor, when x is a slice of it: rows of a ROW
+ * quantisation or columns of a COL one are quantised independently given T). */
+int fp4o_quantize_ex(const uint16_t *x, int64_t rows, int64_t cols, int fmt, int hn, int axis,
+                     const float *amax_in, uint8_t *codes, uint8_t *scales, float *nv_scale_out,
+                     float *nv_amax_out) {
     int bs = fmt == FP4O_MXFP4 ? 32 : 16;
     int64_t R = axis == FP4O_ROW ? rows : cols, C = axis == FP4O_ROW ? cols : rows;
     if (C % bs != 0 || (hn != 0 && C % hn != 0) || C % 2 != 0) return -1;
@@ -262,7 +293,9 @@ int fp4o_quantize(const uint16_t *x, int64_t rows, int64_t cols, int fmt, int hn
     float S = 1.0f;
     if (fmt == FP4O_NVFP4) {
         float T = 0.0f;
-        for (int64_t i = 0; i < R * C; i++) T = fmaxf(T, fabsf(v[i]));
+        if (amax_in) T = *amax_in;
+        else
+            for (int64_t i = 0; i < R * C; i++) T = fmaxf(T, fabsf(v[i]));
         S = fp4o_nv_tensor_scale(T);
         if (nv_scale_out) *nv_scale_out = S;
         if (nv_amax_out) *nv_amax_out = T;
