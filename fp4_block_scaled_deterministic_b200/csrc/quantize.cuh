@@ -66,7 +66,7 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a
 
 // Normalised block FWHT of both lanes: groups of HN along the 32 elements, butterfly
 // strides 1, 2, 4, ... in that order, then x RN(1/sqrt(HN)).
-template <int HN>
+template <int HN, bool kScale = true>
 __device__ __forceinline__ void fwht_x2(float2 (&p)[32]) {
   if constexpr (HN > 0) {
 #pragma unroll
@@ -81,10 +81,12 @@ __device__ __forceinline__ void fwht_x2(float2 (&p)[32]) {
       }
     }
     // 0.25 = 1/sqrt(16) exactly; 0x3E3504F3 = fp32 nearest to 1/sqrt(32)
-    const float c = (HN == 16) ? 0.25f : __uint_as_float(0x3E3504F3u);
-    const float2 c2 = make_float2(c, c);
+    if constexpr (kScale) {
+      const float c = (HN == 16) ? 0.25f : __uint_as_float(0x3E3504F3u);
+      const float2 c2 = make_float2(c, c);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) p[i] = mul2(p[i], c2);
+      for (int i = 0; i < 32; ++i) p[i] = mul2(p[i], c2);
+    }
   }
 }
 
@@ -139,6 +141,33 @@ __device__ __forceinline__ Enc mx_encode_x2(float2 (&p)[32]) {
   e.sx = bx;
   e.sy = by;
   return e;
+}
+
+// MXFP4 after an H16 butterfly whose final x0.25 has NOT been applied: the exact x0.25 is
+// folded into the power-of-two scale, q = v * 2^(-e-2), with e taken from amax*0.25
+// (byte = biased exponent of amax - 4). This equals the two-step RN(RN(v*0.25) * 2^-e)
+// whenever the block amax is >= 2^-100: v*0.25 is then exact unless |v| < 2^-124, and
+// such an element lands below 2^-20 either way (code 0, sign kept). Smaller blocks
+// take the two-step path.
+__device__ __forceinline__ Enc mx_encode_x2_h16fold(float2 (&p)[32]) {
+  const float2 am = amax_x2(p, 0, 32);
+  if (am.x >= 0x1p-100f && am.y >= 0x1p-100f) {
+    const uint32_t bx = ((__float_as_uint(am.x) >> 23) & 0xFFu) - 4u;
+    const uint32_t by = ((__float_as_uint(am.y) >> 23) & 0xFFu) - 4u;
+    const float2 inv = make_float2(__uint_as_float((252u - bx) << 23), __uint_as_float((252u - by) << 23));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) p[i] = mul2(p[i], inv);
+    Enc e;
+    e.cx = make_uint4(cvt8x(p, 0), cvt8x(p, 8), cvt8x(p, 16), cvt8x(p, 24));
+    e.cy = make_uint4(cvt8y(p, 0), cvt8y(p, 8), cvt8y(p, 16), cvt8y(p, 24));
+    e.sx = bx;
+    e.sy = by;
+    return e;
+  }
+  const float2 q = make_float2(0.25f, 0.25f);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) p[i] = mul2(p[i], q);
+  return mx_encode_x2(p);
 }
 
 // True when q lies within 4 units in the last place of a number with at most two
@@ -248,6 +277,8 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
   constexpr bool kRow = (MODE & kModeRow) != 0;
   constexpr bool kCol = (MODE & kModeCol) != 0;
   constexpr bool kDual = kRow && kCol;
+  // MXFP4 + H16 quantise pass: the rotation's x0.25 is folded into the block scale
+  constexpr bool kFoldH16 = FMT == kFmtMX && HN == 16 && !AMAX;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -330,12 +361,12 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
       for (int b = b0; b < b0 + nb; ++b) {
         float2 p[32];
         load_row_job(in, row_r, b, p);
-        fwht_x2<HN>(p);
+        fwht_x2<HN, !kFoldH16>(p);
         if constexpr (AMAX) {
           const float2 m = amax_x2(p, 0, 32);
           amax_r = max3f(amax_r, m.x, m.y);
         } else {
-          const Enc e = encode_x2<FMT>(p, S_r, six_r);
+          const Enc e = kFoldH16 ? mx_encode_x2_h16fold(p) : encode_x2<FMT>(p, S_r, six_r);
           *reinterpret_cast<uint4*>(code_chunk(rcode, row_r, 2 * b)) = e.cx;
           *reinterpret_cast<uint4*>(code_chunk(rcode, row_r, 2 * b + 1)) = e.cy;
           if constexpr (FMT == kFmtMX)  // blocks 2b, 2b+1 of this row: adjacent bytes
@@ -353,12 +384,12 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
       for (int s = s0; s < s0 + ns; ++s) {
         float2 p[32];
         load_col_job(in, col_b, col_w, s, p);
-        fwht_x2<HN>(p);
+        fwht_x2<HN, !kFoldH16>(p);
         if constexpr (AMAX) {
           const float2 m = amax_x2(p, 0, 32);
           amax_c = max3f(amax_c, m.x, m.y);
         } else {
-          const Enc e = encode_x2<FMT>(p, S_c, six_c);
+          const Enc e = kFoldH16 ? mx_encode_x2_h16fold(p) : encode_x2<FMT>(p, S_c, six_c);
           *reinterpret_cast<uint4*>(code_chunk(ccode, col_c, s)) = e.cx;
           *reinterpret_cast<uint4*>(code_chunk(ccode, col_c + 1, s)) = e.cy;
           constexpr int kBytes = FMT == kFmtMX ? 1 : 2;
