@@ -394,7 +394,7 @@ def main():
     peak_fp4 = pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) * FP4_OVER_BF16
     avg_launch_ms = sum(gemm_ms) / len(gemm_ms)
     avg_flops = sum(per_launch_flops) / len(per_launch_flops)
-    traffic = recorded_traffic("gemm_fp4_kernel<mx,*>" if fmt == 0 else "gemm_fp4_kernel<nv,*>")
+    traffic = recorded_traffic("mxfp4" if fmt == 0 else "nvfp4") if a.hadamard == 16 and len(names) == 5 else None
     roof = {"bound": "tensor", "achieved": gemm_tflops, "peak": peak_fp4, "unit": "TFLOP/s",
             "frac": gemm_tflops / peak_fp4, "traffic": traffic,
             "kernel": "gemm_fp4_kernel (tcgen05 block-scaled FP4)",

@@ -282,6 +282,28 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a, const CUtensorMap& b, const C
   return cudaGetLastError();
 }
 
+// Tile order for L2 reuse (see tile_coords). A band of tile rows keeps its A panels in
+// L2 while B is streamed once per band, and the reverse for a band of tile columns. The
+// band is as wide as a panel budget allows (a third of B200's 126 MB L2, which also
+// carries the output stream), and the orientation with fewer estimated HBM operand bytes
+// is taken.
+constexpr double kL2PanelBudget = 40.0 * (1 << 20);
+
+void choose_tile_order(GemmArgs& g, int64_t tile_rows, int64_t K, int block) {
+  const double row_bytes = double(K / 2 + K / block);
+  const double panel_a = double(tile_rows) * row_bytes, panel_b = double(kGBN) * row_bytes;
+  auto fit = [](double panel, int tiles) {
+    const double n = kL2PanelBudget / panel;
+    return n < 1.0 ? 1 : (n >= tiles ? tiles : static_cast<int>(n));
+  };
+  const int ga = fit(panel_a, g.tiles_m), gb = fit(panel_b, g.tiles_n);
+  const double a_all = panel_a * g.tiles_m, b_all = panel_b * g.tiles_n;
+  const double by_rows = a_all + b_all * double(ceil_div(g.tiles_m, ga));
+  const double by_cols = b_all + a_all * double(ceil_div(g.tiles_n, gb));
+  g.band_n = by_cols < by_rows ? 1 : 0;
+  g.band = g.band_n ? gb : ga;
+}
+
 fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void* B,
                      const void* Bs, const float* Bts, void* C, int64_t M, int64_t N, int64_t K,
                      fp4_format fmt, fp4_out_dtype od, cudaStream_t stream) {
@@ -334,6 +356,7 @@ fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void
   if (tiles > INT32_MAX) return FP4_ERR_SHAPE;
   g.num_tiles = static_cast<int>(tiles);
   g.k_tiles = static_cast<int>(ceil_div(K, slab_k));
+  choose_tile_order(g, pair ? 256 : kGBM, K, block_of(fmt));
   g.C = C;
   g.sa = Ats;
   g.sb = Bts;

@@ -53,11 +53,28 @@ struct GemmCfg {
 struct GemmArgs {
   int M, N, K;
   int tiles_m, tiles_n, num_tiles, k_tiles;
+  int band, band_n;  // tile order: see tile_coords
   void* C;
   const float* sa;  // NVFP4 tensor scales (device), or null
   const float* sb;
   uint64_t wait_limit_ns;
 };
+
+// Output tile order. Tiles are numbered in bands of g.band tile rows (g.band_n == 0) or
+// tile columns (g.band_n == 1), the banded index running fastest inside a band. The
+// operand panels of the banded dimension are then reused by every tile of the band while
+// they sit in L2, and the other operand's panels are streamed once per band; the host
+// picks the orientation and width from the operand sizes.
+__device__ __forceinline__ void tile_coords(int tile, const GemmArgs& g, int& tm, int& tn) {
+  const int banded = g.band_n ? g.tiles_n : g.tiles_m;
+  const int other = g.band_n ? g.tiles_m : g.tiles_n;
+  const int first = tile / (g.band * other) * g.band;
+  const int width = min(g.band, banded - first);
+  const int r = tile - first * other;
+  const int a = first + r % width, b = r / width;
+  tm = g.band_n ? b : a;
+  tn = g.band_n ? a : b;
+}
 
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of 128 bytes,
 // 8-row groups 1024 bytes apart (SBO), sm_100 descriptor version 1.
@@ -319,7 +336,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       for (int tile = blockIdx.x; tile < g.num_tiles && !*abort_flag; tile += gridDim.x) {
-        const int tm = tile % g.tiles_m, tn = tile / g.tiles_m;
+        int tm, tn;
+        tile_coords(tile, g, tm, tn);
         for (int kt = 0; kt < g.k_tiles; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, g.wait_limit_ns)) {
             *abort_flag = 1;
@@ -352,7 +370,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
     if constexpr (FMT == kFmtNV) alpha = __fmul_rn(*g.sa, *g.sb);
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < g.num_tiles && !*abort_flag; tile += gridDim.x) {
-      const int tm = tile % g.tiles_m, tn = tile / g.tiles_m;
+      int tm, tn;
+      tile_coords(tile, g, tm, tn);
       if (!mbar_wait(acc_full, acc_phase, g.wait_limit_ns)) {
         *abort_flag = 1;
         break;
@@ -470,7 +489,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       for (int tile = pair; tile < g.num_tiles && !*abort_flag; tile += npairs) {
-        const int tm = tile % g.tiles_m, tn = tile / g.tiles_m;
+        int tm, tn;
+        tile_coords(tile, g, tm, tn);
         for (int kt = 0; kt < g.k_tiles; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, g.wait_limit_ns)) {
             *abort_flag = 1;
@@ -511,7 +531,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
     if constexpr (FMT == kFmtNV) alpha = __fmul_rn(*g.sa, *g.sb);
     uint32_t acc_phase = 0;
     for (int tile = pair; tile < g.num_tiles && !*abort_flag; tile += npairs) {
-      const int tm = tile % g.tiles_m, tn = tile / g.tiles_m;
+      int tm, tn;
+      tile_coords(tile, g, tm, tn);
       if (!mbar_wait(acc_full, acc_phase, g.wait_limit_ns)) {
         *abort_flag = 1;
         break;
