@@ -358,6 +358,7 @@ fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void
   g.k_tiles = static_cast<int>(ceil_div(K, slab_k));
   choose_tile_order(g, pair ? 256 : kGBM, K, block_of(fmt));
   g.C = C;
+  g.c_v8 = (reinterpret_cast<uintptr_t>(C) & 31) == 0 ? 1 : 0;
   g.sa = Ats;
   g.sb = Bts;
   g.wait_limit_ns = kDefaultWaitLimitNs;

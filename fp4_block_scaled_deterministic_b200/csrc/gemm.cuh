@@ -54,6 +54,7 @@ struct GemmArgs {
   int M, N, K;
   int tiles_m, tiles_n, num_tiles, k_tiles;
   int band, band_n;  // tile order: see tile_coords
+  int c_v8;          // output 32-byte aligned: 32-byte stores
   void* C;
   const float* sa;  // NVFP4 tensor scales (device), or null
   const float* sb;
@@ -235,29 +236,49 @@ struct Issuer {
   }
 };
 
+// 32-byte global store (one full L2 sector per thread); the address must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]),
+               "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
 // Scale (NVFP4) and store one thread's row segment of 128 accumulator columns:
 // output row m, columns [n0, n0 + 128), skipping rows >= M and 32-column chunks >= N.
+// Each store writes 32 bytes when the output is 32-byte aligned (g.c_v8; rows then are
+// too, N being a multiple of 32), else 16 bytes.
 template <int FMT, int OUT_BF16>
 __device__ __forceinline__ void store_row_segment(const uint32_t (&r)[128], int m, int n0,
                                                   const GemmArgs& g, float alpha) {
   if (m >= g.M) return;
+  auto val = [&](int i) {
+    const float x = __uint_as_float(r[i]);
+    return FMT == kFmtNV ? __fmul_rn(x, alpha) : x;
+  };
   if constexpr (OUT_BF16) {
     __nv_bfloat16* crow = static_cast<__nv_bfloat16*>(g.C) + static_cast<int64_t>(m) * g.N + n0;
+    auto pack = [&](int i) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(val(i), val(i + 1));
+      return *reinterpret_cast<const uint32_t*>(&h);
+    };
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       if (n0 + 32 * c < g.N) {
+        if (g.c_v8) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          uint32_t w[4];
+          for (int i = 0; i < 2; ++i) {
+            uint32_t w[8];
 #pragma unroll
-          for (int p = 0; p < 4; ++p) {
-            float x0 = __uint_as_float(r[32 * c + 8 * i + 2 * p]);
-            float x1 = __uint_as_float(r[32 * c + 8 * i + 2 * p + 1]);
-            if constexpr (FMT == kFmtNV) { x0 = __fmul_rn(x0, alpha); x1 = __fmul_rn(x1, alpha); }
-            const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
-            w[p] = *reinterpret_cast<const uint32_t*>(&h);
+            for (int p = 0; p < 8; ++p) w[p] = pack(32 * c + 16 * i + 2 * p);
+            st_global_v8(crow + 32 * c + 16 * i, w);
           }
-          *reinterpret_cast<uint4*>(crow + 32 * c + 8 * i) = make_uint4(w[0], w[1], w[2], w[3]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int b = 32 * c + 8 * i;
+            *reinterpret_cast<uint4*>(crow + b) =
+                make_uint4(pack(b), pack(b + 2), pack(b + 4), pack(b + 6));
+          }
         }
       }
     }
@@ -266,18 +287,20 @@ __device__ __forceinline__ void store_row_segment(const uint32_t (&r)[128], int 
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       if (n0 + 32 * c < g.N) {
+        if (g.c_v8) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float4 o;
-          o.x = __uint_as_float(r[32 * c + 4 * i + 0]);
-          o.y = __uint_as_float(r[32 * c + 4 * i + 1]);
-          o.z = __uint_as_float(r[32 * c + 4 * i + 2]);
-          o.w = __uint_as_float(r[32 * c + 4 * i + 3]);
-          if constexpr (FMT == kFmtNV) {
-            o.x = __fmul_rn(o.x, alpha); o.y = __fmul_rn(o.y, alpha);
-            o.z = __fmul_rn(o.z, alpha); o.w = __fmul_rn(o.w, alpha);
+          for (int i = 0; i < 4; ++i) {
+            uint32_t w[8];
+#pragma unroll
+            for (int p = 0; p < 8; ++p) w[p] = __float_as_uint(val(32 * c + 8 * i + p));
+            st_global_v8(crow + 32 * c + 8 * i, w);
           }
-          *reinterpret_cast<float4*>(crow + 32 * c + 4 * i) = o;
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int b = 32 * c + 4 * i;
+            *reinterpret_cast<float4*>(crow + b) = make_float4(val(b), val(b + 1), val(b + 2), val(b + 3));
+          }
         }
       }
     }

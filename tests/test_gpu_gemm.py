@@ -117,3 +117,22 @@ def test_gemm_full_llama_gate_sampled(orc, fmt):
     got = C[torch.from_numpy(ms).cuda(), torch.from_numpy(ns).cuda()].cpu().numpy()
     assert rel_fro(got, ref) <= TOL
     assert torch.equal(Cb.view(torch.int16), C.to(torch.bfloat16).view(torch.int16))
+
+
+@pytest.mark.parametrize("shape", [(160, 96, 224), (384, 512, 1024), (96, 320, 256)])
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_gemm_16byte_aligned_output(orc, fmt, shape):
+    """An output that is 16- but not 32-byte aligned takes the 16-byte store path and
+    holds the same bits as the 32-byte-aligned one."""
+    M, N, K = shape
+    qa, qb, _, _ = _operands(orc, M, N, K, fmt, 16, seed=7 * M + N)
+    for od, dt, off in ((fp4.OUT_F32, torch.float32, 4), (fp4.OUT_BF16, torch.bfloat16, 8)):
+        ref = fp4.gemm(qa, qb, od)
+        buf = torch.full((M * N + off,), float("nan"), dtype=dt, device="cuda")
+        out = buf[off:].view(M, N)
+        assert out.data_ptr() % 32 == 16
+        fp4.gemm(qa, qb, od, out=out)
+        torch.cuda.synchronize()
+        assert fp4.fp4_check_status() == 0
+        assert torch.equal(out.view(torch.int16 if od == fp4.OUT_BF16 else torch.int32),
+                           ref.view(torch.int16 if od == fp4.OUT_BF16 else torch.int32))
