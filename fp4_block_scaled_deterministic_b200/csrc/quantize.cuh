@@ -19,7 +19,7 @@
 //   COL job = two adjacent columns, 32 consecutive rows (32 conflict-free 4-B reads);
 // the rotation runs in registers with packed fp32x2 arithmetic, codes are staged in a
 // 64B-swizzled [128][64 B] tile and written by a TMA store, scale atoms are assembled
-// in shared memory (2- and 4-byte stores) and written by bulk copies. Staging is
+// in shared memory (1-, 2- and 4-byte stores) and written by bulk copies. Staging is
 // double-buffered so stores overlap the next tile.
 #pragma once
 
@@ -276,7 +276,6 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
                     const __grid_constant__ CUtensorMap tm_ccodes, const QuantArgs a) {
   constexpr bool kRow = (MODE & kModeRow) != 0;
   constexpr bool kCol = (MODE & kModeCol) != 0;
-  constexpr bool kDual = kRow && kCol;
   // MXFP4 + H16 quantise pass: the rotation's x0.25 is folded into the block scale
   constexpr bool kFoldH16 = FMT == kFmtMX && HN == 16 && !AMAX;
   extern __shared__ uint8_t smem_raw[];
@@ -332,14 +331,12 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
   }
 
   // Work split of one 128x128 tile over the 256 threads:
-  //   ROW only : thread -> row tid%128, box tid/128                 (1 ROW job)
-  //   COL only : thread -> column pair tid%64, segment tid/64        (1 COL job)
-  //   DUAL     : threads 0-127 -> row tid, boxes 0 and 1              (2 ROW jobs)
-  //              threads 128-255 -> pair t%64, segments 2(t/64)+{0,1} (2 COL jobs)
-  const bool row_thread = kRow && (!kDual || tid < 128);
-  const int ct = kDual ? tid - 128 : tid;
+  //   ROW job : row tid%128, box tid/128
+  //   COL job : column pair tid%64, segment tid/64
+  // A thread takes its ROW job (ROW, DUAL) and its COL job (COL, DUAL), so in the dual
+  // pass every warp carries the same instruction mix and reaches the barriers together.
   const int row_r = tid & 127;
-  const int col_pair = ct & 63, col_b = col_pair >> 5, col_w = col_pair & 31;
+  const int col_pair = tid & 63, col_b = col_pair >> 5, col_w = col_pair & 31;
   const int col_c = 64 * col_b + 2 * col_w;
 
   float amax_r = 0.0f, amax_c = 0.0f;
@@ -355,10 +352,9 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
     uint8_t* rsc = s_rsc + ob * kQScaleBytes;
     uint8_t* csc = s_csc + ob * kQScaleBytes;
 
-    if (row_thread) {
-      const int b0 = kDual ? 0 : (tid >> 7), nb = kDual ? 2 : 1;
-#pragma unroll 1
-      for (int b = b0; b < b0 + nb; ++b) {
+    if constexpr (kRow) {
+      const int b = tid >> 7;
+      {
         float2 p[32];
         load_row_job(in, row_r, b, p);
         fwht_x2<HN, !kFoldH16>(p);
@@ -377,11 +373,9 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
         }
       }
     }
-    if (kCol && !row_thread) {
-      const int s0 = kDual ? 2 * (ct >> 6) : (ct >> 6), ns = kDual ? 2 : 1;
-      uint32_t scx = 0, scy = 0;  // scale bytes of columns c and c+1, segment s0 first
-#pragma unroll 1
-      for (int s = s0; s < s0 + ns; ++s) {
+    if constexpr (kCol) {
+      const int s = tid >> 6;
+      {
         float2 p[32];
         load_col_job(in, col_b, col_w, s, p);
         fwht_x2<HN, !kFoldH16>(p);
@@ -392,26 +386,14 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
           const Enc e = kFoldH16 ? mx_encode_x2_h16fold(p) : encode_x2<FMT>(p, S_c, six_c);
           *reinterpret_cast<uint4*>(code_chunk(ccode, col_c, s)) = e.cx;
           *reinterpret_cast<uint4*>(code_chunk(ccode, col_c + 1, s)) = e.cy;
-          constexpr int kBytes = FMT == kFmtMX ? 1 : 2;
-          scx |= e.sx << (8 * kBytes * (s - s0));
-          scy |= e.sy << (8 * kBytes * (s - s0));
-        }
-      }
-      if constexpr (!AMAX) {
-        // kb of segment s0: s0 (MXFP4) or 2*s0 (NVFP4); ns*kBytes consecutive bytes
-        const int kb0 = FMT == kFmtMX ? s0 : 2 * s0;
-        constexpr int kBytes = FMT == kFmtMX ? 1 : 2;
-        if (kDual || kBytes == 2) {
-          if (ns * kBytes == 4) {
-            *reinterpret_cast<uint32_t*>(csc + atom_off(col_c, kb0)) = scx;
-            *reinterpret_cast<uint32_t*>(csc + atom_off(col_c + 1, kb0)) = scy;
+          // block kb of segment s: s (MXFP4, one byte) or 2s, 2s+1 (NVFP4, two bytes)
+          if constexpr (FMT == kFmtMX) {
+            csc[atom_off(col_c, s)] = static_cast<uint8_t>(e.sx);
+            csc[atom_off(col_c + 1, s)] = static_cast<uint8_t>(e.sy);
           } else {
-            *reinterpret_cast<uint16_t*>(csc + atom_off(col_c, kb0)) = static_cast<uint16_t>(scx);
-            *reinterpret_cast<uint16_t*>(csc + atom_off(col_c + 1, kb0)) = static_cast<uint16_t>(scy);
+            *reinterpret_cast<uint16_t*>(csc + atom_off(col_c, 2 * s)) = static_cast<uint16_t>(e.sx);
+            *reinterpret_cast<uint16_t*>(csc + atom_off(col_c + 1, 2 * s)) = static_cast<uint16_t>(e.sy);
           }
-        } else {
-          csc[atom_off(col_c, kb0)] = static_cast<uint8_t>(scx);
-          csc[atom_off(col_c + 1, kb0)] = static_cast<uint8_t>(scy);
         }
       }
     }
