@@ -397,7 +397,7 @@ def main():
     traffic = recorded_traffic("mxfp4" if fmt == 0 else "nvfp4") if a.hadamard == 16 and len(names) == 5 else None
     roof = {"bound": "tensor", "achieved": gemm_tflops, "peak": peak_fp4, "unit": "TFLOP/s",
             "frac": gemm_tflops / peak_fp4, "traffic": traffic,
-            "kernel": "gemm_fp4_kernel (tcgen05 block-scaled FP4)",
+            "kernel": "gemm_fp4_pair_kernel (tcgen05 block-scaled FP4, CTA pairs)",
             "per_launch": {"avg_flops": avg_flops, "avg_ms": avg_launch_ms,
                            "launches": len(gemm_ms)},
             "peak_source": f"{pk_kind}: bf16_tflops_sustained x {FP4_OVER_BF16} (nominal FP4:BF16)"}

@@ -420,9 +420,11 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
         bulk_commit();
       }
       if (it + kQStages < my_tiles) issue_load(st, tile + kQStages * nctas);
+      // The next tile writes staging buffer ob^1, last read by the stores of the previous
+      // tile: wait for those reads here. Thread 0 joins the next tile's first barrier
+      // only after this, so no barrier of its own is needed.
       if constexpr (!AMAX) bulk_wait_read<1>();
     }
-    __syncthreads();
   }
   if constexpr (!AMAX) {
     if (tid == 0) bulk_wait<0>();
