@@ -79,6 +79,24 @@ def _L():
                                          P, P, P, P, P]
         lib.fp4o_rotated_amax.restype = ctypes.c_float
         lib.fp4o_rotated_amax.argtypes = [P, i64, i64, ctypes.c_int, ctypes.c_int]
+        u64, u32 = ctypes.c_uint64, ctypes.c_uint32
+        lib.fp4o_rotated_amax_opt.restype = ctypes.c_float
+        lib.fp4o_rotated_amax_opt.argtypes = [P, i64, i64, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_int, u64]
+        lib.fp4o_rotate_opt.restype = ctypes.c_int
+        lib.fp4o_rotate_opt.argtypes = [P, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                        u64, P]
+        lib.fp4o_quantize_opt.restype = ctypes.c_int
+        lib.fp4o_quantize_opt.argtypes = [P, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          P, ctypes.c_int, u64, ctypes.c_int, u64, P, P, P, P]
+        lib.fp4o_philox4x32_10.restype = None
+        lib.fp4o_philox4x32_10.argtypes = [P, P, P]
+        lib.fp4o_philox_word.restype = u32
+        lib.fp4o_philox_word.argtypes = [u64, u64, u32]
+        lib.fp4o_e2m1_encode_sr.restype = ctypes.c_uint8
+        lib.fp4o_e2m1_encode_sr.argtypes = [ctypes.c_float, u32]
+        lib.fp4o_rht_negate.restype = ctypes.c_int
+        lib.fp4o_rht_negate.argtypes = [u64, i64]
         lib.fp4o_dequantize.restype = None
         lib.fp4o_dequantize.argtypes = [P, P, ctypes.c_float, i64, i64, ctypes.c_int, P]
         lib.fp4o_gemm_f64.restype = None
@@ -185,28 +203,58 @@ def _bf16_bits(x) -> np.ndarray:
     return np.ascontiguousarray(x.contiguous().view(torch.int16).numpy().view(np.uint16))
 
 
-def rotate(x, hn: int, axis: int = ROW) -> np.ndarray:
+def rotate(x, hn: int, axis: int = ROW, rht_seed: int | None = None) -> np.ndarray:
+    """Widened and rotated matrix ([R][C], transposed for COL); with rht_seed the random
+    signs of the randomised Hadamard variant are applied before the rotation."""
     xb = _bf16_bits(x)
     rows, cols = xb.shape
     R, C = (rows, cols) if axis == ROW else (cols, rows)
     out = np.empty((R, C), np.float32)
-    if _L().fp4o_rotate(_ptr(xb), rows, cols, hn, axis, _ptr(out)) != 0:
+    if _L().fp4o_rotate_opt(_ptr(xb), rows, cols, hn, axis, rht_seed is not None,
+                            rht_seed or 0, _ptr(out)) != 0:
         raise ValueError("rotation group does not divide the axis")
     return out
 
 
-def rotated_amax(x, hn: int, axis: int = ROW) -> float:
+def rotated_amax(x, hn: int, axis: int = ROW, rht_seed: int | None = None) -> float:
     """max |v| over the rotated matrix (NVFP4 tensor amax), computed row by row."""
     xb = _bf16_bits(x)
     rows, cols = xb.shape
-    return float(_L().fp4o_rotated_amax(_ptr(xb), rows, cols, hn, axis))
+    return float(_L().fp4o_rotated_amax_opt(_ptr(xb), rows, cols, hn, axis,
+                                            rht_seed is not None, rht_seed or 0))
 
 
-def quantize(x, fmt: int, hn: int, axis: int = ROW, amax: float | None = None):
+# ----------------------------------------------------------------- random words
+
+def philox4x32_10(ctr, key) -> np.ndarray:
+    """The four output words of Philox4x32-10 for a 4-word counter and 2-word key."""
+    c = np.ascontiguousarray(ctr, dtype=np.uint32)
+    k = np.ascontiguousarray(key, dtype=np.uint32)
+    out = np.empty(4, np.uint32)
+    _L().fp4o_philox4x32_10(_ptr(c), _ptr(k), _ptr(out))
+    return out
+
+
+def philox_word(seed: int, index: int, stream: int) -> int:
+    return int(_L().fp4o_philox_word(seed, index, stream))
+
+
+def e2m1_encode_sr(q: float, w: int) -> int:
+    return int(_L().fp4o_e2m1_encode_sr(q, w))
+
+
+def rht_negate(seed: int, j: int) -> bool:
+    return bool(_L().fp4o_rht_negate(seed, j))
+
+
+def quantize(x, fmt: int, hn: int, axis: int = ROW, amax: float | None = None,
+             sr_seed: int | None = None, rht_seed: int | None = None):
     """Returns (codes [R][C/2] uint8, scales (layout R7) uint8, S, amax) where
     (R, C) = x.shape for ROW and x.shape[::-1] for COL. S and amax are None for MXFP4.
     For NVFP4, `amax` supplies the tensor amax when x is a slice of the tensor (rows of a
-    ROW quantisation or columns of a COL one)."""
+    ROW quantisation or columns of a COL one), or when the caller fixes it.
+    sr_seed: stochastic rounding of the codes; rht_seed: randomised Hadamard signs
+    (both keyed by the given seed; None = off)."""
     xb = _bf16_bits(x)
     rows, cols = xb.shape
     R, C = (rows, cols) if axis == ROW else (cols, rows)
@@ -216,9 +264,10 @@ def quantize(x, fmt: int, hn: int, axis: int = ROW, amax: float | None = None):
     s = np.zeros(1, np.float32)
     t = np.zeros(1, np.float32)
     a_in = None if amax is None else np.array([amax], np.float32)
-    rc = _L().fp4o_quantize_ex(_ptr(xb), rows, cols, fmt, hn, axis,
-                               None if a_in is None else _ptr(a_in), _ptr(codes), _ptr(scales),
-                               _ptr(s), _ptr(t))
+    rc = _L().fp4o_quantize_opt(_ptr(xb), rows, cols, fmt, hn, axis,
+                                None if a_in is None else _ptr(a_in), sr_seed is not None,
+                                sr_seed or 0, rht_seed is not None, rht_seed or 0,
+                                _ptr(codes), _ptr(scales), _ptr(s), _ptr(t))
     if rc != 0:
         raise ValueError(f"oracle quantize rejected shape {xb.shape} fmt={fmt} hn={hn} axis={axis}")
     if fmt == NVFP4:

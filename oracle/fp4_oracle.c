@@ -53,6 +53,28 @@
  *       multiple of 4; padding bytes are zero.
  *   R8  Column-wise ("COL") quantisation of x[R][C] quantises x^T: codes [C][R/2],
  *       scales laid out for a [C][R/bs] scale matrix.
+ *
+ * Variants the pages test and reject as stabilisers ([MXFP4-PT] "방법론" item 3,
+ * "주요 기여 및 발견" section 2: stochastic rounding and randomised Hadamard
+ * rotations both fail to stabilise the full MXFP4 pipeline). The pages give no
+ * numerics for either; the readings below are the plainest deterministic-per-seed
+ * ones. Random words come from Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel
+ * random numbers: as easy as 1, 2, 3", SC 2011), written here from that definition:
+ *   word(seed, index, stream) = Philox4x32-10(counter = (index/4 low 32 bits,
+ *   index/4 high 32 bits, stream, 0), key = (seed low, seed high))[index % 4].
+ *   R12 Stochastic rounding (replaces R4's nearest rounding of the magnitude): for
+ *       |q| >= 6 the magnitude is 6; otherwise lo = the largest E2M1 magnitude <= |q|,
+ *       hi = the next one, and the magnitude is hi when (w >> 8) * 2^-24 <
+ *       (|q| - lo) / (hi - lo), else lo (both sides exact in fp32), with
+ *       w = word(seed, i * C + c, 1 + layout) for element (i, c) of the quantised
+ *       [R][C] matrix, layout 0 = ROW, 1 = COL. The sign is kept as in R4. Block
+ *       scales are those of R2 / R5 unchanged.
+ *   R13 Randomised Hadamard: before R1, the element at index j along the contraction
+ *       axis (column j of the quantised [R][C] matrix) is negated when bit 31 of
+ *       word(seed, j, 0) is set. Both GEMM operands of a pass use the same seed, so
+ *       (X D H)(W D H)^T = X W^T as for the deterministic rotation. The NVFP4 tensor
+ *       amax is taken after this rotation.
+ *   R14 Caller-supplied NVFP4 tensor amax: R5 with T given instead of computed.
  */
 #include <math.h>
 #include <stdint.h>
@@ -100,6 +122,61 @@ uint8_t fp4o_e2m1_encode(float q) {
     else if (a <= 5.0f)  idx = 6;  /* midpoint 5 between 4 (idx 6) and 6 (idx 7) */
     else                 idx = 7;  /* everything above saturates to 6 */
     return (uint8_t)(sign | idx);
+}
+
+/* ---------------------------------------------------------------- Philox4x32-10 */
+
+/* One Philox round: two 32x32 -> 64-bit products of the even counter words with the
+ * round multipliers; the high halves are mixed with the odd words and the key. */
+void fp4o_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]) {
+    uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int round = 0; round < 10; round++) {
+        uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+        uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+        uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        c0 = hi1 ^ c1 ^ k0;
+        c1 = lo1;
+        c2 = hi0 ^ c3 ^ k1;
+        c3 = lo0;
+        k0 += 0x9E3779B9u; /* Weyl key schedule */
+        k1 += 0xBB67AE85u;
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+/* word(seed, index, stream) of R12/R13. */
+uint32_t fp4o_philox_word(uint64_t seed, uint64_t index, uint32_t stream) {
+    uint64_t blk = index / 4;
+    uint32_t ctr[4] = {(uint32_t)blk, (uint32_t)(blk >> 32), stream, 0};
+    uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    uint32_t out[4];
+    fp4o_philox4x32_10(ctr, key, out);
+    return out[index % 4];
+}
+
+/* R12: stochastic E2M1 rounding of q with random word w. */
+uint8_t fp4o_e2m1_encode_sr(float q, uint32_t w) {
+    static const float mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+    uint8_t sign = (f32_to_bits(q) >> 31) ? 8 : 0;
+    float a = fabsf(q);
+    int idx;
+    if (a >= 6.0f) {
+        idx = 7;
+    } else {
+        int lo = 0;
+        while (lo < 6 && mag[lo + 1] <= a) lo++;
+        float p = (a - mag[lo]) / (mag[lo + 1] - mag[lo]);
+        float u = (float)(w >> 8) * 0x1p-24f;
+        idx = u < p ? lo + 1 : lo;
+    }
+    return (uint8_t)(sign | idx);
+}
+
+/* R13: 1 when the element at contraction index j is negated. */
+int fp4o_rht_negate(uint64_t seed, int64_t j) {
+    return (int)(fp4o_philox_word(seed, (uint64_t)j, 0) >> 31);
 }
 
 /* ---------------------------------------------------------------- E8M0 */
@@ -184,12 +261,25 @@ void fp4o_fwht_f32(float *v, int n) {
 /* Rotate a bf16 matrix along its contraction axis. For axis ROW the groups run along
  * each row of x[rows][cols] and out is [rows][cols]; for axis COL they run down each
  * column and out is the transpose, [cols][rows] (R8). hn == 0 only widens. */
+int fp4o_rotate_opt(const uint16_t *x, int64_t rows, int64_t cols, int hn, int axis, int rht,
+                    uint64_t rht_seed, float *out);
+
 int fp4o_rotate(const uint16_t *x, int64_t rows, int64_t cols, int hn, int axis, float *out) {
+    return fp4o_rotate_opt(x, rows, cols, hn, axis, 0, 0, out);
+}
+
+/* As fp4o_rotate; with rht != 0 the random signs of R13 are applied first. */
+int fp4o_rotate_opt(const uint16_t *x, int64_t rows, int64_t cols, int hn, int axis, int rht,
+                    uint64_t rht_seed, float *out) {
     int64_t R = axis == FP4O_ROW ? rows : cols, C = axis == FP4O_ROW ? cols : rows;
     if (hn != 0 && (C % hn) != 0) return -1;
     for (int64_t r = 0; r < R; r++)
         for (int64_t c = 0; c < C; c++)
             out[r * C + c] = fp4o_bf16_to_f32(axis == FP4O_ROW ? x[r * cols + c] : x[c * cols + r]);
+    if (rht)
+        for (int64_t c = 0; c < C; c++)
+            if (fp4o_rht_negate(rht_seed, c))
+                for (int64_t r = 0; r < R; r++) out[r * C + c] = -out[r * C + c];
     if (hn != 0)
         for (int64_t r = 0; r < R; r++)
             for (int64_t g = 0; g < C; g += hn) fp4o_fwht_f32(out + r * C + g, hn);
@@ -198,13 +288,23 @@ int fp4o_rotate(const uint16_t *x, int64_t rows, int64_t cols, int hn, int axis,
 
 /* max |v| over the rotated matrix (the NVFP4 tensor amax of step 3), one row of the
  * rotated matrix at a time. */
+float fp4o_rotated_amax_opt(const uint16_t *x, int64_t rows, int64_t cols, int hn, int axis,
+                            int rht, uint64_t rht_seed);
+
 float fp4o_rotated_amax(const uint16_t *x, int64_t rows, int64_t cols, int hn, int axis) {
+    return fp4o_rotated_amax_opt(x, rows, cols, hn, axis, 0, 0);
+}
+
+float fp4o_rotated_amax_opt(const uint16_t *x, int64_t rows, int64_t cols, int hn, int axis,
+                            int rht, uint64_t rht_seed) {
     int64_t R = axis == FP4O_ROW ? rows : cols, C = axis == FP4O_ROW ? cols : rows;
     float *v = (float *)malloc(sizeof(float) * (size_t)(C > 0 ? C : 1));
     float T = 0.0f;
     for (int64_t r = 0; r < R; r++) {
-        for (int64_t c = 0; c < C; c++)
+        for (int64_t c = 0; c < C; c++) {
             v[c] = fp4o_bf16_to_f32(axis == FP4O_ROW ? x[r * cols + c] : x[c * cols + r]);
+            if (rht && fp4o_rht_negate(rht_seed, c)) v[c] = -v[c];
+        }
         if (hn != 0)
             for (int64_t g = 0; g < C; g += hn) fp4o_fwht_f32(v + g, hn);
         for (int64_t c = 0; c < C; c++) T = fmaxf(T, fabsf(v[c]));
@@ -228,13 +328,23 @@ int64_t fp4o_scale_offset(int64_t r, int64_t kb, int64_t kblocks) {
 /* ---------------------------------------------------------------- block quantisers */
 
 /* MX block (R2, R3): bs values -> bs codes (one per byte, unpacked) and one E8M0 byte. */
-void fp4o_quantize_block_mx(const float *v, int bs, uint8_t *codes, uint8_t *scale_byte) {
+/* w: NULL for nearest rounding (R4), else one random word per element (R12). */
+static uint8_t encode_q(float q, const uint32_t *w, int i) {
+    return w ? fp4o_e2m1_encode_sr(q, w[i]) : fp4o_e2m1_encode(q);
+}
+
+static void quantize_block_mx_w(const float *v, int bs, const uint32_t *w, uint8_t *codes,
+                                uint8_t *scale_byte) {
     float amax = 0.0f;
     for (int i = 0; i < bs; i++) amax = fmaxf(amax, fabsf(v[i]));
     int e = fp4o_mx_scale_exponent(amax);
     float inv = (float)ldexp(1.0, -e); /* 2^-e, exact in fp32 for e in [-127, 127] */
-    for (int i = 0; i < bs; i++) codes[i] = fp4o_e2m1_encode(v[i] * inv);
+    for (int i = 0; i < bs; i++) codes[i] = encode_q(v[i] * inv, w, i);
     *scale_byte = (uint8_t)(e + 127);
+}
+
+void fp4o_quantize_block_mx(const float *v, int bs, uint8_t *codes, uint8_t *scale_byte) {
+    quantize_block_mx_w(v, bs, NULL, codes, scale_byte);
 }
 
 /* NV tensor scale (R5). */
@@ -244,7 +354,8 @@ float fp4o_nv_tensor_scale(float tensor_amax) {
 }
 
 /* NV block (R5): bs values -> bs codes and one UE4M3 byte, under tensor scale S. */
-void fp4o_quantize_block_nv(const float *v, int bs, float S, uint8_t *codes, uint8_t *scale_byte) {
+static void quantize_block_nv_w(const float *v, int bs, float S, const uint32_t *w,
+                                uint8_t *codes, uint8_t *scale_byte) {
     float bmax = 0.0f;
     for (int i = 0; i < bs; i++) bmax = fmaxf(bmax, fabsf(v[i]));
     float six_s = 6.0f * S;
@@ -253,9 +364,13 @@ void fp4o_quantize_block_nv(const float *v, int bs, float S, uint8_t *codes, uin
     float d = (float)fp4o_e4m3_decode(sb) * S; /* decode is exact in fp32; one rounding */
     for (int i = 0; i < bs; i++) {
         if (sb == 0) codes[i] = (f32_to_bits(v[i]) >> 31) ? 8 : 0;
-        else codes[i] = fp4o_e2m1_encode(v[i] / d);
+        else codes[i] = encode_q(v[i] / d, w, i);
     }
     *scale_byte = sb;
+}
+
+void fp4o_quantize_block_nv(const float *v, int bs, float S, uint8_t *codes, uint8_t *scale_byte) {
+    quantize_block_nv_w(v, bs, S, NULL, codes, scale_byte);
 }
 
 /* ---------------------------------------------------------------- tensor quantiser */
@@ -278,9 +393,23 @@ int fp4o_quantize(const uint16_t *x, int64_t rows, int64_t cols, int fmt, int hn
 /* As fp4o_quantize; for NVFP4 a non-NULL amax_in supplies the tensor amax T of step 3
  * (the amax of the whole rotated tensor, when x is a slice of it: rows of a ROW
  * quantisation or columns of a COL one are quantised independently given T). */
+int fp4o_quantize_opt(const uint16_t *x, int64_t rows, int64_t cols, int fmt, int hn, int axis,
+                      const float *amax_in, int sr, uint64_t sr_seed, int rht, uint64_t rht_seed,
+                      uint8_t *codes, uint8_t *scales, float *nv_scale_out, float *nv_amax_out);
+
 int fp4o_quantize_ex(const uint16_t *x, int64_t rows, int64_t cols, int fmt, int hn, int axis,
                      const float *amax_in, uint8_t *codes, uint8_t *scales, float *nv_scale_out,
                      float *nv_amax_out) {
+    return fp4o_quantize_opt(x, rows, cols, fmt, hn, axis, amax_in, 0, 0, 0, 0, codes, scales,
+                             nv_scale_out, nv_amax_out);
+}
+
+/* As fp4o_quantize_ex, with the variants: sr != 0 rounds the codes stochastically
+ * (R12, words keyed by sr_seed), rht != 0 applies the random signs of R13 (keyed by
+ * rht_seed) before the rotation. */
+int fp4o_quantize_opt(const uint16_t *x, int64_t rows, int64_t cols, int fmt, int hn, int axis,
+                      const float *amax_in, int sr, uint64_t sr_seed, int rht, uint64_t rht_seed,
+                      uint8_t *codes, uint8_t *scales, float *nv_scale_out, float *nv_amax_out) {
     int bs = fmt == FP4O_MXFP4 ? 32 : 16;
     int64_t R = axis == FP4O_ROW ? rows : cols, C = axis == FP4O_ROW ? cols : rows;
     if (C % bs != 0 || (hn != 0 && C % hn != 0) || C % 2 != 0) return -1;
@@ -288,7 +417,7 @@ int fp4o_quantize_ex(const uint16_t *x, int64_t rows, int64_t cols, int fmt, int
     float *v = (float *)malloc(sizeof(float) * (size_t)(R * C > 0 ? R * C : 1));
     if (!v) return -2;
     /* steps 1-2: widen, rotate */
-    fp4o_rotate(x, rows, cols, hn, axis, v);
+    fp4o_rotate_opt(x, rows, cols, hn, axis, rht, rht_seed, v);
     /* step 3 (NVFP4 only): tensor amax of the rotated values and the tensor scale */
     float S = 1.0f;
     if (fmt == FP4O_NVFP4) {
@@ -303,12 +432,17 @@ int fp4o_quantize_ex(const uint16_t *x, int64_t rows, int64_t cols, int fmt, int
     /* steps 4-5: block scales and codes; step 6: pack */
     memset(scales, 0, (size_t)fp4o_scale_layout_bytes(R, KB));
     uint8_t blk[32];
+    uint32_t w[32];
     for (int64_t r = 0; r < R; r++) {
         for (int64_t kb = 0; kb < KB; kb++) {
             const float *bv = v + r * C + kb * bs;
+            if (sr)
+                for (int i = 0; i < bs; i++)
+                    w[i] = fp4o_philox_word(sr_seed, (uint64_t)(r * C + kb * bs + i),
+                                            1u + (uint32_t)axis);
             uint8_t sb;
-            if (fmt == FP4O_MXFP4) fp4o_quantize_block_mx(bv, bs, blk, &sb);
-            else fp4o_quantize_block_nv(bv, bs, S, blk, &sb);
+            if (fmt == FP4O_MXFP4) quantize_block_mx_w(bv, bs, sr ? w : NULL, blk, &sb);
+            else quantize_block_nv_w(bv, bs, S, sr ? w : NULL, blk, &sb);
             scales[fp4o_scale_offset(r, kb, KB)] = sb;
             for (int i = 0; i < bs; i += 2)
                 codes[r * (C / 2) + (kb * bs + i) / 2] = (uint8_t)(blk[i] | (blk[i + 1] << 4));
