@@ -40,6 +40,17 @@ WORKLOAD = ("llama3.1-8b layer fwd+bwd: qkv 6144x4096, o 4096x4096, gate/up 1433
             "down 4096x14336; 8192 tokens/rank; MXFP4 + H16")
 
 
+def workload_name(a) -> str:
+    """WORKLOAD for the default run; the same layer with the format / rotation / quantiser
+    variant actually run otherwise."""
+    if a.format == "mxfp4" and a.hadamard == 16 and a.variant == "none":
+        return WORKLOAD
+    tag = f"{a.format.upper()} + " + (f"H{a.hadamard}" if a.hadamard else "no rotation")
+    if a.variant != "none":
+        tag += f" + {a.variant} quantiser variant"
+    return WORKLOAD.rsplit(";", 1)[0] + "; " + tag
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -53,8 +64,13 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--proj", default="qkv,o,gate,up,down",
                     help="comma-separated subset of the layer's projections (profiling cases)")
+    ap.add_argument("--variant", choices=["none", "sr", "rht", "sr+rht", "amax"], default="none",
+                    help="quantiser variant: stochastic rounding, randomised Hadamard signs, "
+                         "both, or (NVFP4) a supplied tensor amax instead of the amax pass")
     a = ap.parse_args()
     a.warmup = max(3, a.warmup)
+    if a.variant == "amax" and a.format != "nvfp4":
+        ap.error("--variant amax needs --format nvfp4")
     return a
 
 
@@ -122,10 +138,11 @@ class Clocks:
 class LlamaLayer:
     """Inputs, quantised operands and outputs of every projection, all on the device."""
 
-    def __init__(self, device, fmt, hn, tokens=8192, seed=0, names=None):
+    def __init__(self, device, fmt, hn, tokens=8192, seed=0, names=None, variant="none"):
         import fp4_block_scaled_deterministic_b200 as fp4
         from fp4_block_scaled_deterministic_b200 import synthetic
         self.fp4, self.fmt, self.hn, self.M = fp4, fmt, hn, tokens
+        self.variant = variant
         self.projs = []
         g = torch.Generator(device=device)
         for i, (name, N, K) in enumerate(synthetic.LLAMA_LAYERS):
@@ -145,6 +162,28 @@ class LlamaLayer:
             p["dW"] = torch.empty(N, K, dtype=torch.float32, device=device)
             self.projs.append(p)
         del g
+        if variant == "amax":
+            # the supplied amax is that of an earlier quantisation of the same tensor: run
+            # one plain quantisation now; its {amax_row, amax_col} (ts[2:4]) stay in place
+            for p in self.projs:
+                for key, (r, c) in self._operands(p):
+                    row, col, ts = p[key + "_row"], p[key + "_col"], p[key + "_ts"]
+                    st = fp4.fp4_quantize_dual(p[key], row[0], row[1], col[0], col[1], ts, r, c,
+                                               fmt, hn, torch.cuda.current_stream().cuda_stream)
+                    assert st == 0
+        self.opts = {}
+        for p in self.projs:
+            for key, _ in self._operands(p):
+                o = None
+                if variant == "amax":
+                    o = fp4.QuantOpts(p[key + "_ts"].data_ptr() + 8, 0, 0, 0, 0)
+                elif variant != "none":
+                    o = fp4.QuantOpts(None, int("sr" in variant), int("rht" in variant),
+                                      0x5EED0000 + seed, 0x51600000 + seed)
+                self.opts[(p["name"], key)] = o
+
+    def _operands(self, p):
+        return (("X", (self.M, p["K"])), ("W", (p["N"], p["K"])), ("dY", (self.M, p["N"])))
 
     def _qbuf(self, r, c, device):
         f = self.fp4
@@ -164,7 +203,8 @@ class LlamaLayer:
         return sum(t.numel() * t.element_size() for p in self.projs for t in (p["Y"], p["dX"], p["dW"]))
 
     def launches_per_step(self):
-        per_q = 1 if self.fmt == 0 else 2  # NVFP4 adds the amax pass (plus a memset)
+        # NVFP4 adds the amax pass (plus a memset) unless the amax is supplied
+        per_q = 1 if self.fmt == 0 or self.variant == "amax" else 2
         return len(self.projs) * (3 * per_q + 3)
 
     def step(self, stream, timers=None, allreduce=None):
@@ -186,12 +226,17 @@ class LlamaLayer:
             return r
 
         for p in self.projs:
-            for key, (r, c) in (("X", (self.M, p["K"])), ("W", (p["N"], p["K"])),
-                                ("dY", (self.M, p["N"]))):
+            for key, (r, c) in self._operands(p):
                 row, col, ts = p[key + "_row"], p[key + "_col"], p[key + "_ts"]
-                st = timed("quant", lambda: f.fp4_quantize_dual(
-                    p[key], row[0], row[1], col[0], col[1], ts if fmt == 1 else None, r, c, fmt,
-                    hn, s))
+                opts = self.opts[(p["name"], key)]
+                if opts is None:
+                    st = timed("quant", lambda: f.fp4_quantize_dual(
+                        p[key], row[0], row[1], col[0], col[1], ts if fmt == 1 else None, r, c,
+                        fmt, hn, s))
+                else:
+                    st = timed("quant", lambda: f.fp4_quantize_dual_opts(
+                        p[key], row[0], row[1], col[0], col[1], ts if fmt == 1 else None, r, c,
+                        fmt, hn, opts, s))
                 assert st == 0, f.status_string(st)
             tsx, tsw, tsy = p["X_ts"], p["W_ts"], p["dY_ts"]
             nv = fmt == 1
@@ -296,7 +341,7 @@ def run_reference(a):
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": t_med * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": WORKLOAD, "format": a.format, "hadamard_n": a.hadamard,
+            "config": {"workload": workload_name(a), "format": a.format, "hadamard_n": a.hadamard,
                        "l2": "n/a (CPU)"},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
                              "sample": desc, "wall_s": wall},
@@ -347,7 +392,7 @@ def main():
     fp4.lib()  # fails loudly if the library is missing
     fmt = 0 if a.format == "mxfp4" else 1
     names = [n.strip() for n in a.proj.split(",") if n.strip()]
-    layer = LlamaLayer(dev, fmt, a.hadamard, seed=1000 * rank, names=names)
+    layer = LlamaLayer(dev, fmt, a.hadamard, seed=1000 * rank, names=names, variant=a.variant)
     stream = torch.cuda.current_stream(dev)
     from fp4_block_scaled_deterministic_b200 import dp
     allreduce = dp.allreduce_wgrad if world > 1 else None
@@ -386,7 +431,8 @@ def main():
     quant_ms = [x.elapsed_time(y) for x, y in timers["quant"]]
     per_launch_flops = gemm_flops_of(layer) * a.steps
     gemm_tflops = sum(per_launch_flops) / (sum(gemm_ms) * 1e-3) / 1e12
-    bpe = 2.0 + 2 * (0.5 + (1 / 32 if fmt == 0 else 1 / 16)) + (2.0 if fmt == 1 else 0.0)
+    amax_pass = fmt == 1 and a.variant != "amax"
+    bpe = 2.0 + 2 * (0.5 + (1 / 32 if fmt == 0 else 1 / 16)) + (2.0 if amax_pass else 0.0)
     q_bytes = layer.quant_elems() * bpe * a.steps
     quant_gbs = q_bytes / (sum(quant_ms) * 1e-3) / 1e9
 
@@ -410,9 +456,10 @@ def main():
            "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms / a.steps,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp4_e2m1",
            "data": "synthetic",
-           "config": {"workload": WORKLOAD if len(names) == 5 else
-                      f"subset {','.join(names)} of: {WORKLOAD}",
-                      "format": a.format, "hadamard_n": a.hadamard, "tokens_per_rank": layer.M,
+           "config": {"workload": workload_name(a) if len(names) == 5 else
+                      f"subset {','.join(names)} of: {workload_name(a)}",
+                      "format": a.format, "hadamard_n": a.hadamard, "variant": a.variant,
+                      "tokens_per_rank": layer.M,
                       "l2": f"inputs larger than L2 ({(layer.bytes_in() + layer.bytes_out()) / 1e9:.1f} GB per step)",
                       "parallelism": f"dp{world}"},
            "gemm_tflops": gemm_tflops, "quantize_gbs": quant_gbs,

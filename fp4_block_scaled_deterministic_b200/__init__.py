@@ -41,6 +41,13 @@ class Fp4Error(RuntimeError):
         super().__init__(f"{where}: {STATUS.get(code, code)} ({status_string(code)})")
 
 
+class QuantOpts(ctypes.Structure):
+    """fp4_quant_opts of include/fp4.h (host struct passed by pointer)."""
+    _fields_ = [("amax", ctypes.c_void_p), ("stochastic", ctypes.c_int),
+                ("random_signs", ctypes.c_int), ("sr_seed", ctypes.c_uint64),
+                ("sign_seed", ctypes.c_uint64)]
+
+
 _lib = None
 
 
@@ -59,6 +66,10 @@ def lib() -> ctypes.CDLL:
             "fp4_scales_bytes": (SZ, [I64, I64, I32]),
             "fp4_quantize": (I32, [P, P, P, P, I64, I64, I32, I32, I32, P]),
             "fp4_quantize_dual": (I32, [P, P, P, P, P, P, I64, I64, I32, I32, P]),
+            "fp4_quantize_opts": (I32, [P, P, P, P, I64, I64, I32, I32, I32,
+                                        ctypes.POINTER(QuantOpts), P]),
+            "fp4_quantize_dual_opts": (I32, [P, P, P, P, P, P, I64, I64, I32, I32,
+                                             ctypes.POINTER(QuantOpts), P]),
             "fp4_gemm": (I32, [P, P, P, P, P, P, P, I64, I64, I64, I32, I32, P]),
             "fp4_linear_workspace_size": (SZ, [I32, I64, I64, I64, I32]),
             "fp4_linear_fprop": (I32, [P, P, P, I64, I64, I64, I32, I32, I32, P, SZ, P]),
@@ -132,6 +143,23 @@ def fp4_quantize_dual(x, row_codes, row_scales, col_codes, col_scales, tensor_sc
                                    hadamard_n, _stream(stream))
 
 
+def _opts(opts):
+    return None if opts is None else ctypes.byref(opts)
+
+
+def fp4_quantize_opts(x, codes, scales, tensor_scale, rows, cols, fmt, hadamard_n, axis, opts,
+                      stream=None):
+    return lib().fp4_quantize_opts(_ptr(x), _ptr(codes), _ptr(scales), _ptr(tensor_scale), rows,
+                                   cols, fmt, hadamard_n, axis, _opts(opts), _stream(stream))
+
+
+def fp4_quantize_dual_opts(x, row_codes, row_scales, col_codes, col_scales, tensor_scale, rows,
+                           cols, fmt, hadamard_n, opts, stream=None):
+    return lib().fp4_quantize_dual_opts(_ptr(x), _ptr(row_codes), _ptr(row_scales),
+                                        _ptr(col_codes), _ptr(col_scales), _ptr(tensor_scale),
+                                        rows, cols, fmt, hadamard_n, _opts(opts), _stream(stream))
+
+
 def fp4_gemm(A, As, Ats, B, Bs, Bts, C, M, N, K, fmt, out_dtype, stream=None):
     return lib().fp4_gemm(_ptr(A), _ptr(As), _ptr(Ats), _ptr(B), _ptr(Bs), _ptr(Bts), _ptr(C), M,
                           N, K, fmt, out_dtype, _stream(stream))
@@ -186,10 +214,25 @@ def _alloc_q(rows, cols, fmt, device):
     return codes, scales
 
 
+def quant_opts(amax: torch.Tensor | None = None, sr_seed: int | None = None,
+               sign_seed: int | None = None) -> QuantOpts | None:
+    """Options of the quantiser variants (None when none is asked for): a device fp32
+    tensor amax per layout, stochastic rounding keyed by sr_seed, random Hadamard signs
+    keyed by sign_seed."""
+    if amax is None and sr_seed is None and sign_seed is None:
+        return None
+    if amax is not None:
+        assert amax.dtype == torch.float32 and amax.is_cuda
+    return QuantOpts(None if amax is None else amax.data_ptr(), int(sr_seed is not None),
+                     int(sign_seed is not None), sr_seed or 0, sign_seed or 0)
+
+
 def quantize(x: torch.Tensor, fmt: int = MXFP4, hadamard_n: int = 16, axis: int = ROW,
-             ts_buf: torch.Tensor | None = None) -> QTensor:
+             ts_buf: torch.Tensor | None = None, amax: torch.Tensor | None = None,
+             sr_seed: int | None = None, sign_seed: int | None = None) -> QTensor:
     """Rotate and quantise a bf16 CUDA matrix along `axis` (COL returns the transposed
-    layout [cols][rows/2])."""
+    layout [cols][rows/2]). amax / sr_seed / sign_seed select the variants of
+    fp4_quantize_opts."""
     assert x.dtype == torch.bfloat16 and x.is_cuda and x.dim() == 2
     x = x.contiguous()
     rows, cols = x.shape
@@ -198,11 +241,19 @@ def quantize(x: torch.Tensor, fmt: int = MXFP4, hadamard_n: int = 16, axis: int 
     ts = None
     if fmt == NVFP4:
         ts = ts_buf if ts_buf is not None else torch.zeros(2, dtype=torch.float32, device=x.device)
-    _check(fp4_quantize(x, codes, scales, ts, rows, cols, fmt, hadamard_n, axis), "fp4_quantize")
+    opts = quant_opts(amax, sr_seed, sign_seed)
+    if opts is None:
+        _check(fp4_quantize(x, codes, scales, ts, rows, cols, fmt, hadamard_n, axis),
+               "fp4_quantize")
+    else:
+        _check(fp4_quantize_opts(x, codes, scales, ts, rows, cols, fmt, hadamard_n, axis, opts),
+               "fp4_quantize_opts")
     return QTensor(codes, scales, None if ts is None else ts[0:1], fmt, R, C)
 
 
-def quantize_dual(x: torch.Tensor, fmt: int = MXFP4, hadamard_n: int = 16):
+def quantize_dual(x: torch.Tensor, fmt: int = MXFP4, hadamard_n: int = 16,
+                  amax: torch.Tensor | None = None, sr_seed: int | None = None,
+                  sign_seed: int | None = None):
     """Row-wise and column-wise (transposed) quantisation from one read of x."""
     assert x.dtype == torch.bfloat16 and x.is_cuda and x.dim() == 2
     x = x.contiguous()
@@ -210,8 +261,13 @@ def quantize_dual(x: torch.Tensor, fmt: int = MXFP4, hadamard_n: int = 16):
     rc, rs = _alloc_q(rows, cols, fmt, x.device)
     cc, cs = _alloc_q(cols, rows, fmt, x.device)
     ts = torch.zeros(4, dtype=torch.float32, device=x.device) if fmt == NVFP4 else None
-    _check(fp4_quantize_dual(x, rc, rs, cc, cs, ts, rows, cols, fmt, hadamard_n),
-           "fp4_quantize_dual")
+    opts = quant_opts(amax, sr_seed, sign_seed)
+    if opts is None:
+        _check(fp4_quantize_dual(x, rc, rs, cc, cs, ts, rows, cols, fmt, hadamard_n),
+               "fp4_quantize_dual")
+    else:
+        _check(fp4_quantize_dual_opts(x, rc, rs, cc, cs, ts, rows, cols, fmt, hadamard_n, opts),
+               "fp4_quantize_dual_opts")
     return (QTensor(rc, rs, None if ts is None else ts[0:1], fmt, rows, cols),
             QTensor(cc, cs, None if ts is None else ts[1:2], fmt, cols, rows))
 

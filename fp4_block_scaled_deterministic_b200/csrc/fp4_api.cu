@@ -103,36 +103,45 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline int block_of(fp4_format f) { return f == FP4_MXFP4 ? 32 : 16; }
 
 // ---------------------------------------------------------------- quantise launch
-template <int FMT, int HN, int MODE, bool AMAX>
+template <int FMT, int HN, int MODE, bool AMAX, bool EXT>
 cudaError_t launch_q(const CUtensorMap& ti, const CUtensorMap& tr, const CUtensorMap& tc,
                      const QuantArgs& a, int grid, int dev, cudaStream_t s) {
   static std::atomic<uint64_t> done{0};
-  auto k = quantize_kernel<FMT, HN, MODE, AMAX>;
+  auto k = quantize_kernel<FMT, HN, MODE, AMAX, EXT>;
   cudaError_t e = ensure_smem(k, kQSmemBytes, dev, done);
   if (e != cudaSuccess) return e;
   k<<<grid, kQThreads, kQSmemBytes, s>>>(ti, tr, tc, a);
   return cudaGetLastError();
 }
 
-template <int FMT, int HN, bool AMAX>
+template <int FMT, int HN, bool AMAX, bool EXT>
 cudaError_t dispatch_mode(int mode, const CUtensorMap& ti, const CUtensorMap& tr,
                           const CUtensorMap& tc, const QuantArgs& a, int grid, int dev,
                           cudaStream_t s) {
   switch (mode) {
-    case kModeRow: return launch_q<FMT, HN, kModeRow, AMAX>(ti, tr, tc, a, grid, dev, s);
-    case kModeCol: return launch_q<FMT, HN, kModeCol, AMAX>(ti, tr, tc, a, grid, dev, s);
-    default: return launch_q<FMT, HN, kModeDual, AMAX>(ti, tr, tc, a, grid, dev, s);
+    case kModeRow: return launch_q<FMT, HN, kModeRow, AMAX, EXT>(ti, tr, tc, a, grid, dev, s);
+    case kModeCol: return launch_q<FMT, HN, kModeCol, AMAX, EXT>(ti, tr, tc, a, grid, dev, s);
+    default: return launch_q<FMT, HN, kModeDual, AMAX, EXT>(ti, tr, tc, a, grid, dev, s);
   }
 }
 
+// ext: the variant kernels (random signs and/or stochastic rounding requested in a)
 template <int FMT, bool AMAX>
 cudaError_t dispatch_hn(int hn, int mode, const CUtensorMap& ti, const CUtensorMap& tr,
                         const CUtensorMap& tc, const QuantArgs& a, int grid, int dev,
                         cudaStream_t s) {
+  const bool ext = a.sr != 0 || a.rht != 0;
+  if (ext) {
+    switch (hn) {
+      case 0: return dispatch_mode<FMT, 0, AMAX, true>(mode, ti, tr, tc, a, grid, dev, s);
+      case 16: return dispatch_mode<FMT, 16, AMAX, true>(mode, ti, tr, tc, a, grid, dev, s);
+      default: return dispatch_mode<FMT, 32, AMAX, true>(mode, ti, tr, tc, a, grid, dev, s);
+    }
+  }
   switch (hn) {
-    case 0: return dispatch_mode<FMT, 0, AMAX>(mode, ti, tr, tc, a, grid, dev, s);
-    case 16: return dispatch_mode<FMT, 16, AMAX>(mode, ti, tr, tc, a, grid, dev, s);
-    default: return dispatch_mode<FMT, 32, AMAX>(mode, ti, tr, tc, a, grid, dev, s);
+    case 0: return dispatch_mode<FMT, 0, AMAX, false>(mode, ti, tr, tc, a, grid, dev, s);
+    case 16: return dispatch_mode<FMT, 16, AMAX, false>(mode, ti, tr, tc, a, grid, dev, s);
+    default: return dispatch_mode<FMT, 32, AMAX, false>(mode, ti, tr, tc, a, grid, dev, s);
   }
 }
 
@@ -151,12 +160,15 @@ fp4_status validate_quant_common(const void* x, int64_t rows, int64_t cols, fp4_
 
 fp4_status quantize_impl(const void* x, void* rcodes, void* rscales, void* ccodes, void* cscales,
                          float* ts, int64_t rows, int64_t cols, fp4_format fmt, int hn, int mode,
-                         cudaStream_t stream) {
+                         cudaStream_t stream, const fp4_quant_opts* opts = nullptr) {
   fp4_status st = validate_quant_common(x, rows, cols, fmt, hn);
   if (st != FP4_OK) return st;
   const bool do_row = mode & kModeRow, do_col = mode & kModeCol;
   if (fmt == FP4_MXFP4 && ts) return FP4_ERR_INVALID_ARG;
   if (fmt == FP4_NVFP4 && !ts) return FP4_ERR_INVALID_ARG;
+  const float* amax_in = opts ? opts->amax : nullptr;
+  if (amax_in && fmt != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
+  if (amax_in && (reinterpret_cast<uintptr_t>(amax_in) & 3u)) return FP4_ERR_ALIGN;
   if (rows == 0 || cols == 0) return FP4_OK;
   if ((do_row && (!rcodes || !rscales)) || (do_col && (!ccodes || !cscales)))
     return FP4_ERR_INVALID_ARG;
@@ -196,6 +208,14 @@ fp4_status quantize_impl(const void* x, void* rcodes, void* rscales, void* ccode
   a.row_kb4 = static_cast<int>(ceil_div(cols / bs, 4));
   a.col_kb4 = static_cast<int>(ceil_div(rows / bs, 4));
   a.wait_limit_ns = kDefaultWaitLimitNs;
+  if (opts) {
+    a.sr = opts->stochastic != 0;
+    a.rht = opts->random_signs != 0;
+    a.sr_key[0] = static_cast<uint32_t>(opts->sr_seed);
+    a.sr_key[1] = static_cast<uint32_t>(opts->sr_seed >> 32);
+    a.sign_key[0] = static_cast<uint32_t>(opts->sign_seed);
+    a.sign_key[1] = static_cast<uint32_t>(opts->sign_seed >> 32);
+  }
   const int resident = kQCtasPerSM * info->sm_count;
   const int grid = a.num_tiles < resident ? a.num_tiles : resident;
 
@@ -218,17 +238,26 @@ fp4_status quantize_impl(const void* x, void* rcodes, void* rscales, void* ccode
       a.s_col_out = ts;
       amax_c = ts + 1;
     }
-    a.amax_row = amax_r;
-    a.amax_col = amax_c;
-    a.amax_row_acc = reinterpret_cast<unsigned*>(amax_r);
-    a.amax_col_acc = reinterpret_cast<unsigned*>(amax_c);
-    float* first = amax_r ? amax_r : amax_c;
-    const size_t nbytes = (amax_r && amax_c) ? 2 * sizeof(float) : sizeof(float);
-    e = cudaMemsetAsync(first, 0, nbytes, stream);
-    if (e == cudaSuccess)
-      e = dispatch_hn<kFmtNV, true>(hn, mode, tm_in, tm_r, tm_c, a, grid, dev, stream);
-    if (e == cudaSuccess)
+    if (amax_in) {
+      // caller-supplied tensor amax: no amax pass; CTA 0 copies T into the amax slots
+      a.amax_row = amax_r ? amax_in : nullptr;
+      a.amax_col = amax_c ? (amax_r ? amax_in + 1 : amax_in) : nullptr;
+      a.amax_row_copy = amax_r;
+      a.amax_col_copy = amax_c;
       e = dispatch_hn<kFmtNV, false>(hn, mode, tm_in, tm_r, tm_c, a, grid, dev, stream);
+    } else {
+      a.amax_row = amax_r;
+      a.amax_col = amax_c;
+      a.amax_row_acc = reinterpret_cast<unsigned*>(amax_r);
+      a.amax_col_acc = reinterpret_cast<unsigned*>(amax_c);
+      float* first = amax_r ? amax_r : amax_c;
+      const size_t nbytes = (amax_r && amax_c) ? 2 * sizeof(float) : sizeof(float);
+      e = cudaMemsetAsync(first, 0, nbytes, stream);
+      if (e == cudaSuccess)
+        e = dispatch_hn<kFmtNV, true>(hn, mode, tm_in, tm_r, tm_c, a, grid, dev, stream);
+      if (e == cudaSuccess)
+        e = dispatch_hn<kFmtNV, false>(hn, mode, tm_in, tm_r, tm_c, a, grid, dev, stream);
+    }
   }
   return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }
@@ -504,7 +533,7 @@ fp4_status noalloc_scratch(void** out) {
 // ==================================================================== C ABI
 extern "C" {
 
-int fp4_abi_version(void) { return 1; }
+int fp4_abi_version(void) { return 2; }
 
 size_t fp4_codes_bytes(int64_t rows, int64_t cols) {
   if (rows <= 0 || cols <= 0) return 0;
@@ -531,6 +560,24 @@ fp4_status fp4_quantize_dual(const void* x, void* row_codes, void* row_scales, v
                              fp4_format fmt, int hn, fp4_stream_t stream) {
   return quantize_impl(x, row_codes, row_scales, col_codes, col_scales, ts, rows, cols, fmt, hn,
                        kModeDual, reinterpret_cast<cudaStream_t>(stream));
+}
+fp4_status fp4_quantize_opts(const void* x, void* codes, void* scales, float* ts, int64_t rows,
+                             int64_t cols, fp4_format fmt, int hn, fp4_axis axis,
+                             const fp4_quant_opts* opts, fp4_stream_t stream) {
+  if (axis != FP4_AXIS_ROW && axis != FP4_AXIS_COL) return FP4_ERR_INVALID_ARG;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (axis == FP4_AXIS_ROW)
+    return quantize_impl(x, codes, scales, nullptr, nullptr, ts, rows, cols, fmt, hn, kModeRow, s,
+                         opts);
+  return quantize_impl(x, nullptr, nullptr, codes, scales, ts, rows, cols, fmt, hn, kModeCol, s,
+                       opts);
+}
+fp4_status fp4_quantize_dual_opts(const void* x, void* row_codes, void* row_scales,
+                                  void* col_codes, void* col_scales, float* ts, int64_t rows,
+                                  int64_t cols, fp4_format fmt, int hn,
+                                  const fp4_quant_opts* opts, fp4_stream_t stream) {
+  return quantize_impl(x, row_codes, row_scales, col_codes, col_scales, ts, rows, cols, fmt, hn,
+                       kModeDual, reinterpret_cast<cudaStream_t>(stream), opts);
 }
 
 fp4_status fp4_gemm(const void* A, const void* As, const float* Ats, const void* B, const void* Bs,

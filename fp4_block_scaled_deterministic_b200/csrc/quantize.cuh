@@ -51,6 +51,10 @@ struct QuantArgs {
   float* s_col_out;
   unsigned* amax_row_acc;  // NVFP4 amax pass: accumulators (bits of a non-negative float)
   unsigned* amax_col_acc;
+  float* amax_row_copy;  // NVFP4 with a caller-supplied amax: CTA 0 copies it here
+  float* amax_col_copy;
+  int sr, rht;           // variant kernels: stochastic rounding, randomised Hadamard signs
+  uint32_t sr_key[2], sign_key[2];
   uint64_t wait_limit_ns;
 };
 
@@ -117,6 +121,94 @@ __device__ __forceinline__ uint32_t cvt8y(const float2 (&p)[32], int b) {
   return cvt_e2m1x8(v);
 }
 
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as 1, 2,
+// 3", SC 2011): ten rounds of two 32x32->64-bit products mixed with the other counter
+// words and the key, the key advanced by the two Weyl increments after each round.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
+    const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return c;
+}
+// The four random words of Philox block `blk` (elements 4*blk .. 4*blk+3) of a stream.
+__device__ __forceinline__ uint4 philox_block(uint64_t blk, uint32_t stream, const uint32_t (&key)[2]) {
+  return philox4x32_10(make_uint4(static_cast<uint32_t>(blk), static_cast<uint32_t>(blk >> 32),
+                                  stream, 0u),
+                       key[0], key[1]);
+}
+
+// Stochastic E2M1 rounding of q with random word w: |q| >= 6 gives 6; otherwise the
+// magnitude rounds up from the E2M1 value lo below |q| to the next one with probability
+// p = (|q| - lo) / step, taken as (w >> 8) * 2^-24 < p. |q| - lo is exact (lo >= |q|/2
+// or lo = 0) and step is a power of two, so p is exact; the sign is kept.
+__device__ __forceinline__ uint32_t e2m1_sr(float q, uint32_t w) {
+  const float a = fabsf(q);
+  uint32_t lo;
+  float base, inv_step;
+  if (a < 2.0f) {
+    lo = static_cast<uint32_t>(a * 2.0f);  // 0, 0.5, 1, 1.5
+    base = static_cast<float>(lo) * 0.5f;
+    inv_step = 2.0f;
+  } else if (a < 4.0f) {
+    const float f = floorf(a);             // 2, 3
+    lo = static_cast<uint32_t>(f) + 2u;
+    base = f;
+    inv_step = 1.0f;
+  } else {
+    lo = 6u;                               // 4
+    base = 4.0f;
+    inv_step = 0.5f;
+  }
+  const float pr = __fmul_rn(__fsub_rn(a, base), inv_step);
+  const float u = static_cast<float>(w >> 8) * 0x1p-24f;
+  const uint32_t idx = a >= 6.0f ? 7u : lo + (u < pr ? 1u : 0u);
+  return ((__float_as_uint(q) >> 31) << 3) | idx;
+}
+
+// Conversion of a job's quotients (two lanes of 32) to packed codes.
+struct RneCodes {
+  static constexpr bool kExactQuotient = false;
+  __device__ __forceinline__ void operator()(const float2 (&p)[32], uint4& cx, uint4& cy) const {
+    cx = make_uint4(cvt8x(p, 0), cvt8x(p, 8), cvt8x(p, 16), cvt8x(p, 24));
+    cy = make_uint4(cvt8y(p, 0), cvt8y(p, 8), cvt8y(p, 16), cvt8y(p, 24));
+  }
+};
+// Stochastic rounding: element i of lane x (y) draws word i of the lane's run of Philox
+// blocks starting at blk_x (blk_y). The quotient must be the exact one.
+struct SrCodes {
+  static constexpr bool kExactQuotient = true;
+  uint64_t blk_x, blk_y;
+  uint32_t stream;
+  const uint32_t* key;
+  __device__ __forceinline__ void operator()(const float2 (&p)[32], uint4& cx, uint4& cy) const {
+    uint32_t wx[8], wy[8];
+    const uint32_t k[2] = {key[0], key[1]};
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      const uint4 rx = philox_block(blk_x + g, stream, k);
+      const uint4 ry = philox_block(blk_y + g, stream, k);
+      const uint32_t ux[4] = {rx.x, rx.y, rx.z, rx.w}, uy[4] = {ry.x, ry.y, ry.z, ry.w};
+      uint32_t bx = 0, by = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        bx |= e2m1_sr(p[4 * g + j].x, ux[j]) << (4 * j);
+        by |= e2m1_sr(p[4 * g + j].y, uy[j]) << (4 * j);
+      }
+      wx[g] = bx;
+      wy[g] = by;
+    }
+    cx = make_uint4(wx[0] | (wx[1] << 16), wx[2] | (wx[3] << 16), wx[4] | (wx[5] << 16),
+                    wx[6] | (wx[7] << 16));
+    cy = make_uint4(wy[0] | (wy[1] << 16), wy[2] | (wy[3] << 16), wy[4] | (wy[5] << 16),
+                    wy[6] | (wy[7] << 16));
+  }
+};
+
 // Encoded job: 16 code bytes per lane and its scale bytes (MXFP4: byte 0; NVFP4: bytes
 // 0 and 1 for the two 16-element blocks).
 struct Enc {
@@ -127,7 +219,8 @@ struct Enc {
 // MXFP4 block of 32 per lane: byte = max(biased exponent of amax - 2, 0), i.e. the byte of
 // e = floor(log2 amax) - 2 clamped at -127 (zero and subnormal amax give 0); codes of
 // v * 2^-e, 2^-e = 2^(127 - byte) built from its bit pattern (byte <= 252).
-__device__ __forceinline__ Enc mx_encode_x2(float2 (&p)[32]) {
+template <class Codes = RneCodes>
+__device__ __forceinline__ Enc mx_encode_x2(float2 (&p)[32], const Codes& codes = Codes()) {
   const float2 am = amax_x2(p, 0, 32);
   const uint32_t ex = (__float_as_uint(am.x) >> 23) & 0xFFu;
   const uint32_t ey = (__float_as_uint(am.y) >> 23) & 0xFFu;
@@ -136,8 +229,7 @@ __device__ __forceinline__ Enc mx_encode_x2(float2 (&p)[32]) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) p[i] = mul2(p[i], inv);
   Enc e;
-  e.cx = make_uint4(cvt8x(p, 0), cvt8x(p, 8), cvt8x(p, 16), cvt8x(p, 24));
-  e.cy = make_uint4(cvt8y(p, 0), cvt8y(p, 8), cvt8y(p, 16), cvt8y(p, 24));
+  codes(p, e.cx, e.cy);
   e.sx = bx;
   e.sy = by;
   return e;
@@ -149,7 +241,8 @@ __device__ __forceinline__ Enc mx_encode_x2(float2 (&p)[32]) {
 // whenever the block amax is >= 2^-100: v*0.25 is then exact unless |v| < 2^-124, and
 // such an element lands below 2^-20 either way (code 0, sign kept). Smaller blocks
 // take the two-step path.
-__device__ __forceinline__ Enc mx_encode_x2_h16fold(float2 (&p)[32]) {
+template <class Codes = RneCodes>
+__device__ __forceinline__ Enc mx_encode_x2_h16fold(float2 (&p)[32], const Codes& codes = Codes()) {
   const float2 am = amax_x2(p, 0, 32);
   if (am.x >= 0x1p-100f && am.y >= 0x1p-100f) {
     const uint32_t bx = ((__float_as_uint(am.x) >> 23) & 0xFFu) - 4u;
@@ -158,8 +251,7 @@ __device__ __forceinline__ Enc mx_encode_x2_h16fold(float2 (&p)[32]) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) p[i] = mul2(p[i], inv);
     Enc e;
-    e.cx = make_uint4(cvt8x(p, 0), cvt8x(p, 8), cvt8x(p, 16), cvt8x(p, 24));
-    e.cy = make_uint4(cvt8y(p, 0), cvt8y(p, 8), cvt8y(p, 16), cvt8y(p, 24));
+    codes(p, e.cx, e.cy);
     e.sx = bx;
     e.sy = by;
     return e;
@@ -167,7 +259,7 @@ __device__ __forceinline__ Enc mx_encode_x2_h16fold(float2 (&p)[32]) {
   const float2 q = make_float2(0.25f, 0.25f);
 #pragma unroll
   for (int i = 0; i < 32; ++i) p[i] = mul2(p[i], q);
-  return mx_encode_x2(p);
+  return mx_encode_x2(p, codes);
 }
 
 // True when q lies within 4 units in the last place of a number with at most two
@@ -183,6 +275,7 @@ __device__ __forceinline__ bool near_e2m1_threshold(float q) {
 // The quotient is formed as v * y with y = RN(1/d): then |v*y - v/d| < 2 ulps, so v*y and
 // RN(v/d) fall on the same side of every E2M1 threshold unless v*y is within 4 ulps of
 // one; those (rare) blocks, and blocks whose 1/d overflows, are divided exactly.
+template <bool kExact = false>
 __device__ __forceinline__ void nv_block_x2(float2 (&p)[32], int b, float S, float six_s,
                                             uint32_t& sbx, uint32_t& sby) {
   const float2 bm = amax_x2(p, b, 16);
@@ -192,7 +285,7 @@ __device__ __forceinline__ void nv_block_x2(float2 (&p)[32], int b, float S, flo
   const float yx = __frcp_rn(dx), yy = __frcp_rn(dy);
   const float2 y2 = make_float2(yx, yy);
   float2 q[16];
-  bool exact = !(yx <= 3.0e38f) || !(yy <= 3.0e38f);
+  bool exact = kExact || !(yx <= 3.0e38f) || !(yy <= 3.0e38f);
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     q[i] = mul2(p[b + i], y2);
@@ -209,22 +302,26 @@ __device__ __forceinline__ void nv_block_x2(float2 (&p)[32], int b, float S, flo
   }
 }
 
-__device__ __forceinline__ Enc nv_encode_x2(float2 (&p)[32], float S, float six_s) {
+// (Stochastic rounding needs the exact quotient, not only its side of each threshold.)
+template <class Codes = RneCodes>
+__device__ __forceinline__ Enc nv_encode_x2(float2 (&p)[32], float S, float six_s,
+                                            const Codes& codes = Codes()) {
   uint32_t x0, y0, x1, y1;
-  nv_block_x2(p, 0, S, six_s, x0, y0);
-  nv_block_x2(p, 16, S, six_s, x1, y1);
+  nv_block_x2<Codes::kExactQuotient>(p, 0, S, six_s, x0, y0);
+  nv_block_x2<Codes::kExactQuotient>(p, 16, S, six_s, x1, y1);
   Enc e;
-  e.cx = make_uint4(cvt8x(p, 0), cvt8x(p, 8), cvt8x(p, 16), cvt8x(p, 24));
-  e.cy = make_uint4(cvt8y(p, 0), cvt8y(p, 8), cvt8y(p, 16), cvt8y(p, 24));
+  codes(p, e.cx, e.cy);
   e.sx = x0 | (x1 << 8);
   e.sy = y0 | (y1 << 8);
   return e;
 }
 
-template <int FMT>
-__device__ __forceinline__ Enc encode_x2(float2 (&p)[32], float S, float six_s) {
-  if constexpr (FMT == kFmtMX) return mx_encode_x2(p);
-  else return nv_encode_x2(p, S, six_s);
+template <int FMT, bool kFold, class Codes = RneCodes>
+__device__ __forceinline__ Enc encode_x2(float2 (&p)[32], float S, float six_s,
+                                         const Codes& codes = Codes()) {
+  if constexpr (FMT == kFmtMX && kFold) return mx_encode_x2_h16fold(p, codes);
+  else if constexpr (FMT == kFmtMX) return mx_encode_x2(p, codes);
+  else return nv_encode_x2(p, S, six_s, codes);
 }
 
 // Offset of scale (row r of the 128-row atom block, block kb of the tile) in a staged
@@ -269,7 +366,9 @@ __device__ __forceinline__ void load_col_job(const uint8_t* in, int b, int w, in
   }
 }
 
-template <int FMT, int HN, int MODE, bool AMAX>
+// EXT kernels also implement the variants selected at run time by a.rht (random +-1
+// signs along the contraction axis before the rotation) and a.sr (stochastic rounding).
+template <int FMT, int HN, int MODE, bool AMAX, bool EXT = false>
 __global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
     quantize_kernel(const __grid_constant__ CUtensorMap tm_in,
                     const __grid_constant__ CUtensorMap tm_rcodes,
@@ -278,6 +377,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
   constexpr bool kCol = (MODE & kModeCol) != 0;
   // MXFP4 + H16 quantise pass: the rotation's x0.25 is folded into the block scale
   constexpr bool kFoldH16 = FMT == kFmtMX && HN == 16 && !AMAX;
+  const bool rht = EXT && a.rht != 0, sr = EXT && a.sr != 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -288,6 +388,9 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
   uint8_t* s_csc = s_rsc + 2 * kQScaleBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(s_csc + 2 * kQScaleBytes);
   float* s_red = reinterpret_cast<float*>(full + kQStages);  // [8 warps][2]
+  // random-sign masks of the tile: [0..3] columns (ROW layout), [4..7] rows (COL layout);
+  // the sign of column c is bit c/4 of word c%4
+  uint32_t* s_sgn = reinterpret_cast<uint32_t*>(s_red + 16);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bid = blockIdx.x, nctas = gridDim.x;
@@ -314,6 +417,8 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
     if (bid == 0 && tid == 0) {
       if constexpr (kRow) *a.s_row_out = S_r;
       if constexpr (kCol) *a.s_col_out = S_c;
+      if constexpr (kRow) if (a.amax_row_copy) *a.amax_row_copy = *a.amax_row;
+      if constexpr (kCol) if (a.amax_col_copy) *a.amax_col_copy = *a.amax_col;
     }
   }
   const float six_r = __fmul_rn(6.0f, S_r), six_c = __fmul_rn(6.0f, S_c);
@@ -344,6 +449,23 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
     const int tile = bid + it * nctas;
     const int tr = tile / a.tiles_c, tc = tile - tr * a.tiles_c;
     const int st = it % kQStages, ob = it & 1;
+    if (rht) {
+      // signs of this tile's 128 columns (warp 0) and 128 rows (warp 1): Philox block
+      // (tile start)/4 + lane holds the words of indices 4*lane .. 4*lane+3 of the tile.
+      // The previous tile's jobs read the masks before its store barrier.
+      if ((kRow && warp == 0) || (kCol && warp == 1)) {
+        const uint64_t first = static_cast<uint64_t>(warp == 0 ? tc : tr) * 32u;
+        const uint4 w = philox_block(first + lane, 0u, a.sign_key);
+        const uint32_t m0 = __ballot_sync(0xffffffffu, w.x >> 31);
+        const uint32_t m1 = __ballot_sync(0xffffffffu, w.y >> 31);
+        const uint32_t m2 = __ballot_sync(0xffffffffu, w.z >> 31);
+        const uint32_t m3 = __ballot_sync(0xffffffffu, w.w >> 31);
+        if (lane == 0) {
+          uint32_t* m = s_sgn + 4 * warp;
+          m[0] = m0; m[1] = m1; m[2] = m2; m[3] = m3;
+        }
+      }
+    }
     const bool ok = mbar_wait(&full[st], static_cast<uint32_t>((it / kQStages) & 1), a.wait_limit_ns);
     if (__syncthreads_or(!ok)) break;  // give up together; the status word says why
     const uint8_t* in = s_in + st * kQInBytes;
@@ -357,12 +479,32 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
       {
         float2 p[32];
         load_row_job(in, row_r, b, p);
+        if (rht) {
+          // lane x holds tile columns 64b + i, lane y 64b + 32 + i
+          const uint32_t m[4] = {s_sgn[0], s_sgn[1], s_sgn[2], s_sgn[3]};
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const uint32_t sx = (m[i & 3] >> (16 * b + (i >> 2))) & 1u;
+            const uint32_t sy = (m[i & 3] >> (16 * b + 8 + (i >> 2))) & 1u;
+            p[i] = make_float2(__uint_as_float(__float_as_uint(p[i].x) ^ (sx << 31)),
+                               __uint_as_float(__float_as_uint(p[i].y) ^ (sy << 31)));
+          }
+        }
         fwht_x2<HN, !kFoldH16>(p);
         if constexpr (AMAX) {
           const float2 m = amax_x2(p, 0, 32);
           amax_r = max3f(amax_r, m.x, m.y);
         } else {
-          const Enc e = kFoldH16 ? mx_encode_x2_h16fold(p) : encode_x2<FMT>(p, S_r, six_r);
+          Enc e;
+          if (sr) {
+            // element (row, column) of the ROW-layout matrix: word of index row*cols + column
+            const uint64_t f = (static_cast<uint64_t>(tr) * 128 + row_r) * static_cast<uint64_t>(a.cols) +
+                               static_cast<uint64_t>(tc) * 128 + 64 * b;
+            const SrCodes codes{f >> 2, (f >> 2) + 8, 1u, a.sr_key};
+            e = encode_x2<FMT, kFoldH16>(p, S_r, six_r, codes);
+          } else {
+            e = encode_x2<FMT, kFoldH16>(p, S_r, six_r);
+          }
           *reinterpret_cast<uint4*>(code_chunk(rcode, row_r, 2 * b)) = e.cx;
           *reinterpret_cast<uint4*>(code_chunk(rcode, row_r, 2 * b + 1)) = e.cy;
           if constexpr (FMT == kFmtMX)  // blocks 2b, 2b+1 of this row: adjacent bytes
@@ -378,12 +520,33 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
       {
         float2 p[32];
         load_col_job(in, col_b, col_w, s, p);
+        if (rht) {
+          // element i of both lanes is tile row 32s + i
+          const uint32_t m[4] = {s_sgn[4], s_sgn[5], s_sgn[6], s_sgn[7]};
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const uint32_t sg = ((m[i & 3] >> (8 * s + (i >> 2))) & 1u) << 31;
+            p[i] = make_float2(__uint_as_float(__float_as_uint(p[i].x) ^ sg),
+                               __uint_as_float(__float_as_uint(p[i].y) ^ sg));
+          }
+        }
         fwht_x2<HN, !kFoldH16>(p);
         if constexpr (AMAX) {
           const float2 m = amax_x2(p, 0, 32);
           amax_c = max3f(amax_c, m.x, m.y);
         } else {
-          const Enc e = kFoldH16 ? mx_encode_x2_h16fold(p) : encode_x2<FMT>(p, S_c, six_c);
+          Enc e;
+          if (sr) {
+            // element (column, row) of the COL-layout matrix: word of index column*rows + row
+            const uint64_t c0 = static_cast<uint64_t>(tc) * 128 + col_c;
+            const uint64_t r0 = static_cast<uint64_t>(tr) * 128 + 32 * s;
+            const uint64_t fx = c0 * static_cast<uint64_t>(a.rows) + r0;
+            const uint64_t fy = fx + static_cast<uint64_t>(a.rows);
+            const SrCodes codes{fx >> 2, fy >> 2, 2u, a.sr_key};
+            e = encode_x2<FMT, kFoldH16>(p, S_c, six_c, codes);
+          } else {
+            e = encode_x2<FMT, kFoldH16>(p, S_c, six_c);
+          }
           *reinterpret_cast<uint4*>(code_chunk(ccode, col_c, s)) = e.cx;
           *reinterpret_cast<uint4*>(code_chunk(ccode, col_c + 1, s)) = e.cy;
           // block kb of segment s: s (MXFP4, one byte) or 2s, 2s+1 (NVFP4, two bytes)

@@ -124,6 +124,58 @@ FP4_API fp4_status fp4_quantize_dual(const void *x_bf16, void *row_codes, void *
                              fp4_stream_t stream);
 
 /*
+ * Quantiser variants. The MXFP4 pre-training summary ("방법론" item 3 and "주요 기여
+ * 및 발견" section 2) names two stabilisers, stochastic rounding and randomised
+ * Hadamard rotations, which it tests and finds do not stabilise the full MXFP4
+ * pipeline. Neither is specified further there. These options implement the plainest
+ * deterministic-per-seed reading of each, plus a caller-supplied NVFP4 tensor amax.
+ *
+ * Random words: word(seed, index, stream) is word index%4 of Philox4x32-10 (Salmon et
+ * al., SC 2011) with counter (index/4 low 32 bits, index/4 high 32 bits, stream, 0)
+ * and key (seed low 32 bits, seed high 32 bits).
+ *
+ *   amax        NVFP4 only: a DEVICE float[1] (single layout) or float[2] {row, col}
+ *               (dual). It holds the tensor amax T of the rotated values of each
+ *               layout, supplied by the caller (e.g. from an earlier step), so the
+ *               amax pass is skipped. S = T/2688 as usual, and T is copied into the
+ *               amax slot(s) of tensor_scale. NULL = computed as in fp4_quantize.
+ *               It must be NULL for MXFP4 and 4-byte aligned.
+ *   stochastic  nonzero: each code's magnitude is rounded stochastically instead
+ *               of to nearest. |q| >= 6 gives 6. Otherwise, with lo the E2M1
+ *               magnitude below |q| and step the gap to the next one, the magnitude
+ *               rounds up iff (w >> 8) * 2^-24 < (|q| - lo) / step, where
+ *               w = word(sr_seed, i*C + c, 1 + axis) for element (i, c) of the
+ *               quantised [R][C] matrix (axis 0 = ROW, 1 = COL). Block scales are
+ *               unchanged. The NVFP4 quotient is the exact IEEE one.
+ *   random_signs nonzero: before the rotation, the element at index j along the
+ *               contraction axis (column j of the quantised [R][C] matrix) is
+ *               negated when bit 31 of word(sign_seed, j, 0) is set. Both operands
+ *               of one GEMM must use the same sign_seed; the product is then
+ *               unchanged, as for the plain rotation. The NVFP4 amax pass applies
+ *               the same signs.
+ *   sr_seed, sign_seed  the keys of the two variants.
+ * A NULL options pointer, or all fields zero, gives exactly fp4_quantize /
+ * fp4_quantize_dual. Errors: as fp4_quantize; FP4_ERR_INVALID_ARG for an amax with
+ * MXFP4, FP4_ERR_ALIGN for a misaligned amax.
+ */
+typedef struct fp4_quant_opts {
+    const float *amax;
+    int stochastic;
+    int random_signs;
+    uint64_t sr_seed;
+    uint64_t sign_seed;
+} fp4_quant_opts;
+
+FP4_API fp4_status fp4_quantize_opts(const void *x_bf16, void *codes, void *scales,
+                             float *tensor_scale, int64_t rows, int64_t cols, fp4_format fmt,
+                             int hadamard_n, fp4_axis axis, const fp4_quant_opts *opts,
+                             fp4_stream_t stream);
+FP4_API fp4_status fp4_quantize_dual_opts(const void *x_bf16, void *row_codes, void *row_scales,
+                                  void *col_codes, void *col_scales, float *tensor_scale,
+                                  int64_t rows, int64_t cols, fp4_format fmt, int hadamard_n,
+                                  const fp4_quant_opts *opts, fp4_stream_t stream);
+
+/*
  * fp4_gemm -- C[M][N] = deq(A)[M][K] * deq(B)[N][K]^T with fp32 accumulation on the
  * sm_100a block-scaled tensor cores (tcgen05.mma kind::mxf4 / kind::mxf4nvf4).
  * [MXFP4 pre-training summary, Methodology item 2; NVFP4/MaxText page, Key facts 5.]

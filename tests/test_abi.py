@@ -25,7 +25,7 @@ def test_every_header_symbol_is_exported():
     L = ctypes.CDLL(fp4.LIB_PATH)
     for s in syms:
         assert hasattr(L, s), s
-    assert fp4.lib().fp4_abi_version() == 1
+    assert fp4.lib().fp4_abi_version() == 2
 
 
 def test_status_strings():
@@ -73,6 +73,24 @@ def test_quantize_dual_validation():
     assert L.fp4_quantize_dual(A16, A16, A16, None, A16, None, 64, 64, 0, 16, None) == INVALID
     assert L.fp4_quantize_dual(A16, A16, A16, A16, MIS, None, 64, 64, 0, 16, None) == ALIGN
     assert L.fp4_quantize_dual(A16, A16, A16, A16, A16, None, 64, 80, 0, 16, None) == SHAPE
+
+
+def qo(opts, fmt=0, ts=None, x=A16):
+    return fp4.lib().fp4_quantize_opts(x, A16, A16, ts, 64, 64, fmt, 16, 0, opts, None)
+
+
+def test_quantize_opts_validation():
+    L = fp4.lib()
+    amax_mx = fp4.QuantOpts(A16, 0, 0, 0, 0)
+    assert qo(ctypes.byref(amax_mx)) == INVALID               # a tensor amax is NVFP4 only
+    mis = fp4.QuantOpts(A16 + 2, 0, 0, 0, 0)
+    assert qo(ctypes.byref(mis), fmt=1, ts=A16) == ALIGN      # amax must be 4-byte aligned
+    sr = fp4.QuantOpts(None, 1, 1, 5, 6)
+    assert qo(ctypes.byref(sr), x=MIS) == ALIGN               # the plain checks still apply
+    assert qo(ctypes.byref(sr), fmt=1, ts=None) == INVALID
+    assert L.fp4_quantize_dual_opts(A16, A16, A16, None, A16, None, 64, 64, 0, 16,
+                                    ctypes.byref(sr), None) == INVALID
+    assert L.fp4_quantize_opts(A16, A16, A16, None, 0, 64, 0, 16, 0, ctypes.byref(sr), None) == OK
 
 
 def g(A=A16, As=A16, Ats=None, B=A16, Bs=A16, Bts=None, C=A16, M=128, N=128, K=128, fmt=0, od=0):
