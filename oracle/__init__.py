@@ -17,9 +17,9 @@ import subprocess
 
 import numpy as np
 
-MXFP4, NVFP4 = 0, 1
+MXFP4, NVFP4, MXFP8 = 0, 1, 2
 ROW, COL = 0, 1
-BLOCK = {MXFP4: 32, NVFP4: 16}
+BLOCK = {MXFP4: 32, NVFP4: 16, MXFP8: 32}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "fp4_oracle.c")
@@ -77,6 +77,8 @@ def _L():
         lib.fp4o_quantize_ex.restype = ctypes.c_int
         lib.fp4o_quantize_ex.argtypes = [P, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          P, P, P, P, P]
+        lib.fp4o_quantize_mxfp8.restype = ctypes.c_int
+        lib.fp4o_quantize_mxfp8.argtypes = [P, i64, i64, ctypes.c_int, ctypes.c_int, P, P]
         lib.fp4o_rotated_amax.restype = ctypes.c_float
         lib.fp4o_rotated_amax.argtypes = [P, i64, i64, ctypes.c_int, ctypes.c_int]
         u64, u32 = ctypes.c_uint64, ctypes.c_uint32
@@ -259,6 +261,13 @@ def quantize(x, fmt: int, hn: int, axis: int = ROW, amax: float | None = None,
     rows, cols = xb.shape
     R, C = (rows, cols) if axis == ROW else (cols, rows)
     bs = BLOCK[fmt]
+    if fmt == MXFP8:
+        assert amax is None and sr_seed is None and rht_seed is None
+        codes = np.zeros((R, C), np.uint8)
+        scales = np.zeros(scale_layout_bytes(R, C // bs), np.uint8)
+        if _L().fp4o_quantize_mxfp8(_ptr(xb), rows, cols, hn, axis, _ptr(codes), _ptr(scales)):
+            raise ValueError(f"oracle quantize rejected shape {xb.shape} fmt={fmt} hn={hn}")
+        return codes, scales, None, None
     codes = np.zeros((R, C // 2), np.uint8)
     scales = np.zeros(scale_layout_bytes(R, C // bs), np.uint8)
     s = np.zeros(1, np.float32)
@@ -276,11 +285,12 @@ def quantize(x, fmt: int, hn: int, axis: int = ROW, amax: float | None = None,
 
 
 def dequantize(codes: np.ndarray, scales: np.ndarray, tensor_scale, fmt: int) -> np.ndarray:
-    R, C2 = codes.shape
-    out = np.empty((R, 2 * C2), np.float64)
+    R, W = codes.shape
+    C = W if fmt == MXFP8 else 2 * W  # MXFP8: one code byte per element
+    out = np.empty((R, C), np.float64)
     ts = 1.0 if tensor_scale is None else float(tensor_scale)
     _L().fp4o_dequantize(_ptr(np.ascontiguousarray(codes)), _ptr(np.ascontiguousarray(scales)),
-                         ts, R, 2 * C2, fmt, _ptr(out))
+                         ts, R, C, fmt, _ptr(out))
     return out
 
 
@@ -300,7 +310,7 @@ def gemm_entries(a_q, b_q, fmt: int, ms, ns) -> np.ndarray:
     a_q = (codes, scales, S) of A [M][K] and b_q likewise of B [N][K]."""
     ac, asc, ats = a_q
     bc, bsc, bts = b_q
-    K = ac.shape[1] * 2
+    K = ac.shape[1] if fmt == MXFP8 else ac.shape[1] * 2
     ms = np.ascontiguousarray(ms, dtype=np.int64)
     ns = np.ascontiguousarray(ns, dtype=np.int64)
     out = np.empty(ms.size, np.float64)
