@@ -35,6 +35,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "FP4 GEMM TFLOPS (fprop/dgrad/wgrad) + H16-quantize GB/s, % of B200 roofline"
 FP4_OVER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput (9 : 2.25 PFLOP/s)
+FP8_OVER_BF16 = 2.0  # nominal dense FP8 : BF16 (4.5 : 2.25 PFLOP/s), for the MXFP8 comparator
+FORMATS = {"mxfp4": 0, "nvfp4": 1, "mxfp8": 2}
 PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 WORKLOAD = ("llama3.1-8b layer fwd+bwd: qkv 6144x4096, o 4096x4096, gate/up 14336x4096, "
             "down 4096x14336; 8192 tokens/rank; MXFP4 + H16")
@@ -57,7 +59,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["fp4", "reference"], default="fp4")
-    ap.add_argument("--format", choices=["mxfp4", "nvfp4"], default="mxfp4")
+    ap.add_argument("--format", choices=list(FORMATS), default="mxfp4",
+                    help="mxfp8 = the FP8 comparator (E4M3, E8M0 scale per 32) on the same step")
     ap.add_argument("--hadamard", type=int, default=16, choices=[0, 16, 32])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -187,7 +190,7 @@ class LlamaLayer:
 
     def _qbuf(self, r, c, device):
         f = self.fp4
-        return (torch.empty(r, c // 2, dtype=torch.uint8, device=device),
+        return (torch.empty(r, c if self.fmt == 2 else c // 2, dtype=torch.uint8, device=device),
                 torch.empty(f.fp4_scales_bytes(r, c, self.fmt), dtype=torch.uint8, device=device))
 
     def flops(self):
@@ -322,7 +325,7 @@ def run_reference(a):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    fmt = 0 if a.format == "mxfp4" else 1
+    fmt = FORMATS[a.format]
     from fp4_block_scaled_deterministic_b200 import synthetic
     flops = sum(3 * 2.0 * 8192 * N * K for _, N, K in synthetic.LLAMA_LAYERS)
     budget = min(20.0, max(2.0, 120.0 / (a.steps + a.warmup)))
@@ -390,7 +393,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     import fp4_block_scaled_deterministic_b200 as fp4
     fp4.lib()  # fails loudly if the library is missing
-    fmt = 0 if a.format == "mxfp4" else 1
+    fmt = FORMATS[a.format]
     names = [n.strip() for n in a.proj.split(",") if n.strip()]
     layer = LlamaLayer(dev, fmt, a.hadamard, seed=1000 * rank, names=names, variant=a.variant)
     stream = torch.cuda.current_stream(dev)
@@ -432,21 +435,26 @@ def main():
     per_launch_flops = gemm_flops_of(layer) * a.steps
     gemm_tflops = sum(per_launch_flops) / (sum(gemm_ms) * 1e-3) / 1e12
     amax_pass = fmt == 1 and a.variant != "amax"
-    bpe = 2.0 + 2 * (0.5 + (1 / 32 if fmt == 0 else 1 / 16)) + (2.0 if amax_pass else 0.0)
+    code_b = 1.0 if fmt == 2 else 0.5                   # bytes per code
+    scale_b = 1 / 16 if fmt == 1 else 1 / 32            # scale bytes per element
+    bpe = 2.0 + 2 * (code_b + scale_b) + (2.0 if amax_pass else 0.0)
     q_bytes = layer.quant_elems() * bpe * a.steps
     quant_gbs = q_bytes / (sum(quant_ms) * 1e-3) / 1e9
 
     pk, pk_kind = peaks()
-    peak_fp4 = pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) * FP4_OVER_BF16
+    ratio = FP8_OVER_BF16 if fmt == 2 else FP4_OVER_BF16
+    peak_fp4 = pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) * ratio
     avg_launch_ms = sum(gemm_ms) / len(gemm_ms)
     avg_flops = sum(per_launch_flops) / len(per_launch_flops)
     traffic = recorded_traffic("mxfp4" if fmt == 0 else "nvfp4") if a.hadamard == 16 and len(names) == 5 else None
     roof = {"bound": "tensor", "achieved": gemm_tflops, "peak": peak_fp4, "unit": "TFLOP/s",
             "frac": gemm_tflops / peak_fp4, "traffic": traffic,
-            "kernel": "gemm_fp4_pair_kernel (tcgen05 block-scaled FP4, CTA pairs)",
+            "kernel": "gemm_fp4_pair_kernel (tcgen05 block-scaled "
+                      f"{'MXFP8, kind::mxf8f6f4' if fmt == 2 else 'FP4'}, CTA pairs)",
             "per_launch": {"avg_flops": avg_flops, "avg_ms": avg_launch_ms,
                            "launches": len(gemm_ms)},
-            "peak_source": f"{pk_kind}: bf16_tflops_sustained x {FP4_OVER_BF16} (nominal FP4:BF16)"}
+            "peak_source": f"{pk_kind}: bf16_tflops_sustained x {ratio} (nominal "
+                           f"{'FP8' if fmt == 2 else 'FP4'}:BF16)"}
     qroof = {"bound": "hbm", "achieved": quant_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
              "frac": quant_gbs / pk["hbm_gbs"], "bytes_per_elem": bpe,
              "kernel": "quantize_kernel dual layout", "launches": len(quant_ms),
@@ -454,7 +462,7 @@ def main():
 
     out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
            "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms / a.steps,
-           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp4_e2m1",
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3" if fmt == 2 else "fp4_e2m1",
            "data": "synthetic",
            "config": {"workload": workload_name(a) if len(names) == 5 else
                       f"subset {','.join(names)} of: {workload_name(a)}",

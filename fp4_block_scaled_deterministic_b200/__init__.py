@@ -20,11 +20,11 @@ from dataclasses import dataclass
 
 import torch
 
-MXFP4, NVFP4 = 0, 1
+MXFP4, NVFP4, MXFP8 = 0, 1, 2  # MXFP8: the FP8 comparator (E4M3 codes, one byte each)
 ROW, COL = 0, 1
 OUT_F32, OUT_BF16 = 0, 1
 FPROP, DGRAD, WGRAD = 0, 1, 2
-BLOCK = {MXFP4: 32, NVFP4: 16}
+BLOCK = {MXFP4: 32, NVFP4: 16, MXFP8: 32}
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libfp4.so")
@@ -63,6 +63,7 @@ def lib() -> ctypes.CDLL:
         sig = {
             "fp4_abi_version": (I32, []),
             "fp4_codes_bytes": (SZ, [I64, I64]),
+            "fp4_codes_bytes_fmt": (SZ, [I64, I64, I32]),
             "fp4_scales_bytes": (SZ, [I64, I64, I32]),
             "fp4_quantize": (I32, [P, P, P, P, I64, I64, I32, I32, I32, P]),
             "fp4_quantize_dual": (I32, [P, P, P, P, P, P, I64, I64, I32, I32, P]),
@@ -209,7 +210,8 @@ class QTensor:
 
 
 def _alloc_q(rows, cols, fmt, device):
-    codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=device)
+    codes = torch.empty(rows, cols if fmt == MXFP8 else cols // 2, dtype=torch.uint8,
+                        device=device)
     scales = torch.empty(max(1, fp4_scales_bytes(rows, cols, fmt)), dtype=torch.uint8, device=device)
     return codes, scales
 

@@ -14,7 +14,8 @@
 namespace fp4k {
 
 // Element formats of the kernels' template parameter.
-enum { kFmtMX = 0, kFmtNV = 1 };
+// kFmtMX8: the MXFP8 comparator (E4M3 elements, E8M0 scale per 32 elements)
+enum { kFmtMX = 0, kFmtNV = 1, kFmtMX8 = 2 };
 
 // ------------------------------------------------------------------ status word
 // Bit flags recorded by kernels instead of trapping; read and cleared by the host.
@@ -356,21 +357,28 @@ __device__ __forceinline__ void tc_cp_32x128b_warpx4_pair(uint32_t taddr, uint64
 }
 // Block-scaled FP4 MMA over a CTA pair: M = 256 (128 rows per CTA), N up to 256 with B
 // split between the two CTAs' shared memory.
-template <bool kMX>
+template <int FMT>
 __device__ __forceinline__ void tc_mma_fp4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                                 uint32_t idesc, uint32_t sfa_tmem,
                                                 uint32_t sfb_tmem, uint32_t accumulate) {
-  if constexpr (kMX) {
+  if constexpr (FMT == kFmtMX) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;"
         "\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
         : "memory");
-  } else {
+  } else if constexpr (FMT == kFmtNV) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], "
+        "[%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale.block32 [%0], %1, %2, %3, [%5], "
         "[%6], p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
         : "memory");

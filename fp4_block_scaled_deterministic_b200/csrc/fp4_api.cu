@@ -100,7 +100,12 @@ cudaError_t ensure_smem(K kernel, int bytes, int dev, std::atomic<uint64_t>& don
 }
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
-inline int block_of(fp4_format f) { return f == FP4_MXFP4 ? 32 : 16; }
+inline int block_of(fp4_format f) { return f == FP4_NVFP4 ? 16 : 32; }
+inline bool valid_format(fp4_format f) {
+  return f == FP4_MXFP4 || f == FP4_NVFP4 || f == FP4_MXFP8;
+}
+// code bytes per element: 1/2 (FP4) or 1 (MXFP8)
+inline int64_t code_bytes(int64_t elems, fp4_format f) { return f == FP4_MXFP8 ? elems : elems / 2; }
 
 // ---------------------------------------------------------------- quantise launch
 template <int FMT, int HN, int MODE, bool AMAX, bool EXT>
@@ -108,9 +113,10 @@ cudaError_t launch_q(const CUtensorMap& ti, const CUtensorMap& tr, const CUtenso
                      const QuantArgs& a, int grid, int dev, cudaStream_t s) {
   static std::atomic<uint64_t> done{0};
   auto k = quantize_kernel<FMT, HN, MODE, AMAX, EXT>;
-  cudaError_t e = ensure_smem(k, kQSmemBytes, dev, done);
+  constexpr int smem = kQSmemBytesOf(FMT);
+  cudaError_t e = ensure_smem(k, smem, dev, done);
   if (e != cudaSuccess) return e;
-  k<<<grid, kQThreads, kQSmemBytes, s>>>(ti, tr, tc, a);
+  k<<<grid, kQThreads, smem, s>>>(ti, tr, tc, a);
   return cudaGetLastError();
 }
 
@@ -147,7 +153,7 @@ cudaError_t dispatch_hn(int hn, int mode, const CUtensorMap& ti, const CUtensorM
 
 fp4_status validate_quant_common(const void* x, int64_t rows, int64_t cols, fp4_format fmt,
                                  int hn) {
-  if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
+  if (!valid_format(fmt)) return FP4_ERR_INVALID_ARG;
   if (hn != 0 && hn != 16 && hn != 32) return FP4_ERR_INVALID_ARG;
   if (rows < 0 || cols < 0) return FP4_ERR_SHAPE;
   if (rows % 32 != 0 || cols % 32 != 0) return FP4_ERR_SHAPE;
@@ -164,8 +170,10 @@ fp4_status quantize_impl(const void* x, void* rcodes, void* rscales, void* ccode
   fp4_status st = validate_quant_common(x, rows, cols, fmt, hn);
   if (st != FP4_OK) return st;
   const bool do_row = mode & kModeRow, do_col = mode & kModeCol;
-  if (fmt == FP4_MXFP4 && ts) return FP4_ERR_INVALID_ARG;
+  if (fmt != FP4_NVFP4 && ts) return FP4_ERR_INVALID_ARG;
   if (fmt == FP4_NVFP4 && !ts) return FP4_ERR_INVALID_ARG;
+  if (fmt == FP4_MXFP8 && opts && (opts->amax || opts->stochastic || opts->random_signs))
+    return FP4_ERR_INVALID_ARG;
   const float* amax_in = opts ? opts->amax : nullptr;
   if (amax_in && fmt != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
   if (amax_in && (reinterpret_cast<uintptr_t>(amax_in) & 3u)) return FP4_ERR_ALIGN;
@@ -187,11 +195,15 @@ fp4_status quantize_impl(const void* x, void* rcodes, void* rscales, void* ccode
   if (!make_map_2d(&tm_in, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, cols, rows, 64, 128,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return FP4_ERR_CUDA;
-  if (do_row && !make_map_2d(&tm_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rcodes, cols / 2, rows, 64,
-                             128, CU_TENSOR_MAP_SWIZZLE_64B))
+  // code tiles: 128 rows x 64 bytes (FP4, 64B swizzle) or x 128 bytes (MXFP8, 128B swizzle)
+  const uint32_t cbox = fmt == FP4_MXFP8 ? 128 : 64;
+  const CUtensorMapSwizzle csw = fmt == FP4_MXFP8 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                                  : CU_TENSOR_MAP_SWIZZLE_64B;
+  if (do_row && !make_map_2d(&tm_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rcodes,
+                             code_bytes(cols, fmt), rows, cbox, 128, csw))
     return FP4_ERR_CUDA;
-  if (do_col && !make_map_2d(&tm_c, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ccodes, rows / 2, cols, 64,
-                             128, CU_TENSOR_MAP_SWIZZLE_64B))
+  if (do_col && !make_map_2d(&tm_c, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ccodes,
+                             code_bytes(rows, fmt), cols, cbox, 128, csw))
     return FP4_ERR_CUDA;
 
   const int bs = block_of(fmt);
@@ -216,12 +228,18 @@ fp4_status quantize_impl(const void* x, void* rcodes, void* rscales, void* ccode
     a.sign_key[0] = static_cast<uint32_t>(opts->sign_seed);
     a.sign_key[1] = static_cast<uint32_t>(opts->sign_seed >> 32);
   }
-  const int resident = kQCtasPerSM * info->sm_count;
+  const int resident = (fmt == FP4_MXFP8 ? kQCtasPerSMOf(kFmtMX8) : kQCtasPerSM) * info->sm_count;
   const int grid = a.num_tiles < resident ? a.num_tiles : resident;
 
   cudaError_t e = cudaSuccess;
   if (fmt == FP4_MXFP4) {
     e = dispatch_hn<kFmtMX, false>(hn, mode, tm_in, tm_r, tm_c, a, grid, dev, stream);
+  } else if (fmt == FP4_MXFP8) {
+    switch (hn) {
+      case 0: e = dispatch_mode<kFmtMX8, 0, false, false>(mode, tm_in, tm_r, tm_c, a, grid, dev, stream); break;
+      case 16: e = dispatch_mode<kFmtMX8, 16, false, false>(mode, tm_in, tm_r, tm_c, a, grid, dev, stream); break;
+      default: e = dispatch_mode<kFmtMX8, 32, false, false>(mode, tm_in, tm_r, tm_c, a, grid, dev, stream);
+    }
   } else {
     // ts layout: single -> {S, amax}; dual -> {S_row, S_col, amax_row, amax_col}
     float* amax_r = nullptr;
@@ -318,8 +336,8 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a, const CUtensorMap& b, const C
 // is taken.
 constexpr double kL2PanelBudget = 40.0 * (1 << 20);
 
-void choose_tile_order(GemmArgs& g, int64_t tile_rows, int64_t K, int block) {
-  const double row_bytes = double(K / 2 + K / block);
+void choose_tile_order(GemmArgs& g, int64_t tile_rows, int64_t row_bytes_i) {
+  const double row_bytes = double(row_bytes_i);  // code + scale bytes of one operand row
   const double panel_a = double(tile_rows) * row_bytes, panel_b = double(kGBN) * row_bytes;
   auto fit = [](double panel, int tiles) {
     const double n = kL2PanelBudget / panel;
@@ -336,13 +354,13 @@ void choose_tile_order(GemmArgs& g, int64_t tile_rows, int64_t K, int block) {
 fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void* B,
                      const void* Bs, const float* Bts, void* C, int64_t M, int64_t N, int64_t K,
                      fp4_format fmt, fp4_out_dtype od, cudaStream_t stream) {
-  if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
+  if (!valid_format(fmt)) return FP4_ERR_INVALID_ARG;
   if (od != FP4_OUT_F32 && od != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || K < 0 || M % 32 || N % 32 || K % 32) return FP4_ERR_SHAPE;
   if (M > (int64_t(1) << 31) - 256 || N > (int64_t(1) << 31) - 256 ||
       K > (int64_t(1) << 31) - 256)
     return FP4_ERR_SHAPE;
-  if (fmt == FP4_MXFP4 && (Ats || Bts)) return FP4_ERR_INVALID_ARG;
+  if (fmt != FP4_NVFP4 && (Ats || Bts)) return FP4_ERR_INVALID_ARG;
   if (fmt == FP4_NVFP4 && (!Ats || !Bts)) return FP4_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return FP4_OK;
   if (!C) return FP4_ERR_INVALID_ARG;
@@ -359,15 +377,20 @@ fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void
   const int64_t kb4 = ceil_div(K / bs, 4);
   // Rows of 256 (M > 128) go to the CTA-pair kernel; a single 128-row band of M to the
   // one-CTA kernel. Each kernel has its own K per pipeline stage.
-  const bool pair = M > 128;
-  const int slab_k = !pair ? kGBK : (fmt == FP4_MXFP4 ? PairCfg<kFmtMX>::kSlabK
-                                                      : PairCfg<kFmtNV>::kSlabK);
+  // (The MXFP8 comparator always takes the pair kernel; M <= 128 is then one zero-filled
+  // 256-row band.)
+  const bool pair = M > 128 || fmt == FP4_MXFP8;
+  const int slab_k = !pair ? kGBK
+                     : fmt == FP4_MXFP4 ? PairCfg<kFmtMX>::kSlabK
+                     : fmt == FP4_NVFP4 ? PairCfg<kFmtNV>::kSlabK
+                                        : PairCfg<kFmtMX8>::kSlabK;
   const int atoms = slab_k / (4 * bs);
   const uint32_t b_box_rows = pair ? 128 : kGBN;
+  const int64_t kbytes = code_bytes(K, fmt);
   CUtensorMap ta, tb, tsa, tsb;
-  if (!make_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K / 2, M, kGBK / 2, kGBM,
+  if (!make_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, kbytes, M, 128, kGBM,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K / 2, N, kGBK / 2, b_box_rows,
+      !make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, kbytes, N, 128, b_box_rows,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&tsa, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, As, kb4 * 64, ceil_div(M, 128),
                    atoms * 64, 1, CU_TENSOR_MAP_SWIZZLE_NONE) ||
@@ -385,7 +408,7 @@ fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void
   if (tiles > INT32_MAX) return FP4_ERR_SHAPE;
   g.num_tiles = static_cast<int>(tiles);
   g.k_tiles = static_cast<int>(ceil_div(K, slab_k));
-  choose_tile_order(g, pair ? 256 : kGBM, K, block_of(fmt));
+  choose_tile_order(g, pair ? 256 : kGBM, kbytes + K / bs);
   g.C = C;
   g.c_v8 = (reinterpret_cast<uintptr_t>(C) & 31) == 0 ? 1 : 0;
   g.sa = Ats;
@@ -398,6 +421,9 @@ fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void
     if (fmt == FP4_MXFP4)
       e = od == FP4_OUT_F32 ? launch_gemm_pair<kFmtMX, 0>(ta, tb, tsa, tsb, g, dev, stream)
                             : launch_gemm_pair<kFmtMX, 1>(ta, tb, tsa, tsb, g, dev, stream);
+    else if (fmt == FP4_MXFP8)
+      e = od == FP4_OUT_F32 ? launch_gemm_pair<kFmtMX8, 0>(ta, tb, tsa, tsb, g, dev, stream)
+                            : launch_gemm_pair<kFmtMX8, 1>(ta, tb, tsa, tsb, g, dev, stream);
     else
       e = od == FP4_OUT_F32 ? launch_gemm_pair<kFmtNV, 0>(ta, tb, tsa, tsb, g, dev, stream)
                             : launch_gemm_pair<kFmtNV, 1>(ta, tb, tsa, tsb, g, dev, stream);
@@ -423,9 +449,9 @@ struct WsPlan {
 WsPlan plan_ws(int64_t ra, int64_t rb, int64_t kc, fp4_format fmt) {
   WsPlan p;
   size_t off = 0;
-  p.a_codes = off;  off += align256(fp4_codes_bytes(ra, kc));
+  p.a_codes = off;  off += align256(fp4_codes_bytes_fmt(ra, kc, fmt));
   p.a_scales = off; off += align256(fp4_scales_bytes(ra, kc, fmt));
-  p.b_codes = off;  off += align256(fp4_codes_bytes(rb, kc));
+  p.b_codes = off;  off += align256(fp4_codes_bytes_fmt(rb, kc, fmt));
   p.b_scales = off; off += align256(fp4_scales_bytes(rb, kc, fmt));
   p.ts = off;       off += 256;
   p.total = off;
@@ -444,7 +470,7 @@ void pass_dims(fp4_pass pass, int64_t M, int64_t N, int64_t K, int64_t* ra, int6
 fp4_status linear_impl(fp4_pass pass, const void* P, const void* Q, void* out, int64_t M,
                        int64_t N, int64_t K, fp4_format fmt, int hn, fp4_out_dtype od, void* ws,
                        size_t ws_bytes, cudaStream_t stream) {
-  if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
+  if (!valid_format(fmt)) return FP4_ERR_INVALID_ARG;
   if (hn != 0 && hn != 16 && hn != 32) return FP4_ERR_INVALID_ARG;
   if (od != FP4_OUT_F32 && od != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || K < 0 || M % 32 || N % 32 || K % 32) return FP4_ERR_SHAPE;
@@ -540,6 +566,11 @@ size_t fp4_codes_bytes(int64_t rows, int64_t cols) {
   return static_cast<size_t>(rows) * static_cast<size_t>(cols) / 2;
 }
 
+size_t fp4_codes_bytes_fmt(int64_t rows, int64_t cols, fp4_format fmt) {
+  if (rows <= 0 || cols <= 0 || !valid_format(fmt)) return 0;
+  return static_cast<size_t>(rows) * static_cast<size_t>(code_bytes(cols, fmt));
+}
+
 size_t fp4_scales_bytes(int64_t rows, int64_t cols, fp4_format fmt) {
   if (rows <= 0 || cols <= 0) return 0;
   const int64_t kb = cols / block_of(fmt);
@@ -589,7 +620,7 @@ fp4_status fp4_gemm(const void* A, const void* As, const float* Ats, const void*
 
 size_t fp4_linear_workspace_size(fp4_pass pass, int64_t M, int64_t N, int64_t K, fp4_format fmt) {
   if (pass != FP4_PASS_FPROP && pass != FP4_PASS_DGRAD && pass != FP4_PASS_WGRAD) return 0;
-  if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return 0;
+  if (!valid_format(fmt)) return 0;
   if (M < 0 || N < 0 || K < 0) return 0;
   int64_t ra, rb, kc;
   pass_dims(pass, M, N, K, &ra, &rb, &kc);

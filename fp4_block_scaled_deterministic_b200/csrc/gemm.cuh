@@ -106,10 +106,13 @@ __device__ __forceinline__ constexpr uint32_t idesc_fp4() {
 
 
 // Instruction descriptor of the pair MMA: as idesc_fp4 with M = 256.
+// Operand formats [7,10) and [10,13): E2M1 = 1 for the mxf4 kinds, E4M3 = 0 for
+// kind::mxf8f6f4; scale type [23]: UE8M0 (MX formats) or UE4M3 (NVFP4).
 template <int FMT>
 __device__ __forceinline__ constexpr uint32_t idesc_fp4_pair() {
-  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(256 >> 3) << 17) |
-         ((FMT == kFmtMX ? 1u : 0u) << 23) | (static_cast<uint32_t>(256 >> 4) << 24);
+  constexpr uint32_t ab = FMT == kFmtMX8 ? 0u : 1u;
+  return (ab << 7) | (ab << 10) | (static_cast<uint32_t>(256 >> 3) << 17) |
+         ((FMT == kFmtNV ? 0u : 1u) << 23) | (static_cast<uint32_t>(256 >> 4) << 24);
 }
 
 
@@ -129,8 +132,8 @@ struct SlabCursor {
 template <int FMT, bool PAIR, int SLAB_K, int STAGES, int A_BYTES, int B_BYTES, int SFA_BYTES,
           int SFB_BYTES, int SF_COLS, int SF_BUFS>
 struct Issuer {
-  static constexpr int kAtoms = SLAB_K / (4 * (FMT == kFmtMX ? 32 : 16));
-  static constexpr int kMMAs = SLAB_K / 64;
+  static constexpr int kAtoms = SLAB_K / (4 * (FMT == kFmtNV ? 16 : 32));
+  static constexpr int kMMAs = SLAB_K / (FMT == kFmtMX8 ? 32 : 64);  // K per MMA: 32 B of codes
   static constexpr int kCopies = 3 * kAtoms;  // A atoms, then B atoms of row blocks 0 and 1
 
   __device__ __forceinline__ static void step(SlabCursor& c, const SlabCursor& base) {
@@ -163,13 +166,17 @@ struct Issuer {
       else tc_cp_32x128b_warpx4(t, d);
     }
   }
-  // MMA j of a slab: K elements [64j, 64j+64).
+  // MMA j of a slab: code bytes [32j, 32j+32) of each row (K elements [64j, 64j+64) of
+  // FP4, [32j, 32j+32) of FP8).
   __device__ __forceinline__ static void mma(const SlabCursor& c, uint32_t tmem_acc, int j,
                                              bool first) {
     // MXFP4: two MMAs share one atom column, bytes {0,1} then {2,3} (scale id 0 / 2);
-    // NVFP4: one atom column per MMA, all four bytes (scale id 0).
-    const int at = FMT == kFmtMX ? (j >> 1) : j;
-    const uint32_t id = FMT == kFmtMX ? static_cast<uint32_t>((j & 1) * 2) : 0u;
+    // NVFP4: one atom column per MMA, all four bytes (scale id 0);
+    // MXFP8: four MMAs share one atom column, one byte each (scale id 0..3).
+    const int at = FMT == kFmtMX ? (j >> 1) : FMT == kFmtNV ? j : (j >> 2);
+    const uint32_t id = FMT == kFmtMX    ? static_cast<uint32_t>((j & 1) * 2)
+                        : FMT == kFmtMX8 ? static_cast<uint32_t>(j & 3)
+                                         : 0u;
     const uint32_t tsfa = (c.t_sf + 4 * at) | (id << 30);
     const uint32_t tsfb = (c.t_sf + 4 * kAtoms + 8 * at) | (id << 30);
     constexpr uint32_t kIdesc = PAIR ? idesc_fp4_pair<FMT>() : idesc_fp4<FMT>();
@@ -177,7 +184,7 @@ struct Issuer {
     const uint64_t koff = (j >> 2) * (128 * 128 >> 4) + 2 * (j & 3);
     const uint32_t acc = first ? 0u : 1u;
     if constexpr (PAIR)
-      tc_mma_fp4_pair<FMT == kFmtMX>(tmem_acc, c.dA + koff, c.dB + koff, idesc, tsfa, tsfb, acc);
+      tc_mma_fp4_pair<FMT>(tmem_acc, c.dA + koff, c.dB + koff, idesc, tsfa, tsfb, acc);
     else
       tc_mma_fp4<FMT == kFmtMX>(tmem_acc, c.dA + koff, c.dB + koff, idesc, tsfa, tsfb, acc);
   }
@@ -435,18 +442,20 @@ __global__ void __launch_bounds__(kGThreads, 1)
 // two CTAs of the pair.
 template <int FMT>
 struct PairCfg {
-  static constexpr int kBlock = FMT == kFmtMX ? 32 : 16;
+  static constexpr int kBlock = FMT == kFmtNV ? 16 : 32;
   // K per stage: 512 for MXFP4 (8 MMAs per barrier wait and commit, 3 stages), 256 for
-  // NVFP4 (whose scale copies are twice as many per K; 5 stages).
-  static constexpr int kSlabK = FMT == kFmtMX ? 512 : 256;
-  static constexpr int kSub = kSlabK / 256;          // 128-byte-wide swizzled sub-tiles
+  // NVFP4 (whose scale copies are twice as many per K; 5 stages), 256 for MXFP8 (the
+  // same 256 code bytes per row as MXFP4, 8 MMAs of K = 32; 3 stages).
+  static constexpr int kSlabK = FMT == kFmtNV ? 256 : (FMT == kFmtMX ? 512 : 256);
+  static constexpr int kRowBytes = FMT == kFmtMX8 ? kSlabK : kSlabK / 2;  // code bytes/row
+  static constexpr int kSub = kRowBytes / 128;       // 128-byte-wide swizzled sub-tiles
   static constexpr int kAtoms = kSlabK / (4 * kBlock);
-  static constexpr int kABytes = 128 * kSlabK / 2;   // this CTA's 128 rows of A
-  static constexpr int kBBytes = 128 * kSlabK / 2;   // this CTA's 128-row half of B
+  static constexpr int kABytes = 128 * kRowBytes;    // this CTA's 128 rows of A
+  static constexpr int kBBytes = 128 * kRowBytes;    // this CTA's 128-row half of B
   static constexpr int kSFABytes = kAtoms * 512;     // scales of this CTA's A rows
   static constexpr int kSFBBytes = 2 * kAtoms * 512; // scales of all 256 B rows
   static constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
-  static constexpr int kStages = FMT == kFmtMX ? 3 : 5;
+  static constexpr int kStages = FMT == kFmtNV ? 5 : 3;
   static constexpr int kSFCols = 12 * kAtoms;
   static constexpr int kSFBufs = 4;
   static constexpr int kTmemSF = 256;
@@ -523,7 +532,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
           const uint32_t bar = leader_full + 8u * stage;
 #pragma unroll
           for (int sub = 0; sub < Cfg::kSub; ++sub) {
-            const int kx = kt * (Cfg::kSlabK / 2) + 128 * sub;
+            const int kx = kt * Cfg::kRowBytes + 128 * sub;
             tma_load_2d_pair(sA + stage * Cfg::kABytes + sub * 16384, &tmA, bar, kx,
                              tm * 256 + 128 * static_cast<int>(rank));
             tma_load_2d_pair(sB + stage * Cfg::kBBytes + sub * 16384, &tmB, bar, kx,

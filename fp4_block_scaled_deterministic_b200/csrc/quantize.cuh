@@ -34,10 +34,16 @@ constexpr int kQCtasPerSM = 2;
 constexpr int kQStages = 2;
 constexpr int kQBoxBytes = 128 * 64 * 2;    // 128 rows x 64 bf16
 constexpr int kQInBytes = 2 * kQBoxBytes;   // a 128 x 128 bf16 tile
-constexpr int kQCodeBytes = 128 * 64;       // 128 rows x 64 code bytes
 constexpr int kQScaleBytes = 1024;          // up to two 512-byte atoms
-constexpr int kQSmemBytes = 1024 /*align*/ + kQStages * kQInBytes + 2 * 2 * kQCodeBytes +
-                            2 * 2 * kQScaleBytes + 256;
+// Staged code tile: 128 rows x 64 code bytes (FP4, 64B swizzle) or x 128 bytes (MXFP8,
+// 128B swizzle). With the larger MXFP8 staging one CTA fits per SM.
+__host__ __device__ constexpr int kQCodeBytesOf(int fmt) { return fmt == kFmtMX8 ? 128 * 128 : 128 * 64; }
+__host__ __device__ constexpr int kQSmemBytesOf(int fmt) {
+  return 1024 /*align*/ + kQStages * kQInBytes + 2 * 2 * kQCodeBytesOf(fmt) +
+         2 * 2 * kQScaleBytes + 256;
+}
+__host__ __device__ constexpr int kQCtasPerSMOf(int fmt) { return fmt == kFmtMX8 ? 1 : kQCtasPerSM; }
+constexpr int kQSmemBytes = kQSmemBytesOf(kFmtMX);
 
 struct QuantArgs {
   int64_t rows, cols;
@@ -324,6 +330,50 @@ __device__ __forceinline__ Enc encode_x2(float2 (&p)[32], float S, float six_s,
   else return nv_encode_x2(p, S, six_s, codes);
 }
 
+// Four fp32 -> E4M3 (RNE, saturating to +-448) in one word, v0 in the low byte.
+__device__ __forceinline__ uint32_t cvt_e4m3x4(float v0, float v1, float v2, float v3) {
+  uint32_t out;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(out)
+      : "f"(v0), "f"(v1), "f"(v2), "f"(v3));
+  return out;
+}
+
+// MXFP8 job: 32 E4M3 code bytes per lane (two 16-byte chunks) and one scale byte.
+struct Enc8 {
+  uint4 cx[2], cy[2];
+  uint32_t sx, sy;
+};
+// MXFP8 block of 32 per lane: byte = max(biased exponent of amax - 8, 0), i.e. the byte of
+// e = floor(log2 amax) - 8 clamped at -127 (8 = largest E4M3 exponent); codes
+// E4M3_RNE_satfinite(v * 2^-e), 2^-e = 2^(127 - byte) built from its bit pattern.
+__device__ __forceinline__ Enc8 mx8_encode_x2(float2 (&p)[32]) {
+  const float2 am = amax_x2(p, 0, 32);
+  const uint32_t ex = (__float_as_uint(am.x) >> 23) & 0xFFu;
+  const uint32_t ey = (__float_as_uint(am.y) >> 23) & 0xFFu;
+  const uint32_t bx = ex > 8u ? ex - 8u : 0u, by = ey > 8u ? ey - 8u : 0u;
+  const float2 inv = make_float2(__uint_as_float((254u - bx) << 23), __uint_as_float((254u - by) << 23));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) p[i] = mul2(p[i], inv);
+  uint32_t wx[8], wy[8];
+#pragma unroll
+  for (int g = 0; g < 8; ++g) {
+    wx[g] = cvt_e4m3x4(p[4 * g].x, p[4 * g + 1].x, p[4 * g + 2].x, p[4 * g + 3].x);
+    wy[g] = cvt_e4m3x4(p[4 * g].y, p[4 * g + 1].y, p[4 * g + 2].y, p[4 * g + 3].y);
+  }
+  Enc8 e;
+  e.cx[0] = make_uint4(wx[0], wx[1], wx[2], wx[3]);
+  e.cx[1] = make_uint4(wx[4], wx[5], wx[6], wx[7]);
+  e.cy[0] = make_uint4(wy[0], wy[1], wy[2], wy[3]);
+  e.cy[1] = make_uint4(wy[4], wy[5], wy[6], wy[7]);
+  e.sx = bx;
+  e.sy = by;
+  return e;
+}
+
 // Offset of scale (row r of the 128-row atom block, block kb of the tile) in a staged
 // scale tile of one or two atoms: atom kb/4, then (r%32)*16 + (r/32)*4 + kb%4.
 __device__ __forceinline__ int atom_off(int r, int kb) {
@@ -332,6 +382,10 @@ __device__ __forceinline__ int atom_off(int r, int kb) {
 // Staged code tile [128 rows][64 B], 64-byte swizzle: 16-byte chunk q of row r.
 __device__ __forceinline__ uint8_t* code_chunk(uint8_t* tile, int r, int q) {
   return tile + r * 64 + ((q ^ ((r >> 1) & 3)) << 4);
+}
+// Staged MXFP8 code tile [128 rows][128 B], 128-byte swizzle: 16-byte chunk q of row r.
+__device__ __forceinline__ uint8_t* code_chunk8(uint8_t* tile, int r, int q) {
+  return tile + r * 128 + ((q ^ (r & 7)) << 4);
 }
 
 // ROW job: tile row r, box b (columns 64b .. 64b+63) = segments 2b (lane x) and 2b+1
@@ -369,7 +423,7 @@ __device__ __forceinline__ void load_col_job(const uint8_t* in, int b, int w, in
 // EXT kernels also implement the variants selected at run time by a.rht (random +-1
 // signs along the contraction axis before the rotation) and a.sr (stochastic rounding).
 template <int FMT, int HN, int MODE, bool AMAX, bool EXT = false>
-__global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
+__global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT))
     quantize_kernel(const __grid_constant__ CUtensorMap tm_in,
                     const __grid_constant__ CUtensorMap tm_rcodes,
                     const __grid_constant__ CUtensorMap tm_ccodes, const QuantArgs a) {
@@ -383,8 +437,9 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* s_in = smem;
   uint8_t* s_rcode = s_in + kQStages * kQInBytes;
-  uint8_t* s_ccode = s_rcode + 2 * kQCodeBytes;
-  uint8_t* s_rsc = s_ccode + 2 * kQCodeBytes;
+  constexpr int kCodeBytes = kQCodeBytesOf(FMT);
+  uint8_t* s_ccode = s_rcode + 2 * kCodeBytes;
+  uint8_t* s_rsc = s_ccode + 2 * kCodeBytes;
   uint8_t* s_csc = s_rsc + 2 * kQScaleBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(s_csc + 2 * kQScaleBytes);
   float* s_red = reinterpret_cast<float*>(full + kQStages);  // [8 warps][2]
@@ -469,8 +524,8 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
     const bool ok = mbar_wait(&full[st], static_cast<uint32_t>((it / kQStages) & 1), a.wait_limit_ns);
     if (__syncthreads_or(!ok)) break;  // give up together; the status word says why
     const uint8_t* in = s_in + st * kQInBytes;
-    uint8_t* rcode = s_rcode + ob * kQCodeBytes;
-    uint8_t* ccode = s_ccode + ob * kQCodeBytes;
+    uint8_t* rcode = s_rcode + ob * kCodeBytes;
+    uint8_t* ccode = s_ccode + ob * kCodeBytes;
     uint8_t* rsc = s_rsc + ob * kQScaleBytes;
     uint8_t* csc = s_csc + ob * kQScaleBytes;
 
@@ -494,6 +549,14 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
         if constexpr (AMAX) {
           const float2 m = amax_x2(p, 0, 32);
           amax_r = max3f(amax_r, m.x, m.y);
+        } else if constexpr (FMT == kFmtMX8) {
+          const Enc8 e = mx8_encode_x2(p);  // lane x: bytes 64b .. +31, lane y: 64b+32 .. +63
+          *reinterpret_cast<uint4*>(code_chunk8(rcode, row_r, 4 * b)) = e.cx[0];
+          *reinterpret_cast<uint4*>(code_chunk8(rcode, row_r, 4 * b + 1)) = e.cx[1];
+          *reinterpret_cast<uint4*>(code_chunk8(rcode, row_r, 4 * b + 2)) = e.cy[0];
+          *reinterpret_cast<uint4*>(code_chunk8(rcode, row_r, 4 * b + 3)) = e.cy[1];
+          *reinterpret_cast<uint16_t*>(rsc + atom_off(row_r, 2 * b)) =
+              static_cast<uint16_t>(e.sx | (e.sy << 8));
         } else {
           Enc e;
           if (sr) {
@@ -534,6 +597,14 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
         if constexpr (AMAX) {
           const float2 m = amax_x2(p, 0, 32);
           amax_c = max3f(amax_c, m.x, m.y);
+        } else if constexpr (FMT == kFmtMX8) {
+          const Enc8 e = mx8_encode_x2(p);  // column c (x) and c+1 (y): rows 32s .. 32s+31
+          *reinterpret_cast<uint4*>(code_chunk8(ccode, col_c, 2 * s)) = e.cx[0];
+          *reinterpret_cast<uint4*>(code_chunk8(ccode, col_c, 2 * s + 1)) = e.cx[1];
+          *reinterpret_cast<uint4*>(code_chunk8(ccode, col_c + 1, 2 * s)) = e.cy[0];
+          *reinterpret_cast<uint4*>(code_chunk8(ccode, col_c + 1, 2 * s + 1)) = e.cy[1];
+          csc[atom_off(col_c, s)] = static_cast<uint8_t>(e.sx);
+          csc[atom_off(col_c + 1, s)] = static_cast<uint8_t>(e.sy);
         } else {
           Enc e;
           if (sr) {
@@ -565,16 +636,17 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSM)
     __syncthreads();
     if (tid == 0) {
       if constexpr (!AMAX) {
-        constexpr int kAtomsPerTile = (FMT == kFmtMX) ? 1 : 2;
+        constexpr int kAtomsPerTile = (FMT == kFmtNV) ? 2 : 1;
+        constexpr int kTileCodeBytes = FMT == kFmtMX8 ? 128 : 64;  // code bytes per tile row
         if constexpr (kRow) {
-          tma_store_2d(&tm_rcodes, rcode, tc * 64, tr * 128);
+          tma_store_2d(&tm_rcodes, rcode, tc * kTileCodeBytes, tr * 128);
           const int first = tc * kAtomsPerTile;
           const int n = (a.row_kb4 - first) < kAtomsPerTile ? (a.row_kb4 - first) : kAtomsPerTile;
           bulk_store(a.row_scales + (static_cast<int64_t>(tr) * a.row_kb4 + first) * 512, rsc,
                      static_cast<uint32_t>(n * 512));
         }
         if constexpr (kCol) {
-          tma_store_2d(&tm_ccodes, ccode, tr * 64, tc * 128);
+          tma_store_2d(&tm_ccodes, ccode, tr * kTileCodeBytes, tc * 128);
           const int first = tr * kAtomsPerTile;
           const int n = (a.col_kb4 - first) < kAtomsPerTile ? (a.col_kb4 - first) : kAtomsPerTile;
           bulk_store(a.col_scales + (static_cast<int64_t>(tc) * a.col_kb4 + first) * 512, csc,

@@ -71,7 +71,14 @@ typedef enum {
     FP4_ERR_WORKSPACE = 7           /* workspace NULL or smaller than required */
 } fp4_status;
 
-typedef enum { FP4_MXFP4 = 0, FP4_NVFP4 = 1 } fp4_format;
+/* FP4_MXFP8 is the FP8 comparator the pages measure FP4 against (MXFP4 pre-training
+ * summary, Methodology item 1: the FP8 baseline; Findings section 3: MXFP4 + H16 20%
+ * faster per step than FP8). Elements are E4M3 (one byte each, codes [R][C]); each
+ * block of 32 shares an E8M0 scale, e = floor(log2 amax) - 8 clamped to [-127, 127]
+ * (amax 0 -> -127), and codes are E4M3_RNE_satfinite(v * 2^-e). Its scales use the
+ * same layout as MXFP4. It has no tensor scale and no quantiser variants (the options
+ * of fp4_quantize_opts). The GEMM is tcgen05.mma kind::mxf8f6f4 with block32 scales. */
+typedef enum { FP4_MXFP4 = 0, FP4_NVFP4 = 1, FP4_MXFP8 = 2 } fp4_format;
 typedef enum { FP4_AXIS_ROW = 0, FP4_AXIS_COL = 1 } fp4_axis;
 typedef enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 } fp4_out_dtype;
 typedef enum { FP4_PASS_FPROP = 0, FP4_PASS_DGRAD = 1, FP4_PASS_WGRAD = 2 } fp4_pass;
@@ -81,6 +88,8 @@ FP4_API int fp4_abi_version(void);
 
 /* Bytes of a packed code matrix with R rows of C elements: R*C/2. */
 FP4_API size_t fp4_codes_bytes(int64_t rows, int64_t cols);
+/* Bytes of a code matrix of format fmt: R*C/2 (FP4 formats) or R*C (FP4_MXFP8). */
+FP4_API size_t fp4_codes_bytes_fmt(int64_t rows, int64_t cols, fp4_format fmt);
 
 /* Bytes of the scale matrix of an [R][C] code matrix in the atom layout above:
  * ceil(R/128)*128 * ceil(C/bs/4)*4. */

@@ -35,9 +35,11 @@ def test_status_strings():
 
 
 @pytest.mark.parametrize("rows,cols", [(32, 32), (160, 224), (128, 4096), (8192, 14336)])
-@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("fmt", [0, 1, 2])
 def test_size_queries_match_layout(orc, rows, cols, fmt):
     assert fp4.fp4_codes_bytes(rows, cols) == rows * cols // 2
+    L = fp4.lib()
+    assert L.fp4_codes_bytes_fmt(rows, cols, fmt) == rows * cols // (1 if fmt == 2 else 2)
     assert fp4.fp4_scales_bytes(rows, cols, fmt) == orc.scale_layout_bytes(rows, cols // orc.BLOCK[fmt])
 
 
@@ -53,7 +55,7 @@ def q(x=A16, codes=A16, scales=A16, ts=None, rows=64, cols=64, fmt=0, hn=16, axi
 
 
 def test_quantize_validation():
-    assert q(fmt=2) == INVALID
+    assert q(fmt=3) == INVALID
     assert q(hn=8) == INVALID
     assert q(axis=3) == INVALID
     assert q(rows=48) == SHAPE
@@ -65,6 +67,7 @@ def test_quantize_validation():
     assert q(scales=None) == INVALID
     assert q(ts=A16) == INVALID            # MXFP4 takes no tensor scale
     assert q(fmt=1, ts=None) == INVALID    # NVFP4 needs one
+    assert q(fmt=2, ts=A16) == INVALID     # nor does the MXFP8 comparator
     assert q(rows=0) == OK and q(cols=0) == OK  # empty: nothing to do
 
 
@@ -91,6 +94,7 @@ def test_quantize_opts_validation():
     assert L.fp4_quantize_dual_opts(A16, A16, A16, None, A16, None, 64, 64, 0, 16,
                                     ctypes.byref(sr), None) == INVALID
     assert L.fp4_quantize_opts(A16, A16, A16, None, 0, 64, 0, 16, 0, ctypes.byref(sr), None) == OK
+    assert qo(ctypes.byref(sr), fmt=2) == INVALID              # no variants for MXFP8
 
 
 def g(A=A16, As=A16, Ats=None, B=A16, Bs=A16, Bts=None, C=A16, M=128, N=128, K=128, fmt=0, od=0):
@@ -99,6 +103,7 @@ def g(A=A16, As=A16, Ats=None, B=A16, Bs=A16, Bts=None, C=A16, M=128, N=128, K=1
 
 def test_gemm_validation():
     assert g(fmt=5) == INVALID
+    assert g(fmt=2, Ats=A16) == INVALID    # the MXFP8 comparator takes no tensor scales
     assert g(od=2) == INVALID
     assert g(M=100) == SHAPE
     assert g(K=48) == SHAPE
