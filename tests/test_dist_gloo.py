@@ -72,11 +72,24 @@ def _run(fn, world, *args):
     procs = [ctx.Process(target=fn, args=(r, world, port, *args, q)) for r in range(world)]
     for p in procs:
         p.start()
+    # drain the queue while the ranks run: a child that has put items exits only after
+    # they are read, so joining first would wait out the whole timeout
+    import queue
+    import time
     results = []
+    deadline = time.monotonic() + 120
+    while time.monotonic() < deadline and any(p.is_alive() for p in procs):
+        try:
+            results.append(q.get(timeout=0.2))
+        except queue.Empty:
+            pass
     for p in procs:
-        p.join(timeout=120)
-    while not q.empty():
-        results.append(q.get())
+        p.join(timeout=max(0.0, deadline - time.monotonic()))
+    while True:
+        try:
+            results.append(q.get(timeout=0.2))
+        except queue.Empty:
+            break
     for p in procs:
         if p.is_alive():
             p.kill()
