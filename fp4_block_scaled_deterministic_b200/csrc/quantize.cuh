@@ -76,11 +76,11 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a
 
 // Normalised block FWHT of both lanes: groups of HN along the 32 elements, butterfly
 // strides 1, 2, 4, ... in that order, then x RN(1/sqrt(HN)).
-template <int HN, bool kScale = true>
+template <int HN, bool kScale = true, int kFirst = 1>
 __device__ __forceinline__ void fwht_x2(float2 (&p)[32]) {
   if constexpr (HN > 0) {
 #pragma unroll
-    for (int h = 1; h < HN; h <<= 1) {
+    for (int h = kFirst; h < HN; h <<= 1) {
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         if ((i & h) == 0) {
@@ -420,6 +420,72 @@ __device__ __forceinline__ void load_col_job(const uint8_t* in, int b, int w, in
   }
 }
 
+// bf16 (low or high half of w) + c in fp32 with one rounding; the widening is exact, so
+// this is RN_fp32(widen(bf16) + c), the stride-1 butterfly of the rotation, issued on
+// the FMA pipe instead of widening on the integer pipe first.
+__device__ __forceinline__ float add_lo(uint32_t w, float c) {
+  float d;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tadd.rn.f32.bf16 %0, l, %2;\n\t}"
+      : "=f"(d) : "r"(w), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float add_hi(uint32_t w, float c) {
+  float d;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tadd.rn.f32.bf16 %0, h, %2;\n\t}"
+      : "=f"(d) : "r"(w), "f"(c));
+  return d;
+}
+// Stride-1 butterfly of two bf16 values u (element 2k) and v (element 2k+1) given as
+// the bf16 u and the widened v: (u + v, u - v), each rounded once.
+__device__ __forceinline__ void bfly1_lo(uint32_t wu, float v, float& s, float& d) {
+  s = add_lo(wu, v);
+  d = add_lo(wu, -v);
+}
+__device__ __forceinline__ void bfly1_hi(uint32_t wu, float v, float& s, float& d) {
+  s = add_hi(wu, v);
+  d = add_hi(wu, -v);
+}
+
+// ROW job with the first (stride-1) butterfly fused into the widening: elements 2k and
+// 2k+1 of a lane are the low and high halves of one 32-bit word.
+__device__ __forceinline__ void load_row_job_bfly1(const uint8_t* in, int r, int b,
+                                                   float2 (&p)[32]) {
+  const uint8_t* rowp = in + b * kQBoxBytes + r * 128;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 wx = *reinterpret_cast<const uint4*>(rowp + ((i ^ (r & 7)) << 4));
+    const uint4 wy = *reinterpret_cast<const uint4*>(rowp + (((4 + i) ^ (r & 7)) << 4));
+    const uint32_t ax[4] = {wx.x, wx.y, wx.z, wx.w}, ay[4] = {wy.x, wy.y, wy.z, wy.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float sx, dx, sy, dy;
+      bfly1_lo(ax[k], add_hi(ax[k], -0.0f), sx, dx);  // x + (-0) widens exactly
+      bfly1_lo(ay[k], add_hi(ay[k], -0.0f), sy, dy);
+      p[8 * i + 2 * k] = make_float2(sx, sy);
+      p[8 * i + 2 * k + 1] = make_float2(dx, dy);
+    }
+  }
+}
+// COL job with the first butterfly fused: elements i and i+1 are consecutive rows, lane x
+// the low halves (column c) and lane y the high halves (column c+1) of the two words.
+__device__ __forceinline__ void load_col_job_bfly1(const uint8_t* in, int b, int w, int s,
+                                                   float2 (&p)[32]) {
+  const uint8_t* boxp = in + b * kQBoxBytes;
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    const int r0 = 32 * s + i, r1 = r0 + 1;
+    const uint32_t v0 = *reinterpret_cast<const uint32_t*>(boxp + r0 * 128 +
+                                                           (((w >> 2) ^ (r0 & 7)) << 4) + ((w & 3) << 2));
+    const uint32_t v1 = *reinterpret_cast<const uint32_t*>(boxp + r1 * 128 +
+                                                           (((w >> 2) ^ (r1 & 7)) << 4) + ((w & 3) << 2));
+    float sx, dx, sy, dy;
+    bfly1_lo(v0, add_lo(v1, -0.0f), sx, dx);
+    bfly1_hi(v0, add_hi(v1, -0.0f), sy, dy);
+    p[i] = make_float2(sx, sy);
+    p[i + 1] = make_float2(dx, dy);
+  }
+}
+
 // EXT kernels also implement the variants selected at run time by a.rht (random +-1
 // signs along the contraction axis before the rotation) and a.sr (stochastic rounding).
 template <int FMT, int HN, int MODE, bool AMAX, bool EXT = false>
@@ -533,7 +599,10 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT))
       const int b = tid >> 7;
       {
         float2 p[32];
-        load_row_job(in, row_r, b, p);
+        // the stride-1 butterfly is fused into the load unless random signs come first
+        constexpr bool kFuse1 = HN > 0 && !EXT;
+        if constexpr (kFuse1) load_row_job_bfly1(in, row_r, b, p);
+        else load_row_job(in, row_r, b, p);
         if (rht) {
           // lane x holds tile columns 64b + i, lane y 64b + 32 + i
           const uint32_t m[4] = {s_sgn[0], s_sgn[1], s_sgn[2], s_sgn[3]};
@@ -545,7 +614,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT))
                                __uint_as_float(__float_as_uint(p[i].y) ^ (sy << 31)));
           }
         }
-        fwht_x2<HN, !kFoldH16>(p);
+        fwht_x2<HN, !kFoldH16, kFuse1 ? 2 : 1>(p);
         if constexpr (AMAX) {
           const float2 m = amax_x2(p, 0, 32);
           amax_r = max3f(amax_r, m.x, m.y);
@@ -582,7 +651,9 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT))
       const int s = tid >> 6;
       {
         float2 p[32];
-        load_col_job(in, col_b, col_w, s, p);
+        constexpr bool kFuse1 = HN > 0 && !EXT;
+        if constexpr (kFuse1) load_col_job_bfly1(in, col_b, col_w, s, p);
+        else load_col_job(in, col_b, col_w, s, p);
         if (rht) {
           // element i of both lanes is tile row 32s + i
           const uint32_t m[4] = {s_sgn[4], s_sgn[5], s_sgn[6], s_sgn[7]};
@@ -593,7 +664,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT))
                                __uint_as_float(__float_as_uint(p[i].y) ^ sg));
           }
         }
-        fwht_x2<HN, !kFoldH16>(p);
+        fwht_x2<HN, !kFoldH16, kFuse1 ? 2 : 1>(p);
         if constexpr (AMAX) {
           const float2 m = amax_x2(p, 0, 32);
           amax_c = max3f(amax_c, m.x, m.y);
