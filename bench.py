@@ -9,6 +9,10 @@ the FP4 tensor cores:
     with N > 1 ranks: data parallel over tokens (8192 per rank), dW all-reduced
     (NCCL) per projection, overlapped with the next projection.
 
+The quantisation of projection p+1 runs on a second stream beside the GEMMs of
+projection p (--side-stream 1, the default), filling the SMs their last tile wave
+leaves idle; per-kernel rooflines are then timed on the same steps run on one stream.
+
 Prints ONE JSON line (rank 0). `value` is the step's GEMM FLOPs divided by the step
 time (quantisation included), summed over ranks. Inputs are synthetic, seeded, and
 resident in HBM before the timed region; the step's working set (~4 GB) is far
@@ -67,6 +71,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--proj", default="qkv,o,gate,up,down",
                     help="comma-separated subset of the layer's projections (profiling cases)")
+    ap.add_argument("--side-stream", type=int, default=1, choices=[0, 1],
+                    help="1: quantise the next projection on a second stream beside the GEMMs "
+                         "(per-kernel rooflines then come from the same steps on one stream)")
     ap.add_argument("--variant", choices=["none", "sr", "rht", "sr+rht", "amax"], default="none",
                     help="quantiser variant: stochastic rounding, randomised Hadamard signs, "
                          "both, or (NVFP4) a supplied tensor amax instead of the amax pass")
@@ -141,11 +148,13 @@ class Clocks:
 class LlamaLayer:
     """Inputs, quantised operands and outputs of every projection, all on the device."""
 
-    def __init__(self, device, fmt, hn, tokens=8192, seed=0, names=None, variant="none"):
+    def __init__(self, device, fmt, hn, tokens=8192, seed=0, names=None, variant="none",
+                 side_stream=False):
         import fp4_block_scaled_deterministic_b200 as fp4
         from fp4_block_scaled_deterministic_b200 import synthetic
         self.fp4, self.fmt, self.hn, self.M = fp4, fmt, hn, tokens
         self.variant = variant
+        self.qstream = torch.cuda.Stream(device) if side_stream else None
         self.projs = []
         g = torch.Generator(device=device)
         for i, (name, N, K) in enumerate(synthetic.LLAMA_LAYERS):
@@ -174,6 +183,7 @@ class LlamaLayer:
                     st = fp4.fp4_quantize_dual(p[key], row[0], row[1], col[0], col[1], ts, r, c,
                                                fmt, hn, torch.cuda.current_stream().cuda_stream)
                     assert st == 0
+        self.gemms_done = []
         self.opts = {}
         for p in self.projs:
             for key, _ in self._operands(p):
@@ -184,6 +194,10 @@ class LlamaLayer:
                     o = fp4.QuantOpts(None, int("sr" in variant), int("rht" in variant),
                                       0x5EED0000 + seed, 0x51600000 + seed)
                 self.opts[(p["name"], key)] = o
+        for _ in self.projs:
+            ev = torch.cuda.Event()
+            ev.record(torch.cuda.current_stream(device))
+            self.gemms_done.append(ev)
 
     def _operands(self, p):
         return (("X", (self.M, p["K"])), ("W", (p["N"], p["K"])), ("dY", (self.M, p["N"])))
@@ -210,37 +224,64 @@ class LlamaLayer:
         per_q = 1 if self.fmt == 0 or self.variant == "amax" else 2
         return len(self.projs) * (3 * per_q + 3)
 
-    def step(self, stream, timers=None, allreduce=None):
+    def step(self, stream, timers=None, allreduce=None, overlap=None):
         """One fwd+bwd pass over every projection. timers: dict kind -> list of event
-        pairs to record around each quantise / GEMM launch."""
+        pairs to record around each quantise / GEMM launch. overlap: quantise on the
+        side stream (default: when the layer has one)."""
         f, fmt, hn = self.fp4, self.fmt, self.hn
+        if overlap is None:
+            overlap = self.qstream is not None
         s = stream.cuda_stream
         pending = []
 
-        def timed(kind, fn):
+        def timed(kind, fn, on=None):
+            on = stream if on is None else on
             if timers is None:
                 return fn()
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
+            e0.record(on)
             r = fn()
-            e1.record(stream)
+            e1.record(on)
             timers[kind].append((e0, e1))
             return r
 
-        for p in self.projs:
+        def quantise(p, qstream):
+            qs = qstream.cuda_stream
             for key, (r, c) in self._operands(p):
                 row, col, ts = p[key + "_row"], p[key + "_col"], p[key + "_ts"]
                 opts = self.opts[(p["name"], key)]
                 if opts is None:
                     st = timed("quant", lambda: f.fp4_quantize_dual(
                         p[key], row[0], row[1], col[0], col[1], ts if fmt == 1 else None, r, c,
-                        fmt, hn, s))
+                        fmt, hn, qs), qstream)
                 else:
                     st = timed("quant", lambda: f.fp4_quantize_dual_opts(
                         p[key], row[0], row[1], col[0], col[1], ts if fmt == 1 else None, r, c,
-                        fmt, hn, opts, s))
+                        fmt, hn, opts, qs), qstream)
                 assert st == 0, f.status_string(st)
+
+        # With a side stream the quantisation of projection p+1 runs beside the GEMMs of
+        # projection p (it fills the SMs their last tile wave leaves idle). Events order
+        # each GEMM after its operands' quantisation, and each quantisation after the
+        # previous step's GEMMs that read the buffers it overwrites.
+        side = self.qstream if overlap else None
+        if side is not None:
+            start = torch.cuda.Event()
+            start.record(stream)          # inputs written on the main stream (e2e copies)
+            side.wait_event(start)
+            ready = []
+            for i, p in enumerate(self.projs):
+                side.wait_event(self.gemms_done[i])
+                quantise(p, side)
+                ev = torch.cuda.Event()
+                ev.record(side)
+                ready.append(ev)
+        for i, p in enumerate(self.projs):
+            if side is None:
+                quantise(p, stream)
+            else:
+                stream.wait_event(ready[i])
             tsx, tsw, tsy = p["X_ts"], p["W_ts"], p["dY_ts"]
             nv = fmt == 1
             M, N, K = self.M, p["N"], p["K"]
@@ -259,6 +300,8 @@ class LlamaLayer:
                 p["dY_col"][0], p["dY_col"][1], tsy[1:2] if nv else None, p["X_col"][0],
                 p["X_col"][1], tsx[1:2] if nv else None, p["dW"], N, K, M, fmt, 0, s))
             assert st == 0
+            if side is not None:
+                self.gemms_done[i].record(stream)
             if allreduce is not None:
                 pending.append(allreduce(p["dW"]))
         for w in pending:
@@ -395,7 +438,8 @@ def main():
     fp4.lib()  # fails loudly if the library is missing
     fmt = FORMATS[a.format]
     names = [n.strip() for n in a.proj.split(",") if n.strip()]
-    layer = LlamaLayer(dev, fmt, a.hadamard, seed=1000 * rank, names=names, variant=a.variant)
+    layer = LlamaLayer(dev, fmt, a.hadamard, seed=1000 * rank, names=names, variant=a.variant,
+                       side_stream=bool(a.side_stream))
     stream = torch.cuda.current_stream(dev)
     from fp4_block_scaled_deterministic_b200 import dp
     allreduce = dp.allreduce_wgrad if world > 1 else None
@@ -411,15 +455,27 @@ def main():
     assert fp4.fp4_check_status() == 0
 
     timers = {"quant": [], "gemm": []}
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if a.side_stream:
+        # Per-kernel durations for the rooflines come from the same steps run on one
+        # stream, where no kernel shares the SMs; the step time below overlaps them.
+        for _ in range(a.warmup):
+            layer.step(stream, None, allreduce, overlap=False)
+        barrier()
+        for _ in range(a.steps):
+            layer.step(stream, timers, allreduce, overlap=False)
+        barrier()
+        for _ in range(a.warmup):
+            layer.step(stream, None, allreduce)
+        barrier()
     clocks = Clocks(local)
     clocks.start()
     time.sleep(0.3)
     barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(a.steps):
-        layer.step(stream, timers, allreduce)
+        layer.step(stream, None if a.side_stream else timers, allreduce)
     e1.record(stream)
     barrier()
     clk = clocks.stop()
@@ -453,6 +509,9 @@ def main():
                       f"{'MXFP8, kind::mxf8f6f4' if fmt == 2 else 'FP4'}, CTA pairs)",
             "per_launch": {"avg_flops": avg_flops, "avg_ms": avg_launch_ms,
                            "launches": len(gemm_ms)},
+            "timing": ("CUDA events around each launch over the timed steps" if not a.side_stream
+                       else "CUDA events around each launch over the same number of steps run "
+                            "on one stream just before the overlapped timed region"),
             "peak_source": f"{pk_kind}: bf16_tflops_sustained x {ratio} (nominal "
                            f"{'FP8' if fmt == 2 else 'FP4'}:BF16)"}
     qroof = {"bound": "hbm", "achieved": quant_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
@@ -467,6 +526,7 @@ def main():
            "config": {"workload": workload_name(a) if len(names) == 5 else
                       f"subset {','.join(names)} of: {workload_name(a)}",
                       "format": a.format, "hadamard_n": a.hadamard, "variant": a.variant,
+                      "streams": 2 if a.side_stream else 1,
                       "tokens_per_rank": layer.M,
                       "l2": f"inputs larger than L2 ({(layer.bytes_in() + layer.bytes_out()) / 1e9:.1f} GB per step)",
                       "parallelism": f"dp{world}"},
