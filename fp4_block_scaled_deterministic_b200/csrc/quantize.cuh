@@ -40,7 +40,7 @@ constexpr int kQScaleBytes = 1024;          // up to two 512-byte atoms
 __host__ __device__ constexpr int kQCodeBytesOf(int fmt) { return fmt == kFmtMX8 ? 128 * 128 : 128 * 64; }
 __host__ __device__ constexpr int kQSmemBytesOf(int fmt) {
   return 1024 /*align*/ + kQStages * kQInBytes + 2 * 2 * kQCodeBytesOf(fmt) +
-         2 * 2 * kQScaleBytes + 256;
+         2 * 2 * kQScaleBytes + 256 + 1024 /* random-sign masks */;
 }
 __host__ __device__ constexpr int kQCtasPerSMOf(int fmt) { return fmt == kFmtMX8 ? 1 : kQCtasPerSM; }
 constexpr int kQSmemBytes = kQSmemBytesOf(kFmtMX);
@@ -133,8 +133,11 @@ __device__ __forceinline__ uint32_t cvt8y(const float2 (&p)[32], int b) {
 __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
 #pragma unroll
   for (int r = 0; r < 10; ++r) {
-    const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
-    const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
+    // one 32x32 -> 64-bit product each (both halves from one wide multiply)
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c.x;
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c.z;
+    const uint32_t lo0 = static_cast<uint32_t>(p0), hi0 = static_cast<uint32_t>(p0 >> 32);
+    const uint32_t lo1 = static_cast<uint32_t>(p1), hi1 = static_cast<uint32_t>(p1 >> 32);
     c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
     k0 += 0x9E3779B9u;
     k1 += 0xBB67AE85u;
@@ -390,12 +393,24 @@ __device__ __forceinline__ uint8_t* code_chunk8(uint8_t* tile, int r, int q) {
 
 // ROW job: tile row r, box b (columns 64b .. 64b+63) = segments 2b (lane x) and 2b+1
 // (lane y); 8 conflict-free 16-byte reads of the 128B-swizzled box row.
-__device__ __forceinline__ void load_row_job(const uint8_t* in, int r, int b, float2 (&p)[32]) {
+// Random signs as XOR masks on the raw bf16x2 words: cm[q] flips the two columns of
+// column pair q of the tile (bits 15 and 31), rm[r] both halves of tile row r.
+__device__ __forceinline__ uint4 xor4(uint4 a, uint4 m) {
+  return make_uint4(a.x ^ m.x, a.y ^ m.y, a.z ^ m.z, a.w ^ m.w);
+}
+
+template <bool kSigns = false>
+__device__ __forceinline__ void load_row_job(const uint8_t* in, int r, int b, float2 (&p)[32],
+                                             const uint32_t* cm = nullptr) {
   const uint8_t* rowp = in + b * kQBoxBytes + r * 128;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const uint4 wx = *reinterpret_cast<const uint4*>(rowp + ((i ^ (r & 7)) << 4));
-    const uint4 wy = *reinterpret_cast<const uint4*>(rowp + (((4 + i) ^ (r & 7)) << 4));
+    uint4 wx = *reinterpret_cast<const uint4*>(rowp + ((i ^ (r & 7)) << 4));
+    uint4 wy = *reinterpret_cast<const uint4*>(rowp + (((4 + i) ^ (r & 7)) << 4));
+    if constexpr (kSigns) {  // pairs 32b + 4i .. (lane x) and 32b + 16 + 4i .. (lane y)
+      wx = xor4(wx, *reinterpret_cast<const uint4*>(cm + 32 * b + 4 * i));
+      wy = xor4(wy, *reinterpret_cast<const uint4*>(cm + 32 * b + 16 + 4 * i));
+    }
     p[8 * i + 0] = make_float2(bf16lo(wx.x), bf16lo(wy.x));
     p[8 * i + 1] = make_float2(bf16hi(wx.x), bf16hi(wy.x));
     p[8 * i + 2] = make_float2(bf16lo(wx.y), bf16lo(wy.y));
@@ -408,14 +423,16 @@ __device__ __forceinline__ void load_row_job(const uint8_t* in, int r, int b, fl
 }
 // COL job: tile columns c = 64b + 2w (lane x) and c + 1 (lane y), rows 32s .. 32s+31;
 // 32 conflict-free 4-byte reads.
+template <bool kSigns = false>
 __device__ __forceinline__ void load_col_job(const uint8_t* in, int b, int w, int s,
-                                             float2 (&p)[32]) {
+                                             float2 (&p)[32], const uint32_t* rm = nullptr) {
   const uint8_t* boxp = in + b * kQBoxBytes;
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
     const int r = 32 * s + i;
-    const uint32_t v = *reinterpret_cast<const uint32_t*>(boxp + r * 128 +
-                                                          (((w >> 2) ^ (r & 7)) << 4) + ((w & 3) << 2));
+    uint32_t v = *reinterpret_cast<const uint32_t*>(boxp + r * 128 +
+                                                    (((w >> 2) ^ (r & 7)) << 4) + ((w & 3) << 2));
+    if constexpr (kSigns) v ^= rm[r];
     p[i] = make_float2(bf16lo(v), bf16hi(v));
   }
 }
@@ -448,13 +465,18 @@ __device__ __forceinline__ void bfly1_hi(uint32_t wu, float v, float& s, float& 
 
 // ROW job with the first (stride-1) butterfly fused into the widening: elements 2k and
 // 2k+1 of a lane are the low and high halves of one 32-bit word.
+template <bool kSigns = false>
 __device__ __forceinline__ void load_row_job_bfly1(const uint8_t* in, int r, int b,
-                                                   float2 (&p)[32]) {
+                                                   float2 (&p)[32], const uint32_t* cm = nullptr) {
   const uint8_t* rowp = in + b * kQBoxBytes + r * 128;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const uint4 wx = *reinterpret_cast<const uint4*>(rowp + ((i ^ (r & 7)) << 4));
-    const uint4 wy = *reinterpret_cast<const uint4*>(rowp + (((4 + i) ^ (r & 7)) << 4));
+    uint4 wx = *reinterpret_cast<const uint4*>(rowp + ((i ^ (r & 7)) << 4));
+    uint4 wy = *reinterpret_cast<const uint4*>(rowp + (((4 + i) ^ (r & 7)) << 4));
+    if constexpr (kSigns) {
+      wx = xor4(wx, *reinterpret_cast<const uint4*>(cm + 32 * b + 4 * i));
+      wy = xor4(wy, *reinterpret_cast<const uint4*>(cm + 32 * b + 16 + 4 * i));
+    }
     const uint32_t ax[4] = {wx.x, wx.y, wx.z, wx.w}, ay[4] = {wy.x, wy.y, wy.z, wy.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -468,16 +490,21 @@ __device__ __forceinline__ void load_row_job_bfly1(const uint8_t* in, int r, int
 }
 // COL job with the first butterfly fused: elements i and i+1 are consecutive rows, lane x
 // the low halves (column c) and lane y the high halves (column c+1) of the two words.
+template <bool kSigns = false>
 __device__ __forceinline__ void load_col_job_bfly1(const uint8_t* in, int b, int w, int s,
-                                                   float2 (&p)[32]) {
+                                                   float2 (&p)[32], const uint32_t* rm = nullptr) {
   const uint8_t* boxp = in + b * kQBoxBytes;
 #pragma unroll
   for (int i = 0; i < 32; i += 2) {
     const int r0 = 32 * s + i, r1 = r0 + 1;
-    const uint32_t v0 = *reinterpret_cast<const uint32_t*>(boxp + r0 * 128 +
-                                                           (((w >> 2) ^ (r0 & 7)) << 4) + ((w & 3) << 2));
-    const uint32_t v1 = *reinterpret_cast<const uint32_t*>(boxp + r1 * 128 +
-                                                           (((w >> 2) ^ (r1 & 7)) << 4) + ((w & 3) << 2));
+    uint32_t v0 = *reinterpret_cast<const uint32_t*>(boxp + r0 * 128 +
+                                                     (((w >> 2) ^ (r0 & 7)) << 4) + ((w & 3) << 2));
+    uint32_t v1 = *reinterpret_cast<const uint32_t*>(boxp + r1 * 128 +
+                                                     (((w >> 2) ^ (r1 & 7)) << 4) + ((w & 3) << 2));
+    if constexpr (kSigns) {
+      v0 ^= rm[r0];
+      v1 ^= rm[r1];
+    }
     float sx, dx, sy, dy;
     bfly1_lo(v0, add_lo(v1, -0.0f), sx, dx);
     bfly1_hi(v0, add_hi(v1, -0.0f), sy, dy);
@@ -509,9 +536,11 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT))
   uint8_t* s_csc = s_rsc + 2 * kQScaleBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(s_csc + 2 * kQScaleBytes);
   float* s_red = reinterpret_cast<float*>(full + kQStages);  // [8 warps][2]
-  // random-sign masks of the tile: [0..3] columns (ROW layout), [4..7] rows (COL layout);
-  // the sign of column c is bit c/4 of word c%4
-  uint32_t* s_sgn = reinterpret_cast<uint32_t*>(s_red + 16);
+  // random-sign XOR masks of the tile: 64 column-pair words (ROW jobs), 128 row words
+  // (COL jobs); 16-byte aligned (s_red is 16 floats after 8-byte barriers)
+  uint32_t* s_cmask = reinterpret_cast<uint32_t*>(
+      (reinterpret_cast<uintptr_t>(s_red + 16) + 15) & ~static_cast<uintptr_t>(15));
+  uint32_t* s_rmask = s_cmask + 64;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bid = blockIdx.x, nctas = gridDim.x;
@@ -574,17 +603,18 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT))
       // signs of this tile's 128 columns (warp 0) and 128 rows (warp 1): Philox block
       // (tile start)/4 + lane holds the words of indices 4*lane .. 4*lane+3 of the tile.
       // The previous tile's jobs read the masks before its store barrier.
-      if ((kRow && warp == 0) || (kCol && warp == 1)) {
-        const uint64_t first = static_cast<uint64_t>(warp == 0 ? tc : tr) * 32u;
-        const uint4 w = philox_block(first + lane, 0u, a.sign_key);
-        const uint32_t m0 = __ballot_sync(0xffffffffu, w.x >> 31);
-        const uint32_t m1 = __ballot_sync(0xffffffffu, w.y >> 31);
-        const uint32_t m2 = __ballot_sync(0xffffffffu, w.z >> 31);
-        const uint32_t m3 = __ballot_sync(0xffffffffu, w.w >> 31);
-        if (lane == 0) {
-          uint32_t* m = s_sgn + 4 * warp;
-          m[0] = m0; m[1] = m1; m[2] = m2; m[3] = m3;
-        }
+      if (kRow && warp == 0) {
+        const uint4 w = philox_block(static_cast<uint64_t>(tc) * 32u + lane, 0u, a.sign_key);
+        // column pairs 2*lane (columns 4*lane, +1) and 2*lane+1 (columns 4*lane+2, +3)
+        *reinterpret_cast<uint2*>(s_cmask + 2 * lane) =
+            make_uint2(((w.x >> 31) << 15) | (w.y & 0x80000000u),
+                       ((w.z >> 31) << 15) | (w.w & 0x80000000u));
+      }
+      if (kCol && warp == 1) {
+        const uint4 w = philox_block(static_cast<uint64_t>(tr) * 32u + lane, 0u, a.sign_key);
+        *reinterpret_cast<uint4*>(s_rmask + 4 * lane) =
+            make_uint4((w.x >> 31) * 0x80008000u, (w.y >> 31) * 0x80008000u,
+                       (w.z >> 31) * 0x80008000u, (w.w >> 31) * 0x80008000u);
       }
     }
     const bool ok = mbar_wait(&full[st], static_cast<uint32_t>((it / kQStages) & 1), a.wait_limit_ns);
@@ -599,20 +629,15 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT))
       const int b = tid >> 7;
       {
         float2 p[32];
-        // the stride-1 butterfly is fused into the load unless random signs come first
-        constexpr bool kFuse1 = HN > 0 && !EXT;
-        if constexpr (kFuse1) load_row_job_bfly1(in, row_r, b, p);
-        else load_row_job(in, row_r, b, p);
+        // the stride-1 butterfly is fused into the widening; random signs (EXT) are
+        // XORed into the raw bf16 words before it
+        constexpr bool kFuse1 = HN > 0;
         if (rht) {
-          // lane x holds tile columns 64b + i, lane y 64b + 32 + i
-          const uint32_t m[4] = {s_sgn[0], s_sgn[1], s_sgn[2], s_sgn[3]};
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const uint32_t sx = (m[i & 3] >> (16 * b + (i >> 2))) & 1u;
-            const uint32_t sy = (m[i & 3] >> (16 * b + 8 + (i >> 2))) & 1u;
-            p[i] = make_float2(__uint_as_float(__float_as_uint(p[i].x) ^ (sx << 31)),
-                               __uint_as_float(__float_as_uint(p[i].y) ^ (sy << 31)));
-          }
+          if constexpr (kFuse1) load_row_job_bfly1<true>(in, row_r, b, p, s_cmask);
+          else load_row_job<true>(in, row_r, b, p, s_cmask);
+        } else {
+          if constexpr (kFuse1) load_row_job_bfly1(in, row_r, b, p);
+          else load_row_job(in, row_r, b, p);
         }
         fwht_x2<HN, !kFoldH16, kFuse1 ? 2 : 1>(p);
         if constexpr (AMAX) {
@@ -651,18 +676,13 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT))
       const int s = tid >> 6;
       {
         float2 p[32];
-        constexpr bool kFuse1 = HN > 0 && !EXT;
-        if constexpr (kFuse1) load_col_job_bfly1(in, col_b, col_w, s, p);
-        else load_col_job(in, col_b, col_w, s, p);
+        constexpr bool kFuse1 = HN > 0;
         if (rht) {
-          // element i of both lanes is tile row 32s + i
-          const uint32_t m[4] = {s_sgn[4], s_sgn[5], s_sgn[6], s_sgn[7]};
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const uint32_t sg = ((m[i & 3] >> (8 * s + (i >> 2))) & 1u) << 31;
-            p[i] = make_float2(__uint_as_float(__float_as_uint(p[i].x) ^ sg),
-                               __uint_as_float(__float_as_uint(p[i].y) ^ sg));
-          }
+          if constexpr (kFuse1) load_col_job_bfly1<true>(in, col_b, col_w, s, p, s_rmask);
+          else load_col_job<true>(in, col_b, col_w, s, p, s_rmask);
+        } else {
+          if constexpr (kFuse1) load_col_job_bfly1(in, col_b, col_w, s, p);
+          else load_col_job(in, col_b, col_w, s, p);
         }
         fwht_x2<HN, !kFoldH16, kFuse1 ? 2 : 1>(p);
         if constexpr (AMAX) {
