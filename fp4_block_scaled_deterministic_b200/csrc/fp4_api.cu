@@ -113,7 +113,7 @@ cudaError_t launch_q(const CUtensorMap& ti, const CUtensorMap& tr, const CUtenso
                      const QuantArgs& a, int grid, int dev, cudaStream_t s) {
   static std::atomic<uint64_t> done{0};
   auto k = quantize_kernel<FMT, HN, MODE, AMAX, EXT>;
-  constexpr int smem = kQSmemBytesOf(FMT);
+  constexpr int smem = kQSmemBytesOf(FMT, EXT);
   cudaError_t e = ensure_smem(k, smem, dev, done);
   if (e != cudaSuccess) return e;
   k<<<grid, kQThreads, smem, s>>>(ti, tr, tc, a);
@@ -228,7 +228,11 @@ fp4_status quantize_impl(const void* x, void* rcodes, void* rscales, void* ccode
     a.sign_key[0] = static_cast<uint32_t>(opts->sign_seed);
     a.sign_key[1] = static_cast<uint32_t>(opts->sign_seed >> 32);
   }
-  const int resident = (fmt == FP4_MXFP8 ? kQCtasPerSMOf(kFmtMX8) : kQCtasPerSM) * info->sm_count;
+  const bool ext = a.sr != 0 || a.rht != 0;
+  const int per_sm = fmt == FP4_MXFP8 ? kQCtasPerSMOf(kFmtMX8, false)
+                     : fmt == FP4_MXFP4 ? kQCtasPerSMOf(kFmtMX, ext)
+                                        : kQCtasPerSMOf(kFmtNV, ext);
+  const int resident = per_sm * info->sm_count;
   const int grid = a.num_tiles < resident ? a.num_tiles : resident;
 
   cudaError_t e = cudaSuccess;

@@ -30,20 +30,23 @@ namespace fp4k {
 enum { kModeRow = 1, kModeCol = 2, kModeDual = 3 };
 
 constexpr int kQThreads = 256;
-constexpr int kQCtasPerSM = 2;
-constexpr int kQStages = 2;
+// Input pipeline depth and CTAs per SM: two tiles in flight per CTA, two CTAs per SM
+// (one for MXFP8, whose 128-byte code tiles take more shared memory). One tile in
+// flight at three CTAs per SM (70 KB each) was measured 6% slower for MXFP4.
+__host__ __device__ constexpr int kQStagesOf(int fmt, bool ext) { return 2; }
 constexpr int kQBoxBytes = 128 * 64 * 2;    // 128 rows x 64 bf16
 constexpr int kQInBytes = 2 * kQBoxBytes;   // a 128 x 128 bf16 tile
 constexpr int kQScaleBytes = 1024;          // up to two 512-byte atoms
 // Staged code tile: 128 rows x 64 code bytes (FP4, 64B swizzle) or x 128 bytes (MXFP8,
 // 128B swizzle). With the larger MXFP8 staging one CTA fits per SM.
 __host__ __device__ constexpr int kQCodeBytesOf(int fmt) { return fmt == kFmtMX8 ? 128 * 128 : 128 * 64; }
-__host__ __device__ constexpr int kQSmemBytesOf(int fmt) {
-  return 1024 /*align*/ + kQStages * kQInBytes + 2 * 2 * kQCodeBytesOf(fmt) +
+__host__ __device__ constexpr int kQSmemBytesOf(int fmt, bool ext) {
+  return 1024 /*align*/ + kQStagesOf(fmt, ext) * kQInBytes + 2 * 2 * kQCodeBytesOf(fmt) +
          2 * 2 * kQScaleBytes + 256 + 1024 /* random-sign masks */;
 }
-__host__ __device__ constexpr int kQCtasPerSMOf(int fmt) { return fmt == kFmtMX8 ? 1 : kQCtasPerSM; }
-constexpr int kQSmemBytes = kQSmemBytesOf(kFmtMX);
+__host__ __device__ constexpr int kQCtasPerSMOf(int fmt, bool ext) {
+  return fmt == kFmtMX8 ? 1 : 2;
+}
 
 struct QuantArgs {
   int64_t rows, cols;
@@ -516,7 +519,7 @@ __device__ __forceinline__ void load_col_job_bfly1(const uint8_t* in, int b, int
 // EXT kernels also implement the variants selected at run time by a.rht (random +-1
 // signs along the contraction axis before the rotation) and a.sr (stochastic rounding).
 template <int FMT, int HN, int MODE, bool AMAX, bool EXT = false>
-__global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT))
+__global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
     quantize_kernel(const __grid_constant__ CUtensorMap tm_in,
                     const __grid_constant__ CUtensorMap tm_rcodes,
                     const __grid_constant__ CUtensorMap tm_ccodes, const QuantArgs a) {
@@ -529,6 +532,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT))
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* s_in = smem;
+  constexpr int kQStages = kQStagesOf(FMT, EXT);
   uint8_t* s_rcode = s_in + kQStages * kQInBytes;
   constexpr int kCodeBytes = kQCodeBytesOf(FMT);
   uint8_t* s_ccode = s_rcode + 2 * kCodeBytes;
