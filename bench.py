@@ -46,15 +46,28 @@ WORKLOAD = ("llama3.1-8b layer fwd+bwd: qkv 6144x4096, o 4096x4096, gate/up 1433
             "down 4096x14336; 8192 tokens/rank; MXFP4 + H16")
 
 
+WORKLOAD_GPT3 = ("gpt3-175b layer fwd+bwd: qkv 36864x12288, o 12288x12288, fc1 49152x12288, "
+                 "fc2 12288x49152; 4096 tokens/rank")
+
+
+def layer_table(a):
+    """(projections (name, N, K), tokens, X outlier factor) of the workload."""
+    from fp4_block_scaled_deterministic_b200 import synthetic
+    if a.workload == "gpt3":
+        return synthetic.GPT3_LAYERS, synthetic.GPT3_TOKENS, 100.0
+    return synthetic.LLAMA_LAYERS, 8192, 50.0
+
+
 def workload_name(a) -> str:
     """WORKLOAD for the default run; the same layer with the format / rotation / quantiser
     variant actually run otherwise."""
-    if a.format == "mxfp4" and a.hadamard == 16 and a.variant == "none":
+    if a.workload == "llama" and a.format == "mxfp4" and a.hadamard == 16 and a.variant == "none":
         return WORKLOAD
     tag = f"{a.format.upper()} + " + (f"H{a.hadamard}" if a.hadamard else "no rotation")
     if a.variant != "none":
         tag += f" + {a.variant} quantiser variant"
-    return WORKLOAD.rsplit(";", 1)[0] + "; " + tag
+    base = WORKLOAD_GPT3 if a.workload == "gpt3" else WORKLOAD.rsplit(";", 1)[0]
+    return base + "; " + tag
 
 
 def parse():
@@ -71,6 +84,11 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--proj", default="qkv,o,gate,up,down",
                     help="comma-separated subset of the layer's projections (profiling cases)")
+    ap.add_argument("--workload", choices=["llama", "gpt3"], default="llama",
+                    help="gpt3: the GPT-3 175B layer shapes on 4096 tokens (a parity config, "
+                         "measured for the record; the headline line is the Llama layer)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="quantise-only bandwidth sweep (one JSON line per case) instead of the step")
     ap.add_argument("--side-stream", type=int, default=1, choices=[0, 1],
                     help="1: quantise the next projection on a second stream beside the GEMMs "
                          "(per-kernel rooflines then come from the same steps on one stream)")
@@ -149,7 +167,7 @@ class LlamaLayer:
     """Inputs, quantised operands and outputs of every projection, all on the device."""
 
     def __init__(self, device, fmt, hn, tokens=8192, seed=0, names=None, variant="none",
-                 side_stream=False):
+                 side_stream=False, layers=None, outlier_mult=50.0):
         import fp4_block_scaled_deterministic_b200 as fp4
         from fp4_block_scaled_deterministic_b200 import synthetic
         self.fp4, self.fmt, self.hn, self.M = fp4, fmt, hn, tokens
@@ -157,11 +175,11 @@ class LlamaLayer:
         self.qstream = torch.cuda.Stream(device) if side_stream else None
         self.projs = []
         g = torch.Generator(device=device)
-        for i, (name, N, K) in enumerate(synthetic.LLAMA_LAYERS):
+        for i, (name, N, K) in enumerate(layers or synthetic.LLAMA_LAYERS):
             if names is not None and name not in names:
                 continue
             X = synthetic.normal(tokens, K, 1.0, seed=seed + i, outlier_frac=0.001,
-                                 outlier_mult=50.0, device=device)
+                                 outlier_mult=outlier_mult, device=device)
             W = synthetic.normal(N, K, 0.02, seed=seed + 100 + i, device=device)
             dY = synthetic.heavy_tailed_grad(tokens, N, 1e-3, seed=seed + 200 + i, device=device)
             p = {"name": name, "N": N, "K": K, "X": X, "W": W, "dY": dY}
@@ -420,6 +438,62 @@ def kernel_source_hash():
     return h.hexdigest()
 
 
+# ---------------------------------------------------------------- quantise-only sweep
+def run_sweep(a, dev):
+    """Quantise-only bandwidth sweep: tensors of 2^p elements with rows of L elements,
+    single (ROW, COL) and dual layouts; algorithmic GB/s per launch against measured HBM.
+    One JSON line per case."""
+    import fp4_block_scaled_deterministic_b200 as fp4
+    from fp4_block_scaled_deterministic_b200 import synthetic
+    fmt = FORMATS[a.format]
+    pk, pk_kind = peaks()
+    stream = torch.cuda.current_stream(dev)
+    code_b = 1.0 if fmt == 2 else 0.5
+    scale_b = 1 / 16 if fmt == 1 else 1 / 32
+    for p in (24, 28, 30):
+        for L in (4096, 14336, 49152):
+            x = synthetic.sweep_tensor(p, L, seed=p, device=dev)
+            rows, cols = x.shape
+            ts = torch.zeros(4, dtype=torch.float32, device=dev) if fmt == 1 else None
+            rq = fp4._alloc_q(rows, cols, fmt, dev)
+            cq = fp4._alloc_q(cols, rows, fmt, dev)
+            for mode in ("row", "col", "dual"):
+                def launch():
+                    if mode == "dual":
+                        st = fp4.fp4_quantize_dual(x, rq[0], rq[1], cq[0], cq[1], ts, rows, cols,
+                                                   fmt, a.hadamard, stream.cuda_stream)
+                    else:
+                        q = rq if mode == "row" else cq
+                        st = fp4.fp4_quantize(x, q[0], q[1], ts, rows, cols, fmt, a.hadamard,
+                                              fp4.ROW if mode == "row" else fp4.COL,
+                                              stream.cuda_stream)
+                    assert st == 0
+                for _ in range(3):
+                    launch()
+                torch.cuda.synchronize(dev)
+                n = 20 if p < 30 else 8
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for _ in range(n):
+                    launch()
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                ms = e0.elapsed_time(e1) / n
+                outs = 2 if mode == "dual" else 1
+                bpe = 2.0 + outs * (code_b + scale_b) + (2.0 if fmt == 1 else 0.0)
+                gbs = rows * cols * bpe / (ms * 1e-3) / 1e9
+                print(json.dumps({"sweep": "quantise", "elements": rows * cols, "p": p,
+                                  "shape": [rows, cols], "format": a.format,
+                                  "hadamard_n": a.hadamard, "mode": mode, "ms": ms,
+                                  "gbs": gbs, "bytes_per_elem": bpe,
+                                  "frac_hbm": gbs / pk["hbm_gbs"], "peak_source": pk_kind}),
+                      flush=True)
+            del x, rq, cq
+            torch.cuda.empty_cache()
+    assert fp4.fp4_check_status() == 0
+
+
 # ---------------------------------------------------------------- main
 def main():
     a = parse()
@@ -437,9 +511,14 @@ def main():
     import fp4_block_scaled_deterministic_b200 as fp4
     fp4.lib()  # fails loudly if the library is missing
     fmt = FORMATS[a.format]
-    names = [n.strip() for n in a.proj.split(",") if n.strip()]
-    layer = LlamaLayer(dev, fmt, a.hadamard, seed=1000 * rank, names=names, variant=a.variant,
-                       side_stream=bool(a.side_stream))
+    if a.sweep:
+        return run_sweep(a, dev)
+    layers, tokens, omult = layer_table(a)
+    all_names = [n for n, _, _ in layers]
+    names = [n.strip() for n in a.proj.split(",") if n.strip() in all_names] or all_names
+    layer = LlamaLayer(dev, fmt, a.hadamard, tokens=tokens, seed=1000 * rank, names=names,
+                       variant=a.variant, side_stream=bool(a.side_stream), layers=layers,
+                       outlier_mult=omult)
     stream = torch.cuda.current_stream(dev)
     from fp4_block_scaled_deterministic_b200 import dp
     allreduce = dp.allreduce_wgrad if world > 1 else None
@@ -502,7 +581,9 @@ def main():
     peak_fp4 = pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) * ratio
     avg_launch_ms = sum(gemm_ms) / len(gemm_ms)
     avg_flops = sum(per_launch_flops) / len(per_launch_flops)
-    traffic = recorded_traffic("mxfp4" if fmt == 0 else "nvfp4") if a.hadamard == 16 and len(names) == 5 else None
+    traffic = (recorded_traffic("mxfp4" if fmt == 0 else "nvfp4")
+               if a.workload == "llama" and a.hadamard == 16 and len(names) == len(all_names)
+               else None)
     roof = {"bound": "tensor", "achieved": gemm_tflops, "peak": peak_fp4, "unit": "TFLOP/s",
             "frac": gemm_tflops / peak_fp4, "traffic": traffic,
             "kernel": "gemm_fp4_pair_kernel (tcgen05 block-scaled "
@@ -523,7 +604,7 @@ def main():
            "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms / a.steps,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3" if fmt == 2 else "fp4_e2m1",
            "data": "synthetic",
-           "config": {"workload": workload_name(a) if len(names) == 5 else
+           "config": {"workload": workload_name(a) if len(names) == len(all_names) else
                       f"subset {','.join(names)} of: {workload_name(a)}",
                       "format": a.format, "hadamard_n": a.hadamard, "variant": a.variant,
                       "streams": 2 if a.side_stream else 1,
@@ -566,7 +647,8 @@ def main():
     else:
         out["e2e"] = None
 
-    if rank == 0 and world == 1 and not a.no_cpu_baseline and len(names) == 5:
+    if (rank == 0 and world == 1 and not a.no_cpu_baseline and a.workload == "llama"
+            and len(names) == len(all_names)):
         t_step, desc, cores = cpu_oracle_rate(a.cpu_seconds, fmt, a.hadamard)
         out["cpu_baseline"] = {"value": flops_step / t_step / 1e12, "unit": "TFLOP/s",
                                "cores": cores, "kind": "oracle", "sample": desc}

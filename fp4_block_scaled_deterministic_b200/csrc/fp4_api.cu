@@ -108,16 +108,28 @@ inline bool valid_format(fp4_format f) {
 inline int64_t code_bytes(int64_t elems, fp4_format f) { return f == FP4_MXFP8 ? elems : elems / 2; }
 
 // ---------------------------------------------------------------- quantise launch
-template <int FMT, int HN, int MODE, bool AMAX, bool EXT>
-cudaError_t launch_q(const CUtensorMap& ti, const CUtensorMap& tr, const CUtensorMap& tc,
-                     const QuantArgs& a, int grid, int dev, cudaStream_t s) {
+template <int FMT, int HN, int MODE, bool AMAX, bool EXT, bool BANDED>
+cudaError_t launch_q_kernel(const CUtensorMap& ti, const CUtensorMap& tr, const CUtensorMap& tc,
+                            const QuantArgs& a, int grid, int dev, cudaStream_t s) {
   static std::atomic<uint64_t> done{0};
-  auto k = quantize_kernel<FMT, HN, MODE, AMAX, EXT>;
+  auto k = quantize_kernel<FMT, HN, MODE, AMAX, EXT, BANDED>;
   constexpr int smem = kQSmemBytesOf(FMT, EXT);
   cudaError_t e = ensure_smem(k, smem, dev, done);
   if (e != cudaSuccess) return e;
   k<<<grid, kQThreads, smem, s>>>(ti, tr, tc, a);
   return cudaGetLastError();
+}
+
+// Banded tile order (a.band_c < a.tiles_c) only for the column-layout modes of the
+// plain kernels; everything else walks tiles row-major.
+template <int FMT, int HN, int MODE, bool AMAX, bool EXT>
+cudaError_t launch_q(const CUtensorMap& ti, const CUtensorMap& tr, const CUtensorMap& tc,
+                     const QuantArgs& a, int grid, int dev, cudaStream_t s) {
+  if constexpr (MODE != kModeRow && !EXT) {
+    if (a.band_c < a.tiles_c)
+      return launch_q_kernel<FMT, HN, MODE, AMAX, EXT, true>(ti, tr, tc, a, grid, dev, s);
+  }
+  return launch_q_kernel<FMT, HN, MODE, AMAX, EXT, false>(ti, tr, tc, a, grid, dev, s);
 }
 
 template <int FMT, int HN, bool AMAX, bool EXT>
@@ -212,7 +224,14 @@ fp4_status quantize_impl(const void* x, void* rcodes, void* rscales, void* ccode
   a.rows = rows;
   a.cols = cols;
   a.tiles_c = static_cast<int>(ceil_div(cols, 128));
-  const int64_t tiles = ceil_div(rows, 128) * a.tiles_c;
+  a.tiles_r = static_cast<int>(ceil_div(rows, 128));
+  const int64_t tiles = int64_t(a.tiles_r) * a.tiles_c;
+  // Bands of 32 tile columns once the column-layout codes are far larger than L2
+  // (measured: a 2^30-element dual pass 0.57 -> 0.70 of HBM; at 2^27 and below plain
+  // row-major order was 4% faster).
+  a.band_c = (do_col && !(opts && (opts->stochastic || opts->random_signs)) && a.tiles_c > 32 &&
+              code_bytes(rows * cols, fmt) > (int64_t(256) << 20))
+                 ? 32 : a.tiles_c;
   if (tiles > INT32_MAX) return FP4_ERR_SHAPE;
   a.num_tiles = static_cast<int>(tiles);
   a.row_scales = static_cast<uint8_t*>(rscales);

@@ -50,7 +50,8 @@ __host__ __device__ constexpr int kQCtasPerSMOf(int fmt, bool ext) {
 
 struct QuantArgs {
   int64_t rows, cols;
-  int tiles_c, num_tiles;
+  int tiles_c, tiles_r, num_tiles;
+  int band_c;  // tile order: see qtile_coords
   uint8_t* row_scales;   // ROW layout scales (scale matrix [rows][cols/bs])
   uint8_t* col_scales;   // COL layout scales (scale matrix [cols][rows/bs])
   int row_kb4, col_kb4;  // 512-byte atoms per 128-row block of each layout
@@ -516,9 +517,30 @@ __device__ __forceinline__ void load_col_job_bfly1(const uint8_t* in, int b, int
   }
 }
 
+// Tile order. Row-major (tile column fastest) keeps the input rows of the tiles in
+// flight long and sequential, which is best while the column-layout (transposed)
+// codes, written 64 bytes per output row per tile, can still be merged in L2. For
+// tensors whose column-layout codes far exceed L2 the host launches the BANDED kernels:
+// bands of a.band_c (32) tile columns with the tile column fastest inside a band. The
+// tiles in flight then cover about nine tile rows of one band, and each column-layout
+// row receives a 576-byte run instead of scattered 64-byte pieces.
+template <bool BANDED>
+__device__ __forceinline__ void qtile_coords(int tile, const QuantArgs& a, int& tr, int& tc) {
+  if constexpr (!BANDED) {
+    tr = tile / a.tiles_c;
+    tc = tile - tr * a.tiles_c;
+    return;
+  }
+  const int first = tile / (a.band_c * a.tiles_r) * a.band_c;
+  const int width = min(a.band_c, a.tiles_c - first);
+  const int r = tile - first * a.tiles_r;
+  tc = first + r % width;
+  tr = r / width;
+}
+
 // EXT kernels also implement the variants selected at run time by a.rht (random +-1
 // signs along the contraction axis before the rotation) and a.sr (stochastic rounding).
-template <int FMT, int HN, int MODE, bool AMAX, bool EXT = false>
+template <int FMT, int HN, int MODE, bool AMAX, bool EXT = false, bool BANDED = false>
 __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
     quantize_kernel(const __grid_constant__ CUtensorMap tm_in,
                     const __grid_constant__ CUtensorMap tm_rcodes,
@@ -578,7 +600,8 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
   const float six_r = __fmul_rn(6.0f, S_r), six_c = __fmul_rn(6.0f, S_c);
 
   auto issue_load = [&](int stage, int tile) {
-    const int tr = tile / a.tiles_c, tc = tile - tr * a.tiles_c;
+    int tr, tc;
+    qtile_coords<BANDED>(tile, a, tr, tc);
     uint8_t* dst = s_in + stage * kQInBytes;
     mbar_arrive_expect_tx(&full[stage], kQInBytes);
     tma_load_2d(dst, &tm_in, &full[stage], tc * 128, tr * 128);
@@ -601,7 +624,8 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
   float amax_r = 0.0f, amax_c = 0.0f;
   for (int it = 0; it < my_tiles; ++it) {
     const int tile = bid + it * nctas;
-    const int tr = tile / a.tiles_c, tc = tile - tr * a.tiles_c;
+    int tr, tc;
+    qtile_coords<BANDED>(tile, a, tr, tc);
     const int st = it % kQStages, ob = it & 1;
     if (rht) {
       // signs of this tile's 128 columns (warp 0) and 128 rows (warp 1): Philox block
