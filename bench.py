@@ -201,7 +201,7 @@ class LlamaLayer:
                     st = fp4.fp4_quantize_dual(p[key], row[0], row[1], col[0], col[1], ts, r, c,
                                                fmt, hn, torch.cuda.current_stream().cuda_stream)
                     assert st == 0
-        self.gemms_done = []
+        self.gemms_done, self.quant_done = [], []
         self.opts = {}
         for p in self.projs:
             for key, _ in self._operands(p):
@@ -213,9 +213,10 @@ class LlamaLayer:
                                       0x5EED0000 + seed, 0x51600000 + seed)
                 self.opts[(p["name"], key)] = o
         for _ in self.projs:
-            ev = torch.cuda.Event()
-            ev.record(torch.cuda.current_stream(device))
-            self.gemms_done.append(ev)
+            for lst in (self.gemms_done, self.quant_done):
+                ev = torch.cuda.Event()
+                ev.record(torch.cuda.current_stream(device))
+                lst.append(ev)
 
     def _operands(self, p):
         return (("X", (self.M, p["K"])), ("W", (p["N"], p["K"])), ("dY", (self.M, p["N"])))
@@ -242,10 +243,13 @@ class LlamaLayer:
         per_q = 1 if self.fmt == 0 or self.variant == "amax" else 2
         return len(self.projs) * (3 * per_q + 3)
 
-    def step(self, stream, timers=None, allreduce=None, overlap=None):
+    def step(self, stream, timers=None, allreduce=None, overlap=None, inputs_ready=None,
+             outputs_free=None):
         """One fwd+bwd pass over every projection. timers: dict kind -> list of event
         pairs to record around each quantise / GEMM launch. overlap: quantise on the
-        side stream (default: when the layer has one)."""
+        side stream (default: when the layer has one). inputs_ready[i] / outputs_free[i]:
+        events the quantisation / the GEMMs of projection i wait for (the end-to-end
+        copies); self.quant_done[i] and self.gemms_done[i] are recorded after them."""
         f, fmt, hn = self.fp4, self.fmt, self.hn
         if overlap is None:
             overlap = self.qstream is not None
@@ -265,6 +269,9 @@ class LlamaLayer:
             return r
 
         def quantise(p, qstream):
+            i = self.projs.index(p)
+            if inputs_ready is not None:
+                qstream.wait_event(inputs_ready[i])
             qs = qstream.cuda_stream
             for key, (r, c) in self._operands(p):
                 row, col, ts = p[key + "_row"], p[key + "_col"], p[key + "_ts"]
@@ -292,14 +299,16 @@ class LlamaLayer:
             for i, p in enumerate(self.projs):
                 side.wait_event(self.gemms_done[i])
                 quantise(p, side)
-                ev = torch.cuda.Event()
-                ev.record(side)
-                ready.append(ev)
+                self.quant_done[i].record(side)
+                ready.append(self.quant_done[i])
         for i, p in enumerate(self.projs):
             if side is None:
                 quantise(p, stream)
+                self.quant_done[i].record(stream)
             else:
                 stream.wait_event(ready[i])
+            if outputs_free is not None:
+                stream.wait_event(outputs_free[i])
             tsx, tsw, tsy = p["X_ts"], p["W_ts"], p["dY_ts"]
             nv = fmt == 1
             M, N, K = self.M, p["N"], p["K"]
@@ -318,8 +327,7 @@ class LlamaLayer:
                 p["dY_col"][0], p["dY_col"][1], tsy[1:2] if nv else None, p["X_col"][0],
                 p["X_col"][1], tsx[1:2] if nv else None, p["dW"], N, K, M, fmt, 0, s))
             assert st == 0
-            if side is not None:
-                self.gemms_done[i].record(stream)
+            self.gemms_done[i].record(stream)
             if allreduce is not None:
                 pending.append(allreduce(p["dW"]))
         for w in pending:
@@ -622,16 +630,37 @@ def main():
                      for t in (p["Y"], p["dX"], p["dW"])] for p in layer.projs]
         barrier()
 
+        # Copies run on their own streams, per projection: the inputs of projection i
+        # arrive while earlier projections compute, and its outputs leave while later
+        # ones compute (PCIe carries both directions at once). Events keep every copy
+        # ordered with the kernels that read or overwrite the same buffers.
+        h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        n = len(layer.projs)
+        in_ready = [torch.cuda.Event() for _ in range(n)]
+        out_free = [torch.cuda.Event() for _ in range(n)]
+        for ev in out_free:
+            ev.record(stream)
+
         def e2e_step():
-            for p, hin in zip(layer.projs, host_in):
-                p["X"].copy_(hin[0], non_blocking=True)
-                p["W"].copy_(hin[1], non_blocking=True)
-                p["dY"].copy_(hin[2], non_blocking=True)
-            layer.step(stream, None, allreduce)
-            for p, hout in zip(layer.projs, host_out):
-                hout[0].copy_(p["Y"], non_blocking=True)
-                hout[1].copy_(p["dX"], non_blocking=True)
-                hout[2].copy_(p["dW"], non_blocking=True)
+            for i, (p, hin) in enumerate(zip(layer.projs, host_in)):
+                h2d.wait_event(layer.quant_done[i])  # last step's readers of these inputs
+                with torch.cuda.stream(h2d):
+                    p["X"].copy_(hin[0], non_blocking=True)
+                    p["W"].copy_(hin[1], non_blocking=True)
+                    p["dY"].copy_(hin[2], non_blocking=True)
+                in_ready[i].record(h2d)
+            layer.step(stream, None, allreduce, inputs_ready=in_ready, outputs_free=out_free)
+            if allreduce is not None:
+                d2h.wait_stream(stream)  # dW is final only after its all-reduce
+            for i, (p, hout) in enumerate(zip(layer.projs, host_out)):
+                d2h.wait_event(layer.gemms_done[i])
+                with torch.cuda.stream(d2h):
+                    hout[0].copy_(p["Y"], non_blocking=True)
+                    hout[1].copy_(p["dX"], non_blocking=True)
+                    hout[2].copy_(p["dW"], non_blocking=True)
+                out_free[i].record(d2h)
+            stream.wait_event(out_free[n - 1])  # the step ends when its last output is home
+            stream.wait_stream(d2h)
 
         e2e_step()
         barrier()
