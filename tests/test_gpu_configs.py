@@ -141,3 +141,22 @@ def test_sweep_large_sampled_rows(orc, row_len, p, fmt, hn):
     cols = np.sort(rng.choice(cq.rows, 16, replace=False))
     _check_rows(orc, rq, _oracle_rows(orc, xc, ROW, rows, fmt, hn), rows, fmt)
     _check_rows(orc, cq, _oracle_rows(orc, xc, COL, cols, fmt, hn), cols, fmt)
+
+
+@pytest.mark.parametrize("fmt,row_len", [(0, 14336), (0, 49152), (1, 49152)])
+def test_sweep_2p30_banded_tile_order_sampled_rows(orc, fmt, row_len):
+    """2^30-element tensors whose column-layout codes exceed 256 MB take the banded tile
+    order (bands of 32 tile columns): sampled rows of both layouts bit-exact, tensor
+    scales of both layouts bit-exact for NVFP4."""
+    x = synthetic.sweep_tensor(30, row_len, seed=9, device="cuda")
+    assert x.shape[1] // 128 > 32 and x.numel() // 2 > (256 << 20)
+    rq, cq = fp4.quantize_dual(x, fmt, 16)
+    torch.cuda.synchronize()
+    assert fp4.fp4_check_status() == 0
+    xc = x.cpu()
+    del x
+    rng = np.random.default_rng(10)
+    rows = np.sort(rng.choice(rq.rows, 12, replace=False))
+    cols = np.sort(rng.choice(cq.rows, 12, replace=False))
+    _check_rows(orc, rq, _oracle_rows(orc, xc, ROW, rows, fmt, 16), rows, fmt)
+    _check_rows(orc, cq, _oracle_rows(orc, xc, COL, cols, fmt, 16), cols, fmt)
