@@ -31,7 +31,7 @@ def _deq(orc, q, fmt):
 
 @pytest.mark.parametrize("shape", [(256, 384, 512), (160, 96, 224), (1024, 768, 256)])
 @pytest.mark.parametrize("hn", [16, 32])
-@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("fmt", [0, 1, 2])  # MXFP4, NVFP4, the MXFP8 comparator
 def test_three_passes(orc, fmt, hn, shape):
     M, N, K = shape
     X, W, dY = _inputs(M, N, K, seed=M + K)
