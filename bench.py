@@ -82,6 +82,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-budget", type=float, default=None,
+                    help="reference arm: oracle seconds per step (default: fills ~2 minutes)")
     ap.add_argument("--proj", default="qkv,o,gate,up,down",
                     help="comma-separated subset of the layer's projections (profiling cases)")
     ap.add_argument("--workload", choices=["llama", "gpt3"], default="llama",
@@ -342,7 +344,8 @@ def gemm_flops_of(layer):
 
 
 # ---------------------------------------------------------------- CPU baseline
-def cpu_oracle_rate(seconds_budget: float, fmt: int, hn: int):
+def cpu_oracle_rate(seconds_budget: float, fmt: int, hn: int, layers=None, tokens: int = 8192,
+                    outlier_mult: float = 50.0):
     """Time the oracle on a bounded sample of the same step: dual quantisation of a
     row slice of every operand and a sample of GEMM outputs of every pass. Returns
     (extrapolated seconds per full step, description, cores used)."""
@@ -350,7 +353,8 @@ def cpu_oracle_rate(seconds_budget: float, fmt: int, hn: int):
     import oracle
     from fp4_block_scaled_deterministic_b200 import synthetic
     oracle.build()
-    M = 8192
+    layers = layers or synthetic.LLAMA_LAYERS
+    M = tokens
     rows = 64
     n_ent = 48
     q_time, q_elems, g_time, g_macs = 0.0, 0, 0.0, 0
@@ -358,9 +362,9 @@ def cpu_oracle_rate(seconds_budget: float, fmt: int, hn: int):
     rounds = 0
     # repeat the per-projection sample until the time budget is used (at least once)
     while rounds == 0 or time.perf_counter() - t_start < seconds_budget:
-        for i, (name, N, K) in enumerate(synthetic.LLAMA_LAYERS):
+        for i, (name, N, K) in enumerate(layers):
             X = synthetic.normal(rows * 2, K, 1.0, seed=i + 10 * rounds, outlier_frac=0.001,
-                                 outlier_mult=50.0)
+                                 outlier_mult=outlier_mult)
             W = synthetic.normal(rows * 2, K, 0.02, seed=100 + i + 10 * rounds)
             t0 = time.perf_counter()
             xq = oracle.quantize(X, fmt, hn, oracle.ROW)
@@ -378,7 +382,7 @@ def cpu_oracle_rate(seconds_budget: float, fmt: int, hn: int):
         rounds += 1
     # full step: dual quantisation of X, W, dY of each projection, and 3 GEMMs
     step_elems, step_macs = 0, 0
-    for name, N, K in synthetic.LLAMA_LAYERS:
+    for name, N, K in layers:
         step_elems += 2 * (M * K + N * K + M * N)
         step_macs += 3 * M * N * K
     t_step = q_time / q_elems * step_elems + g_time / g_macs * step_macs
@@ -395,16 +399,17 @@ def run_reference(a):
     if rank != 0:
         return
     fmt = FORMATS[a.format]
-    from fp4_block_scaled_deterministic_b200 import synthetic
-    flops = sum(3 * 2.0 * 8192 * N * K for _, N, K in synthetic.LLAMA_LAYERS)
-    budget = min(20.0, max(2.0, 120.0 / (a.steps + a.warmup)))
+    layers, tokens, omult = layer_table(a)
+    flops = sum(3 * 2.0 * tokens * N * K for _, N, K in layers)
+    budget = min(20.0, max(2.0, 120.0 / (a.steps + a.warmup))) if a.cpu_budget is None \
+        else a.cpu_budget
     for _ in range(a.warmup):
-        cpu_oracle_rate(1.0, fmt, a.hadamard)
+        cpu_oracle_rate(min(1.0, budget), fmt, a.hadamard, layers, tokens, omult)
     ts = []
     desc = ""
     t0 = time.perf_counter()
     for _ in range(a.steps):
-        t_step, desc, cores = cpu_oracle_rate(budget, fmt, a.hadamard)
+        t_step, desc, cores = cpu_oracle_rate(budget, fmt, a.hadamard, layers, tokens, omult)
         ts.append(t_step)
     wall = time.perf_counter() - t0
     t_med = statistics.median(ts)

@@ -1,0 +1,73 @@
+"""Host logic of bench.py that needs no GPU: argument defaults, workload naming, the
+GEMM traffic record's source check, and the reference arm (the oracle timed on the
+host cores) printing its JSON line."""
+import io
+import json
+import os
+import sys
+from contextlib import redirect_stdout
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _args(*argv):
+    old = sys.argv
+    sys.argv = ["bench.py", *argv]
+    try:
+        return bench.parse()
+    finally:
+        sys.argv = old
+
+
+def test_defaults_follow_the_contract():
+    a = _args()
+    assert a.gpus == 1 and a.steps >= 1 and a.warmup >= 3 and a.impl == "fp4"
+    assert a.format == "mxfp4" and a.hadamard == 16 and a.side_stream == 1
+    assert _args("--warmup", "1").warmup == 3  # at least three warm-up steps
+
+
+def test_workload_names():
+    assert bench.workload_name(_args()) == bench.WORKLOAD
+    assert "NVFP4 + H32" in bench.workload_name(_args("--format", "nvfp4", "--hadamard", "32"))
+    assert "sr quantiser variant" in bench.workload_name(_args("--variant", "sr"))
+    g = bench.workload_name(_args("--workload", "gpt3", "--hadamard", "0"))
+    assert g.startswith("gpt3-175b") and "no rotation" in g
+    with pytest.raises(SystemExit):
+        _args("--variant", "amax")  # a supplied amax is NVFP4 only
+
+
+def test_layer_tables():
+    from fp4_block_scaled_deterministic_b200 import synthetic
+    layers, tokens, mult = bench.layer_table(_args("--workload", "gpt3"))
+    assert layers == synthetic.GPT3_LAYERS and tokens == 4096 and mult == 100.0
+    layers, tokens, mult = bench.layer_table(_args())
+    assert layers == synthetic.LLAMA_LAYERS and tokens == 8192 and mult == 50.0
+
+
+def test_traffic_record_is_tied_to_the_gemm_sources():
+    rec = json.load(open(os.path.join(ROOT, "profiles", "gemm_llama_traffic.json")))
+    assert bench.kernel_source_hash() == bench.kernel_source_hash()
+    got = bench.recorded_traffic("mxfp4")
+    if rec["source_sha1"] == bench.kernel_source_hash():
+        assert got == rec["per_launch_bytes"]["mxfp4"] and got > 0
+    else:
+        assert got is None  # the kernel changed since the counters were taken
+    assert bench.recorded_traffic("no-such-kernel") is None
+
+
+def test_reference_arm_prints_one_json_line():
+    a = _args("--impl", "reference", "--steps", "1", "--warmup", "3", "--cpu-budget", "0.1")
+    out = io.StringIO()
+    with redirect_stdout(out):
+        bench.run_reference(a)
+    lines = [ln for ln in out.getvalue().splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["higher_is_better"] is True
+    assert d["config"]["workload"] == bench.WORKLOAD
