@@ -4,9 +4,15 @@
 //
 // with deq = e2m1 * 2^(byte-127) (MXFP4, 32-element blocks) or e2m1 * ue4m3(byte)
 // (NVFP4, 16-element blocks; the fp32 tensor scales S_A * S_B are applied in the
-// epilogue). Accumulation is fp32 in tensor memory. [gist.science summary of arXiv
+// epilogue), or e4m3 * 2^(byte-127) for the MXFP8 comparator (one byte per element).
+// Accumulation is fp32 in tensor memory. [gist.science summary of arXiv
 // 2605.09825, Methodology item 2 (all three GEMM passes in FP4); molayo1419.me
 // NVFP4/MaxText page, Key facts bullet 5 (FP4 tensor cores on Blackwell).]
+//
+// Two kernels share the MMA issue loop (Issuer) and the epilogue (store_row_segment):
+// gemm_fp4_pair_kernel (CTA pairs, cta_group::2, 256x256 tiles; every M > 128, and
+// all MXFP8) and gemm_fp4_kernel (one CTA, 128x256 tiles; FP4 with M <= 128), the
+// latter described here:
 //
 // Design (one CTA per SM, persistent over 128x256 output tiles, K in slabs of 256):
 //   warp 0   : TMA producer. Per slab it loads A 128x128 B, B 256x128 B (128B swizzle)

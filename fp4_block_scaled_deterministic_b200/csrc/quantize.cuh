@@ -17,10 +17,16 @@
 // memory in jobs of two 32-element vectors held lane-wise in float2 registers:
 //   ROW job = one row, 64 consecutive columns (two segments; 8 conflict-free 16-B reads);
 //   COL job = two adjacent columns, 32 consecutive rows (32 conflict-free 4-B reads);
-// the rotation runs in registers with packed fp32x2 arithmetic, codes are staged in a
-// 64B-swizzled [128][64 B] tile and written by a TMA store, scale atoms are assembled
-// in shared memory (1-, 2- and 4-byte stores) and written by bulk copies. Staging is
-// double-buffered so stores overlap the next tile.
+// the rotation runs in registers with packed fp32x2 arithmetic (its first stage fused
+// into the bf16 widening), codes are staged in a 64B-swizzled [128][64 B] tile and
+// written by a TMA store, scale atoms are assembled in shared memory (1-, 2- and 4-byte
+// stores) and written by bulk copies. Staging is double-buffered so stores overlap the
+// next tile.
+//
+// Also here: the MXFP8 comparator (E4M3 codes, one byte each, 128-byte code tiles,
+// one CTA per SM); the EXT instances with the quantiser variants (random Hadamard
+// signs, Philox-driven stochastic rounding); the BANDED instances, whose tile order
+// suits tensors with very large column-layout outputs.
 #pragma once
 
 #include "common.cuh"
