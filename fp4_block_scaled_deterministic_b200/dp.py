@@ -30,8 +30,10 @@ def token_shard(total_tokens: int, rank: int, world: int, block: int = 32) -> tu
 
 
 def allreduce_wgrad(dW: torch.Tensor, group=None, async_op: bool = True):
-    """Sum the partial weight gradients of all ranks in place (fixed NCCL/gloo
-    algorithm per world size, so the result is run-to-run deterministic)."""
+    """Sum the partial weight gradients of all ranks in place. The sum's rounding
+    order is that of the collective's algorithm: NCCL picks it from the message size
+    and the topology (ring, tree or in-switch NVLS), the same choice on every run of
+    one configuration; NCCL_ALGO=Ring pins one fixed order across configurations."""
     return dist.all_reduce(dW, op=dist.ReduceOp.SUM, group=group, async_op=async_op)
 
 
