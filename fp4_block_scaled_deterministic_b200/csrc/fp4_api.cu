@@ -331,7 +331,7 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a, const CUtensorMap& b, const C
   std::call_once(once[dev], [&] {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * g_dev[dev].sm_count / 2, 1, 1);
-    cfg.blockDim = dim3(kGThreads, 1, 1);
+    cfg.blockDim = dim3(PairCfg<FMT>::kThreads, 1, 1);
     cfg.dynamicSmemBytes = PairCfg<FMT>::kSmemBytes;
     cudaLaunchAttribute attr;
     attr.id = cudaLaunchAttributeClusterDimension;
@@ -348,7 +348,7 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a, const CUtensorMap& b, const C
     max_pairs[dev] = n;
   });
   const int pairs = g.num_tiles < max_pairs[dev] ? g.num_tiles : max_pairs[dev];
-  k<<<2 * pairs, kGThreads, PairCfg<FMT>::kSmemBytes, s>>>(a, b, sa, sb, g);
+  k<<<2 * pairs, PairCfg<FMT>::kThreads, PairCfg<FMT>::kSmemBytes, s>>>(a, b, sa, sb, g);
   return cudaGetLastError();
 }
 

@@ -38,6 +38,9 @@ namespace fp4k {
 constexpr int kGBM = 128, kGBN = 256, kGBK = 256;  // tile M, tile N, K elements per slab
 constexpr int kGStages = 4;
 constexpr int kGThreads = 320;
+// Scale-copy threads of the pair kernel (warps 10, 11, ...; see Issuer::run_copies).
+constexpr int kGPairCopyThreads = 2;
+static_assert(kGPairCopyThreads >= 1 && kGPairCopyThreads <= 2, "one or two copy threads");
 constexpr int kGABytes = kGBM * kGBK / 2;  // 16 KB
 constexpr int kGBBytes = kGBN * kGBK / 2;  // 32 KB
 
@@ -132,7 +135,7 @@ struct SlabCursor {
   int stage;
   uint32_t phase;
   uint64_t dA, dB, dSA, dSB;
-  uint32_t t_sf, slot;
+  uint32_t t_sf, slot, sf_phase;
 };
 
 template <int FMT, bool PAIR, int SLAB_K, int STAGES, int A_BYTES, int B_BYTES, int SFA_BYTES,
@@ -151,7 +154,13 @@ struct Issuer {
       c.dA += A_BYTES >> 4; c.dB += B_BYTES >> 4;
       c.dSA += SFA_BYTES >> 4; c.dSB += SFB_BYTES >> 4;
     }
-    if (++c.slot == SF_BUFS) { c.slot = 0; c.t_sf = base.t_sf; } else { c.t_sf += SF_COLS; }
+    if (++c.slot == SF_BUFS) {
+      c.slot = 0;
+      c.t_sf = base.t_sf;
+      c.sf_phase ^= 1u;
+    } else {
+      c.t_sf += SF_COLS;
+    }
   }
   // Scale-factor copies [lo, hi) of a slab into its TMEM ring slot (t_sfb = t_sfa + 4*atoms).
   template <int LO, int HI>
@@ -207,20 +216,96 @@ struct Issuer {
     else tc_commit(bar);
   }
 
+  __device__ __forceinline__ static SlabCursor make_base(uint32_t tmem, uint8_t* sA, uint8_t* sB,
+                                                         uint8_t* sSFA, uint8_t* sSFB) {
+    SlabCursor b;
+    b.stage = 0;
+    b.phase = 0;
+    b.dA = desc_kmajor_sw128(smem_u32(sA));
+    b.dB = desc_kmajor_sw128(smem_u32(sB));
+    b.dSA = desc_sf_atom(smem_u32(sSFA));
+    b.dSB = desc_sf_atom(smem_u32(sSFB));
+    b.t_sf = tmem + 256;
+    b.slot = 0;
+    b.sf_phase = 0;
+    return b;
+  }
+
+  // Split issue (pair kernel). Issuing a slab's scale copies and its MMAs from one thread
+  // takes that thread longer than the tensor cores take to run the MMAs, so the copies go
+  // to other threads (run_copies, each a share [LO, HI) of the slab's copies) that walk
+  // the same slabs: each waits for the stage, copies its scales into the slab's ring slot
+  // and commits them to sf_full[slot], which completes when every copy thread has
+  // arrived; the MMA thread (run_split) waits on sf_full instead of the stage barrier. The TMA
+  // data of the stage is complete before the copy thread sees full[stage], hence before
+  // sf_full[slot] completes. A slot is rewritten only after full[] of a slab SF_BUFS
+  // later, whose load waited for the MMAs of the slab STAGES back; SF_BUFS >= STAGES makes
+  // those the slot's previous readers (or later ones), so no slot is overwritten early.
+  static_assert(SF_BUFS >= STAGES, "scale ring must cover the stage ring");
+  template <int LO, int HI>
+  __device__ static void run_copies(uint32_t tmem, uint8_t* sA, uint8_t* sB, uint8_t* sSFA,
+                                    uint8_t* sSFB, uint64_t* full, uint64_t* sf_full,
+                                    uint64_t* drained, volatile int* abort_flag, int first,
+                                    int stride, const GemmArgs& g) {
+    const SlabCursor base = make_base(tmem, sA, sB, sSFA, sSFB);
+    SlabCursor cur = base;
+    const int my_tiles = first < g.num_tiles ? (g.num_tiles - first + stride - 1) / stride : 0;
+    for (int t = 0; t < my_tiles && !*abort_flag; ++t) {
+      bool ok = true;
+      for (int kt = 0; kt < g.k_tiles; ++kt) {
+        if (!mbar_wait(&full[cur.stage], cur.phase, g.wait_limit_ns)) {
+          ok = false;
+          break;
+        }
+        copies<LO, HI>(cur);
+        tc_commit_pair_mc(&sf_full[cur.slot], 0x1);
+        step(cur, base);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        break;
+      }
+    }
+    // Every copy this thread issued has landed before TMEM can be released.
+    tc_commit_pair_mc(drained, 0x1);
+    if (!mbar_wait(drained, 0u, g.wait_limit_ns)) *abort_flag = 1;
+  }
+  __device__ static void run_split(uint32_t tmem, uint8_t* sA, uint8_t* sB, uint8_t* sSFA,
+                                   uint8_t* sSFB, uint64_t* sf_full, uint64_t* empty,
+                                   uint64_t* acc_full, uint64_t* acc_empty,
+                                   volatile int* abort_flag, int first, int stride,
+                                   const GemmArgs& g) {
+    const SlabCursor base = make_base(tmem, sA, sB, sSFA, sSFB);
+    SlabCursor cur = base;
+    const int my_tiles = first < g.num_tiles ? (g.num_tiles - first + stride - 1) / stride : 0;
+    uint32_t acc_phase = 0;
+    for (int t = 0; t < my_tiles; ++t) {
+      if (!mbar_wait(acc_empty, acc_phase ^ 1u, g.wait_limit_ns) || *abort_flag) {
+        *abort_flag = 1;
+        return;
+      }
+      tc_fence_after();
+      for (int kt = 0; kt < g.k_tiles; ++kt) {
+        if (!mbar_wait(&sf_full[cur.slot], cur.sf_phase, g.wait_limit_ns)) {
+          *abort_flag = 1;
+          return;
+        }
+        tc_fence_after();
+        slab_mmas<0>(cur, tmem, kt == 0);
+        commit(&empty[cur.stage]);
+        step(cur, base);
+      }
+      commit(acc_full);
+      acc_phase ^= 1u;
+    }
+  }
+
   // Runs all tiles of this CTA (or CTA pair): tiles first, first+stride, ... < num_tiles.
   __device__ static void run(uint32_t tmem, uint8_t* sA, uint8_t* sB, uint8_t* sSFA,
                              uint8_t* sSFB, uint64_t* full, uint64_t* empty, uint64_t* acc_full,
                              uint64_t* acc_empty, volatile int* abort_flag, int first,
                              int stride, const GemmArgs& g) {
-    SlabCursor base;
-    base.stage = 0;
-    base.phase = 0;
-    base.dA = desc_kmajor_sw128(smem_u32(sA));
-    base.dB = desc_kmajor_sw128(smem_u32(sB));
-    base.dSA = desc_sf_atom(smem_u32(sSFA));
-    base.dSB = desc_sf_atom(smem_u32(sSFB));
-    base.t_sf = tmem + 256;
-    base.slot = 0;
+    SlabCursor base = make_base(tmem, sA, sB, sSFA, sSFB);
     SlabCursor cur = base;
     const int my_tiles = first < g.num_tiles ? (g.num_tiles - first + stride - 1) / stride : 0;
     uint32_t acc_phase = 0;
@@ -462,21 +547,30 @@ struct PairCfg {
   static constexpr int kSFBBytes = 2 * kAtoms * 512; // scales of all 256 B rows
   static constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
   static constexpr int kStages = FMT == kFmtNV ? 5 : 3;
+  // MXFP8 (6 copies per 8 MMAs) keeps the copies in the MMA thread: there the extra wait
+  // of the split issue costs more than it saves.
+  static constexpr int kCopyThreads = FMT == kFmtMX8 ? 0 : kGPairCopyThreads;
+  static constexpr int kThreads = kGThreads + 32 * kCopyThreads;
   static constexpr int kSFCols = 12 * kAtoms;
-  static constexpr int kSFBufs = 4;
+  // At least one ring slot per stage (the split issue's reuse rule): 5 x 48 columns for
+  // NVFP4, 4 x 48 for MXFP4, 4 x 24 for MXFP8, after the 256 accumulator columns.
+  static constexpr int kSFBufs = kStages > 4 ? kStages : 4;
   static constexpr int kTmemSF = 256;
+  static_assert(kTmemSF + kSFBufs * kSFCols <= 512, "TMEM columns");
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 256;
 };
 
 
 template <int FMT, int OUT_BF16>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<FMT>::kThreads, 1)
     gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmSFA,
                          const __grid_constant__ CUtensorMap tmSFB, const GemmArgs g) {
   using Cfg = PairCfg<FMT>;
   constexpr int S = Cfg::kStages;
+  using PairIssuer = Issuer<FMT, true, Cfg::kSlabK, S, Cfg::kABytes, Cfg::kBBytes,
+                            Cfg::kSFABytes, Cfg::kSFBBytes, Cfg::kSFCols, Cfg::kSFBufs>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -489,8 +583,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
   uint64_t* empty = bars + S;
   uint64_t* acc_full = bars + 2 * S;
   uint64_t* acc_empty = acc_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  uint64_t* sf_full = acc_empty + 1;           // one per scale ring slot
+  uint64_t* cp_drained = sf_full + Cfg::kSFBufs;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cp_drained + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  static_assert((2 * S + 3 + Cfg::kSFBufs) * 8 + 8 <= 256, "barrier area");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -507,6 +604,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 16);  // 8 epilogue warps in each CTA of the pair
+    if constexpr (Cfg::kCopyThreads > 0) {
+      for (int i = 0; i < Cfg::kSFBufs; ++i) mbar_init(&sf_full[i], Cfg::kCopyThreads);
+      mbar_init(cp_drained, Cfg::kCopyThreads);
+    }
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -555,10 +656,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
       // ------------------------------------------------------------ MMA issuer (leader)
-      Issuer<FMT, true, Cfg::kSlabK, S, Cfg::kABytes, Cfg::kBBytes, Cfg::kSFABytes,
-             Cfg::kSFBBytes, Cfg::kSFCols, Cfg::kSFBufs>::run(tmem, sA, sB, sSFA, sSFB, full,
-                                                              empty, acc_full, acc_empty,
-                                                              abort_flag, pair, npairs, g);
+      if constexpr (Cfg::kCopyThreads > 0)
+        PairIssuer::run_split(tmem, sA, sB, sSFA, sSFB, sf_full, empty, acc_full, acc_empty,
+                              abort_flag, pair, npairs, g);
+      else
+        PairIssuer::run(tmem, sA, sB, sSFA, sSFB, full, empty, acc_full, acc_empty,
+                        abort_flag, pair, npairs, g);
+    }
+  } else if (warp >= kGThreads / 32) {
+    if (lane == 0 && rank == 0) {
+      // ------------------------------------------------------------ scale copies (leader)
+      constexpr int kC = PairIssuer::kCopies;
+      constexpr int kN = Cfg::kCopyThreads > 0 ? Cfg::kCopyThreads : 1;
+      const int ci = warp - kGThreads / 32;
+      if (ci == 0)
+        PairIssuer::template run_copies<0, kC / kN>(tmem, sA, sB, sSFA, sSFB, full, sf_full,
+                                                    cp_drained, abort_flag, pair, npairs, g);
+      else
+        PairIssuer::template run_copies<kC / kN, kC>(tmem, sA, sB, sSFA, sSFB, full, sf_full,
+                                                     cp_drained, abort_flag, pair, npairs, g);
     }
   } else {
     // -------------------------------------------------------------- epilogue (both CTAs)
