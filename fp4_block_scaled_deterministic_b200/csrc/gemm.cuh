@@ -529,6 +529,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
 // pair-wide MMAs; both CTAs load through TMA into their own shared memory with the
 // transfers counted on the leader's barrier, and both drain their own half of the
 // accumulator (rows 128*rank ... +128, all 256 columns) from their own TMEM.
+// Roles: warp 0 of both CTAs loads; in the leader, warp 1 issues the MMAs and (MXFP4,
+// NVFP4) warps 10 and 11 issue the scale copies, half a slab each (Issuer::run_copies);
+// warps 2-9 of both CTAs run the epilogue. MXFP8 launches without warps 10-11 and
+// copies its scales from the MMA thread.
 // The loads carry no multicast; only the tcgen05.commit arrivals are multicast to the
 // two CTAs of the pair.
 template <int FMT>
