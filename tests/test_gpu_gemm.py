@@ -99,7 +99,9 @@ def test_gemm_is_deterministic(orc):
 def test_gemm_full_llama_gate_sampled(orc, fmt):
     """Fprop of the Llama-3.1-8B gate projection at full size (M=8192, N=14336,
     K=4096, H16), the benchmark's launch configuration: operands bit-exact against
-    the oracle, 512 sampled outputs within the tolerance, bf16 = RN(fp32)."""
+    the oracle, 512 sampled outputs within the tolerance against the oracle's own
+    sums, the whole output within the tolerance against an fp64 library matmul of the
+    oracle-dequantised operands, bf16 = RN(fp32)."""
     X, W, _ = synthetic.llama_layer("gate")
     qa = fp4.quantize(X.cuda(), fmt, 16)
     qb = fp4.quantize(W.cuda(), fmt, 16)
@@ -117,6 +119,13 @@ def test_gemm_full_llama_gate_sampled(orc, fmt):
     got = C[torch.from_numpy(ms).cuda(), torch.from_numpy(ns).cuda()].cpu().numpy()
     assert rel_fro(got, ref) <= TOL
     assert torch.equal(Cb.view(torch.int16), C.to(torch.bfloat16).view(torch.int16))
+    # Whole output: deq(A) deq(B)^T in fp64 (operands dequantised by the oracle).
+    da = torch.from_numpy(orc.dequantize(*oa, fmt)).cuda()
+    db = torch.from_numpy(orc.dequantize(*ob, fmt)).cuda()
+    full = da @ db.T
+    del da, db
+    err = float((C.double() - full).norm() / full.norm())
+    assert err <= TOL, err
 
 
 @pytest.mark.parametrize("shape", [(160, 96, 224), (384, 512, 1024), (96, 320, 256)])
