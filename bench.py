@@ -40,6 +40,7 @@ sys.path.insert(0, ROOT)
 METRIC = "FP4 GEMM TFLOPS (fprop/dgrad/wgrad) + H16-quantize GB/s, % of B200 roofline"
 FP4_OVER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput (9 : 2.25 PFLOP/s)
 FP8_OVER_BF16 = 2.0  # nominal dense FP8 : BF16 (4.5 : 2.25 PFLOP/s), for the MXFP8 comparator
+DATASHEET_TFLOPS = {"fp4": 9000.0, "fp8": 4500.0}  # B200 dense tensor peaks (HGX datasheet)
 FORMATS = {"mxfp4": 0, "nvfp4": 1, "mxfp8": 2}
 PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 WORKLOAD = ("llama3.1-8b layer fwd+bwd: qkv 6144x4096, o 4096x4096, gate/up 14336x4096, "
@@ -81,7 +82,8 @@ def parse():
     ap.add_argument("--hadamard", type=int, default=16, choices=[0, 16, 32])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=20.0,
+                    help="oracle seconds of the CPU baseline (half on one thread, half on all)")
     ap.add_argument("--cpu-budget", type=float, default=None,
                     help="reference arm: oracle seconds per step (default: fills ~2 minutes)")
     ap.add_argument("--proj", default="qkv,o,gate,up,down",
@@ -169,7 +171,7 @@ class LlamaLayer:
     """Inputs, quantised operands and outputs of every projection, all on the device."""
 
     def __init__(self, device, fmt, hn, tokens=8192, seed=0, names=None, variant="none",
-                 side_stream=False, layers=None, outlier_mult=50.0):
+                 side_stream=False, layers=None, outlier_mult=50.0, w_seed=0):
         import fp4_block_scaled_deterministic_b200 as fp4
         from fp4_block_scaled_deterministic_b200 import synthetic
         self.fp4, self.fmt, self.hn, self.M = fp4, fmt, hn, tokens
@@ -182,7 +184,7 @@ class LlamaLayer:
                 continue
             X = synthetic.normal(tokens, K, 1.0, seed=seed + i, outlier_frac=0.001,
                                  outlier_mult=outlier_mult, device=device)
-            W = synthetic.normal(N, K, 0.02, seed=seed + 100 + i, device=device)
+            W = synthetic.normal(N, K, 0.02, seed=w_seed + 100 + i, device=device)
             dY = synthetic.heavy_tailed_grad(tokens, N, 1e-3, seed=seed + 200 + i, device=device)
             p = {"name": name, "N": N, "K": K, "X": X, "W": W, "dY": dY}
             for key, (r, c) in (("X", (tokens, K)), ("W", (N, K)), ("dY", (tokens, N))):
@@ -344,15 +346,44 @@ def gemm_flops_of(layer):
 
 
 # ---------------------------------------------------------------- CPU baseline
+def host_facts() -> dict:
+    """The host the CPU baseline ran on: logical CPUs, the affinity mask of this
+    process, and the CPU model."""
+    model = None
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                model = ln.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    aff = sorted(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else []
+    runs, start = [], None
+    for i, c in enumerate(aff):  # compress the mask to ranges, e.g. "0-63,128-191"
+        if start is None:
+            start = c
+        if i + 1 == len(aff) or aff[i + 1] != c + 1:
+            runs.append(f"{start}-{c}" if c != start else f"{c}")
+            start = None
+    return {"cpu_count": os.cpu_count(), "affinity": ",".join(runs),
+            "affinity_cpus": len(aff), "cpu_model": model}
+
+
+def host_threads() -> int:
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+
+
 def cpu_oracle_rate(seconds_budget: float, fmt: int, hn: int, layers=None, tokens: int = 8192,
-                    outlier_mult: float = 50.0):
+                    outlier_mult: float = 50.0, threads: int = 1):
     """Time the oracle on a bounded sample of the same step: dual quantisation of a
-    row slice of every operand and a sample of GEMM outputs of every pass. Returns
-    (extrapolated seconds per full step, description, cores used)."""
+    row slice of every operand and a sample of GEMM outputs of every pass, on
+    `threads` host threads (1 = the serial build). Returns (extrapolated seconds per
+    full step, description, threads used)."""
     import numpy as np
     import oracle
     from fp4_block_scaled_deterministic_b200 import synthetic
     oracle.build()
+    threads = oracle.set_threads(threads)
     layers = layers or synthetic.LLAMA_LAYERS
     M = tokens
     rows = 64
@@ -386,11 +417,14 @@ def cpu_oracle_rate(seconds_budget: float, fmt: int, hn: int, layers=None, token
         step_elems += 2 * (M * K + N * K + M * N)
         step_macs += 3 * M * N * K
     t_step = q_time / q_elems * step_elems + g_time / g_macs * step_macs
-    desc = (f"oracle (scalar C, 1 thread): {rounds} rounds of dual quantisation of {rows * 2}-row "
+    oracle.set_threads(1)
+    desc = (f"oracle (scalar C, {threads} thread{'s' if threads > 1 else ''}"
+            f"{', OpenMP over rows and entries' if threads > 1 else ''}): {rounds} rounds of "
+            f"dual quantisation of {rows * 2}-row "
             f"slices of X and W of each projection and {n_ent} GEMM outputs per projection "
             f"({q_elems} elements, {g_macs} MACs, {q_time + g_time:.1f} s of oracle time), "
             f"extrapolated linearly to the full step")
-    return t_step, desc, 1
+    return t_step, desc, threads
 
 
 # ---------------------------------------------------------------- reference arm
@@ -403,13 +437,16 @@ def run_reference(a):
     flops = sum(3 * 2.0 * tokens * N * K for _, N, K in layers)
     budget = min(20.0, max(2.0, 120.0 / (a.steps + a.warmup))) if a.cpu_budget is None \
         else a.cpu_budget
+    threads = host_threads()
     for _ in range(a.warmup):
-        cpu_oracle_rate(min(1.0, budget), fmt, a.hadamard, layers, tokens, omult)
+        cpu_oracle_rate(min(1.0, budget), fmt, a.hadamard, layers, tokens, omult, threads)
     ts = []
     desc = ""
+    cores = threads
     t0 = time.perf_counter()
     for _ in range(a.steps):
-        t_step, desc, cores = cpu_oracle_rate(budget, fmt, a.hadamard, layers, tokens, omult)
+        t_step, desc, cores = cpu_oracle_rate(budget, fmt, a.hadamard, layers, tokens, omult,
+                                              threads)
         ts.append(t_step)
     wall = time.perf_counter() - t0
     t_med = statistics.median(ts)
@@ -420,8 +457,10 @@ def run_reference(a):
             "data": "synthetic", "impl": "reference",
             "config": {"workload": workload_name(a), "format": a.format, "hadamard_n": a.hadamard,
                        "l2": "n/a (CPU)"},
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-                             "sample": desc, "wall_s": wall},
+            "extrapolated": True,
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": desc, "wall_s": wall, "extrapolated": True,
+                             "host": host_facts()},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -508,10 +547,36 @@ def run_sweep(a, dev):
 
 
 # ---------------------------------------------------------------- main
+def spawn_ranks(a) -> int:
+    """`--gpus N` (N > 1) started as a plain process: re-launch this command as N ranks
+    of one node through torch.distributed.run (one process per GPU, rendezvous on
+    127.0.0.1), and return its exit status. Fails loudly when fewer than N GPUs are
+    visible."""
+    import socket
+    have = torch.cuda.device_count()
+    if have < a.gpus:
+        print(f"bench.py: --gpus {a.gpus} needs {a.gpus} visible CUDA devices, found {have}",
+              file=sys.stderr, flush=True)
+        return 2
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={a.gpus}", "--master-addr=127.0.0.1", f"--master-port={port}",
+           os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
 def main():
     a = parse()
     if a.impl == "reference":
         return run_reference(a)
+    if a.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(spawn_ranks(a))
+    if a.gpus != int(os.environ.get("WORLD_SIZE", "1")):
+        print(f"bench.py: --gpus {a.gpus} but WORLD_SIZE={os.environ.get('WORLD_SIZE', '1')}",
+              file=sys.stderr, flush=True)
+        sys.exit(2)
     import torch.distributed as dist
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -529,12 +594,13 @@ def main():
     layers, tokens, omult = layer_table(a)
     all_names = [n for n, _, _ in layers]
     names = [n.strip() for n in a.proj.split(",") if n.strip() in all_names] or all_names
+    # data parallel: every rank holds the same W (replicated weights) and its own tokens
     layer = LlamaLayer(dev, fmt, a.hadamard, tokens=tokens, seed=1000 * rank, names=names,
                        variant=a.variant, side_stream=bool(a.side_stream), layers=layers,
-                       outlier_mult=omult)
+                       outlier_mult=omult, w_seed=0)
     stream = torch.cuda.current_stream(dev)
     from fp4_block_scaled_deterministic_b200 import dp
-    allreduce = dp.allreduce_wgrad if world > 1 else None
+    allreduce = (lambda t: dp.allreduce_wgrad(t, async_op=True)) if world > 1 else None
 
     def barrier():
         if world > 1:
@@ -591,7 +657,11 @@ def main():
 
     pk, pk_kind = peaks()
     ratio = FP8_OVER_BF16 if fmt == 2 else FP4_OVER_BF16
-    peak_fp4 = pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) * ratio
+    # the GEMM is timed launch by launch in a sub-second loop: the burst bf16 figure x the
+    # nominal FP4 (FP8) : BF16 ratio; the datasheet dense peak and the sustained figure
+    # are reported beside it
+    peak_fp4 = pk["bf16_tflops"] * ratio
+    sheet = DATASHEET_TFLOPS["fp8" if fmt == 2 else "fp4"]
     avg_launch_ms = sum(gemm_ms) / len(gemm_ms)
     avg_flops = sum(per_launch_flops) / len(per_launch_flops)
     traffic = (recorded_traffic("mxfp4" if fmt == 0 else "nvfp4")
@@ -599,6 +669,9 @@ def main():
                else None)
     roof = {"bound": "tensor", "achieved": gemm_tflops, "peak": peak_fp4, "unit": "TFLOP/s",
             "frac": gemm_tflops / peak_fp4, "traffic": traffic,
+            "frac_datasheet": gemm_tflops / sheet, "peak_datasheet": sheet,
+            "frac_sustained": gemm_tflops / (pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+                                             * ratio),
             "kernel": "gemm_fp4_pair_kernel (tcgen05 block-scaled "
                       f"{'MXFP8, kind::mxf8f6f4' if fmt == 2 else 'FP4'}, CTA pairs)",
             "per_launch": {"avg_flops": avg_flops, "avg_ms": avg_launch_ms,
@@ -606,8 +679,9 @@ def main():
             "timing": ("CUDA events around each launch over the timed steps" if not a.side_stream
                        else "CUDA events around each launch over the same number of steps run "
                             "on one stream just before the overlapped timed region"),
-            "peak_source": f"{pk_kind}: bf16_tflops_sustained x {ratio} (nominal "
-                           f"{'FP8' if fmt == 2 else 'FP4'}:BF16)"}
+            "peak_source": f"{pk_kind}: bf16_tflops (burst) x {ratio} (nominal "
+                           f"{'FP8' if fmt == 2 else 'FP4'}:BF16); frac_datasheet against the "
+                           f"B200 dense {'FP8' if fmt == 2 else 'FP4'} datasheet peak"}
     qroof = {"bound": "hbm", "achieved": quant_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
              "frac": quant_gbs / pk["hbm_gbs"], "bytes_per_elem": bpe,
              "kernel": "quantize_kernel dual layout", "launches": len(quant_ms),
@@ -617,6 +691,7 @@ def main():
            "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms / a.steps,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3" if fmt == 2 else "fp4_e2m1",
            "data": "synthetic",
+           "dw_reduction": (dp.REDUCTION if world > 1 else None),
            "config": {"workload": workload_name(a) if len(names) == len(all_names) else
                       f"subset {','.join(names)} of: {workload_name(a)}",
                       "format": a.format, "hadamard_n": a.hadamard, "variant": a.variant,
@@ -683,9 +758,14 @@ def main():
 
     if (rank == 0 and world == 1 and not a.no_cpu_baseline and a.workload == "llama"
             and len(names) == len(all_names)):
-        t_step, desc, cores = cpu_oracle_rate(a.cpu_seconds, fmt, a.hadamard)
-        out["cpu_baseline"] = {"value": flops_step / t_step / 1e12, "unit": "TFLOP/s",
-                               "cores": cores, "kind": "oracle", "sample": desc}
+        t1, desc1, _ = cpu_oracle_rate(a.cpu_seconds / 2, fmt, a.hadamard, threads=1)
+        tn, descn, cores = cpu_oracle_rate(a.cpu_seconds / 2, fmt, a.hadamard,
+                                           threads=host_threads())
+        out["cpu_baseline"] = {"value": flops_step / tn / 1e12, "unit": "TFLOP/s",
+                               "cores": cores, "kind": "oracle", "sample": descn,
+                               "extrapolated": True, "host": host_facts(),
+                               "single_thread": {"value": flops_step / t1 / 1e12,
+                                                 "cores": 1, "sample": desc1}}
     if world > 1:
         dist.barrier(device_ids=[local])
         dist.destroy_process_group()

@@ -559,23 +559,30 @@ __global__ void wait_selftest_kernel(uint64_t limit_ns) {
 // stand-in); it passes the device address looked up once per device below.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[FP4_NOALLOC_SCRATCH_BYTES];
 
-void* g_noalloc_ptr[kMaxDevices];
-cudaError_t g_noalloc_err[kMaxDevices];
-std::once_flag g_noalloc_once[kMaxDevices];
+std::atomic<void*> g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mutex;
 
-// Device address of the scratch array on the current device (looked up on the first
-// call for that device, with that device current).
+// Device address of the scratch array on the current device, looked up with that
+// device current. Only a successful lookup is cached: a failed one (for example a
+// module load refused during a stream capture) clears the CUDA error it raised, so
+// later calls and status checks do not see it, and is retried on the next call.
 fp4_status noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FP4_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return FP4_ERR_UNSUPPORTED_DEVICE;
-  std::call_once(g_noalloc_once[dev], [dev] {
-    void* p = nullptr;
-    g_noalloc_err[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    g_noalloc_ptr[dev] = g_noalloc_err[dev] == cudaSuccess ? p : nullptr;
-  });
-  if (g_noalloc_err[dev] != cudaSuccess || !g_noalloc_ptr[dev]) return FP4_ERR_CUDA;
-  *out = g_noalloc_ptr[dev];
+  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (!p) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    p = g_noalloc_ptr[dev].load(std::memory_order_relaxed);
+    if (!p) {
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+        (void)cudaGetLastError();
+        return FP4_ERR_CUDA;
+      }
+      g_noalloc_ptr[dev].store(p, std::memory_order_release);
+    }
+  }
+  *out = p;
   return FP4_OK;
 }
 

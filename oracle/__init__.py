@@ -24,25 +24,56 @@ BLOCK = {MXFP4: 32, NVFP4: 16, MXFP8: 32}
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "fp4_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
+_LIB_OMP = os.path.join(_HERE, "liboracle_omp.so")
 _lib = None
+_libs = {}
+_threads = 1
+
+
+def _compile(out: str, extra) -> None:
+    if os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(_SRC):
+        return
+    cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
+           "-shared", *extra, _SRC, "-o", out + ".tmp", "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(out + ".tmp", out)
 
 
 def build(force: bool = False) -> str:
-    """Compile fp4_oracle.c with gcc. No fast-math and no FP contraction, so every
+    """Compile fp4_oracle.c with gcc, twice: serial (liboracle.so, the default) and
+    with OpenMP (liboracle_omp.so, for the all-core CPU baseline; its pragmas only
+    split independent rows or entries). No fast-math and no FP contraction, so every
     fp32 operation rounds once, as IEEE 754 prescribes."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
-               "-shared", _SRC, "-o", _LIB + ".tmp", "-lm"]
-        subprocess.run(cmd, check=True)
-        os.replace(_LIB + ".tmp", _LIB)
+    if force:
+        for f in (_LIB, _LIB_OMP):
+            if os.path.exists(f):
+                os.remove(f)
+    _compile(_LIB, [])
+    _compile(_LIB_OMP, ["-fopenmp"])
     return _LIB
+
+
+def set_threads(n: int) -> int:
+    """Run the oracle on n host threads from now on (1 = the serial build, the
+    default; n > 1 = the OpenMP build). Returns the thread count in use."""
+    global _lib, _threads
+    _threads = max(1, int(n))
+    _lib = None
+    return _L().fp4o_set_threads(_threads)
 
 
 def _L():
     global _lib
     if _lib is None:
         build()
-        lib = ctypes.CDLL(_LIB)
+        path = _LIB if _threads == 1 else _LIB_OMP
+        if path in _libs:
+            _lib = _libs[path]
+            _lib.fp4o_set_threads(_threads)
+            return _lib
+        lib = ctypes.CDLL(path)
+        lib.fp4o_set_threads.restype = ctypes.c_int
+        lib.fp4o_set_threads.argtypes = [ctypes.c_int]
         P = ctypes.c_void_p
         i64 = ctypes.c_int64
         lib.fp4o_e2m1_decode.restype = ctypes.c_double
@@ -112,6 +143,8 @@ def _L():
             f = getattr(lib, name)
             f.restype = None
             f.argtypes = [t_in, t_out, i64]
+        lib.fp4o_set_threads(_threads)
+        _libs[path] = lib
         _lib = lib
     return _lib
 

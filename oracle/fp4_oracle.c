@@ -88,6 +88,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define FP4O_MXFP4 0
 #define FP4O_NVFP4 1
@@ -282,16 +285,21 @@ int fp4o_rotate_opt(const uint16_t *x, int64_t rows, int64_t cols, int hn, int a
                     uint64_t rht_seed, float *out) {
     int64_t R = axis == FP4O_ROW ? rows : cols, C = axis == FP4O_ROW ? cols : rows;
     if (hn != 0 && (C % hn) != 0) return -1;
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < R; r++)
         for (int64_t c = 0; c < C; c++)
             out[r * C + c] = fp4o_bf16_to_f32(axis == FP4O_ROW ? x[r * cols + c] : x[c * cols + r]);
-    if (rht)
+    if (rht) {
+#pragma omp parallel for schedule(static)
         for (int64_t c = 0; c < C; c++)
             if (fp4o_rht_negate(rht_seed, c))
                 for (int64_t r = 0; r < R; r++) out[r * C + c] = -out[r * C + c];
-    if (hn != 0)
+    }
+    if (hn != 0) {
+#pragma omp parallel for schedule(static)
         for (int64_t r = 0; r < R; r++)
             for (int64_t g = 0; g < C; g += hn) fp4o_fwht_f32(out + r * C + g, hn);
+    }
     return 0;
 }
 
@@ -431,18 +439,23 @@ int fp4o_quantize_opt(const uint16_t *x, int64_t rows, int64_t cols, int fmt, in
     float S = 1.0f;
     if (fmt == FP4O_NVFP4) {
         float T = 0.0f;
-        if (amax_in) T = *amax_in;
-        else
+        if (amax_in) {
+            T = *amax_in;
+        } else {
+            /* a max is exact and order independent, so splitting it changes nothing */
+#pragma omp parallel for schedule(static) reduction(max : T)
             for (int64_t i = 0; i < R * C; i++) T = fmaxf(T, fabsf(v[i]));
+        }
         S = fp4o_nv_tensor_scale(T);
         if (nv_scale_out) *nv_scale_out = S;
         if (nv_amax_out) *nv_amax_out = T;
     }
     /* steps 4-5: block scales and codes; step 6: pack */
     memset(scales, 0, (size_t)fp4o_scale_layout_bytes(R, KB));
-    uint8_t blk[32];
-    uint32_t w[32];
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < R; r++) {
+        uint8_t blk[32];
+        uint32_t w[32];
         for (int64_t kb = 0; kb < KB; kb++) {
             const float *bv = v + r * C + kb * bs;
             if (sr)
@@ -471,6 +484,7 @@ int fp4o_quantize_mxfp8(const uint16_t *x, int64_t rows, int64_t cols, int hn, i
     if (!v) return -2;
     fp4o_rotate(x, rows, cols, hn, axis, v);
     memset(scales, 0, (size_t)fp4o_scale_layout_bytes(R, KB));
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < R; r++) {
         for (int64_t kb = 0; kb < KB; kb++) {
             const float *bv = v + r * C + kb * 32;
@@ -514,6 +528,7 @@ static double deq_elem(const uint8_t *codes, const uint8_t *scales, double S, in
 void fp4o_dequantize(const uint8_t *codes, const uint8_t *scales, float tensor_scale, int64_t R,
                      int64_t C, int fmt, double *out) {
     double S = fmt == FP4O_NVFP4 ? (double)tensor_scale : 1.0;
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < R; r++)
         for (int64_t c = 0; c < C; c++) out[r * C + c] = deq_elem(codes, scales, S, C, fmt, r, c);
 }
@@ -522,6 +537,7 @@ void fp4o_dequantize(const uint8_t *codes, const uint8_t *scales, float tensor_s
 
 /* C[m][n] = sum_k A[m][k] * B[n][k] in fp64 (both operands K-major). */
 void fp4o_gemm_f64(const double *A, const double *B, double *Cm, int64_t M, int64_t N, int64_t K) {
+#pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; m++)
         for (int64_t n = 0; n < N; n++) {
             double acc = 0.0;
@@ -537,6 +553,7 @@ void fp4o_gemm_entries(const uint8_t *a_codes, const uint8_t *a_scales, float a_
                        int fmt, const int64_t *ms, const int64_t *ns, int64_t count, double *out) {
     double SA = fmt == FP4O_NVFP4 ? (double)a_ts : 1.0;
     double SB = fmt == FP4O_NVFP4 ? (double)b_ts : 1.0;
+#pragma omp parallel for schedule(dynamic, 1)
     for (int64_t i = 0; i < count; i++) {
         double acc = 0.0;
         for (int64_t k = 0; k < K; k++)
@@ -558,4 +575,19 @@ void fp4o_e4m3_encode_array(const float *t, uint8_t *out, int64_t n) {
 
 void fp4o_mx_scale_exponent_array(const float *a, int32_t *out, int64_t n) {
     for (int64_t i = 0; i < n; i++) out[i] = fp4o_mx_scale_exponent(a[i]);
+}
+
+/* ---------------------------------------------------------------- threads */
+
+/* Threads of the OpenMP build (the same source compiled with -fopenmp; the pragmas
+ * above split independent rows, columns or entries and never a rounding step).
+ * n > 0 sets the count; returns the count in use (1 in the serial build). */
+int fp4o_set_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
 }

@@ -14,6 +14,11 @@ def pytest_configure(config):
 
 @pytest.fixture(scope="session")
 def orc():
+    """The CPU oracle, on every host thread this process may use (its OpenMP build
+    splits independent rows and entries only, so the results are those of the serial
+    build)."""
     import oracle
     oracle.build()
+    n = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    oracle.set_threads(n)
     return oracle

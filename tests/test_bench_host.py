@@ -68,6 +68,31 @@ def test_reference_arm_prints_one_json_line():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["value"] > 0
-    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["extrapolated"] is True and d["cpu_baseline"]["extrapolated"] is True
+    host = d["cpu_baseline"]["host"]
+    assert host["cpu_count"] >= 1 and host["affinity_cpus"] >= 1 and "cpu_model" in host
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["higher_is_better"] is True
     assert d["config"]["workload"] == bench.WORKLOAD
+
+
+def test_host_facts_and_threads():
+    h = bench.host_facts()
+    assert h["cpu_count"] == os.cpu_count() and h["affinity_cpus"] == bench.host_threads()
+    assert h["affinity"]  # e.g. "0-7"
+
+
+def test_gpus_n_spawns_ranks_or_fails_loudly():
+    """`bench.py --gpus 2` as a plain process re-launches itself as two ranks; without
+    two visible GPUs it stops with a clear error and exit status 2 instead of running
+    one rank and calling it two."""
+    import subprocess
+    import torch
+    if torch.cuda.device_count() >= 2:
+        pytest.skip("host has two GPUs: the spawn would run the real benchmark")
+    env = dict(os.environ)
+    env.pop("WORLD_SIZE", None)
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                        "--steps", "1"], capture_output=True, text=True, env=env, timeout=300)
+    assert r.returncode == 2
+    assert "needs 2 visible CUDA devices" in r.stderr

@@ -33,17 +33,31 @@ def _init(rank, world, port, timeout_s=30):
                             timeout=timedelta(seconds=timeout_s))
 
 
+def _partial_dw(oracle, X, dY, rank, world, fmt):
+    """This rank's fp32 partial dW: the oracle's Wgrad of its token shard (the GPU GEMM
+    writes fp32 dW)."""
+    a, b = dp.token_shard(X.shape[0], rank, world)
+    Xs, dYs = X[a:b].contiguous(), dY[a:b].contiguous()
+    qa = oracle.quantize(dYs, fmt, 16, oracle.COL)
+    qb = oracle.quantize(Xs, fmt, 16, oracle.COL)
+    part = oracle.gemm_f64(oracle.dequantize(*qa[:3], fmt), oracle.dequantize(*qb[:3], fmt))
+    return part.astype(np.float32), (Xs, dYs)
+
+
+def _inputs(M=128, N=64, K=96):
+    X = synthetic.normal(M, K, 1.0, seed=3, outlier_frac=0.02, outlier_mult=50.0)
+    dY = synthetic.heavy_tailed_grad(M, N, seed=4)
+    return X, dY
+
+
 def _wgrad_worker(rank, world, port, fmt, out_q):
     try:
         import sys
         sys.path.insert(0, ROOT)
         import oracle
         _init(rank, world, port)
-        M, N, K = 128, 64, 96
-        X = synthetic.normal(M, K, 1.0, seed=3, outlier_frac=0.02, outlier_mult=50.0)
-        dY = synthetic.heavy_tailed_grad(M, N, seed=4)
-        a, b = dp.token_shard(M, rank, world)
-        Xs, dYs = X[a:b].contiguous(), dY[a:b].contiguous()
+        X, dY = _inputs()
+        part, (Xs, dYs) = _partial_dw(oracle, X, dY, rank, world, fmt)
         if fmt == oracle.NVFP4:
             # global tensor amax: each rank's amax of its rotated shard, max over ranks
             amax = torch.tensor([oracle.rotate(dYs, 16, oracle.COL).__abs__().max(),
@@ -51,10 +65,7 @@ def _wgrad_worker(rank, world, port, fmt, out_q):
                                 dtype=torch.float32)
             dp.allreduce_amax_(amax)
             out_q.put((rank, "amax", amax.numpy().tolist()))
-        qa = oracle.quantize(dYs, fmt, 16, oracle.COL)
-        qb = oracle.quantize(Xs, fmt, 16, oracle.COL)
-        part = oracle.gemm_f64(oracle.dequantize(*qa[:3], fmt), oracle.dequantize(*qb[:3], fmt))
-        t = torch.from_numpy(part)
+        t = torch.from_numpy(part.copy())
         work = dp.allreduce_wgrad(t, async_op=True)
         work.wait()
         slowest = dp.max_over_ranks(float(rank + 1), "cpu")
@@ -96,23 +107,39 @@ def _run(fn, world, *args):
     return results
 
 
-@pytest.mark.parametrize("fmt", [0])
-def test_dp_wgrad_equals_single_rank_wgrad(orc, fmt):
-    res = _run(_wgrad_worker, 2, fmt)
-    errs = [r for r in res if r[1] == "error"]
-    assert not errs, errs[0][2]
-    dws = [r for r in res if r[1] == "dW"]
-    assert len(dws) == 2
-    M, N, K = 128, 64, 96
-    X = synthetic.normal(M, K, 1.0, seed=3, outlier_frac=0.02, outlier_mult=50.0)
-    dY = synthetic.heavy_tailed_grad(M, N, seed=4)
+@pytest.mark.parametrize("world", [2, 4])
+def test_dp_wgrad_is_the_rank_ordered_sum(orc, world):
+    """The reduced dW equals, bit for bit, the sum of the ranks' fp32 partials added in
+    rank order, on every rank and on two runs; it is within fp32 rounding of the
+    single-rank Wgrad over all tokens."""
+    fmt = 0
+    runs = []
+    for _ in range(2):
+        res = _run(_wgrad_worker, world, fmt)
+        errs = [r for r in res if r[1] == "error"]
+        assert not errs, errs[0][2]
+        dws = sorted((r for r in res if r[1] == "dW"), key=lambda r: r[0])
+        assert len(dws) == world
+        assert all(r[3] == float(world) for r in dws)  # max over ranks of (rank + 1)
+        runs.append([r[2] for r in dws])
+    X, dY = _inputs()
+    acc = _partial_dw(orc, X, dY, 0, world, fmt)[0].copy()
+    for r in range(1, world):
+        acc += _partial_dw(orc, X, dY, r, world, fmt)[0]  # one fp32 rounding per addition
+    for run in runs:
+        for d in run:
+            assert d.dtype == np.float32 and np.array_equal(d.view(np.uint32), acc.view(np.uint32))
     qa = orc.quantize(dY, fmt, 16, orc.COL)
     qb = orc.quantize(X, fmt, 16, orc.COL)
     full = orc.gemm_f64(orc.dequantize(*qa[:3], fmt), orc.dequantize(*qb[:3], fmt))
-    for r in dws:
-        assert np.allclose(r[2], full, rtol=1e-12, atol=1e-12)
-        assert r[3] == 2.0  # max over ranks of (rank + 1)
-    assert np.array_equal(dws[0][2], dws[1][2])
+    assert np.linalg.norm(acc - full) <= 1e-6 * np.linalg.norm(full)
+
+
+def test_rank_ordered_sum_is_sequential():
+    parts = torch.tensor([[1.0], [2.0 ** -24], [2.0 ** -24]], dtype=torch.float32)
+    # ((1 + 2^-24) + 2^-24) = 1 in fp32 (each tie rounds to even); 1 + (2^-24 + 2^-24) would not
+    assert dp.rank_ordered_sum_(parts).item() == 1.0
+    assert dp.rank_ordered_sum_(parts.flip(0)).item() == 1.0 + 2.0 ** -23
 
 
 def test_nvfp4_global_amax_matches_single_rank(orc):
@@ -121,9 +148,7 @@ def test_nvfp4_global_amax_matches_single_rank(orc):
     assert not errs, errs[0][2]
     amaxes = [r[2] for r in res if r[1] == "amax"]
     assert len(amaxes) == 2 and amaxes[0] == amaxes[1]
-    M, N, K = 128, 64, 96
-    X = synthetic.normal(M, K, 1.0, seed=3, outlier_frac=0.02, outlier_mult=50.0)
-    dY = synthetic.heavy_tailed_grad(M, N, seed=4)
+    X, dY = _inputs()
     full_dy = orc.quantize(dY, 1, 16, orc.COL)[3]
     full_x = orc.quantize(X, 1, 16, orc.COL)[3]
     assert np.float32(amaxes[0][0]) == np.float32(full_dy)
