@@ -62,11 +62,14 @@ def layer_table(a):
 def workload_name(a) -> str:
     """WORKLOAD for the default run; the same layer with the format / rotation / quantiser
     variant actually run otherwise."""
-    if a.workload == "llama" and a.format == "mxfp4" and a.hadamard == 16 and a.variant == "none":
+    if (a.workload == "llama" and a.format == "mxfp4" and a.hadamard == 16 and a.variant == "none"
+            and getattr(a, "next_layer_quant", "none") == "none"):
         return WORKLOAD
     tag = f"{a.format.upper()} + " + (f"H{a.hadamard}" if a.hadamard else "no rotation")
     if a.variant != "none":
         tag += f" + {a.variant} quantiser variant"
+    if getattr(a, "next_layer_quant", "none") != "none":
+        tag += f" + Y quantised for the next layer ({a.next_layer_quant})"
     base = WORKLOAD_GPT3 if a.workload == "gpt3" else WORKLOAD.rsplit(";", 1)[0]
     return base + "; " + tag
 
@@ -96,6 +99,10 @@ def parse():
     ap.add_argument("--side-stream", type=int, default=1, choices=[0, 1],
                     help="1: quantise the next projection on a second stream beside the GEMMs "
                          "(per-kernel rooflines then come from the same steps on one stream)")
+    ap.add_argument("--next-layer-quant", choices=["none", "standalone", "fused"], default="none",
+                    help="also quantise each Fprop output Y row-wise (MXFP4, same rotation) for "
+                         "the next layer: by a separate quantise launch after the GEMM, or in "
+                         "the GEMM's epilogue (fp4_gemm_quant)")
     ap.add_argument("--variant", choices=["none", "sr", "rht", "sr+rht", "amax"], default="none",
                     help="quantiser variant: stochastic rounding, randomised Hadamard signs, "
                          "both, or (NVFP4) a supplied tensor amax instead of the amax pass")
@@ -103,6 +110,8 @@ def parse():
     a.warmup = max(3, a.warmup)
     if a.variant == "amax" and a.format != "nvfp4":
         ap.error("--variant amax needs --format nvfp4")
+    if a.next_layer_quant != "none" and a.format != "mxfp4":
+        ap.error("--next-layer-quant quantises Y as MXFP4: it needs --format mxfp4")
     return a
 
 
@@ -171,11 +180,12 @@ class LlamaLayer:
     """Inputs, quantised operands and outputs of every projection, all on the device."""
 
     def __init__(self, device, fmt, hn, tokens=8192, seed=0, names=None, variant="none",
-                 side_stream=False, layers=None, outlier_mult=50.0, w_seed=0):
+                 side_stream=False, layers=None, outlier_mult=50.0, w_seed=0, next_quant="none"):
         import fp4_block_scaled_deterministic_b200 as fp4
         from fp4_block_scaled_deterministic_b200 import synthetic
         self.fp4, self.fmt, self.hn, self.M = fp4, fmt, hn, tokens
         self.variant = variant
+        self.next_quant = next_quant
         self.qstream = torch.cuda.Stream(device) if side_stream else None
         self.projs = []
         g = torch.Generator(device=device)
@@ -192,6 +202,8 @@ class LlamaLayer:
                 p[key + "_col"] = self._qbuf(c, r, device)
                 p[key + "_ts"] = torch.zeros(4, dtype=torch.float32, device=device)
             p["Y"] = torch.empty(tokens, N, dtype=torch.bfloat16, device=device)
+            if next_quant != "none":  # Y quantised row-wise (along N) for the next layer
+                p["Yq"] = self._qbuf(tokens, N, device)
             p["dX"] = torch.empty(tokens, K, dtype=torch.bfloat16, device=device)
             p["dW"] = torch.empty(N, K, dtype=torch.float32, device=device)
             self.projs.append(p)
@@ -245,7 +257,7 @@ class LlamaLayer:
     def launches_per_step(self):
         # NVFP4 adds the amax pass (plus a memset) unless the amax is supplied
         per_q = 1 if self.fmt == 0 or self.variant == "amax" else 2
-        return len(self.projs) * (3 * per_q + 3)
+        return len(self.projs) * (3 * per_q + 3 + (self.next_quant == "standalone"))
 
     def step(self, stream, timers=None, allreduce=None, overlap=None, inputs_ready=None,
              outputs_free=None):
@@ -317,10 +329,19 @@ class LlamaLayer:
             nv = fmt == 1
             M, N, K = self.M, p["N"], p["K"]
             # Fprop: Y[M][N] = X_row . W_row^T
-            st = timed("gemm", lambda: f.fp4_gemm(
-                p["X_row"][0], p["X_row"][1], tsx[0:1] if nv else None, p["W_row"][0],
-                p["W_row"][1], tsw[0:1] if nv else None, p["Y"], M, N, K, fmt, 1, s))
+            if self.next_quant == "fused":  # and Q_row(Y) from the same epilogue
+                st = timed("gemm", lambda: f.fp4_gemm_quant(
+                    p["X_row"][0], p["X_row"][1], None, p["W_row"][0], p["W_row"][1], None,
+                    p["Y"], p["Yq"][0], p["Yq"][1], M, N, K, fmt, hn, s))
+            else:
+                st = timed("gemm", lambda: f.fp4_gemm(
+                    p["X_row"][0], p["X_row"][1], tsx[0:1] if nv else None, p["W_row"][0],
+                    p["W_row"][1], tsw[0:1] if nv else None, p["Y"], M, N, K, fmt, 1, s))
             assert st == 0
+            if self.next_quant == "standalone":  # Q_row(Y) by a separate launch
+                st = timed("quant_y", lambda: f.fp4_quantize(
+                    p["Y"], p["Yq"][0], p["Yq"][1], None, M, N, fmt, hn, 0, s))
+                assert st == 0
             # Dgrad: dX[M][K] = dY_row . W_col^T  (contraction over N)
             st = timed("gemm", lambda: f.fp4_gemm(
                 p["dY_row"][0], p["dY_row"][1], tsy[0:1] if nv else None, p["W_col"][0],
@@ -597,7 +618,7 @@ def main():
     # data parallel: every rank holds the same W (replicated weights) and its own tokens
     layer = LlamaLayer(dev, fmt, a.hadamard, tokens=tokens, seed=1000 * rank, names=names,
                        variant=a.variant, side_stream=bool(a.side_stream), layers=layers,
-                       outlier_mult=omult, w_seed=0)
+                       outlier_mult=omult, w_seed=0, next_quant=a.next_layer_quant)
     stream = torch.cuda.current_stream(dev)
     from fp4_block_scaled_deterministic_b200 import dp
     allreduce = (lambda t: dp.allreduce_wgrad(t, async_op=True)) if world > 1 else None
@@ -612,7 +633,7 @@ def main():
     barrier()
     assert fp4.fp4_check_status() == 0
 
-    timers = {"quant": [], "gemm": []}
+    timers = {"quant": [], "gemm": [], "quant_y": []}
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     if a.side_stream:
@@ -695,6 +716,7 @@ def main():
            "config": {"workload": workload_name(a) if len(names) == len(all_names) else
                       f"subset {','.join(names)} of: {workload_name(a)}",
                       "format": a.format, "hadamard_n": a.hadamard, "variant": a.variant,
+                      "next_layer_quant": a.next_layer_quant,
                       "streams": 2 if a.side_stream else 1,
                       "tokens_per_rank": layer.M,
                       "l2": f"inputs larger than L2 ({(layer.bytes_in() + layer.bytes_out()) / 1e9:.1f} GB per step)",
@@ -702,6 +724,13 @@ def main():
            "gemm_tflops": gemm_tflops, "quantize_gbs": quant_gbs,
            "roofline": roof, "roofline_quantize": qroof, "clocks": clk,
            "gpu_launches": layer.launches_per_step() * a.steps}
+    if a.next_layer_quant != "none":
+        qy = [x.elapsed_time(y) for x, y in timers["quant_y"]]
+        out["next_layer_quant"] = {
+            "mode": a.next_layer_quant,
+            "what": "each Fprop output Y quantised row-wise (MXFP4, same rotation) for the next "
+                    "layer, by a separate launch (standalone) or in the GEMM epilogue (fused)",
+            "standalone_launch_avg_ms": (sum(qy) / len(qy)) if qy else None}
 
     # end to end through the C ABI from pinned host buffers (inputs H2D, outputs D2H)
     if not a.no_e2e:

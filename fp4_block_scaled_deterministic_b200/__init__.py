@@ -27,12 +27,15 @@ FPROP, DGRAD, WGRAD = 0, 1, 2
 BLOCK = {MXFP4: 32, NVFP4: 16, MXFP8: 32}
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libfp4.so")
+# FP4_DEBUG_BOUNDS=1 in the environment selects the debug build (device-side range
+# checks; fp4_check_status reports FP4_ERR_BOUNDS), same ABI and results.
+LIB_PATH = os.path.join(_PKG, "libfp4_debug.so" if os.environ.get("FP4_DEBUG_BOUNDS") == "1"
+                        else "libfp4.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "fp4.h")
 
 STATUS = {0: "FP4_OK", 1: "FP4_ERR_INVALID_ARG", 2: "FP4_ERR_SHAPE", 3: "FP4_ERR_ALIGN",
           4: "FP4_ERR_UNSUPPORTED_DEVICE", 5: "FP4_ERR_CUDA", 6: "FP4_ERR_TIMEOUT",
-          7: "FP4_ERR_WORKSPACE"}
+          7: "FP4_ERR_WORKSPACE", 8: "FP4_ERR_BOUNDS"}
 
 
 class Fp4Error(RuntimeError):
@@ -56,7 +59,7 @@ def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"libfp4.so not built at {LIB_PATH}; run "
+            raise RuntimeError(f"{os.path.basename(LIB_PATH)} not built at {LIB_PATH}; run "
                                "python -m fp4_block_scaled_deterministic_b200.build")
         L = ctypes.CDLL(LIB_PATH)
         P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
@@ -72,6 +75,7 @@ def lib() -> ctypes.CDLL:
             "fp4_quantize_dual_opts": (I32, [P, P, P, P, P, P, I64, I64, I32, I32,
                                              ctypes.POINTER(QuantOpts), P]),
             "fp4_gemm": (I32, [P, P, P, P, P, P, P, I64, I64, I64, I32, I32, P]),
+            "fp4_gemm_quant": (I32, [P, P, P, P, P, P, P, P, P, I64, I64, I64, I32, I32, P]),
             "fp4_linear_workspace_size": (SZ, [I32, I64, I64, I64, I32]),
             "fp4_linear_fprop": (I32, [P, P, P, I64, I64, I64, I32, I32, I32, P, SZ, P]),
             "fp4_linear_dgrad": (I32, [P, P, P, I64, I64, I64, I32, I32, I32, P, SZ, P]),
@@ -164,6 +168,11 @@ def fp4_quantize_dual_opts(x, row_codes, row_scales, col_codes, col_scales, tens
 def fp4_gemm(A, As, Ats, B, Bs, Bts, C, M, N, K, fmt, out_dtype, stream=None):
     return lib().fp4_gemm(_ptr(A), _ptr(As), _ptr(Ats), _ptr(B), _ptr(Bs), _ptr(Bts), _ptr(C), M,
                           N, K, fmt, out_dtype, _stream(stream))
+
+
+def fp4_gemm_quant(A, As, Ats, B, Bs, Bts, C, Qc, Qs, M, N, K, fmt, q_hn, stream=None):
+    return lib().fp4_gemm_quant(_ptr(A), _ptr(As), _ptr(Ats), _ptr(B), _ptr(Bs), _ptr(Bts),
+                                _ptr(C), _ptr(Qc), _ptr(Qs), M, N, K, fmt, q_hn, _stream(stream))
 
 
 def fp4_linear_fprop(X, W, Y, M, N, K, fmt, hn, out_dtype, ws, ws_bytes, stream=None):
@@ -284,6 +293,19 @@ def gemm(a: QTensor, b: QTensor, out_dtype: int = OUT_F32, out: torch.Tensor | N
     _check(fp4_gemm(a.codes, a.scales, a.tensor_scale, b.codes, b.scales, b.tensor_scale, out, M,
                     N, K, a.fmt, out_dtype), "fp4_gemm")
     return out
+
+
+def gemm_quant(a: QTensor, b: QTensor, q_hn: int = 16, with_output: bool = True):
+    """Y = RN_bf16(deq(a) @ deq(b)^T) and its row-wise MXFP4 quantisation (rotation q_hn
+    along N) from the same epilogue. Returns (Y or None, QTensor of Y)."""
+    assert a.fmt == b.fmt and a.cols == b.cols
+    M, N, K = a.rows, b.rows, a.cols
+    dev = a.codes.device
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev) if with_output else None
+    codes, scales = _alloc_q(M, N, MXFP4, dev)
+    _check(fp4_gemm_quant(a.codes, a.scales, a.tensor_scale, b.codes, b.scales, b.tensor_scale,
+                          Y, codes, scales, M, N, K, a.fmt, q_hn), "fp4_gemm_quant")
+    return Y, QTensor(codes, scales, None, MXFP4, M, N)
 
 
 def _linear(pass_, P, Q, out_shape, M, N, K, fmt, hn, out_dtype, ws, out):

@@ -1,6 +1,6 @@
 """Build libfp4.so (the C-ABI CUDA library) in-tree for sm_100a with nvcc.
 
-    python -m fp4_block_scaled_deterministic_b200.build [--force]
+    python -m fp4_block_scaled_deterministic_b200.build [--force] [--debug]
 
 The library is one translation unit (csrc/fp4_api.cu including the kernel headers),
 compiled with -gencode arch=compute_100a,code=sm_100a and linked against the static
@@ -18,6 +18,10 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libfp4.so")
+# The same sources with -DFP4_DEBUG_BOUNDS: every kernel range-checks its computed
+# shared-memory offsets, TMEM columns, tile coordinates and global indices, records a
+# failure in the status word and skips the access (fp4_check_status -> FP4_ERR_BOUNDS).
+LIB_DEBUG = os.path.join(PKG, "libfp4_debug.so")
 SOURCES = [os.path.join(CSRC, f) for f in ("fp4_api.cu",)]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("common.cuh", "quantize.cuh", "gemm.cuh")] + [
     os.path.join(ROOT, "include", "fp4.h")]
@@ -36,26 +40,41 @@ def flags(extra=()):
             "-I", os.path.join(ROOT, "include"), *extra]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(d) <= t for d in DEPS)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    tmp = LIB + ".tmp"
-    cmd = [nvcc(), *flags(), "-shared", "-o", tmp, *SOURCES]
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Compile libfp4.so (debug=True: libfp4_debug.so with the device-side range checks)."""
+    lib = LIB_DEBUG if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
+    tmp = lib + ".tmp"
+    cmd = [nvcc(), *flags(["-DFP4_DEBUG_BOUNDS"] if debug else []), "-shared", "-o", tmp,
+           *SOURCES]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
+
+
+def build_all(force: bool = False) -> None:
+    """Both libraries, compiled in parallel."""
+    import concurrent.futures as cf
+    with cf.ThreadPoolExecutor(2) as ex:
+        for f in [ex.submit(build, force, False, d) for d in (False, True)]:
+            f.result()
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="-v" in sys.argv)
-    print(LIB)
+    if "--debug" in sys.argv:
+        print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, debug=True))
+    else:
+        build_all(force="--force" in sys.argv)
+        print(LIB)
+        print(LIB_DEBUG)

@@ -20,8 +20,23 @@ enum { kFmtMX = 0, kFmtNV = 1, kFmtMX8 = 2 };
 // ------------------------------------------------------------------ status word
 // Bit flags recorded by kernels instead of trapping; read and cleared by the host.
 constexpr unsigned kDevErrTimeout = 1u;
+constexpr unsigned kDevErrBounds = 2u;
 
 __device__ unsigned int g_status_word;
+
+// Debug build (-DFP4_DEBUG_BOUNDS): the kernels range-check every computed
+// shared-memory offset, TMEM column, tile coordinate and global index before using it.
+// A failed check records kDevErrBounds in the status word and the access is skipped;
+// nothing traps. In the release build FP4_IN_BOUNDS(c) is the constant true.
+#ifdef FP4_DEBUG_BOUNDS
+__device__ __forceinline__ bool bounds_ok(bool ok) {
+  if (!ok) atomicOr(&g_status_word, kDevErrBounds);
+  return ok;
+}
+#define FP4_IN_BOUNDS(cond) (::fp4k::bounds_ok(static_cast<bool>(cond)))
+#else
+#define FP4_IN_BOUNDS(cond) (static_cast<void>(sizeof(cond)), true)  // not evaluated
+#endif
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;

@@ -10,6 +10,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/fp4.h"
 #include "common.cuh"
 #include "gemm.cuh"
@@ -18,6 +20,16 @@
 using namespace fp4k;
 
 namespace {
+
+// NVTX range around each compute entry point (named after it), so that a profiler's
+// timeline shows which ABI call launched which kernels. Header-only NVTX: without a
+// profiler attached a push/pop is a check of one pointer.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 constexpr int kMaxDevices = 64;
 constexpr uint64_t kDefaultWaitLimitNs = 1000000000ull;  // 1 s per pipeline wait
@@ -319,13 +331,13 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtens
 // CTA-pair kernel: the grid is two CTAs per pair tile, capped at the number of CTA pairs
 // the device can hold at once (queried once per device), so the persistent loop never
 // waits for a pair that is not resident.
-template <int FMT, int OUT>
+template <int FMT, int OUT, int QHN = -1>
 cudaError_t launch_gemm_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& sa,
                              const CUtensorMap& sb, const GemmArgs& g, int dev, cudaStream_t s) {
   static std::atomic<uint64_t> done{0};
   static int max_pairs[kMaxDevices];
   static std::once_flag once[kMaxDevices];
-  auto k = gemm_fp4_pair_kernel<FMT, OUT>;
+  auto k = gemm_fp4_pair_kernel<FMT, OUT, QHN>;
   cudaError_t e = ensure_smem(k, PairCfg<FMT>::kSmemBytes, dev, done);
   if (e != cudaSuccess) return e;
   std::call_once(once[dev], [&] {
@@ -374,11 +386,29 @@ void choose_tile_order(GemmArgs& g, int64_t tile_rows, int64_t row_bytes_i) {
   g.band = g.band_n ? gb : ga;
 }
 
+// With q_hn >= 0 (fp4_gemm_quant) the output is bf16 and the epilogue also writes its
+// row-wise MXFP4 quantisation (rotation q_hn along N) to q_codes / q_scales; C may then
+// be null.
+template <int FMT>
+cudaError_t launch_gemm_pair_quant(const CUtensorMap& a, const CUtensorMap& b,
+                                   const CUtensorMap& sa, const CUtensorMap& sb,
+                                   const GemmArgs& g, int q_hn, int dev, cudaStream_t s) {
+  switch (q_hn) {
+    case 0: return launch_gemm_pair<FMT, 1, 0>(a, b, sa, sb, g, dev, s);
+    case 16: return launch_gemm_pair<FMT, 1, 16>(a, b, sa, sb, g, dev, s);
+    default: return launch_gemm_pair<FMT, 1, 32>(a, b, sa, sb, g, dev, s);
+  }
+}
+
 fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void* B,
                      const void* Bs, const float* Bts, void* C, int64_t M, int64_t N, int64_t K,
-                     fp4_format fmt, fp4_out_dtype od, cudaStream_t stream) {
+                     fp4_format fmt, fp4_out_dtype od, cudaStream_t stream,
+                     void* q_codes = nullptr, void* q_scales = nullptr, int q_hn = -1) {
   if (!valid_format(fmt)) return FP4_ERR_INVALID_ARG;
   if (od != FP4_OUT_F32 && od != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
+  const bool quant = q_hn >= 0;
+  if (quant && (fmt == FP4_MXFP8 || od != FP4_OUT_BF16 || (q_hn != 0 && q_hn != 16 && q_hn != 32)))
+    return FP4_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || K < 0 || M % 32 || N % 32 || K % 32) return FP4_ERR_SHAPE;
   if (M > (int64_t(1) << 31) - 256 || N > (int64_t(1) << 31) - 256 ||
       K > (int64_t(1) << 31) - 256)
@@ -386,11 +416,13 @@ fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void
   if (fmt != FP4_NVFP4 && (Ats || Bts)) return FP4_ERR_INVALID_ARG;
   if (fmt == FP4_NVFP4 && (!Ats || !Bts)) return FP4_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return FP4_OK;
-  if (!C) return FP4_ERR_INVALID_ARG;
+  if (!C && !quant) return FP4_ERR_INVALID_ARG;
+  if (quant && (!q_codes || !q_scales)) return FP4_ERR_INVALID_ARG;
   if (K == 0) return FP4_ERR_SHAPE;  // an empty contraction is not a launch the tiles express
   if (!A || !As || !B || !Bs) return FP4_ERR_INVALID_ARG;
-  if (!aligned16(A) || !aligned16(As) || !aligned16(B) || !aligned16(Bs) || !aligned16(C))
+  if (!aligned16(A) || !aligned16(As) || !aligned16(B) || !aligned16(Bs) || (C && !aligned16(C)))
     return FP4_ERR_ALIGN;
+  if (quant && (!aligned16(q_codes) || !aligned16(q_scales))) return FP4_ERR_ALIGN;
   int dev;
   const DeviceInfo* info;
   fp4_status st = current_device(&dev, &info);
@@ -402,7 +434,7 @@ fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void
   // one-CTA kernel. Each kernel has its own K per pipeline stage.
   // (The MXFP8 comparator always takes the pair kernel; M <= 128 is then one zero-filled
   // 256-row band.)
-  const bool pair = M > 128 || fmt == FP4_MXFP8;
+  const bool pair = M > 128 || fmt == FP4_MXFP8 || quant;
   const int slab_k = !pair ? kGBK
                      : fmt == FP4_MXFP4 ? PairCfg<kFmtMX>::kSlabK
                      : fmt == FP4_NVFP4 ? PairCfg<kFmtNV>::kSlabK
@@ -437,10 +469,18 @@ fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void
   g.sa = Ats;
   g.sb = Bts;
   g.wait_limit_ns = kDefaultWaitLimitNs;
+  g.q_codes = static_cast<uint8_t*>(q_codes);
+  g.q_scales = static_cast<uint8_t*>(q_scales);
+  g.q_kb4 = static_cast<int>(ceil_div(N / 32, 4));
+  g.m_pad = static_cast<int>(ceil_div(M, 128) * 128);
   const int grid = g.num_tiles < info->sm_count ? g.num_tiles : info->sm_count;
 
   cudaError_t e;
-  if (pair) {
+  if (quant) {
+    e = fmt == FP4_MXFP4
+            ? launch_gemm_pair_quant<kFmtMX>(ta, tb, tsa, tsb, g, q_hn, dev, stream)
+            : launch_gemm_pair_quant<kFmtNV>(ta, tb, tsa, tsb, g, q_hn, dev, stream);
+  } else if (pair) {
     if (fmt == FP4_MXFP4)
       e = od == FP4_OUT_F32 ? launch_gemm_pair<kFmtMX, 0>(ta, tb, tsa, tsb, g, dev, stream)
                             : launch_gemm_pair<kFmtMX, 1>(ta, tb, tsa, tsb, g, dev, stream);
@@ -609,6 +649,7 @@ size_t fp4_scales_bytes(int64_t rows, int64_t cols, fp4_format fmt) {
 
 fp4_status fp4_quantize(const void* x, void* codes, void* scales, float* ts, int64_t rows,
                         int64_t cols, fp4_format fmt, int hn, fp4_axis axis, fp4_stream_t stream) {
+  NvtxRange nvtx_range("fp4_quantize");
   if (axis != FP4_AXIS_ROW && axis != FP4_AXIS_COL) return FP4_ERR_INVALID_ARG;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (axis == FP4_AXIS_ROW)
@@ -619,12 +660,14 @@ fp4_status fp4_quantize(const void* x, void* codes, void* scales, float* ts, int
 fp4_status fp4_quantize_dual(const void* x, void* row_codes, void* row_scales, void* col_codes,
                              void* col_scales, float* ts, int64_t rows, int64_t cols,
                              fp4_format fmt, int hn, fp4_stream_t stream) {
+  NvtxRange nvtx_range("fp4_quantize_dual");
   return quantize_impl(x, row_codes, row_scales, col_codes, col_scales, ts, rows, cols, fmt, hn,
                        kModeDual, reinterpret_cast<cudaStream_t>(stream));
 }
 fp4_status fp4_quantize_opts(const void* x, void* codes, void* scales, float* ts, int64_t rows,
                              int64_t cols, fp4_format fmt, int hn, fp4_axis axis,
                              const fp4_quant_opts* opts, fp4_stream_t stream) {
+  NvtxRange nvtx_range("fp4_quantize_opts");
   if (axis != FP4_AXIS_ROW && axis != FP4_AXIS_COL) return FP4_ERR_INVALID_ARG;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (axis == FP4_AXIS_ROW)
@@ -637,6 +680,7 @@ fp4_status fp4_quantize_dual_opts(const void* x, void* row_codes, void* row_scal
                                   void* col_codes, void* col_scales, float* ts, int64_t rows,
                                   int64_t cols, fp4_format fmt, int hn,
                                   const fp4_quant_opts* opts, fp4_stream_t stream) {
+  NvtxRange nvtx_range("fp4_quantize_dual_opts");
   return quantize_impl(x, row_codes, row_scales, col_codes, col_scales, ts, rows, cols, fmt, hn,
                        kModeDual, reinterpret_cast<cudaStream_t>(stream), opts);
 }
@@ -644,8 +688,19 @@ fp4_status fp4_quantize_dual_opts(const void* x, void* row_codes, void* row_scal
 fp4_status fp4_gemm(const void* A, const void* As, const float* Ats, const void* B, const void* Bs,
                     const float* Bts, void* C, int64_t M, int64_t N, int64_t K, fp4_format fmt,
                     fp4_out_dtype od, fp4_stream_t stream) {
+  NvtxRange nvtx_range("fp4_gemm");
   return gemm_impl(A, As, Ats, B, Bs, Bts, C, M, N, K, fmt, od,
                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+fp4_status fp4_gemm_quant(const void* A, const void* As, const float* Ats, const void* B,
+                          const void* Bs, const float* Bts, void* C, void* Q_codes,
+                          void* Q_scales, int64_t M, int64_t N, int64_t K, fp4_format fmt,
+                          int q_hadamard_n, fp4_stream_t stream) {
+  NvtxRange nvtx_range("fp4_gemm_quant");
+  if (q_hadamard_n != 0 && q_hadamard_n != 16 && q_hadamard_n != 32) return FP4_ERR_INVALID_ARG;
+  return gemm_impl(A, As, Ats, B, Bs, Bts, C, M, N, K, fmt, FP4_OUT_BF16,
+                   reinterpret_cast<cudaStream_t>(stream), Q_codes, Q_scales, q_hadamard_n);
 }
 
 size_t fp4_linear_workspace_size(fp4_pass pass, int64_t M, int64_t N, int64_t K, fp4_format fmt) {
@@ -660,6 +715,7 @@ size_t fp4_linear_workspace_size(fp4_pass pass, int64_t M, int64_t N, int64_t K,
 fp4_status fp4_linear_fprop(const void* X, const void* W, void* Y, int64_t M, int64_t N, int64_t K,
                             fp4_format fmt, int hn, fp4_out_dtype od, void* ws, size_t ws_bytes,
                             fp4_stream_t stream) {
+  NvtxRange nvtx_range("fp4_linear_fprop");
   return linear_impl(FP4_PASS_FPROP, X, W, Y, M, N, K, fmt, hn, od, ws, ws_bytes,
                      reinterpret_cast<cudaStream_t>(stream));
 }
@@ -667,6 +723,7 @@ fp4_status fp4_linear_fprop(const void* X, const void* W, void* Y, int64_t M, in
 fp4_status fp4_linear_dgrad(const void* dY, const void* W, void* dX, int64_t M, int64_t N,
                             int64_t K, fp4_format fmt, int hn, fp4_out_dtype od, void* ws,
                             size_t ws_bytes, fp4_stream_t stream) {
+  NvtxRange nvtx_range("fp4_linear_dgrad");
   return linear_impl(FP4_PASS_DGRAD, dY, W, dX, M, N, K, fmt, hn, od, ws, ws_bytes,
                      reinterpret_cast<cudaStream_t>(stream));
 }
@@ -674,6 +731,7 @@ fp4_status fp4_linear_dgrad(const void* dY, const void* W, void* dX, int64_t M, 
 fp4_status fp4_linear_wgrad(const void* dY, const void* X, void* dW, int64_t M, int64_t N,
                             int64_t K, fp4_format fmt, int hn, fp4_out_dtype od, void* ws,
                             size_t ws_bytes, fp4_stream_t stream) {
+  NvtxRange nvtx_range("fp4_linear_wgrad");
   return linear_impl(FP4_PASS_WGRAD, dY, X, dW, M, N, K, fmt, hn, od, ws, ws_bytes,
                      reinterpret_cast<cudaStream_t>(stream));
 }
@@ -681,6 +739,7 @@ fp4_status fp4_linear_wgrad(const void* dY, const void* X, void* dW, int64_t M, 
 fp4_status fp4_linear_fprop_noalloc(const void* X, const void* W, void* Y, int64_t M, int64_t N,
                                     int64_t K, fp4_format fmt, int hn, fp4_out_dtype od,
                                     fp4_stream_t stream) {
+  NvtxRange nvtx_range("fp4_linear_fprop_noalloc");
   if (fp4_linear_workspace_size(FP4_PASS_FPROP, M, N, K, fmt) > FP4_NOALLOC_SCRATCH_BYTES)
     return FP4_ERR_WORKSPACE;
   int dev;
@@ -702,10 +761,12 @@ fp4_status fp4_check_status(fp4_stream_t stream) {
   if (cudaMemcpyFromSymbol(&word, g_status_word, sizeof(word)) != cudaSuccess) return FP4_ERR_CUDA;
   if (word != 0 && cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero)) != cudaSuccess)
     return FP4_ERR_CUDA;
+  if (word & kDevErrBounds) return FP4_ERR_BOUNDS;
   return (word & kDevErrTimeout) ? FP4_ERR_TIMEOUT : FP4_OK;
 }
 
 fp4_status fp4_selftest_timeout(uint64_t timeout_ns, fp4_stream_t stream) {
+  NvtxRange nvtx_range("fp4_selftest_timeout");
   int dev;
   const DeviceInfo* info;
   fp4_status st = current_device(&dev, &info);
@@ -724,6 +785,7 @@ const char* fp4_status_string(fp4_status s) {
     case FP4_ERR_CUDA: return "CUDA error";
     case FP4_ERR_TIMEOUT: return "device pipeline wait timed out";
     case FP4_ERR_WORKSPACE: return "workspace missing or too small";
+    case FP4_ERR_BOUNDS: return "device-side bounds check failed (debug build)";
   }
   return "unknown status";
 }

@@ -32,6 +32,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "quantize.cuh"
 
 namespace fp4k {
 
@@ -64,10 +65,16 @@ struct GemmArgs {
   int tiles_m, tiles_n, num_tiles, k_tiles;
   int band, band_n;  // tile order: see tile_coords
   int c_v8;          // output 32-byte aligned: 32-byte stores
-  void* C;
+  void* C;           // output; may be null when the epilogue quantises it (fp4_gemm_quant)
   const float* sa;  // NVFP4 tensor scales (device), or null
   const float* sb;
   uint64_t wait_limit_ns;
+  // Fused output quantisation (gemm_fp4_pair_kernel with QHN >= 0): row-wise MXFP4
+  // codes [M][N/2] and scales (128-row x 4-block atoms, q_kb4 atoms per 128 rows) of
+  // RN_bf16(C); rows [M, m_pad) get zero scale bytes (the layout's padding).
+  uint8_t* q_codes;
+  uint8_t* q_scales;
+  int q_kb4, m_pad;
 };
 
 // Output tile order. Tiles are numbered in bands of g.band tile rows (g.band_n == 0) or
@@ -84,6 +91,10 @@ __device__ __forceinline__ void tile_coords(int tile, const GemmArgs& g, int& tm
   const int a = first + r % width, b = r / width;
   tm = g.band_n ? b : a;
   tn = g.band_n ? a : b;
+  if (!FP4_IN_BOUNDS(tm >= 0 && tm < g.tiles_m && tn >= 0 && tn < g.tiles_n)) {
+    tm = 0;  // debug build: an in-range tile keeps every pipeline count intact
+    tn = 0;
+  }
 }
 
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of 128 bytes,
@@ -177,6 +188,7 @@ struct Issuer {
         t = c.t_sf + 4 * kAtoms + 8 * at + 4 * rb;
         d = c.dSB + rb * (kAtoms * 32) + 32 * at;
       }
+      if (!FP4_IN_BOUNDS((t & 0xFFFFu) + 4u <= 512u)) continue;  // TMEM columns of the copy
       if constexpr (PAIR) tc_cp_32x128b_warpx4_pair(t, d);
       else tc_cp_32x128b_warpx4(t, d);
     }
@@ -198,6 +210,8 @@ struct Issuer {
     const uint32_t idesc = kIdesc | (id << 29) | (id << 4);
     const uint64_t koff = (j >> 2) * (128 * 128 >> 4) + 2 * (j & 3);
     const uint32_t acc = first ? 0u : 1u;
+    if (!FP4_IN_BOUNDS((c.t_sf & 0xFFFFu) + SF_COLS <= 512u && (tmem_acc & 0xFFFFu) + 256u <= 512u))
+      return;  // TMEM columns of the scale slot or the accumulator
     if constexpr (PAIR)
       tc_mma_fp4_pair<FMT>(tmem_acc, c.dA + koff, c.dB + koff, idesc, tsfa, tsfb, acc);
     else
@@ -405,6 +419,85 @@ __device__ __forceinline__ void store_row_segment(const uint32_t (&r)[128], int 
   }
 }
 
+// Epilogue with the output quantised for the next layer, row-wise along N (the next
+// contraction axis): the thread's 128 accumulator columns of row m are rounded to bf16
+// (the layer output Y, stored when g.C is set), widened back exactly, rotated in groups
+// of QHN consecutive columns and quantised to MXFP4 in four 32-column blocks -- the
+// quantiser's own ROW-job arithmetic (fused first butterfly, H16 scale fold), so the
+// codes and scales equal a separate quantisation of the stored bf16 Y. Columns >= N
+// are not stored; their scale bytes, in the same 4-byte word, are the layout's padding
+// and come out zero because those accumulator columns are zero (B rows >= N are
+// zero-filled by TMA).
+template <int FMT, int QHN>
+__device__ __forceinline__ void store_row_segment_quant(const uint32_t (&r)[128], int m, int n0,
+                                                        const GemmArgs& g, float alpha) {
+  // A segment wholly beyond N owns no output column and no scale byte (its scale word
+  // would fall into the next atom).
+  if (n0 >= g.N) return;
+  const int64_t sc_off = (static_cast<int64_t>(m >> 7) * g.q_kb4 + (n0 >> 7)) * 512 +
+                         (m & 31) * 16 + ((m & 127) >> 5) * 4;
+  const int64_t sc_bytes = static_cast<int64_t>(g.m_pad) * g.q_kb4 * 4;
+  if (m >= g.M) {  // rows [M, m_pad): the layout's zero padding; rows beyond: nothing
+    if (m < g.m_pad && FP4_IN_BOUNDS(sc_off + 4 <= sc_bytes))
+      *reinterpret_cast<uint32_t*>(g.q_scales + sc_off) = 0u;
+    return;
+  }
+  if (!FP4_IN_BOUNDS(m >= 0 && n0 >= 0 && (n0 & 127) == 0 && sc_off + 4 <= sc_bytes)) return;
+  uint32_t w[64];  // bf16x2 words: w[k] holds columns 2k (low half) and 2k+1 (high half)
+#pragma unroll
+  for (int k = 0; k < 64; ++k) {
+    float x0 = __uint_as_float(r[2 * k]), x1 = __uint_as_float(r[2 * k + 1]);
+    if constexpr (FMT == kFmtNV) {
+      x0 = __fmul_rn(x0, alpha);
+      x1 = __fmul_rn(x1, alpha);
+    }
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    w[k] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  if (g.C) {
+    __nv_bfloat16* crow = static_cast<__nv_bfloat16*>(g.C) + static_cast<int64_t>(m) * g.N + n0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (n0 + 32 * c < g.N) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          *reinterpret_cast<uint4*>(crow + 32 * c + 8 * i) =
+              make_uint4(w[16 * c + 4 * i], w[16 * c + 4 * i + 1], w[16 * c + 4 * i + 2],
+                         w[16 * c + 4 * i + 3]);
+      }
+    }
+  }
+  constexpr bool kFold = QHN == 16;  // MXFP4 + H16: the x0.25 goes into the scale
+  constexpr bool kFuse1 = QHN > 0;   // first butterfly fused into the widening
+  uint8_t* qrow = g.q_codes + static_cast<int64_t>(m) * (g.N >> 1) + (n0 >> 1);
+  uint32_t sbytes = 0;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    // lane x = columns 64*half + 0..31, lane y = 64*half + 32..63 (words wx, wy)
+    float2 p[32];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const uint32_t wx = w[32 * half + k], wy = w[32 * half + 16 + k];
+      if constexpr (kFuse1) {
+        float sx, dx, sy, dy;
+        bfly1_lo(wx, add_hi(wx, -0.0f), sx, dx);
+        bfly1_lo(wy, add_hi(wy, -0.0f), sy, dy);
+        p[2 * k] = make_float2(sx, sy);
+        p[2 * k + 1] = make_float2(dx, dy);
+      } else {
+        p[2 * k] = make_float2(bf16lo(wx), bf16lo(wy));
+        p[2 * k + 1] = make_float2(bf16hi(wx), bf16hi(wy));
+      }
+    }
+    fwht_x2<QHN, !kFold, kFuse1 ? 2 : 1>(p);
+    const Enc e = encode_x2<kFmtMX, kFold>(p, 1.0f, 6.0f);
+    if (n0 + 64 * half < g.N) *reinterpret_cast<uint4*>(qrow + 32 * half) = e.cx;
+    if (n0 + 64 * half + 32 < g.N) *reinterpret_cast<uint4*>(qrow + 32 * half + 16) = e.cy;
+    sbytes |= (e.sx | (e.sy << 8)) << (16 * half);
+  }
+  *reinterpret_cast<uint32_t*>(g.q_scales + sc_off) = sbytes;
+}
+
 template <int FMT, int OUT_BF16>
 __global__ void __launch_bounds__(kGThreads, 1)
     gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -538,10 +631,13 @@ __global__ void __launch_bounds__(kGThreads, 1)
 template <int FMT>
 struct PairCfg {
   static constexpr int kBlock = FMT == kFmtNV ? 16 : 32;
-  // K per stage: 512 for MXFP4 (8 MMAs per barrier wait and commit, 3 stages), 256 for
-  // NVFP4 (whose scale copies are twice as many per K; 5 stages), 256 for MXFP8 (the
-  // same 256 code bytes per row as MXFP4, 8 MMAs of K = 32; 3 stages).
-  static constexpr int kSlabK = FMT == kFmtNV ? 256 : (FMT == kFmtMX ? 512 : 256);
+  // K per stage: 256 for MXFP4 (4 MMAs per barrier wait and commit, 6 stages) and NVFP4
+  // (5 stages), 256 for MXFP8 (the same 256 code bytes per row as 512 K of MXFP4, 8 MMAs
+  // of K = 32; 3 stages). The mainloop is bound by how long a stage stays occupied (load
+  // latency + MMAs), not by barrier waits: six 35 KB MXFP4 stages keep the same bytes in
+  // flight as three 70 KB ones but free each after 512 MMA cycles instead of 1024
+  // (measured 5165 -> 5396 TFLOP/s over the Llama layer's GEMMs).
+  static constexpr int kSlabK = 256;
   static constexpr int kRowBytes = FMT == kFmtMX8 ? kSlabK : kSlabK / 2;  // code bytes/row
   static constexpr int kSub = kRowBytes / 128;       // 128-byte-wide swizzled sub-tiles
   static constexpr int kAtoms = kSlabK / (4 * kBlock);
@@ -550,14 +646,14 @@ struct PairCfg {
   static constexpr int kSFABytes = kAtoms * 512;     // scales of this CTA's A rows
   static constexpr int kSFBBytes = 2 * kAtoms * 512; // scales of all 256 B rows
   static constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
-  static constexpr int kStages = FMT == kFmtNV ? 5 : 3;
+  static constexpr int kStages = FMT == kFmtNV ? 5 : (FMT == kFmtMX ? 6 : 3);
   // MXFP8 (6 copies per 8 MMAs) keeps the copies in the MMA thread: there the extra wait
   // of the split issue costs more than it saves.
   static constexpr int kCopyThreads = FMT == kFmtMX8 ? 0 : kGPairCopyThreads;
   static constexpr int kThreads = kGThreads + 32 * kCopyThreads;
   static constexpr int kSFCols = 12 * kAtoms;
   // At least one ring slot per stage (the split issue's reuse rule): 5 x 48 columns for
-  // NVFP4, 4 x 48 for MXFP4, 4 x 24 for MXFP8, after the 256 accumulator columns.
+  // NVFP4, 6 x 24 for MXFP4, 4 x 24 for MXFP8, after the 256 accumulator columns.
   static constexpr int kSFBufs = kStages > 4 ? kStages : 4;
   static constexpr int kTmemSF = 256;
   static_assert(kTmemSF + kSFBufs * kSFCols <= 512, "TMEM columns");
@@ -565,7 +661,9 @@ struct PairCfg {
 };
 
 
-template <int FMT, int OUT_BF16>
+// QHN >= 0: the epilogue also quantises the output (store_row_segment_quant, rotation
+// QHN along N); OUT_BF16 is then 1.
+template <int FMT, int OUT_BF16, int QHN = -1>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<FMT>::kThreads, 1)
     gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB,
@@ -706,9 +804,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<FMT>::kThrea
       // about a microsecond per tile.
       if (lane == 0) mbar_arrive_cluster_cta_release(leader_acc_empty);
       acc_phase ^= 1u;
-      store_row_segment<FMT, OUT_BF16>(r, tm * 256 + 128 * static_cast<int>(rank) + 32 * quarter +
-                                              lane,
-                                       tn * kGBN + 128 * half, g, alpha);
+      const int m = tm * 256 + 128 * static_cast<int>(rank) + 32 * quarter + lane;
+      if constexpr (QHN >= 0)
+        store_row_segment_quant<FMT, QHN>(r, m, tn * kGBN + 128 * half, g, alpha);
+      else
+        store_row_segment<FMT, OUT_BF16>(r, m, tn * kGBN + 128 * half, g, alpha);
     }
   }
   __syncwarp();

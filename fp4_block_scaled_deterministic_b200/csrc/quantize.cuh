@@ -48,7 +48,7 @@ constexpr int kQScaleBytes = 1024;          // up to two 512-byte atoms
 __host__ __device__ constexpr int kQCodeBytesOf(int fmt) { return fmt == kFmtMX8 ? 128 * 128 : 128 * 64; }
 __host__ __device__ constexpr int kQSmemBytesOf(int fmt, bool ext) {
   return 1024 /*align*/ + kQStagesOf(fmt, ext) * kQInBytes + 2 * 2 * kQCodeBytesOf(fmt) +
-         2 * 2 * kQScaleBytes + 256 + 1024 /* random-sign masks */;
+         2 * 2 * kQScaleBytes + 256 + 2048 /* random-sign masks, two tiles */;
 }
 __host__ __device__ constexpr int kQCtasPerSMOf(int fmt, bool ext) {
   return fmt == kFmtMX8 ? 1 : 2;
@@ -115,15 +115,36 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-// max |x| over elements [b, b+n) of each lane.
-__device__ __forceinline__ float2 amax_x2(const float2 (&p)[32], int b, int n) {
-  float m0 = 0.0f, m1 = 0.0f;
+// Max of N non-negative floats as a tree of three-input maxes (depth ~log3 N instead of
+// a chain of N/2 dependent instructions; max is exact, so the order does not matter).
+template <int N>
+__device__ __forceinline__ float tree_max(const float* v) {
+  if constexpr (N == 1) {
+    return v[0];
+  } else if constexpr (N == 2) {
+    return fmaxf(v[0], v[1]);
+  } else {
+    constexpr int G = (N + 2) / 3;  // groups of three (the last may be shorter)
+    float m[G];
 #pragma unroll
-  for (int i = 0; i < n; i += 2) {
-    m0 = max3f(m0, fabsf(p[b + i].x), fabsf(p[b + i + 1].x));
-    m1 = max3f(m1, fabsf(p[b + i].y), fabsf(p[b + i + 1].y));
+    for (int g = 0; g < G; ++g) {
+      if (3 * g + 2 < N) m[g] = max3f(v[3 * g], v[3 * g + 1], v[3 * g + 2]);
+      else if (3 * g + 1 < N) m[g] = fmaxf(v[3 * g], v[3 * g + 1]);
+      else m[g] = v[3 * g];
+    }
+    return tree_max<G>(m);
   }
-  return make_float2(m0, m1);
+}
+// max |x| over elements [B, B+N) of each lane.
+template <int B, int N>
+__device__ __forceinline__ float2 amax_x2(const float2 (&p)[32]) {
+  float ax[N], ay[N];
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    ax[i] = fabsf(p[B + i].x);
+    ay[i] = fabsf(p[B + i].y);
+  }
+  return make_float2(tree_max<N>(ax), tree_max<N>(ay));
 }
 
 __device__ __forceinline__ uint32_t cvt8x(const float2 (&p)[32], int b) {
@@ -240,7 +261,7 @@ struct Enc {
 // v * 2^-e, 2^-e = 2^(127 - byte) built from its bit pattern (byte <= 252).
 template <class Codes = RneCodes>
 __device__ __forceinline__ Enc mx_encode_x2(float2 (&p)[32], const Codes& codes = Codes()) {
-  const float2 am = amax_x2(p, 0, 32);
+  const float2 am = amax_x2<0, 32>(p);
   const uint32_t ex = (__float_as_uint(am.x) >> 23) & 0xFFu;
   const uint32_t ey = (__float_as_uint(am.y) >> 23) & 0xFFu;
   const uint32_t bx = ex > 2u ? ex - 2u : 0u, by = ey > 2u ? ey - 2u : 0u;
@@ -262,7 +283,7 @@ __device__ __forceinline__ Enc mx_encode_x2(float2 (&p)[32], const Codes& codes 
 // take the two-step path.
 template <class Codes = RneCodes>
 __device__ __forceinline__ Enc mx_encode_x2_h16fold(float2 (&p)[32], const Codes& codes = Codes()) {
-  const float2 am = amax_x2(p, 0, 32);
+  const float2 am = amax_x2<0, 32>(p);
   if (am.x >= 0x1p-100f && am.y >= 0x1p-100f) {
     const uint32_t bx = ((__float_as_uint(am.x) >> 23) & 0xFFu) - 4u;
     const uint32_t by = ((__float_as_uint(am.y) >> 23) & 0xFFu) - 4u;
@@ -294,10 +315,10 @@ __device__ __forceinline__ bool near_e2m1_threshold(float q) {
 // The quotient is formed as v * y with y = RN(1/d): then |v*y - v/d| < 2 ulps, so v*y and
 // RN(v/d) fall on the same side of every E2M1 threshold unless v*y is within 4 ulps of
 // one; those (rare) blocks, and blocks whose 1/d overflows, are divided exactly.
-template <bool kExact = false>
-__device__ __forceinline__ void nv_block_x2(float2 (&p)[32], int b, float S, float six_s,
+template <int b, bool kExact = false>
+__device__ __forceinline__ void nv_block_x2(float2 (&p)[32], float S, float six_s,
                                             uint32_t& sbx, uint32_t& sby) {
-  const float2 bm = amax_x2(p, b, 16);
+  const float2 bm = amax_x2<b, 16>(p);
   sbx = cvt_e4m3(__fdiv_rn(bm.x, six_s));
   sby = cvt_e4m3(__fdiv_rn(bm.y, six_s));
   const float dx = __fmul_rn(e4m3_to_f32(sbx), S), dy = __fmul_rn(e4m3_to_f32(sby), S);
@@ -326,8 +347,8 @@ template <class Codes = RneCodes>
 __device__ __forceinline__ Enc nv_encode_x2(float2 (&p)[32], float S, float six_s,
                                             const Codes& codes = Codes()) {
   uint32_t x0, y0, x1, y1;
-  nv_block_x2<Codes::kExactQuotient>(p, 0, S, six_s, x0, y0);
-  nv_block_x2<Codes::kExactQuotient>(p, 16, S, six_s, x1, y1);
+  nv_block_x2<0, Codes::kExactQuotient>(p, S, six_s, x0, y0);
+  nv_block_x2<16, Codes::kExactQuotient>(p, S, six_s, x1, y1);
   Enc e;
   codes(p, e.cx, e.cy);
   e.sx = x0 | (x1 << 8);
@@ -364,7 +385,7 @@ struct Enc8 {
 // e = floor(log2 amax) - 8 clamped at -127 (8 = largest E4M3 exponent); codes
 // E4M3_RNE_satfinite(v * 2^-e), 2^-e = 2^(127 - byte) built from its bit pattern.
 __device__ __forceinline__ Enc8 mx8_encode_x2(float2 (&p)[32]) {
-  const float2 am = amax_x2(p, 0, 32);
+  const float2 am = amax_x2<0, 32>(p);
   const uint32_t ex = (__float_as_uint(am.x) >> 23) & 0xFFu;
   const uint32_t ey = (__float_as_uint(am.y) >> 23) & 0xFFu;
   const uint32_t bx = ex > 8u ? ex - 8u : 0u, by = ey > 8u ? ey - 8u : 0u;
@@ -400,6 +421,22 @@ __device__ __forceinline__ uint8_t* code_chunk(uint8_t* tile, int r, int q) {
 __device__ __forceinline__ uint8_t* code_chunk8(uint8_t* tile, int r, int q) {
   return tile + r * 128 + ((q ^ (r & 7)) << 4);
 }
+// Debug-build range checks of the offsets into the staged tiles (always true otherwise):
+// 16-byte code chunk q of tile row r (nq chunks per row), `bytes` scale bytes at
+// atom_off(r, kb), and the base of a ROW job (row r of box b) or a COL job (column pair
+// w of box b, rows 32s .. 32s+31) of the input tile.
+__device__ __forceinline__ bool code_ok(int r, int q, int nq) {
+  return FP4_IN_BOUNDS(r >= 0 && r < 128 && q >= 0 && q < nq);
+}
+__device__ __forceinline__ bool scale_ok(int r, int kb, int bytes) {
+  return FP4_IN_BOUNDS(r >= 0 && r < 128 && kb >= 0 && atom_off(r, kb) + bytes <= kQScaleBytes);
+}
+__device__ __forceinline__ bool row_job_ok(int r, int b) {
+  return FP4_IN_BOUNDS(r >= 0 && r < 128 && b >= 0 && b * kQBoxBytes + r * 128 + 128 <= kQInBytes);
+}
+__device__ __forceinline__ bool col_job_ok(int b, int w, int s) {
+  return FP4_IN_BOUNDS(b >= 0 && b < 2 && w >= 0 && w < 32 && s >= 0 && s < 4);
+}
 
 // ROW job: tile row r, box b (columns 64b .. 64b+63) = segments 2b (lane x) and 2b+1
 // (lane y); 8 conflict-free 16-byte reads of the 128B-swizzled box row.
@@ -412,6 +449,11 @@ __device__ __forceinline__ uint4 xor4(uint4 a, uint4 m) {
 template <bool kSigns = false>
 __device__ __forceinline__ void load_row_job(const uint8_t* in, int r, int b, float2 (&p)[32],
                                              const uint32_t* cm = nullptr) {
+  if (!row_job_ok(r, b)) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) p[i] = make_float2(0.0f, 0.0f);
+    return;
+  }
   const uint8_t* rowp = in + b * kQBoxBytes + r * 128;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -436,6 +478,11 @@ __device__ __forceinline__ void load_row_job(const uint8_t* in, int r, int b, fl
 template <bool kSigns = false>
 __device__ __forceinline__ void load_col_job(const uint8_t* in, int b, int w, int s,
                                              float2 (&p)[32], const uint32_t* rm = nullptr) {
+  if (!col_job_ok(b, w, s)) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) p[i] = make_float2(0.0f, 0.0f);
+    return;
+  }
   const uint8_t* boxp = in + b * kQBoxBytes;
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
@@ -478,6 +525,11 @@ __device__ __forceinline__ void bfly1_hi(uint32_t wu, float v, float& s, float& 
 template <bool kSigns = false>
 __device__ __forceinline__ void load_row_job_bfly1(const uint8_t* in, int r, int b,
                                                    float2 (&p)[32], const uint32_t* cm = nullptr) {
+  if (!row_job_ok(r, b)) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) p[i] = make_float2(0.0f, 0.0f);
+    return;
+  }
   const uint8_t* rowp = in + b * kQBoxBytes + r * 128;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -503,6 +555,11 @@ __device__ __forceinline__ void load_row_job_bfly1(const uint8_t* in, int r, int
 template <bool kSigns = false>
 __device__ __forceinline__ void load_col_job_bfly1(const uint8_t* in, int b, int w, int s,
                                                    float2 (&p)[32], const uint32_t* rm = nullptr) {
+  if (!col_job_ok(b, w, s)) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) p[i] = make_float2(0.0f, 0.0f);
+    return;
+  }
   const uint8_t* boxp = in + b * kQBoxBytes;
 #pragma unroll
   for (int i = 0; i < 32; i += 2) {
@@ -568,21 +625,42 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
   uint8_t* s_csc = s_rsc + 2 * kQScaleBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(s_csc + 2 * kQScaleBytes);
   float* s_red = reinterpret_cast<float*>(full + kQStages);  // [8 warps][2]
-  // random-sign XOR masks of the tile: 64 column-pair words (ROW jobs), 128 row words
-  // (COL jobs); 16-byte aligned (s_red is 16 floats after 8-byte barriers)
-  uint32_t* s_cmask = reinterpret_cast<uint32_t*>(
+  // random-sign XOR masks of a tile, double-buffered by tile parity: 64 column-pair
+  // words (ROW jobs) and 128 row words (COL jobs) per buffer; 16-byte aligned (s_red is
+  // 16 floats after 8-byte barriers)
+  uint32_t* s_masks = reinterpret_cast<uint32_t*>(
       (reinterpret_cast<uintptr_t>(s_red + 16) + 15) & ~static_cast<uintptr_t>(15));
-  uint32_t* s_rmask = s_cmask + 64;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bid = blockIdx.x, nctas = gridDim.x;
   const int my_tiles = bid < a.num_tiles ? (a.num_tiles - bid + nctas - 1) / nctas : 0;
 
+  // Signs of a tile's 128 columns (warp 0) and 128 rows (warp 1) into mask buffer `buf`:
+  // Philox block (tile start)/4 + lane holds the words of indices 4*lane .. 4*lane+3.
+  auto write_masks = [&](int tile, int buf) {
+    int tr, tc;
+    qtile_coords<BANDED>(tile, a, tr, tc);
+    uint32_t* cm = s_masks + 192 * buf;
+    if (kRow && warp == 0) {
+      const uint4 w = philox_block(static_cast<uint64_t>(tc) * 32u + lane, 0u, a.sign_key);
+      // column pairs 2*lane (columns 4*lane, +1) and 2*lane+1 (columns 4*lane+2, +3)
+      *reinterpret_cast<uint2*>(cm + 2 * lane) =
+          make_uint2(((w.x >> 31) << 15) | (w.y & 0x80000000u),
+                     ((w.z >> 31) << 15) | (w.w & 0x80000000u));
+    }
+    if (kCol && warp == 1) {
+      const uint4 w = philox_block(static_cast<uint64_t>(tr) * 32u + lane, 0u, a.sign_key);
+      *reinterpret_cast<uint4*>(cm + 64 + 4 * lane) =
+          make_uint4((w.x >> 31) * 0x80008000u, (w.y >> 31) * 0x80008000u,
+                     (w.z >> 31) * 0x80008000u, (w.w >> 31) * 0x80008000u);
+    }
+  };
   if (tid == 0) {
     tma_prefetch_desc(&tm_in);
     for (int s = 0; s < kQStages; ++s) mbar_init(&full[s], 1);
     mbar_fence_init();
   }
+  if (rht && my_tiles > 0) write_masks(bid, 0);
   __syncthreads();
 
   // NVFP4 tensor scales of the quantise pass: S = amax / 2688 (1 when amax is 0).
@@ -609,6 +687,12 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
     int tr, tc;
     qtile_coords<BANDED>(tile, a, tr, tc);
     uint8_t* dst = s_in + stage * kQInBytes;
+    if (!FP4_IN_BOUNDS(tile < a.num_tiles && tr >= 0 && tr < a.tiles_r && tc >= 0 &&
+                       tc < a.tiles_c)) {
+      tr = 0;  // an in-range tile: the barrier still gets its bytes and nothing hangs
+      tc = 0;
+    }
+    if (!FP4_IN_BOUNDS(stage >= 0 && stage < kQStages)) return;  // the bounded waits report it
     mbar_arrive_expect_tx(&full[stage], kQInBytes);
     tma_load_2d(dst, &tm_in, &full[stage], tc * 128, tr * 128);
     tma_load_2d(dst + kQBoxBytes, &tm_in, &full[stage], tc * 128 + 64, tr * 128);
@@ -633,26 +717,14 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
     int tr, tc;
     qtile_coords<BANDED>(tile, a, tr, tc);
     const int st = it % kQStages, ob = it & 1;
-    if (rht) {
-      // signs of this tile's 128 columns (warp 0) and 128 rows (warp 1): Philox block
-      // (tile start)/4 + lane holds the words of indices 4*lane .. 4*lane+3 of the tile.
-      // The previous tile's jobs read the masks before its store barrier.
-      if (kRow && warp == 0) {
-        const uint4 w = philox_block(static_cast<uint64_t>(tc) * 32u + lane, 0u, a.sign_key);
-        // column pairs 2*lane (columns 4*lane, +1) and 2*lane+1 (columns 4*lane+2, +3)
-        *reinterpret_cast<uint2*>(s_cmask + 2 * lane) =
-            make_uint2(((w.x >> 31) << 15) | (w.y & 0x80000000u),
-                       ((w.z >> 31) << 15) | (w.w & 0x80000000u));
-      }
-      if (kCol && warp == 1) {
-        const uint4 w = philox_block(static_cast<uint64_t>(tr) * 32u + lane, 0u, a.sign_key);
-        *reinterpret_cast<uint4*>(s_rmask + 4 * lane) =
-            make_uint4((w.x >> 31) * 0x80008000u, (w.y >> 31) * 0x80008000u,
-                       (w.z >> 31) * 0x80008000u, (w.w >> 31) * 0x80008000u);
-      }
-    }
+    // One barrier per tile (at its end). The next tile's signs go to the other mask
+    // buffer, whose readers (the tile before this one) finished before the last barrier.
+    if (rht && it + 1 < my_tiles) write_masks(tile + nctas, (it + 1) & 1);
+    const uint32_t* s_cmask = s_masks + 192 * (it & 1);
+    const uint32_t* s_rmask = s_cmask + 64;
+    // A wait that runs out is acted on at the barrier below, together: the jobs then
+    // read stale (never faulting) shared memory, and nothing of this tile is stored.
     const bool ok = mbar_wait(&full[st], static_cast<uint32_t>((it / kQStages) & 1), a.wait_limit_ns);
-    if (__syncthreads_or(!ok)) break;  // give up together; the status word says why
     const uint8_t* in = s_in + st * kQInBytes;
     uint8_t* rcode = s_rcode + ob * kCodeBytes;
     uint8_t* ccode = s_ccode + ob * kCodeBytes;
@@ -675,16 +747,19 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
         }
         fwht_x2<HN, !kFoldH16, kFuse1 ? 2 : 1>(p);
         if constexpr (AMAX) {
-          const float2 m = amax_x2(p, 0, 32);
+          const float2 m = amax_x2<0, 32>(p);
           amax_r = max3f(amax_r, m.x, m.y);
         } else if constexpr (FMT == kFmtMX8) {
           const Enc8 e = mx8_encode_x2(p);  // lane x: bytes 64b .. +31, lane y: 64b+32 .. +63
-          *reinterpret_cast<uint4*>(code_chunk8(rcode, row_r, 4 * b)) = e.cx[0];
-          *reinterpret_cast<uint4*>(code_chunk8(rcode, row_r, 4 * b + 1)) = e.cx[1];
-          *reinterpret_cast<uint4*>(code_chunk8(rcode, row_r, 4 * b + 2)) = e.cy[0];
-          *reinterpret_cast<uint4*>(code_chunk8(rcode, row_r, 4 * b + 3)) = e.cy[1];
-          *reinterpret_cast<uint16_t*>(rsc + atom_off(row_r, 2 * b)) =
-              static_cast<uint16_t>(e.sx | (e.sy << 8));
+          if (code_ok(row_r, 4 * b + 3, 8)) {
+            *reinterpret_cast<uint4*>(code_chunk8(rcode, row_r, 4 * b)) = e.cx[0];
+            *reinterpret_cast<uint4*>(code_chunk8(rcode, row_r, 4 * b + 1)) = e.cx[1];
+            *reinterpret_cast<uint4*>(code_chunk8(rcode, row_r, 4 * b + 2)) = e.cy[0];
+            *reinterpret_cast<uint4*>(code_chunk8(rcode, row_r, 4 * b + 3)) = e.cy[1];
+          }
+          if (scale_ok(row_r, 2 * b, 2))
+            *reinterpret_cast<uint16_t*>(rsc + atom_off(row_r, 2 * b)) =
+                static_cast<uint16_t>(e.sx | (e.sy << 8));
         } else {
           Enc e;
           if (sr) {
@@ -696,13 +771,18 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
           } else {
             e = encode_x2<FMT, kFoldH16>(p, S_r, six_r);
           }
-          *reinterpret_cast<uint4*>(code_chunk(rcode, row_r, 2 * b)) = e.cx;
-          *reinterpret_cast<uint4*>(code_chunk(rcode, row_r, 2 * b + 1)) = e.cy;
-          if constexpr (FMT == kFmtMX)  // blocks 2b, 2b+1 of this row: adjacent bytes
-            *reinterpret_cast<uint16_t*>(rsc + atom_off(row_r, 2 * b)) =
-                static_cast<uint16_t>(e.sx | (e.sy << 8));
-          else  // blocks 4b .. 4b+3: one 4-byte group of atom b
-            *reinterpret_cast<uint32_t*>(rsc + atom_off(row_r, 4 * b)) = e.sx | (e.sy << 16);
+          if (code_ok(row_r, 2 * b + 1, 4)) {
+            *reinterpret_cast<uint4*>(code_chunk(rcode, row_r, 2 * b)) = e.cx;
+            *reinterpret_cast<uint4*>(code_chunk(rcode, row_r, 2 * b + 1)) = e.cy;
+          }
+          if constexpr (FMT == kFmtMX) {  // blocks 2b, 2b+1 of this row: adjacent bytes
+            if (scale_ok(row_r, 2 * b, 2))
+              *reinterpret_cast<uint16_t*>(rsc + atom_off(row_r, 2 * b)) =
+                  static_cast<uint16_t>(e.sx | (e.sy << 8));
+          } else {  // blocks 4b .. 4b+3: one 4-byte group of atom b
+            if (scale_ok(row_r, 4 * b, 4))
+              *reinterpret_cast<uint32_t*>(rsc + atom_off(row_r, 4 * b)) = e.sx | (e.sy << 16);
+          }
         }
       }
     }
@@ -720,16 +800,20 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
         }
         fwht_x2<HN, !kFoldH16, kFuse1 ? 2 : 1>(p);
         if constexpr (AMAX) {
-          const float2 m = amax_x2(p, 0, 32);
+          const float2 m = amax_x2<0, 32>(p);
           amax_c = max3f(amax_c, m.x, m.y);
         } else if constexpr (FMT == kFmtMX8) {
           const Enc8 e = mx8_encode_x2(p);  // column c (x) and c+1 (y): rows 32s .. 32s+31
-          *reinterpret_cast<uint4*>(code_chunk8(ccode, col_c, 2 * s)) = e.cx[0];
-          *reinterpret_cast<uint4*>(code_chunk8(ccode, col_c, 2 * s + 1)) = e.cx[1];
-          *reinterpret_cast<uint4*>(code_chunk8(ccode, col_c + 1, 2 * s)) = e.cy[0];
-          *reinterpret_cast<uint4*>(code_chunk8(ccode, col_c + 1, 2 * s + 1)) = e.cy[1];
-          csc[atom_off(col_c, s)] = static_cast<uint8_t>(e.sx);
-          csc[atom_off(col_c + 1, s)] = static_cast<uint8_t>(e.sy);
+          if (code_ok(col_c + 1, 2 * s + 1, 8)) {
+            *reinterpret_cast<uint4*>(code_chunk8(ccode, col_c, 2 * s)) = e.cx[0];
+            *reinterpret_cast<uint4*>(code_chunk8(ccode, col_c, 2 * s + 1)) = e.cx[1];
+            *reinterpret_cast<uint4*>(code_chunk8(ccode, col_c + 1, 2 * s)) = e.cy[0];
+            *reinterpret_cast<uint4*>(code_chunk8(ccode, col_c + 1, 2 * s + 1)) = e.cy[1];
+          }
+          if (scale_ok(col_c + 1, s, 1)) {
+            csc[atom_off(col_c, s)] = static_cast<uint8_t>(e.sx);
+            csc[atom_off(col_c + 1, s)] = static_cast<uint8_t>(e.sy);
+          }
         } else {
           Enc e;
           if (sr) {
@@ -743,13 +827,17 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
           } else {
             e = encode_x2<FMT, kFoldH16>(p, S_c, six_c);
           }
-          *reinterpret_cast<uint4*>(code_chunk(ccode, col_c, s)) = e.cx;
-          *reinterpret_cast<uint4*>(code_chunk(ccode, col_c + 1, s)) = e.cy;
+          if (code_ok(col_c + 1, s, 4)) {
+            *reinterpret_cast<uint4*>(code_chunk(ccode, col_c, s)) = e.cx;
+            *reinterpret_cast<uint4*>(code_chunk(ccode, col_c + 1, s)) = e.cy;
+          }
           // block kb of segment s: s (MXFP4, one byte) or 2s, 2s+1 (NVFP4, two bytes)
           if constexpr (FMT == kFmtMX) {
-            csc[atom_off(col_c, s)] = static_cast<uint8_t>(e.sx);
-            csc[atom_off(col_c + 1, s)] = static_cast<uint8_t>(e.sy);
-          } else {
+            if (scale_ok(col_c + 1, s, 1)) {
+              csc[atom_off(col_c, s)] = static_cast<uint8_t>(e.sx);
+              csc[atom_off(col_c + 1, s)] = static_cast<uint8_t>(e.sy);
+            }
+          } else if (scale_ok(col_c + 1, 2 * s, 2)) {
             *reinterpret_cast<uint16_t*>(csc + atom_off(col_c, 2 * s)) = static_cast<uint16_t>(e.sx);
             *reinterpret_cast<uint16_t*>(csc + atom_off(col_c + 1, 2 * s)) = static_cast<uint16_t>(e.sy);
           }
@@ -757,33 +845,37 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
       }
     }
 
-    if constexpr (!AMAX) fence_proxy_async_smem();
-    __syncthreads();
+    if constexpr (!AMAX) {
+      fence_proxy_async_smem();
+      // The next tile writes staging buffer ob^1, which the stores issued after the last
+      // barrier are reading: wait for those reads before this barrier releases it.
+      if (tid == 0) bulk_wait_read<0>();
+    }
+    if (__syncthreads_or(!ok)) break;  // give up together; the status word says why
     if (tid == 0) {
       if constexpr (!AMAX) {
         constexpr int kAtomsPerTile = (FMT == kFmtNV) ? 2 : 1;
         constexpr int kTileCodeBytes = FMT == kFmtMX8 ? 128 : 64;  // code bytes per tile row
+        const bool tile_ok = FP4_IN_BOUNDS(tr >= 0 && tr < a.tiles_r && tc >= 0 && tc < a.tiles_c);
         if constexpr (kRow) {
-          tma_store_2d(&tm_rcodes, rcode, tc * kTileCodeBytes, tr * 128);
           const int first = tc * kAtomsPerTile;
           const int n = (a.row_kb4 - first) < kAtomsPerTile ? (a.row_kb4 - first) : kAtomsPerTile;
-          bulk_store(a.row_scales + (static_cast<int64_t>(tr) * a.row_kb4 + first) * 512, rsc,
-                     static_cast<uint32_t>(n * 512));
+          if (tile_ok) tma_store_2d(&tm_rcodes, rcode, tc * kTileCodeBytes, tr * 128);
+          if (tile_ok && FP4_IN_BOUNDS(n > 0 && first + n <= a.row_kb4))
+            bulk_store(a.row_scales + (static_cast<int64_t>(tr) * a.row_kb4 + first) * 512, rsc,
+                       static_cast<uint32_t>(n * 512));
         }
         if constexpr (kCol) {
-          tma_store_2d(&tm_ccodes, ccode, tr * kTileCodeBytes, tc * 128);
           const int first = tr * kAtomsPerTile;
           const int n = (a.col_kb4 - first) < kAtomsPerTile ? (a.col_kb4 - first) : kAtomsPerTile;
-          bulk_store(a.col_scales + (static_cast<int64_t>(tc) * a.col_kb4 + first) * 512, csc,
-                     static_cast<uint32_t>(n * 512));
+          if (tile_ok) tma_store_2d(&tm_ccodes, ccode, tr * kTileCodeBytes, tc * 128);
+          if (tile_ok && FP4_IN_BOUNDS(n > 0 && first + n <= a.col_kb4))
+            bulk_store(a.col_scales + (static_cast<int64_t>(tc) * a.col_kb4 + first) * 512, csc,
+                       static_cast<uint32_t>(n * 512));
         }
         bulk_commit();
       }
       if (it + kQStages < my_tiles) issue_load(st, tile + kQStages * nctas);
-      // The next tile writes staging buffer ob^1, last read by the stores of the previous
-      // tile: wait for those reads here. Thread 0 joins the next tile's first barrier
-      // only after this, so no barrier of its own is needed.
-      if constexpr (!AMAX) bulk_wait_read<1>();
     }
   }
   if constexpr (!AMAX) {

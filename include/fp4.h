@@ -68,7 +68,9 @@ typedef enum {
     FP4_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not compute capability 10.x */
     FP4_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed */
     FP4_ERR_TIMEOUT = 6,            /* a device-side pipeline wait gave up (fp4_check_status) */
-    FP4_ERR_WORKSPACE = 7           /* workspace NULL or smaller than required */
+    FP4_ERR_WORKSPACE = 7,          /* workspace NULL or smaller than required */
+    FP4_ERR_BOUNDS = 8              /* a device-side range check failed (debug build only,
+                                       see fp4_check_status) */
 } fp4_status;
 
 /* FP4_MXFP8 is the FP8 comparator the pages measure FP4 against (MXFP4 pre-training
@@ -86,13 +88,16 @@ typedef enum { FP4_PASS_FPROP = 0, FP4_PASS_DGRAD = 1, FP4_PASS_WGRAD = 2 } fp4_
 /* Version of this ABI; bumped on any incompatible change. */
 FP4_API int fp4_abi_version(void);
 
-/* Bytes of a packed code matrix with R rows of C elements: R*C/2. */
+/* Bytes of a packed code matrix with R rows of C elements: R*C/2 (two 4-bit codes per
+ * byte: NVFP4/MaxText page, Key facts bullet 2). */
 FP4_API size_t fp4_codes_bytes(int64_t rows, int64_t cols);
 /* Bytes of a code matrix of format fmt: R*C/2 (FP4 formats) or R*C (FP4_MXFP8). */
 FP4_API size_t fp4_codes_bytes_fmt(int64_t rows, int64_t cols, fp4_format fmt);
 
 /* Bytes of the scale matrix of an [R][C] code matrix in the atom layout above:
- * ceil(R/128)*128 * ceil(C/bs/4)*4. */
+ * ceil(R/128)*128 * ceil(C/bs/4)*4 (one shared scale per block of bs elements: the
+ * block scales of the NVFP4/MaxText page's first paragraph and of MXFP4 in the
+ * pre-training summary, Methodology item 2). */
 FP4_API size_t fp4_scales_bytes(int64_t rows, int64_t cols, fp4_format fmt);
 
 /*
@@ -121,7 +126,10 @@ FP4_API fp4_status fp4_quantize(const void *x_bf16, void *codes, void *scales, f
 /*
  * fp4_quantize_dual -- both layouts of fp4_quantize from ONE read of x: the row-wise
  * result (row_codes, row_scales) and the column-wise transposed one (col_codes,
- * col_scales), bit-identical to two separate fp4_quantize calls.
+ * col_scales), bit-identical to two separate fp4_quantize calls. Each activation and
+ * gradient of a training step is needed in both: along its rows for Fprop / Dgrad and
+ * along the token axis for Wgrad, the pass the pre-training summary finds most
+ * sensitive to quantisation (Methodology item 2; Findings section 1).
  *   tensor_scale: NVFP4 -> device float[4], written {S_row, S_col, amax_row, amax_col}
  *                 (each layout is scaled by the amax of its own rotation).
  *                 MXFP4 -> must be NULL.
@@ -202,6 +210,29 @@ FP4_API fp4_status fp4_gemm(const void *A_codes, const void *A_scales, const flo
                     fp4_out_dtype out_dtype, fp4_stream_t stream);
 
 /*
+ * fp4_gemm_quant -- fp4_gemm with a bf16 output whose epilogue also quantises it for
+ * the next layer: Q = the row-wise MXFP4 quantisation, with rotation q_hadamard_n
+ * (0, 16, 32) along N, of Y = RN_bf16(C) -- bit-identical to
+ * fp4_quantize(Y, ..., FP4_MXFP4, q_hadamard_n, FP4_AXIS_ROW) of the stored Y, without
+ * reading Y back from memory. [Producer-fused quantisation: the rotated FP4 operand of
+ * the next GEMM comes out of the previous one, with custom kernels fusing the
+ * quantisation into the training step (NVFP4/MaxText pages: the JAX/MaxText section
+ * on fused low-precision kernels); MXFP4 + H16 as the pre-training summary, Methodology
+ * items 2-3.]
+ *   A, B, tensor scales, fmt (FP4_MXFP4 or FP4_NVFP4 operands), M, N, K: as fp4_gemm.
+ *   C: bf16 [M][N] output, or NULL to write only the quantised output.
+ *   Q_codes [M][N/2] and Q_scales (fp4_scales_bytes(M, N, FP4_MXFP4) bytes, the atom
+ *   layout above, padding written as zero): device, 16-byte aligned.
+ *   Errors: FP4_ERR_INVALID_ARG for FP4_MXFP8 operands, a NULL Q buffer or another
+ *   q_hadamard_n; otherwise as fp4_gemm.
+ */
+FP4_API fp4_status fp4_gemm_quant(const void *A_codes, const void *A_scales,
+                                  const float *A_tensor_scale, const void *B_codes,
+                                  const void *B_scales, const float *B_tensor_scale, void *C,
+                                  void *Q_codes, void *Q_scales, int64_t M, int64_t N, int64_t K,
+                                  fp4_format fmt, int q_hadamard_n, fp4_stream_t stream);
+
+/*
  * The three passes of a linear layer Y = X W^T with X [M][K], W [N][K], dY [M][N],
  * each quantising its operands along its own contraction axis and multiplying them.
  * [MXFP4 pre-training summary, Methodology item 2: Fprop, Dgrad, Wgrad.]
@@ -252,9 +283,13 @@ FP4_API fp4_status fp4_linear_fprop_noalloc(const void *X, const void *W, void *
 
 /*
  * fp4_check_status -- synchronises `stream`, then returns and clears the device
- * status word of the current device: FP4_ERR_TIMEOUT if any kernel's bounded wait
- * gave up since the last check, FP4_ERR_CUDA if the synchronisation failed, else
- * FP4_OK.
+ * status word of the current device: FP4_ERR_BOUNDS if a range check of the debug
+ * build failed, else FP4_ERR_TIMEOUT if any kernel's bounded wait gave up since the
+ * last check, FP4_ERR_CUDA if the synchronisation failed, else FP4_OK.
+ *   Debug build (libfp4_debug.so, compiled with -DFP4_DEBUG_BOUNDS): every kernel
+ *   range-checks its computed shared-memory offsets, TMEM columns, tile coordinates
+ *   and global indices before use; a failed check skips that access (no trap) and
+ *   sets the bit reported here. Same ABI and results as the release library.
  */
 FP4_API fp4_status fp4_check_status(fp4_stream_t stream);
 

@@ -29,7 +29,7 @@ def test_every_header_symbol_is_exported():
 
 
 def test_status_strings():
-    for code in range(8):
+    for code in range(9):
         assert fp4.status_string(code)
     assert fp4.status_string(99) == "unknown status"
 
@@ -113,6 +113,20 @@ def test_gemm_validation():
     assert g(B=MIS) == ALIGN
     assert g(K=0) == SHAPE
     assert g(M=0) == OK
+
+
+def gq(C=A16, Qc=A16, Qs=A16, M=128, N=128, K=128, fmt=0, qhn=16):
+    return fp4.lib().fp4_gemm_quant(A16, A16, None, A16, A16, None, C, Qc, Qs, M, N, K, fmt, qhn,
+                                    None)
+
+
+def test_gemm_quant_validation():
+    assert gq(qhn=8) == INVALID
+    assert gq(fmt=2) == INVALID           # the MXFP8 comparator has no fused output
+    assert gq(Qc=None) == INVALID and gq(Qs=None) == INVALID
+    assert gq(Qc=MIS) == ALIGN and gq(C=MIS) == ALIGN
+    assert gq(N=100) == SHAPE
+    assert gq(M=0) == OK
 
 
 def test_linear_validation():
