@@ -99,6 +99,9 @@ def parse():
     ap.add_argument("--side-stream", type=int, default=1, choices=[0, 1],
                     help="1: quantise the next projection on a second stream beside the GEMMs "
                          "(per-kernel rooflines then come from the same steps on one stream)")
+    ap.add_argument("--quant-batch", type=int, default=1, choices=[0, 1],
+                    help="1: quantise each projection's X, W and dY in one batched launch "
+                         "(fp4_quantize_dual_batch); 0: one launch per tensor")
     ap.add_argument("--next-layer-quant", choices=["none", "standalone", "fused"], default="none",
                     help="also quantise each Fprop output Y row-wise (MXFP4, same rotation) for "
                          "the next layer: by a separate quantise launch after the GEMM, or in "
@@ -180,12 +183,15 @@ class LlamaLayer:
     """Inputs, quantised operands and outputs of every projection, all on the device."""
 
     def __init__(self, device, fmt, hn, tokens=8192, seed=0, names=None, variant="none",
-                 side_stream=False, layers=None, outlier_mult=50.0, w_seed=0, next_quant="none"):
+                 side_stream=False, layers=None, outlier_mult=50.0, w_seed=0, next_quant="none",
+                 quant_batch=True):
         import fp4_block_scaled_deterministic_b200 as fp4
         from fp4_block_scaled_deterministic_b200 import synthetic
         self.fp4, self.fmt, self.hn, self.M = fp4, fmt, hn, tokens
         self.variant = variant
         self.next_quant = next_quant
+        # the plain quantiser takes a projection's three tensors in one batched launch
+        self.quant_batch = quant_batch and variant == "none"
         self.qstream = torch.cuda.Stream(device) if side_stream else None
         self.projs = []
         g = torch.Generator(device=device)
@@ -220,6 +226,13 @@ class LlamaLayer:
         self.gemms_done, self.quant_done = [], []
         self.opts = {}
         for p in self.projs:
+            # batched quantisation: one fp4_quant_item per operand, built once
+            p["qitems"] = (fp4.QuantItem * 3)(*[
+                fp4.QuantItem(p[key].data_ptr(), p[key + "_row"][0].data_ptr(),
+                              p[key + "_row"][1].data_ptr(), p[key + "_col"][0].data_ptr(),
+                              p[key + "_col"][1].data_ptr(),
+                              p[key + "_ts"].data_ptr() if fmt == 1 else None, r, c)
+                for key, (r, c) in self._operands(p)])
             for key, _ in self._operands(p):
                 o = None
                 if variant == "amax":
@@ -256,8 +269,9 @@ class LlamaLayer:
 
     def launches_per_step(self):
         # NVFP4 adds the amax pass (plus a memset) unless the amax is supplied
-        per_q = 1 if self.fmt == 0 or self.variant == "amax" else 2
-        return len(self.projs) * (3 * per_q + 3 + (self.next_quant == "standalone"))
+        per_q = 1 if self.fmt != 1 or self.variant == "amax" else 2
+        q_launches = per_q if self.quant_batch else 3 * per_q
+        return len(self.projs) * (q_launches + 3 + (self.next_quant == "standalone"))
 
     def step(self, stream, timers=None, allreduce=None, overlap=None, inputs_ready=None,
              outputs_free=None):
@@ -289,6 +303,11 @@ class LlamaLayer:
             if inputs_ready is not None:
                 qstream.wait_event(inputs_ready[i])
             qs = qstream.cuda_stream
+            if self.quant_batch:
+                st = timed("quant", lambda: f.lib().fp4_quantize_dual_batch(
+                    p["qitems"], 3, fmt, hn, qs), qstream)
+                assert st == 0, f.status_string(st)
+                return
             for key, (r, c) in self._operands(p):
                 row, col, ts = p[key + "_row"], p[key + "_col"], p[key + "_ts"]
                 opts = self.opts[(p["name"], key)]
@@ -618,7 +637,8 @@ def main():
     # data parallel: every rank holds the same W (replicated weights) and its own tokens
     layer = LlamaLayer(dev, fmt, a.hadamard, tokens=tokens, seed=1000 * rank, names=names,
                        variant=a.variant, side_stream=bool(a.side_stream), layers=layers,
-                       outlier_mult=omult, w_seed=0, next_quant=a.next_layer_quant)
+                       outlier_mult=omult, w_seed=0, next_quant=a.next_layer_quant,
+                       quant_batch=bool(a.quant_batch))
     stream = torch.cuda.current_stream(dev)
     from fp4_block_scaled_deterministic_b200 import dp
     allreduce = (lambda t: dp.allreduce_wgrad(t, async_op=True)) if world > 1 else None
@@ -705,7 +725,9 @@ def main():
                            f"B200 dense {'FP8' if fmt == 2 else 'FP4'} datasheet peak"}
     qroof = {"bound": "hbm", "achieved": quant_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
              "frac": quant_gbs / pk["hbm_gbs"], "bytes_per_elem": bpe,
-             "kernel": "quantize_kernel dual layout", "launches": len(quant_ms),
+             "kernel": ("quantize_kernel dual layout, "
+                        + ("X, W, dY of a projection per launch" if layer.quant_batch
+                           else "one tensor per launch")), "launches": len(quant_ms),
              "avg_ms": sum(quant_ms) / len(quant_ms), "peak_source": f"{pk_kind}: hbm_gbs"}
 
     out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -717,6 +739,8 @@ def main():
                       f"subset {','.join(names)} of: {workload_name(a)}",
                       "format": a.format, "hadamard_n": a.hadamard, "variant": a.variant,
                       "next_layer_quant": a.next_layer_quant,
+                      "quant_launch": ("one batched launch per projection (X, W, dY)"
+                                       if layer.quant_batch else "one launch per tensor"),
                       "streams": 2 if a.side_stream else 1,
                       "tokens_per_rank": layer.M,
                       "l2": f"inputs larger than L2 ({(layer.bytes_in() + layer.bytes_out()) / 1e9:.1f} GB per step)",

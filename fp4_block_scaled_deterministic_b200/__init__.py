@@ -44,6 +44,14 @@ class Fp4Error(RuntimeError):
         super().__init__(f"{where}: {STATUS.get(code, code)} ({status_string(code)})")
 
 
+class QuantItem(ctypes.Structure):
+    """fp4_quant_item of include/fp4.h (one tensor of fp4_quantize_dual_batch)."""
+    _fields_ = [("x_bf16", ctypes.c_void_p), ("row_codes", ctypes.c_void_p),
+                ("row_scales", ctypes.c_void_p), ("col_codes", ctypes.c_void_p),
+                ("col_scales", ctypes.c_void_p), ("tensor_scale", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
+
+
 class QuantOpts(ctypes.Structure):
     """fp4_quant_opts of include/fp4.h (host struct passed by pointer)."""
     _fields_ = [("amax", ctypes.c_void_p), ("stochastic", ctypes.c_int),
@@ -74,6 +82,7 @@ def lib() -> ctypes.CDLL:
                                         ctypes.POINTER(QuantOpts), P]),
             "fp4_quantize_dual_opts": (I32, [P, P, P, P, P, P, I64, I64, I32, I32,
                                              ctypes.POINTER(QuantOpts), P]),
+            "fp4_quantize_dual_batch": (I32, [ctypes.POINTER(QuantItem), I32, I32, I32, P]),
             "fp4_gemm": (I32, [P, P, P, P, P, P, P, I64, I64, I64, I32, I32, P]),
             "fp4_gemm_quant": (I32, [P, P, P, P, P, P, P, P, P, I64, I64, I64, I32, I32, P]),
             "fp4_linear_workspace_size": (SZ, [I32, I64, I64, I64, I32]),
@@ -146,6 +155,14 @@ def fp4_quantize_dual(x, row_codes, row_scales, col_codes, col_scales, tensor_sc
     return lib().fp4_quantize_dual(_ptr(x), _ptr(row_codes), _ptr(row_scales), _ptr(col_codes),
                                    _ptr(col_scales), _ptr(tensor_scale), rows, cols, fmt,
                                    hadamard_n, _stream(stream))
+
+
+def fp4_quantize_dual_batch(items, fmt, hadamard_n, stream=None):
+    """items: a sequence of (x, row_codes, row_scales, col_codes, col_scales, tensor_scale,
+    rows, cols) -- tensors or pointers as for fp4_quantize_dual."""
+    arr = (QuantItem * len(items))(*[QuantItem(*[_ptr(v) for v in it[:6]], it[6], it[7])
+                                     for it in items])
+    return lib().fp4_quantize_dual_batch(arr, len(items), fmt, hadamard_n, _stream(stream))
 
 
 def _opts(opts):
@@ -281,6 +298,24 @@ def quantize_dual(x: torch.Tensor, fmt: int = MXFP4, hadamard_n: int = 16,
                "fp4_quantize_dual_opts")
     return (QTensor(rc, rs, None if ts is None else ts[0:1], fmt, rows, cols),
             QTensor(cc, cs, None if ts is None else ts[1:2], fmt, cols, rows))
+
+
+def quantize_dual_batch(xs, fmt: int = MXFP4, hadamard_n: int = 16):
+    """quantize_dual of every bf16 CUDA matrix in xs, in as few launches as possible.
+    Returns [(row QTensor, column QTensor), ...] in the order of xs."""
+    items, outs = [], []
+    for x in xs:
+        assert x.dtype == torch.bfloat16 and x.is_cuda and x.dim() == 2
+        x = x.contiguous()
+        rows, cols = x.shape
+        rc, rs = _alloc_q(rows, cols, fmt, x.device)
+        cc, cs = _alloc_q(cols, rows, fmt, x.device)
+        ts = torch.zeros(4, dtype=torch.float32, device=x.device) if fmt == NVFP4 else None
+        items.append((x, rc, rs, cc, cs, ts, rows, cols))
+        outs.append((QTensor(rc, rs, None if ts is None else ts[0:1], fmt, rows, cols),
+                     QTensor(cc, cs, None if ts is None else ts[1:2], fmt, cols, rows)))
+    _check(fp4_quantize_dual_batch(items, fmt, hadamard_n), "fp4_quantize_dual_batch")
+    return outs
 
 
 def gemm(a: QTensor, b: QTensor, out_dtype: int = OUT_F32, out: torch.Tensor | None = None):

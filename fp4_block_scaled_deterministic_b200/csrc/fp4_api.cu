@@ -9,6 +9,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include <nvtx3/nvToolsExt.h>
 
@@ -120,58 +121,72 @@ inline bool valid_format(fp4_format f) {
 inline int64_t code_bytes(int64_t elems, fp4_format f) { return f == FP4_MXFP8 ? elems : elems / 2; }
 
 // ---------------------------------------------------------------- quantise launch
-template <int FMT, int HN, int MODE, bool AMAX, bool EXT, bool BANDED>
-cudaError_t launch_q_kernel(const CUtensorMap& ti, const CUtensorMap& tr, const CUtensorMap& tc,
-                            const QuantArgs& a, int grid, int dev, cudaStream_t s) {
+// The plain NVFP4 instances run the 512-thread quantize_wide_kernel (measured 2027 ->
+// 2384 GB/s over the Llama layer's dual quantisations); MXFP4 (where the 256-thread
+// kernel measured 4% faster), the variants (EXT) and MXFP8 run quantize_kernel. Both
+// take two CTAs per SM.
+template <int FMT, int HN, int MODE, bool AMAX, bool EXT, bool BANDED, int NITEMS = 1>
+cudaError_t launch_q_kernel(const QuantBatch& qb, int grid, int dev, cudaStream_t s) {
   static std::atomic<uint64_t> done{0};
-  auto k = quantize_kernel<FMT, HN, MODE, AMAX, EXT, BANDED>;
-  constexpr int smem = kQSmemBytesOf(FMT, EXT);
-  cudaError_t e = ensure_smem(k, smem, dev, done);
-  if (e != cudaSuccess) return e;
-  k<<<grid, kQThreads, smem, s>>>(ti, tr, tc, a);
+  if constexpr (!EXT && FMT == kFmtNV) {
+    auto k = quantize_wide_kernel<FMT, HN, MODE, AMAX, BANDED, NITEMS>;
+    cudaError_t e = ensure_smem(k, kQWSmemBytes, dev, done);
+    if (e != cudaSuccess) return e;
+    k<<<grid, kQWThreads, kQWSmemBytes, s>>>(qb);
+  } else {
+    auto k = quantize_kernel<FMT, HN, MODE, AMAX, EXT, BANDED, NITEMS>;
+    constexpr int smem = kQSmemBytesOf(FMT, EXT);
+    cudaError_t e = ensure_smem(k, smem, dev, done);
+    if (e != cudaSuccess) return e;
+    k<<<grid, kQThreads, smem, s>>>(qb);
+  }
   return cudaGetLastError();
 }
 
-// Banded tile order (a.band_c < a.tiles_c) only for the column-layout modes of the
-// plain kernels; everything else walks tiles row-major.
+// Banded tile order (band_c < tiles_c) only for single-tensor launches of the
+// column-layout modes of the plain kernels; everything else walks tiles row-major.
+// Batches of several tensors (dual layout, plain quantiser only) take the instances
+// compiled for kQMaxItems tensors.
 template <int FMT, int HN, int MODE, bool AMAX, bool EXT>
-cudaError_t launch_q(const CUtensorMap& ti, const CUtensorMap& tr, const CUtensorMap& tc,
-                     const QuantArgs& a, int grid, int dev, cudaStream_t s) {
-  if constexpr (MODE != kModeRow && !EXT) {
-    if (a.band_c < a.tiles_c)
-      return launch_q_kernel<FMT, HN, MODE, AMAX, EXT, true>(ti, tr, tc, a, grid, dev, s);
+cudaError_t launch_q(const QuantBatch& qb, int grid, int dev, cudaStream_t s) {
+  if (qb.n > 1) {
+    if constexpr (MODE == kModeDual && !EXT)
+      return launch_q_kernel<FMT, HN, MODE, AMAX, EXT, false, kQMaxItems>(qb, grid, dev, s);
+    else
+      return cudaErrorInvalidValue;  // not reached: batches are dual and plain
   }
-  return launch_q_kernel<FMT, HN, MODE, AMAX, EXT, false>(ti, tr, tc, a, grid, dev, s);
+  if constexpr (MODE != kModeRow && !EXT) {
+    if (qb.item[0].a.band_c < qb.item[0].a.tiles_c)
+      return launch_q_kernel<FMT, HN, MODE, AMAX, EXT, true>(qb, grid, dev, s);
+  }
+  return launch_q_kernel<FMT, HN, MODE, AMAX, EXT, false>(qb, grid, dev, s);
 }
 
 template <int FMT, int HN, bool AMAX, bool EXT>
-cudaError_t dispatch_mode(int mode, const CUtensorMap& ti, const CUtensorMap& tr,
-                          const CUtensorMap& tc, const QuantArgs& a, int grid, int dev,
-                          cudaStream_t s) {
+cudaError_t dispatch_mode(int mode, const QuantBatch& qb, int grid, int dev, cudaStream_t s) {
   switch (mode) {
-    case kModeRow: return launch_q<FMT, HN, kModeRow, AMAX, EXT>(ti, tr, tc, a, grid, dev, s);
-    case kModeCol: return launch_q<FMT, HN, kModeCol, AMAX, EXT>(ti, tr, tc, a, grid, dev, s);
-    default: return launch_q<FMT, HN, kModeDual, AMAX, EXT>(ti, tr, tc, a, grid, dev, s);
+    case kModeRow: return launch_q<FMT, HN, kModeRow, AMAX, EXT>(qb, grid, dev, s);
+    case kModeCol: return launch_q<FMT, HN, kModeCol, AMAX, EXT>(qb, grid, dev, s);
+    default: return launch_q<FMT, HN, kModeDual, AMAX, EXT>(qb, grid, dev, s);
   }
 }
 
-// ext: the variant kernels (random signs and/or stochastic rounding requested in a)
+// ext: the variant kernels (random signs and/or stochastic rounding requested)
 template <int FMT, bool AMAX>
-cudaError_t dispatch_hn(int hn, int mode, const CUtensorMap& ti, const CUtensorMap& tr,
-                        const CUtensorMap& tc, const QuantArgs& a, int grid, int dev,
+cudaError_t dispatch_hn(int hn, int mode, const QuantBatch& qb, int grid, int dev,
                         cudaStream_t s) {
-  const bool ext = a.sr != 0 || a.rht != 0;
+  const bool ext = qb.item[0].a.sr != 0 || qb.item[0].a.rht != 0;
   if (ext) {
     switch (hn) {
-      case 0: return dispatch_mode<FMT, 0, AMAX, true>(mode, ti, tr, tc, a, grid, dev, s);
-      case 16: return dispatch_mode<FMT, 16, AMAX, true>(mode, ti, tr, tc, a, grid, dev, s);
-      default: return dispatch_mode<FMT, 32, AMAX, true>(mode, ti, tr, tc, a, grid, dev, s);
+      case 0: return dispatch_mode<FMT, 0, AMAX, true>(mode, qb, grid, dev, s);
+      case 16: return dispatch_mode<FMT, 16, AMAX, true>(mode, qb, grid, dev, s);
+      default: return dispatch_mode<FMT, 32, AMAX, true>(mode, qb, grid, dev, s);
     }
   }
   switch (hn) {
-    case 0: return dispatch_mode<FMT, 0, AMAX, false>(mode, ti, tr, tc, a, grid, dev, s);
-    case 16: return dispatch_mode<FMT, 16, AMAX, false>(mode, ti, tr, tc, a, grid, dev, s);
-    default: return dispatch_mode<FMT, 32, AMAX, false>(mode, ti, tr, tc, a, grid, dev, s);
+    case 0: return dispatch_mode<FMT, 0, AMAX, false>(mode, qb, grid, dev, s);
+    case 16: return dispatch_mode<FMT, 16, AMAX, false>(mode, qb, grid, dev, s);
+    default: return dispatch_mode<FMT, 32, AMAX, false>(mode, qb, grid, dev, s);
   }
 }
 
@@ -188,9 +203,12 @@ fp4_status validate_quant_common(const void* x, int64_t rows, int64_t cols, fp4_
   return FP4_OK;
 }
 
-fp4_status quantize_impl(const void* x, void* rcodes, void* rscales, void* ccodes, void* cscales,
-                         float* ts, int64_t rows, int64_t cols, fp4_format fmt, int hn, int mode,
-                         cudaStream_t stream, const fp4_quant_opts* opts = nullptr) {
+// Host-side checks of one tensor of a quantise call (no device access). *skip is set
+// for an empty tensor (nothing to do).
+fp4_status check_item(bool* skip, const void* x, void* rcodes, void* rscales, void* ccodes,
+                      void* cscales, float* ts, int64_t rows, int64_t cols, fp4_format fmt,
+                      int hn, int mode, const fp4_quant_opts* opts) {
+  *skip = false;
   fp4_status st = validate_quant_common(x, rows, cols, fmt, hn);
   if (st != FP4_OK) return st;
   const bool do_row = mode & kModeRow, do_col = mode & kModeCol;
@@ -201,38 +219,51 @@ fp4_status quantize_impl(const void* x, void* rcodes, void* rscales, void* ccode
   const float* amax_in = opts ? opts->amax : nullptr;
   if (amax_in && fmt != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
   if (amax_in && (reinterpret_cast<uintptr_t>(amax_in) & 3u)) return FP4_ERR_ALIGN;
-  if (rows == 0 || cols == 0) return FP4_OK;
+  if (rows == 0 || cols == 0) {
+    *skip = true;
+    return FP4_OK;
+  }
   if ((do_row && (!rcodes || !rscales)) || (do_col && (!ccodes || !cscales)))
     return FP4_ERR_INVALID_ARG;
   if ((do_row && (!aligned16(rcodes) || !aligned16(rscales))) ||
       (do_col && (!aligned16(ccodes) || !aligned16(cscales))) ||
       (ts && (reinterpret_cast<uintptr_t>(ts) & 3u)))
     return FP4_ERR_ALIGN;
-  int dev;
-  const DeviceInfo* info;
-  st = current_device(&dev, &info);
-  if (st != FP4_OK) return st;
+  return FP4_OK;
+}
 
-  CUtensorMap tm_in, tm_r, tm_c;
-  std::memset(&tm_r, 0, sizeof(tm_r));
-  std::memset(&tm_c, 0, sizeof(tm_c));
-  if (!make_map_2d(&tm_in, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, cols, rows, 64, 128,
+// One tensor of a quantise launch: validated arguments, TMA maps and kernel arguments.
+// *skip is set for an empty tensor (nothing to do). For NVFP4 without a supplied amax,
+// *amax_cells / *amax_bytes name the reduction cells the amax pass needs zeroed first.
+fp4_status prepare_item(QuantItem* item, bool* skip, float** amax_cells, size_t* amax_bytes,
+                        const void* x, void* rcodes, void* rscales, void* ccodes, void* cscales,
+                        float* ts, int64_t rows, int64_t cols, fp4_format fmt, int hn, int mode,
+                        const fp4_quant_opts* opts) {
+  *amax_cells = nullptr;
+  *amax_bytes = 0;
+  fp4_status st = check_item(skip, x, rcodes, rscales, ccodes, cscales, ts, rows, cols, fmt, hn,
+                             mode, opts);
+  if (st != FP4_OK || *skip) return st;
+  const bool do_row = mode & kModeRow, do_col = mode & kModeCol;
+  const float* amax_in = opts ? opts->amax : nullptr;
+
+  std::memset(item, 0, sizeof(*item));
+  if (!make_map_2d(&item->in, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, cols, rows, 64, 128,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return FP4_ERR_CUDA;
   // code tiles: 128 rows x 64 bytes (FP4, 64B swizzle) or x 128 bytes (MXFP8, 128B swizzle)
   const uint32_t cbox = fmt == FP4_MXFP8 ? 128 : 64;
   const CUtensorMapSwizzle csw = fmt == FP4_MXFP8 ? CU_TENSOR_MAP_SWIZZLE_128B
                                                   : CU_TENSOR_MAP_SWIZZLE_64B;
-  if (do_row && !make_map_2d(&tm_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rcodes,
+  if (do_row && !make_map_2d(&item->rcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rcodes,
                              code_bytes(cols, fmt), rows, cbox, 128, csw))
     return FP4_ERR_CUDA;
-  if (do_col && !make_map_2d(&tm_c, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ccodes,
+  if (do_col && !make_map_2d(&item->ccodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ccodes,
                              code_bytes(rows, fmt), cols, cbox, 128, csw))
     return FP4_ERR_CUDA;
 
   const int bs = block_of(fmt);
-  QuantArgs a;
-  std::memset(&a, 0, sizeof(a));
+  QuantArgs& a = item->a;
   a.rows = rows;
   a.cols = cols;
   a.tiles_c = static_cast<int>(ceil_div(cols, 128));
@@ -259,23 +290,7 @@ fp4_status quantize_impl(const void* x, void* rcodes, void* rscales, void* ccode
     a.sign_key[0] = static_cast<uint32_t>(opts->sign_seed);
     a.sign_key[1] = static_cast<uint32_t>(opts->sign_seed >> 32);
   }
-  const bool ext = a.sr != 0 || a.rht != 0;
-  const int per_sm = fmt == FP4_MXFP8 ? kQCtasPerSMOf(kFmtMX8, false)
-                     : fmt == FP4_MXFP4 ? kQCtasPerSMOf(kFmtMX, ext)
-                                        : kQCtasPerSMOf(kFmtNV, ext);
-  const int resident = per_sm * info->sm_count;
-  const int grid = a.num_tiles < resident ? a.num_tiles : resident;
-
-  cudaError_t e = cudaSuccess;
-  if (fmt == FP4_MXFP4) {
-    e = dispatch_hn<kFmtMX, false>(hn, mode, tm_in, tm_r, tm_c, a, grid, dev, stream);
-  } else if (fmt == FP4_MXFP8) {
-    switch (hn) {
-      case 0: e = dispatch_mode<kFmtMX8, 0, false, false>(mode, tm_in, tm_r, tm_c, a, grid, dev, stream); break;
-      case 16: e = dispatch_mode<kFmtMX8, 16, false, false>(mode, tm_in, tm_r, tm_c, a, grid, dev, stream); break;
-      default: e = dispatch_mode<kFmtMX8, 32, false, false>(mode, tm_in, tm_r, tm_c, a, grid, dev, stream);
-    }
-  } else {
+  if (fmt == FP4_NVFP4) {
     // ts layout: single -> {S, amax}; dual -> {S_row, S_col, amax_row, amax_col}
     float* amax_r = nullptr;
     float* amax_c = nullptr;
@@ -297,22 +312,79 @@ fp4_status quantize_impl(const void* x, void* rcodes, void* rscales, void* ccode
       a.amax_col = amax_c ? (amax_r ? amax_in + 1 : amax_in) : nullptr;
       a.amax_row_copy = amax_r;
       a.amax_col_copy = amax_c;
-      e = dispatch_hn<kFmtNV, false>(hn, mode, tm_in, tm_r, tm_c, a, grid, dev, stream);
     } else {
       a.amax_row = amax_r;
       a.amax_col = amax_c;
       a.amax_row_acc = reinterpret_cast<unsigned*>(amax_r);
       a.amax_col_acc = reinterpret_cast<unsigned*>(amax_c);
-      float* first = amax_r ? amax_r : amax_c;
-      const size_t nbytes = (amax_r && amax_c) ? 2 * sizeof(float) : sizeof(float);
-      e = cudaMemsetAsync(first, 0, nbytes, stream);
-      if (e == cudaSuccess)
-        e = dispatch_hn<kFmtNV, true>(hn, mode, tm_in, tm_r, tm_c, a, grid, dev, stream);
-      if (e == cudaSuccess)
-        e = dispatch_hn<kFmtNV, false>(hn, mode, tm_in, tm_r, tm_c, a, grid, dev, stream);
+      *amax_cells = amax_r ? amax_r : amax_c;
+      *amax_bytes = (amax_r && amax_c) ? 2 * sizeof(float) : sizeof(float);
     }
   }
+  return FP4_OK;
+}
+
+// Launch the kernels of up to kQMaxItems prepared tensors of one format, rotation and
+// mode: NVFP4 without supplied amaxes zeroes the amax cells, runs the amax pass and then
+// the quantise pass; the other formats one quantise pass. `need_amax_pass` is whether
+// the (all-alike) tensors take the amax pass.
+fp4_status launch_batch(QuantBatch& qb, const float* const* amax_cells, const size_t* amax_bytes,
+                        fp4_format fmt, int hn, int mode, bool need_amax_pass,
+                        const DeviceInfo* info, int dev, cudaStream_t stream) {
+  int tiles = 0;
+  for (int k = 0; k < qb.n; ++k) {
+    qb.item[k].tile0 = tiles;
+    if (int64_t(tiles) + qb.item[k].a.num_tiles > INT32_MAX) return FP4_ERR_SHAPE;
+    tiles += qb.item[k].a.num_tiles;
+  }
+  qb.num_tiles = tiles;
+  if (qb.n == 0 || tiles == 0) return FP4_OK;
+  const bool ext = qb.item[0].a.sr != 0 || qb.item[0].a.rht != 0;
+  const int per_sm = fmt == FP4_MXFP8 ? kQCtasPerSMOf(kFmtMX8, false)
+                     : fmt == FP4_MXFP4 ? kQCtasPerSMOf(kFmtMX, ext)
+                                        : kQCtasPerSMOf(kFmtNV, ext);
+  const int resident = per_sm * info->sm_count;
+  const int grid = tiles < resident ? tiles : resident;
+  cudaError_t e = cudaSuccess;
+  if (fmt == FP4_MXFP4) {
+    e = dispatch_hn<kFmtMX, false>(hn, mode, qb, grid, dev, stream);
+  } else if (fmt == FP4_MXFP8) {
+    switch (hn) {
+      case 0: e = dispatch_mode<kFmtMX8, 0, false, false>(mode, qb, grid, dev, stream); break;
+      case 16: e = dispatch_mode<kFmtMX8, 16, false, false>(mode, qb, grid, dev, stream); break;
+      default: e = dispatch_mode<kFmtMX8, 32, false, false>(mode, qb, grid, dev, stream);
+    }
+  } else {
+    if (need_amax_pass) {
+      for (int k = 0; k < qb.n && e == cudaSuccess; ++k)
+        e = cudaMemsetAsync(const_cast<float*>(amax_cells[k]), 0, amax_bytes[k], stream);
+      if (e == cudaSuccess) e = dispatch_hn<kFmtNV, true>(hn, mode, qb, grid, dev, stream);
+    }
+    if (e == cudaSuccess) e = dispatch_hn<kFmtNV, false>(hn, mode, qb, grid, dev, stream);
+  }
   return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+}
+
+fp4_status quantize_impl(const void* x, void* rcodes, void* rscales, void* ccodes, void* cscales,
+                         float* ts, int64_t rows, int64_t cols, fp4_format fmt, int hn, int mode,
+                         cudaStream_t stream, const fp4_quant_opts* opts = nullptr) {
+  // thread-local storage keeps the batch (2.3 KB of tensor maps and arguments) off
+  // small host stacks
+  static thread_local QuantBatch qb;
+  bool skip;
+  float* cells;
+  size_t cell_bytes;
+  fp4_status st = prepare_item(&qb.item[0], &skip, &cells, &cell_bytes, x, rcodes, rscales,
+                               ccodes, cscales, ts, rows, cols, fmt, hn, mode, opts);
+  if (st != FP4_OK || skip) return st;
+  int dev;
+  const DeviceInfo* info;
+  st = current_device(&dev, &info);
+  if (st != FP4_OK) return st;
+  qb.n = 1;
+  const float* cell_list[1] = {cells};
+  return launch_batch(qb, cell_list, &cell_bytes, fmt, hn, mode, cells != nullptr, info, dev,
+                      stream);
 }
 
 // ---------------------------------------------------------------- GEMM launch
@@ -683,6 +755,66 @@ fp4_status fp4_quantize_dual_opts(const void* x, void* row_codes, void* row_scal
   NvtxRange nvtx_range("fp4_quantize_dual_opts");
   return quantize_impl(x, row_codes, row_scales, col_codes, col_scales, ts, rows, cols, fmt, hn,
                        kModeDual, reinterpret_cast<cudaStream_t>(stream), opts);
+}
+
+fp4_status fp4_quantize_dual_batch(const fp4_quant_item* items, int n, fp4_format fmt, int hn,
+                                   fp4_stream_t stream) {
+  NvtxRange nvtx_range("fp4_quantize_dual_batch");
+  if (n < 0 || (n > 0 && !items)) return FP4_ERR_INVALID_ARG;
+  // every tensor is checked, then every map built, before anything is launched
+  for (int i = 0; i < n; ++i) {
+    const fp4_quant_item& t = items[i];
+    bool skip;
+    const fp4_status st = check_item(&skip, t.x_bf16, t.row_codes, t.row_scales, t.col_codes,
+                                     t.col_scales, t.tensor_scale, t.rows, t.cols, fmt, hn,
+                                     kModeDual, nullptr);
+    if (st != FP4_OK) return st;
+  }
+  std::vector<QuantItem> prepared;
+  std::vector<float*> cells;
+  std::vector<size_t> cell_bytes;
+  prepared.reserve(n);
+  for (int i = 0; i < n; ++i) {
+    const fp4_quant_item& t = items[i];
+    QuantItem q;
+    bool skip;
+    float* c;
+    size_t cb;
+    const fp4_status st =
+        prepare_item(&q, &skip, &c, &cb, t.x_bf16, t.row_codes, t.row_scales, t.col_codes,
+                     t.col_scales, t.tensor_scale, t.rows, t.cols, fmt, hn, kModeDual, nullptr);
+    if (st != FP4_OK) return st;
+    if (skip) continue;
+    prepared.push_back(q);
+    cells.push_back(c);
+    cell_bytes.push_back(cb);
+  }
+  if (prepared.empty()) return FP4_OK;
+  int dev;
+  const DeviceInfo* info;
+  fp4_status st = current_device(&dev, &info);
+  if (st != FP4_OK) return st;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  static thread_local QuantBatch qb;
+  // tensors whose transposed codes want the banded tile order go alone; the rest in
+  // groups of up to kQMaxItems, in the order given
+  size_t i = 0;
+  while (i < prepared.size() && st == FP4_OK) {
+    qb.n = 0;
+    const float* group_cells[kQMaxItems];
+    size_t group_bytes[kQMaxItems];
+    while (i < prepared.size() && qb.n < kQMaxItems) {
+      const bool banded = prepared[i].a.band_c < prepared[i].a.tiles_c;
+      if (banded && qb.n > 0) break;
+      group_cells[qb.n] = cells[i];
+      group_bytes[qb.n] = cell_bytes[i];
+      qb.item[qb.n++] = prepared[i++];
+      if (banded) break;
+    }
+    st = launch_batch(qb, group_cells, group_bytes, fmt, hn, kModeDual, fmt == FP4_NVFP4, info,
+                      dev, s);
+  }
+  return st;
 }
 
 fp4_status fp4_gemm(const void* A, const void* As, const float* Ats, const void* B, const void* Bs,

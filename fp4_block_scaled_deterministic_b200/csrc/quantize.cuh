@@ -74,6 +74,59 @@ struct QuantArgs {
   uint64_t wait_limit_ns;
 };
 
+// One launch quantises up to kQMaxItems tensors (e.g. the X, W and dY of one projection
+// of a training step), so that the launch's fixed costs -- start-up, pipeline fill,
+// drain and the last partial wave of tiles -- are paid once. Tiles are numbered one
+// tensor after the other (tensor k's first tile is tile0); each tensor has its own TMA
+// maps and arguments. A single-tensor call is a batch of one.
+constexpr int kQMaxItems = 4;
+struct QuantItem {
+  CUtensorMap in, rcodes, ccodes;
+  QuantArgs a;
+  int tile0;
+};
+struct QuantBatch {
+  QuantItem item[kQMaxItems];
+  int n, num_tiles;
+};
+// Tensor of global tile `tile`. NITEMS (a kernel template argument) is 1 for
+// single-tensor launches, whose code then indexes item 0 at compile time.
+template <int NITEMS>
+__device__ __forceinline__ int batch_item(const QuantBatch& qb, int tile) {
+  if constexpr (NITEMS == 1) return 0;
+  int k = 0;
+#pragma unroll
+  for (int j = 1; j < NITEMS; ++j) k += (j < qb.n && tile >= qb.item[j].tile0) ? 1 : 0;
+  return k;
+}
+// NVFP4 tensor scales of every tensor of the batch into s_S[2k] (row) and s_S[2k+1]
+// (column layout): S = amax / 2688 (1 when amax is 0); CTA 0 also publishes them (and
+// copies a caller-supplied amax). Thread 0 of each CTA calls this before its first barrier.
+template <bool kRow, bool kCol, int NITEMS>
+__device__ __forceinline__ void batch_tensor_scales(const QuantBatch& qb, float* s_S, bool publish) {
+  const int n = NITEMS == 1 ? 1 : qb.n;
+  for (int k = 0; k < n; ++k) {
+    const QuantArgs& a = qb.item[k].a;
+    float S_r = 1.0f, S_c = 1.0f;
+    if constexpr (kRow) {
+      const float T = *a.amax_row;
+      S_r = T > 0.0f ? __fdiv_rn(T, 2688.0f) : 1.0f;
+    }
+    if constexpr (kCol) {
+      const float T = *a.amax_col;
+      S_c = T > 0.0f ? __fdiv_rn(T, 2688.0f) : 1.0f;
+    }
+    s_S[2 * k] = S_r;
+    s_S[2 * k + 1] = S_c;
+    if (publish) {
+      if constexpr (kRow) *a.s_row_out = S_r;
+      if constexpr (kCol) *a.s_col_out = S_c;
+      if constexpr (kRow) if (a.amax_row_copy) *a.amax_row_copy = *a.amax_row;
+      if constexpr (kCol) if (a.amax_col_copy) *a.amax_col_copy = *a.amax_col;
+    }
+  }
+}
+
 // Every unit of work ("job") is two independent 32-element vectors held lane-wise in
 // float2 registers (.x = first vector, .y = second), so the butterflies, scalings and
 // quotients use the packed fp32x2 instructions; each lane is rounded exactly as the
@@ -136,8 +189,8 @@ __device__ __forceinline__ float tree_max(const float* v) {
   }
 }
 // max |x| over elements [B, B+N) of each lane.
-template <int B, int N>
-__device__ __forceinline__ float2 amax_x2(const float2 (&p)[32]) {
+template <int B, int N, int L>
+__device__ __forceinline__ float2 amax_x2(const float2 (&p)[L]) {
   float ax[N], ay[N];
 #pragma unroll
   for (int i = 0; i < N; ++i) {
@@ -315,8 +368,8 @@ __device__ __forceinline__ bool near_e2m1_threshold(float q) {
 // The quotient is formed as v * y with y = RN(1/d): then |v*y - v/d| < 2 ulps, so v*y and
 // RN(v/d) fall on the same side of every E2M1 threshold unless v*y is within 4 ulps of
 // one; those (rare) blocks, and blocks whose 1/d overflows, are divided exactly.
-template <int b, bool kExact = false>
-__device__ __forceinline__ void nv_block_x2(float2 (&p)[32], float S, float six_s,
+template <int b, bool kExact = false, int L = 32>
+__device__ __forceinline__ void nv_block_x2(float2 (&p)[L], float S, float six_s,
                                             uint32_t& sbx, uint32_t& sby) {
   const float2 bm = amax_x2<b, 16>(p);
   sbx = cvt_e4m3(__fdiv_rn(bm.x, six_s));
@@ -324,21 +377,30 @@ __device__ __forceinline__ void nv_block_x2(float2 (&p)[32], float S, float six_
   const float dx = __fmul_rn(e4m3_to_f32(sbx), S), dy = __fmul_rn(e4m3_to_f32(sby), S);
   const float yx = __frcp_rn(dx), yy = __frcp_rn(dy);
   const float2 y2 = make_float2(yx, yy);
-  float2 q[16];
+  // Two passes (the quotients are not kept between them, which saves registers): find
+  // whether any reciprocal product lands near a threshold, then overwrite each value
+  // with its quotient, divided exactly when so.
   bool exact = kExact || !(yx <= 3.0e38f) || !(yy <= 3.0e38f);
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    q[i] = mul2(p[b + i], y2);
-    exact |= near_e2m1_threshold(q[i].x) | near_e2m1_threshold(q[i].y);
+    const float2 q = mul2(p[b + i], y2);
+    exact |= near_e2m1_threshold(q.x) | near_e2m1_threshold(q.y);
   }
+  // A zero block scale gives zeros that keep the sign of the element itself (the
+  // quotient by d = 0 is an infinity, or a NaN for a zero element).
+  const bool zx = sbx == 0u, zy = sby == 0u;
+  auto put = [&](int i, float2 q) {
+    const float2 v = p[b + i];
+    p[b + i] = make_float2(zx ? __uint_as_float(__float_as_uint(v.x) & 0x80000000u) : q.x,
+                           zy ? __uint_as_float(__float_as_uint(v.y) & 0x80000000u) : q.y);
+  };
   if (exact) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) q[i] = make_float2(__fdiv_rn(p[b + i].x, dx), __fdiv_rn(p[b + i].y, dy));
-  }
+    for (int i = 0; i < 16; ++i)
+      put(i, make_float2(__fdiv_rn(p[b + i].x, dx), __fdiv_rn(p[b + i].y, dy)));
+  } else {
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    p[b + i].x = sbx == 0u ? __uint_as_float(__float_as_uint(p[b + i].x) & 0x80000000u) : q[i].x;
-    p[b + i].y = sby == 0u ? __uint_as_float(__float_as_uint(p[b + i].y) & 0x80000000u) : q[i].y;
+    for (int i = 0; i < 16; ++i) put(i, mul2(p[b + i], y2));
   }
 }
 
@@ -603,16 +665,16 @@ __device__ __forceinline__ void qtile_coords(int tile, const QuantArgs& a, int& 
 
 // EXT kernels also implement the variants selected at run time by a.rht (random +-1
 // signs along the contraction axis before the rotation) and a.sr (stochastic rounding).
-template <int FMT, int HN, int MODE, bool AMAX, bool EXT = false, bool BANDED = false>
+template <int FMT, int HN, int MODE, bool AMAX, bool EXT = false, bool BANDED = false,
+          int NITEMS = 1>
 __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
-    quantize_kernel(const __grid_constant__ CUtensorMap tm_in,
-                    const __grid_constant__ CUtensorMap tm_rcodes,
-                    const __grid_constant__ CUtensorMap tm_ccodes, const QuantArgs a) {
+    quantize_kernel(const __grid_constant__ QuantBatch qb) {
   constexpr bool kRow = (MODE & kModeRow) != 0;
   constexpr bool kCol = (MODE & kModeCol) != 0;
   // MXFP4 + H16 quantise pass: the rotation's x0.25 is folded into the block scale
   constexpr bool kFoldH16 = FMT == kFmtMX && HN == 16 && !AMAX;
-  const bool rht = EXT && a.rht != 0, sr = EXT && a.sr != 0;
+  // variants come one tensor per launch
+  const bool rht = EXT && qb.item[0].a.rht != 0, sr = EXT && qb.item[0].a.sr != 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -624,22 +686,26 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
   uint8_t* s_rsc = s_ccode + 2 * kCodeBytes;
   uint8_t* s_csc = s_rsc + 2 * kQScaleBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(s_csc + 2 * kQScaleBytes);
-  float* s_red = reinterpret_cast<float*>(full + kQStages);  // [8 warps][2]
+  // per-tensor amax accumulators of the amax pass (bits of non-negative floats) and
+  // NVFP4 tensor scales {row, col} of the batch's tensors
+  unsigned* s_amax = reinterpret_cast<unsigned*>(full + kQStages);  // [kQMaxItems][2]
+  float* s_S = reinterpret_cast<float*>(s_amax + 2 * kQMaxItems);   // [kQMaxItems][2]
   // random-sign XOR masks of a tile, double-buffered by tile parity: 64 column-pair
-  // words (ROW jobs) and 128 row words (COL jobs) per buffer; 16-byte aligned (s_red is
-  // 16 floats after 8-byte barriers)
+  // words (ROW jobs) and 128 row words (COL jobs) per buffer; 16-byte aligned
   uint32_t* s_masks = reinterpret_cast<uint32_t*>(
-      (reinterpret_cast<uintptr_t>(s_red + 16) + 15) & ~static_cast<uintptr_t>(15));
+      (reinterpret_cast<uintptr_t>(s_S + 2 * kQMaxItems) + 15) & ~static_cast<uintptr_t>(15));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bid = blockIdx.x, nctas = gridDim.x;
-  const int my_tiles = bid < a.num_tiles ? (a.num_tiles - bid + nctas - 1) / nctas : 0;
+  const int my_tiles = bid < qb.num_tiles ? (qb.num_tiles - bid + nctas - 1) / nctas : 0;
 
   // Signs of a tile's 128 columns (warp 0) and 128 rows (warp 1) into mask buffer `buf`:
   // Philox block (tile start)/4 + lane holds the words of indices 4*lane .. 4*lane+3.
   auto write_masks = [&](int tile, int buf) {
+    const QuantItem& I = qb.item[batch_item<NITEMS>(qb, tile)];
+    const QuantArgs& a = I.a;
     int tr, tc;
-    qtile_coords<BANDED>(tile, a, tr, tc);
+    qtile_coords<BANDED>(tile - I.tile0, a, tr, tc);
     uint32_t* cm = s_masks + 192 * buf;
     if (kRow && warp == 0) {
       const uint4 w = philox_block(static_cast<uint64_t>(tc) * 32u + lane, 0u, a.sign_key);
@@ -656,46 +722,29 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
     }
   };
   if (tid == 0) {
-    tma_prefetch_desc(&tm_in);
+    for (int k = 0; k < (NITEMS == 1 ? 1 : qb.n); ++k) tma_prefetch_desc(&qb.item[k].in);
     for (int s = 0; s < kQStages; ++s) mbar_init(&full[s], 1);
+    for (int k = 0; k < 2 * kQMaxItems; ++k) s_amax[k] = 0u;
+    if constexpr (FMT == kFmtNV && !AMAX) batch_tensor_scales<kRow, kCol, NITEMS>(qb, s_S, bid == 0);
     mbar_fence_init();
   }
   if (rht && my_tiles > 0) write_masks(bid, 0);
   __syncthreads();
 
-  // NVFP4 tensor scales of the quantise pass: S = amax / 2688 (1 when amax is 0).
-  float S_r = 1.0f, S_c = 1.0f;
-  if constexpr (FMT == kFmtNV && !AMAX) {
-    if constexpr (kRow) {
-      const float T = *a.amax_row;
-      S_r = T > 0.0f ? __fdiv_rn(T, 2688.0f) : 1.0f;
-    }
-    if constexpr (kCol) {
-      const float T = *a.amax_col;
-      S_c = T > 0.0f ? __fdiv_rn(T, 2688.0f) : 1.0f;
-    }
-    if (bid == 0 && tid == 0) {
-      if constexpr (kRow) *a.s_row_out = S_r;
-      if constexpr (kCol) *a.s_col_out = S_c;
-      if constexpr (kRow) if (a.amax_row_copy) *a.amax_row_copy = *a.amax_row;
-      if constexpr (kCol) if (a.amax_col_copy) *a.amax_col_copy = *a.amax_col;
-    }
-  }
-  const float six_r = __fmul_rn(6.0f, S_r), six_c = __fmul_rn(6.0f, S_c);
-
   auto issue_load = [&](int stage, int tile) {
+    const QuantItem& I = qb.item[batch_item<NITEMS>(qb, tile)];
     int tr, tc;
-    qtile_coords<BANDED>(tile, a, tr, tc);
+    qtile_coords<BANDED>(tile - I.tile0, I.a, tr, tc);
     uint8_t* dst = s_in + stage * kQInBytes;
-    if (!FP4_IN_BOUNDS(tile < a.num_tiles && tr >= 0 && tr < a.tiles_r && tc >= 0 &&
-                       tc < a.tiles_c)) {
+    if (!FP4_IN_BOUNDS(tile < qb.num_tiles && tr >= 0 && tr < I.a.tiles_r && tc >= 0 &&
+                       tc < I.a.tiles_c)) {
       tr = 0;  // an in-range tile: the barrier still gets its bytes and nothing hangs
       tc = 0;
     }
     if (!FP4_IN_BOUNDS(stage >= 0 && stage < kQStages)) return;  // the bounded waits report it
     mbar_arrive_expect_tx(&full[stage], kQInBytes);
-    tma_load_2d(dst, &tm_in, &full[stage], tc * 128, tr * 128);
-    tma_load_2d(dst + kQBoxBytes, &tm_in, &full[stage], tc * 128 + 64, tr * 128);
+    tma_load_2d(dst, &I.in, &full[stage], tc * 128, tr * 128);
+    tma_load_2d(dst + kQBoxBytes, &I.in, &full[stage], tc * 128 + 64, tr * 128);
   };
   if (tid == 0) {
     const int pro = my_tiles < kQStages ? my_tiles : kQStages;
@@ -714,8 +763,17 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
   float amax_r = 0.0f, amax_c = 0.0f;
   for (int it = 0; it < my_tiles; ++it) {
     const int tile = bid + it * nctas;
+    const int item = batch_item<NITEMS>(qb, tile);
+    const QuantItem& I = qb.item[item];
+    const QuantArgs& a = I.a;
     int tr, tc;
-    qtile_coords<BANDED>(tile, a, tr, tc);
+    qtile_coords<BANDED>(tile - I.tile0, a, tr, tc);
+    float S_r = 1.0f, S_c = 1.0f;  // NVFP4 tensor scales of this tile's tensor
+    if constexpr (FMT == kFmtNV && !AMAX) {
+      S_r = s_S[2 * item];
+      S_c = s_S[2 * item + 1];
+    }
+    const float six_r = __fmul_rn(6.0f, S_r), six_c = __fmul_rn(6.0f, S_c);
     const int st = it % kQStages, ob = it & 1;
     // One barrier per tile (at its end). The next tile's signs go to the other mask
     // buffer, whose readers (the tile before this one) finished before the last barrier.
@@ -850,6 +908,19 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
       // The next tile writes staging buffer ob^1, which the stores issued after the last
       // barrier are reading: wait for those reads before this barrier releases it.
       if (tid == 0) bulk_wait_read<0>();
+    } else {
+      // this tile's amax into its tensor's accumulator (a max: exact in any order)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        amax_r = fmaxf(amax_r, __shfl_xor_sync(0xffffffffu, amax_r, o));
+        amax_c = fmaxf(amax_c, __shfl_xor_sync(0xffffffffu, amax_c, o));
+      }
+      if (lane == 0) {
+        if constexpr (kRow) atomicMax(&s_amax[2 * item], __float_as_uint(amax_r));
+        if constexpr (kCol) atomicMax(&s_amax[2 * item + 1], __float_as_uint(amax_c));
+      }
+      amax_r = 0.0f;
+      amax_c = 0.0f;
     }
     if (__syncthreads_or(!ok)) break;  // give up together; the status word says why
     if (tid == 0) {
@@ -860,7 +931,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
         if constexpr (kRow) {
           const int first = tc * kAtomsPerTile;
           const int n = (a.row_kb4 - first) < kAtomsPerTile ? (a.row_kb4 - first) : kAtomsPerTile;
-          if (tile_ok) tma_store_2d(&tm_rcodes, rcode, tc * kTileCodeBytes, tr * 128);
+          if (tile_ok) tma_store_2d(&I.rcodes, rcode, tc * kTileCodeBytes, tr * 128);
           if (tile_ok && FP4_IN_BOUNDS(n > 0 && first + n <= a.row_kb4))
             bulk_store(a.row_scales + (static_cast<int64_t>(tr) * a.row_kb4 + first) * 512, rsc,
                        static_cast<uint32_t>(n * 512));
@@ -868,7 +939,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
         if constexpr (kCol) {
           const int first = tr * kAtomsPerTile;
           const int n = (a.col_kb4 - first) < kAtomsPerTile ? (a.col_kb4 - first) : kAtomsPerTile;
-          if (tile_ok) tma_store_2d(&tm_ccodes, ccode, tr * kTileCodeBytes, tc * 128);
+          if (tile_ok) tma_store_2d(&I.ccodes, ccode, tr * kTileCodeBytes, tc * 128);
           if (tile_ok && FP4_IN_BOUNDS(n > 0 && first + n <= a.col_kb4))
             bulk_store(a.col_scales + (static_cast<int64_t>(tc) * a.col_kb4 + first) * 512, csc,
                        static_cast<uint32_t>(n * 512));
@@ -881,26 +952,472 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
   if constexpr (!AMAX) {
     if (tid == 0) bulk_wait<0>();
   } else {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      amax_r = fmaxf(amax_r, __shfl_xor_sync(0xffffffffu, amax_r, o));
-      amax_c = fmaxf(amax_c, __shfl_xor_sync(0xffffffffu, amax_c, o));
-    }
-    if (lane == 0) {
-      s_red[2 * warp] = amax_r;
-      s_red[2 * warp + 1] = amax_c;
-    }
     __syncthreads();
     if (tid == 0) {
-      float mr = 0.0f, mc = 0.0f;
-      for (int w = 0; w < kQThreads / 32; ++w) {
-        mr = fmaxf(mr, s_red[2 * w]);
-        mc = fmaxf(mc, s_red[2 * w + 1]);
-      }
       // non-negative floats order like their bit patterns: max is exact and
       // independent of the order in which CTAs arrive
-      if constexpr (kRow) atomicMax(a.amax_row_acc, __float_as_uint(mr));
-      if constexpr (kCol) atomicMax(a.amax_col_acc, __float_as_uint(mc));
+      for (int k = 0; k < (NITEMS == 1 ? 1 : qb.n); ++k) {
+        if constexpr (kRow) atomicMax(qb.item[k].a.amax_row_acc, s_amax[2 * k]);
+        if constexpr (kCol) atomicMax(qb.item[k].a.amax_col_acc, s_amax[2 * k + 1]);
+      }
+    }
+  }
+}
+
+
+// ====================================================================================
+// quantize_wide_kernel: the plain MXFP4 / NVFP4 quantiser (no variant) with twice the
+// warps per SM. The same tiles, TMA pipeline, staging and stores as quantize_kernel, but
+// 512 threads per CTA whose jobs hold 32 values (32 registers) instead of 64, so two
+// CTAs of 16 warps fit per SM: the ALU and FMA pipes, not warp latency, then set the
+// pace. Per 128x128 tile every thread takes
+//   one ROW job : row t%128, columns 32q .. 32q+31 (q = t/128) -- one MX block or two NV
+//                 blocks -- as 16 pairs (v[2k], v[2k+1]), so strides >= 2 of the
+//                 butterfly and the scaling are packed fp32x2 ops;
+//   one COL job : columns c, c+1 (lanes x, y) of 16 consecutive rows; lanes 0-15 and
+//                 16-31 of a warp hold the two 16-row halves of the same 32-row MX
+//                 block, whose amax (and the H32 stride-16 butterfly) they complete
+//                 with one warp shuffle.
+// The arithmetic of every value is the one quantize_kernel (and the oracle) performs.
+constexpr int kQWThreads = 512;
+constexpr int kQWSmemBytes = 1024 + 2 * kQInBytes + 2 * 2 * kQCodeBytesOf(kFmtMX) +
+                             2 * 2 * kQScaleBytes + 256;
+
+// ROW job loader: row r, columns 32q .. 32q+31 as pairs q2[k] = (v[2k], v[2k+1]); with
+// kFuse1 the stride-1 butterfly is done here (q2[k] = (v[2k] + v[2k+1], v[2k] - v[2k+1])).
+template <bool kFuse1>
+__device__ __forceinline__ void load_row_v(const uint8_t* in, int r, int q, float2 (&q2)[16]) {
+  if (!FP4_IN_BOUNDS(r >= 0 && r < 128 && q >= 0 && q < 4)) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) q2[i] = make_float2(0.0f, 0.0f);
+    return;
+  }
+  const uint8_t* rowp = in + (q >> 1) * kQBoxBytes + r * 128;
+  const int cb = (q & 1) * 4;  // first 16-byte chunk of the 32 columns in the box row
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint4 w = *reinterpret_cast<const uint4*>(rowp + (((cb + j) ^ (r & 7)) << 4));
+    const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if constexpr (kFuse1) {
+        float sm, df;
+        bfly1_lo(a[k], add_hi(a[k], -0.0f), sm, df);
+        q2[4 * j + k] = make_float2(sm, df);
+      } else {
+        q2[4 * j + k] = make_float2(bf16lo(a[k]), bf16hi(a[k]));
+      }
+    }
+  }
+}
+
+// COL job loader: columns 2*cp, 2*cp+1 of the tile (lanes x, y), rows r0 .. r0+15
+// (r0 a multiple of 16), p[i] = row r0+i; kFuse1 as for the ROW job.
+template <bool kFuse1>
+__device__ __forceinline__ void load_col_v(const uint8_t* in, int cp, int r0, float2 (&p)[16]) {
+  if (!FP4_IN_BOUNDS(cp >= 0 && cp < 64 && r0 >= 0 && r0 + 16 <= 128 && (r0 & 15) == 0)) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) p[i] = make_float2(0.0f, 0.0f);
+    return;
+  }
+  const int wc = cp & 31;
+  const uint8_t* colp = in + (cp >> 5) * kQBoxBytes + r0 * 128 + ((wc & 3) << 2);
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) {
+    // rows r0+i, r0+i+1: (r0 + i) & 7 == i & 7, a compile-time swizzle per step
+    const uint32_t v0 = *reinterpret_cast<const uint32_t*>(colp + i * 128 + (((wc >> 2) ^ (i & 7)) << 4));
+    const uint32_t v1 =
+        *reinterpret_cast<const uint32_t*>(colp + (i + 1) * 128 + (((wc >> 2) ^ ((i + 1) & 7)) << 4));
+    if constexpr (kFuse1) {
+      float sx, dx, sy, dy;
+      bfly1_lo(v0, add_lo(v1, -0.0f), sx, dx);
+      bfly1_hi(v0, add_hi(v1, -0.0f), sy, dy);
+      p[i] = make_float2(sx, sy);
+      p[i + 1] = make_float2(dx, dy);
+    } else {
+      p[i] = make_float2(bf16lo(v0), bf16hi(v0));
+      p[i + 1] = make_float2(bf16lo(v1), bf16hi(v1));
+    }
+  }
+}
+
+// Rotation stages after the fused stride-1 stage, and the final x c (unless folded).
+// ROW: strides 2 .. HN/2 pair q2[j] with q2[j + h/2] (both values of a pair share bit h).
+template <int HN, bool kScale>
+__device__ __forceinline__ void fwht_row_v(float2 (&q2)[16]) {
+  if constexpr (HN > 0) {
+#pragma unroll
+    for (int h = 2; h < HN; h <<= 1) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if ((j & (h >> 1)) == 0) {
+          const float2 a = q2[j], b = q2[j + (h >> 1)];
+          q2[j] = add2(a, b);
+          q2[j + (h >> 1)] = sub2(a, b);
+        }
+      }
+    }
+    if constexpr (kScale) {
+      const float c = (HN == 16) ? 0.25f : __uint_as_float(0x3E3504F3u);
+      const float2 c2 = make_float2(c, c);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) q2[i] = mul2(q2[i], c2);
+    }
+  }
+}
+// COL: strides 2 .. 8 inside the 16 rows; for H32 the stride-16 stage pairs row i of the
+// lower half-warp (a) with row i of the upper one (b): lower keeps a + b, upper a - b.
+template <int HN, bool kScale>
+__device__ __forceinline__ void fwht_col_v(float2 (&p)[16], bool upper) {
+  if constexpr (HN > 0) {
+#pragma unroll
+    for (int h = 2; h < HN && h < 16; h <<= 1) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if ((i & h) == 0) {
+          const float2 a = p[i], b = p[i + h];
+          p[i] = add2(a, b);
+          p[i + h] = sub2(a, b);
+        }
+      }
+    }
+    if constexpr (HN == 32) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float2 o = make_float2(__shfl_xor_sync(0xffffffffu, p[i].x, 16),
+                                     __shfl_xor_sync(0xffffffffu, p[i].y, 16));
+        // lower: p + o; upper: o + (-p) = o - p, each rounded once
+        const float2 x = upper ? o : p[i];
+        const float2 y = upper ? make_float2(-p[i].x, -p[i].y) : o;
+        p[i] = add2(x, y);
+      }
+    }
+    if constexpr (kScale) {
+      const float c = (HN == 16) ? 0.25f : __uint_as_float(0x3E3504F3u);
+      const float2 c2 = make_float2(c, c);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) p[i] = mul2(p[i], c2);
+    }
+  }
+}
+
+// MX scale byte and multiplier 2^-e from a block amax (R2), with the H16 fold when kFold:
+// byte = biased exponent of amax - 4 and the multiplier takes the x0.25 along
+// (valid when amax >= 2^-100, else *two_step is set and the caller multiplies by 0.25
+// first and uses the plain rule).
+__device__ __forceinline__ uint32_t mx_byte(float amax) {
+  const uint32_t e = (__float_as_uint(amax) >> 23) & 0xFFu;
+  return e > 2u ? e - 2u : 0u;
+}
+__device__ __forceinline__ float mx_inv(uint32_t byte) { return __uint_as_float((254u - byte) << 23); }
+
+// Codes of 16 pairs (v[2k] low nibble, v[2k+1] high) as four words, byte k = pair k.
+__device__ __forceinline__ uint4 codes_row16(const float2 (&q2)[16]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const float v[8] = {q2[4 * m].x,     q2[4 * m].y,     q2[4 * m + 1].x, q2[4 * m + 1].y,
+                        q2[4 * m + 2].x, q2[4 * m + 2].y, q2[4 * m + 3].x, q2[4 * m + 3].y};
+    w[m] = cvt_e2m1x8(v);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+// Codes of one lane of 16 consecutive entries (8 bytes).
+__device__ __forceinline__ uint2 codes_col16x(const float2 (&p)[16]) {
+  const float a[8] = {p[0].x, p[1].x, p[2].x, p[3].x, p[4].x, p[5].x, p[6].x, p[7].x};
+  const float b[8] = {p[8].x, p[9].x, p[10].x, p[11].x, p[12].x, p[13].x, p[14].x, p[15].x};
+  return make_uint2(cvt_e2m1x8(a), cvt_e2m1x8(b));
+}
+__device__ __forceinline__ uint2 codes_col16y(const float2 (&p)[16]) {
+  const float a[8] = {p[0].y, p[1].y, p[2].y, p[3].y, p[4].y, p[5].y, p[6].y, p[7].y};
+  const float b[8] = {p[8].y, p[9].y, p[10].y, p[11].y, p[12].y, p[13].y, p[14].y, p[15].y};
+  return make_uint2(cvt_e2m1x8(a), cvt_e2m1x8(b));
+}
+
+// NVFP4 block of 16 values held as 8 pairs q2[B .. B+8) (ROW job): scale byte, and the
+// pairs replaced by their quotients (or signed zeros); the arithmetic of nv_block_x2.
+template <int B>
+__device__ __forceinline__ uint32_t nv_block_row_v(float2 (&q2)[16], float S, float six_s) {
+  float a[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    a[2 * i] = fabsf(q2[B + i].x);
+    a[2 * i + 1] = fabsf(q2[B + i].y);
+  }
+  const float bm = tree_max<16>(a);
+  const uint32_t sb = cvt_e4m3(__fdiv_rn(bm, six_s));
+  const float d = __fmul_rn(e4m3_to_f32(sb), S);
+  const float y = __frcp_rn(d);
+  const float2 y2 = make_float2(y, y);
+  bool exact = !(y <= 3.0e38f);  // two passes, as in nv_block_x2
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float2 q = mul2(q2[B + i], y2);
+    exact |= near_e2m1_threshold(q.x) | near_e2m1_threshold(q.y);
+  }
+  if (sb == 0u) {  // a zero block scale: zeros that keep the sign of each element
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      q2[B + i] = make_float2(__uint_as_float(__float_as_uint(q2[B + i].x) & 0x80000000u),
+                              __uint_as_float(__float_as_uint(q2[B + i].y) & 0x80000000u));
+  } else if (exact) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) q2[B + i] = make_float2(__fdiv_rn(q2[B + i].x, d), __fdiv_rn(q2[B + i].y, d));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) q2[B + i] = mul2(q2[B + i], y2);
+  }
+  return sb;
+}
+
+template <int FMT, int HN, int MODE, bool AMAX, bool BANDED = false, int NITEMS = 1>
+__global__ void __launch_bounds__(kQWThreads, 2)
+    quantize_wide_kernel(const __grid_constant__ QuantBatch qb) {
+  static_assert(FMT == kFmtMX || FMT == kFmtNV, "FP4 formats only");
+  constexpr bool kRow = (MODE & kModeRow) != 0;
+  constexpr bool kCol = (MODE & kModeCol) != 0;
+  constexpr bool kFold = FMT == kFmtMX && HN == 16 && !AMAX;
+  constexpr bool kFuse1 = HN > 0;
+  constexpr int kStages = 2;
+  constexpr int kCodeBytes = kQCodeBytesOf(FMT);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* s_in = smem;
+  uint8_t* s_rcode = s_in + kStages * kQInBytes;
+  uint8_t* s_ccode = s_rcode + 2 * kCodeBytes;
+  uint8_t* s_rsc = s_ccode + 2 * kCodeBytes;
+  uint8_t* s_csc = s_rsc + 2 * kQScaleBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_csc + 2 * kQScaleBytes);
+  unsigned* s_amax = reinterpret_cast<unsigned*>(full + kStages);  // [kQMaxItems][2]
+  float* s_S = reinterpret_cast<float*>(s_amax + 2 * kQMaxItems);   // [kQMaxItems][2]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bid = blockIdx.x, nctas = gridDim.x;
+  const int my_tiles = bid < qb.num_tiles ? (qb.num_tiles - bid + nctas - 1) / nctas : 0;
+
+  if (tid == 0) {
+    for (int k = 0; k < (NITEMS == 1 ? 1 : qb.n); ++k) tma_prefetch_desc(&qb.item[k].in);
+    for (int st = 0; st < kStages; ++st) mbar_init(&full[st], 1);
+    for (int k = 0; k < 2 * kQMaxItems; ++k) s_amax[k] = 0u;
+    if constexpr (FMT == kFmtNV && !AMAX) batch_tensor_scales<kRow, kCol, NITEMS>(qb, s_S, bid == 0);
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  auto issue_load = [&](int stage, int tile) {
+    const QuantItem& I = qb.item[batch_item<NITEMS>(qb, tile)];
+    int tr, tc;
+    qtile_coords<BANDED>(tile - I.tile0, I.a, tr, tc);
+    uint8_t* dst = s_in + stage * kQInBytes;
+    if (!FP4_IN_BOUNDS(tile < qb.num_tiles && tr >= 0 && tr < I.a.tiles_r && tc >= 0 &&
+                       tc < I.a.tiles_c)) {
+      tr = 0;
+      tc = 0;
+    }
+    if (!FP4_IN_BOUNDS(stage >= 0 && stage < kStages)) return;
+    mbar_arrive_expect_tx(&full[stage], kQInBytes);
+    tma_load_2d(dst, &I.in, &full[stage], tc * 128, tr * 128);
+    tma_load_2d(dst + kQBoxBytes, &I.in, &full[stage], tc * 128 + 64, tr * 128);
+  };
+  if (tid == 0) {
+    const int pro = my_tiles < kStages ? my_tiles : kStages;
+    for (int st = 0; st < pro; ++st) issue_load(st, bid + st * nctas);
+  }
+
+  // job coordinates (fixed for the kernel)
+  const int row_r = tid & 127, row_q = tid >> 7;
+  const int col_cp = (warp & 3) * 16 + (lane & 15);  // column pair 0 .. 63
+  const int col_s = warp >> 2;                        // 32-row block 0 .. 3
+  const bool col_upper = lane >= 16;                  // rows 16 .. 31 of the block
+  const int col_r0 = 32 * col_s + (col_upper ? 16 : 0);
+  const int col_c = 2 * col_cp;
+
+  float amax_r = 0.0f, amax_c = 0.0f;
+  for (int it = 0; it < my_tiles; ++it) {
+    const int tile = bid + it * nctas;
+    const int item = batch_item<NITEMS>(qb, tile);
+    const QuantItem& I = qb.item[item];
+    const QuantArgs& a = I.a;
+    int tr, tc;
+    qtile_coords<BANDED>(tile - I.tile0, a, tr, tc);
+    float S_r = 1.0f, S_c = 1.0f;  // NVFP4 tensor scales of this tile's tensor
+    if constexpr (FMT == kFmtNV && !AMAX) {
+      S_r = s_S[2 * item];
+      S_c = s_S[2 * item + 1];
+    }
+    const float six_r = __fmul_rn(6.0f, S_r), six_c = __fmul_rn(6.0f, S_c);
+    const int st = it % kStages, ob = it & 1;
+    const bool ok =
+        mbar_wait(&full[st], static_cast<uint32_t>((it / kStages) & 1), a.wait_limit_ns);
+    const uint8_t* in = s_in + st * kQInBytes;
+    uint8_t* rcode = s_rcode + ob * kCodeBytes;
+    uint8_t* ccode = s_ccode + ob * kCodeBytes;
+    uint8_t* rsc = s_rsc + ob * kQScaleBytes;
+    uint8_t* csc = s_csc + ob * kQScaleBytes;
+
+    if constexpr (kRow) {
+      float2 q2[16];
+      load_row_v<kFuse1>(in, row_r, row_q, q2);
+      fwht_row_v<HN, !kFold>(q2);
+      if constexpr (AMAX) {
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          v[2 * i] = fabsf(q2[i].x);
+          v[2 * i + 1] = fabsf(q2[i].y);
+        }
+        amax_r = fmaxf(amax_r, tree_max<32>(v));
+      } else if constexpr (FMT == kFmtMX) {
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          v[2 * i] = fabsf(q2[i].x);
+          v[2 * i + 1] = fabsf(q2[i].y);
+        }
+        const float am = tree_max<32>(v);
+        uint32_t byte;
+        float inv;
+        if (kFold && am >= 0x1p-100f) {  // the x0.25 of H16 folded into the scale
+          byte = ((__float_as_uint(am) >> 23) & 0xFFu) - 4u;
+          inv = __uint_as_float((252u - byte) << 23);
+        } else {
+          if constexpr (kFold) {  // tiny block: the two-step rule
+            const float2 c2 = make_float2(0.25f, 0.25f);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) q2[i] = mul2(q2[i], c2);
+            byte = mx_byte(__fmul_rn(am, 0.25f));
+          } else {
+            byte = mx_byte(am);
+          }
+          inv = mx_inv(byte);
+        }
+        const float2 inv2 = make_float2(inv, inv);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) q2[i] = mul2(q2[i], inv2);
+        if (code_ok(row_r, row_q, 4))
+          *reinterpret_cast<uint4*>(code_chunk(rcode, row_r, row_q)) = codes_row16(q2);
+        if (scale_ok(row_r, row_q, 1)) rsc[atom_off(row_r, row_q)] = static_cast<uint8_t>(byte);
+      } else {  // NVFP4: blocks 2q and 2q+1
+        const uint32_t b0 = nv_block_row_v<0>(q2, S_r, six_r);
+        const uint32_t b1 = nv_block_row_v<8>(q2, S_r, six_r);
+        if (code_ok(row_r, row_q, 4))
+          *reinterpret_cast<uint4*>(code_chunk(rcode, row_r, row_q)) = codes_row16(q2);
+        if (scale_ok(row_r, 2 * row_q, 2))
+          *reinterpret_cast<uint16_t*>(rsc + atom_off(row_r, 2 * row_q)) =
+              static_cast<uint16_t>(b0 | (b1 << 8));
+      }
+    }
+    if constexpr (kCol) {
+      float2 p[16];
+      load_col_v<kFuse1>(in, col_cp, col_r0, p);
+      fwht_col_v<HN, !kFold>(p, col_upper);
+      if constexpr (AMAX) {
+        const float2 m = amax_x2<0, 16>(p);
+        amax_c = max3f(amax_c, m.x, m.y);
+      } else if constexpr (FMT == kFmtMX) {
+        float2 m = amax_x2<0, 16>(p);  // this half's 16 rows, then the other half's
+        m.x = fmaxf(m.x, __shfl_xor_sync(0xffffffffu, m.x, 16));
+        m.y = fmaxf(m.y, __shfl_xor_sync(0xffffffffu, m.y, 16));
+        uint32_t bx, by;
+        float2 inv;
+        if (kFold && m.x >= 0x1p-100f && m.y >= 0x1p-100f) {
+          bx = ((__float_as_uint(m.x) >> 23) & 0xFFu) - 4u;
+          by = ((__float_as_uint(m.y) >> 23) & 0xFFu) - 4u;
+          inv = make_float2(__uint_as_float((252u - bx) << 23), __uint_as_float((252u - by) << 23));
+        } else {
+          if constexpr (kFold) {
+            const float2 c2 = make_float2(0.25f, 0.25f);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) p[i] = mul2(p[i], c2);
+            bx = mx_byte(__fmul_rn(m.x, 0.25f));
+            by = mx_byte(__fmul_rn(m.y, 0.25f));
+          } else {
+            bx = mx_byte(m.x);
+            by = mx_byte(m.y);
+          }
+          inv = make_float2(mx_inv(bx), mx_inv(by));
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) p[i] = mul2(p[i], inv);
+        if (code_ok(col_c + 1, col_s, 4)) {
+          *reinterpret_cast<uint2*>(code_chunk(ccode, col_c, col_s) + (col_upper ? 8 : 0)) =
+              codes_col16x(p);
+          *reinterpret_cast<uint2*>(code_chunk(ccode, col_c + 1, col_s) + (col_upper ? 8 : 0)) =
+              codes_col16y(p);
+        }
+        if (!col_upper && scale_ok(col_c + 1, col_s, 1)) {
+          csc[atom_off(col_c, col_s)] = static_cast<uint8_t>(bx);
+          csc[atom_off(col_c + 1, col_s)] = static_cast<uint8_t>(by);
+        }
+      } else {  // NVFP4: the 16 rows are one block per column
+        uint32_t sbx, sby;
+        nv_block_x2<0, false, 16>(p, S_c, six_c, sbx, sby);
+        if (code_ok(col_c + 1, col_s, 4)) {
+          *reinterpret_cast<uint2*>(code_chunk(ccode, col_c, col_s) + (col_upper ? 8 : 0)) =
+              codes_col16x(p);
+          *reinterpret_cast<uint2*>(code_chunk(ccode, col_c + 1, col_s) + (col_upper ? 8 : 0)) =
+              codes_col16y(p);
+        }
+        const int kb = 2 * col_s + (col_upper ? 1 : 0);
+        if (scale_ok(col_c + 1, kb, 1)) {
+          csc[atom_off(col_c, kb)] = static_cast<uint8_t>(sbx);
+          csc[atom_off(col_c + 1, kb)] = static_cast<uint8_t>(sby);
+        }
+      }
+    }
+
+    if constexpr (!AMAX) {
+      fence_proxy_async_smem();
+      if (tid == 0) bulk_wait_read<0>();  // staging ob^1 free before the barrier releases it
+    } else {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        amax_r = fmaxf(amax_r, __shfl_xor_sync(0xffffffffu, amax_r, o));
+        amax_c = fmaxf(amax_c, __shfl_xor_sync(0xffffffffu, amax_c, o));
+      }
+      if (lane == 0) {
+        if constexpr (kRow) atomicMax(&s_amax[2 * item], __float_as_uint(amax_r));
+        if constexpr (kCol) atomicMax(&s_amax[2 * item + 1], __float_as_uint(amax_c));
+      }
+      amax_r = 0.0f;
+      amax_c = 0.0f;
+    }
+    if (__syncthreads_or(!ok)) break;  // give up together; the status word says why
+    if (tid == 0) {
+      if constexpr (!AMAX) {
+        constexpr int kAtomsPerTile = (FMT == kFmtNV) ? 2 : 1;
+        const bool tile_ok = FP4_IN_BOUNDS(tr >= 0 && tr < a.tiles_r && tc >= 0 && tc < a.tiles_c);
+        if constexpr (kRow) {
+          const int first = tc * kAtomsPerTile;
+          const int n = (a.row_kb4 - first) < kAtomsPerTile ? (a.row_kb4 - first) : kAtomsPerTile;
+          if (tile_ok) tma_store_2d(&I.rcodes, rcode, tc * 64, tr * 128);
+          if (tile_ok && FP4_IN_BOUNDS(n > 0 && first + n <= a.row_kb4))
+            bulk_store(a.row_scales + (static_cast<int64_t>(tr) * a.row_kb4 + first) * 512, rsc,
+                       static_cast<uint32_t>(n * 512));
+        }
+        if constexpr (kCol) {
+          const int first = tr * kAtomsPerTile;
+          const int n = (a.col_kb4 - first) < kAtomsPerTile ? (a.col_kb4 - first) : kAtomsPerTile;
+          if (tile_ok) tma_store_2d(&I.ccodes, ccode, tr * 64, tc * 128);
+          if (tile_ok && FP4_IN_BOUNDS(n > 0 && first + n <= a.col_kb4))
+            bulk_store(a.col_scales + (static_cast<int64_t>(tc) * a.col_kb4 + first) * 512, csc,
+                       static_cast<uint32_t>(n * 512));
+        }
+        bulk_commit();
+      }
+      if (it + kStages < my_tiles) issue_load(st, tile + kStages * nctas);
+    }
+  }
+  if constexpr (!AMAX) {
+    if (tid == 0) bulk_wait<0>();
+  } else {
+    __syncthreads();
+    if (tid == 0) {
+      for (int k = 0; k < (NITEMS == 1 ? 1 : qb.n); ++k) {
+        if constexpr (kRow) atomicMax(qb.item[k].a.amax_row_acc, s_amax[2 * k]);
+        if constexpr (kCol) atomicMax(qb.item[k].a.amax_col_acc, s_amax[2 * k + 1]);
+      }
     }
   }
 }

@@ -141,6 +141,34 @@ FP4_API fp4_status fp4_quantize_dual(const void *x_bf16, void *row_codes, void *
                              fp4_stream_t stream);
 
 /*
+ * fp4_quantize_dual_batch -- fp4_quantize_dual of n tensors of one format and rotation,
+ * grouped into as few launches as possible (up to four tensors per launch; a tensor
+ * whose column-layout codes exceed 256 MB goes alone). Each item is exactly one
+ * fp4_quantize_dual call: the outputs are bit-identical. A training step quantises the
+ * activation, the weight and the upstream gradient of every projection in both layouts
+ * (pre-training summary, Methodology item 2); one launch for all of them pays the
+ * launch's fixed costs (start-up, pipeline fill and drain, the last partial wave of
+ * tiles) once instead of three times.
+ *   items: host array of n descriptions (read during the call only); tensor_scale as
+ *          for fp4_quantize_dual (NVFP4: device float[4]; MXFP4 / MXFP8: NULL).
+ *   Every item is validated before anything is launched; errors as fp4_quantize_dual.
+ *   NVFP4: one memset per item, then one amax launch and one quantise launch per group.
+ */
+typedef struct fp4_quant_item {
+    const void *x_bf16;
+    void *row_codes;
+    void *row_scales;
+    void *col_codes;
+    void *col_scales;
+    float *tensor_scale;
+    int64_t rows;
+    int64_t cols;
+} fp4_quant_item;
+
+FP4_API fp4_status fp4_quantize_dual_batch(const fp4_quant_item *items, int n, fp4_format fmt,
+                                           int hadamard_n, fp4_stream_t stream);
+
+/*
  * Quantiser variants. The MXFP4 pre-training summary ("방법론" item 3 and "주요 기여
  * 및 발견" section 2) names two stabilisers, stochastic rounding and randomised
  * Hadamard rotations, which it tests and finds do not stabilise the full MXFP4

@@ -129,6 +129,21 @@ def test_gemm_quant_validation():
     assert gq(M=0) == OK
 
 
+def test_quantize_batch_validation():
+    L = fp4.lib()
+    item = fp4.QuantItem(A16, A16, A16, A16, A16, None, 64, 64)
+    bad_shape = fp4.QuantItem(A16, A16, A16, A16, A16, None, 64, 40)
+    misaligned = fp4.QuantItem(MIS, A16, A16, A16, A16, None, 64, 64)
+    arr = lambda *its: (fp4.QuantItem * len(its))(*its)
+    assert L.fp4_quantize_dual_batch(None, -1, 0, 16, None) == INVALID
+    assert L.fp4_quantize_dual_batch(None, 2, 0, 16, None) == INVALID
+    assert L.fp4_quantize_dual_batch(None, 0, 0, 16, None) == OK
+    assert L.fp4_quantize_dual_batch(arr(item, bad_shape), 2, 0, 16, None) == SHAPE
+    assert L.fp4_quantize_dual_batch(arr(item, misaligned), 2, 0, 16, None) == ALIGN
+    assert L.fp4_quantize_dual_batch(arr(item), 1, 0, 12, None) == INVALID
+    assert L.fp4_quantize_dual_batch(arr(item), 1, 1, 16, None) == INVALID  # NVFP4 needs scales
+
+
 def test_linear_validation():
     L = fp4.lib()
     need = fp4.fp4_linear_workspace_size(0, 64, 64, 64, 0)

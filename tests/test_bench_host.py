@@ -38,6 +38,10 @@ def test_workload_names():
     assert g.startswith("gpt3-175b") and "no rotation" in g
     with pytest.raises(SystemExit):
         _args("--variant", "amax")  # a supplied amax is NVFP4 only
+    assert "next layer (fused)" in bench.workload_name(_args("--next-layer-quant", "fused"))
+    assert _args().next_layer_quant == "none"
+    with pytest.raises(SystemExit):
+        _args("--next-layer-quant", "fused", "--format", "nvfp4")  # Y is quantised as MXFP4
 
 
 def test_layer_tables():
