@@ -178,6 +178,59 @@ class Clocks:
                 "samples": len(sm)}
 
 
+class NvmlClocks:
+    """SM clock and clock-event reasons read through NVML every few milliseconds, so
+    that windows of a few hundred milliseconds (the per-kernel timing pass, the timed
+    region) get tens of samples; window(t0, t1) summarises those in [t0, t1] (host
+    perf_counter seconds). Reads only: nothing is set."""
+    REASONS = (("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"))
+
+    def __init__(self, dev: int, period_s: float = 0.005):
+        self.dev, self.period, self.samples, self.ok = dev, period_s, [], False
+        self.stop_flag = threading.Event()
+
+    def start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(self.dev)
+            self.bits = {n: getattr(pynvml, c) for n, c in self.REASONS}
+            self.ok = True
+        except Exception:  # no NVML: the nvidia-smi sampler still reports
+            return
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_flag.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                break
+            self.samples.append((time.perf_counter(), mhz, rs))
+            time.sleep(self.period)
+
+    def stop(self):
+        self.stop_flag.set()
+        if self.ok:
+            self.t.join(timeout=2)
+
+    def window(self, t0: float, t1: float):
+        w = [(m, r) for t, m, r in self.samples if t0 <= t <= t1]
+        if not w:
+            return None
+        mhz = sorted(m for m, _ in w)
+        reasons = sorted(n for n, b in self.bits.items() if any(r & b for _, r in w))
+        return {"sm_mhz_median": statistics.median(mhz), "sm_mhz_min": mhz[0],
+                "sm_mhz_max": mhz[-1], "samples": len(w), "reasons": reasons}
+
+
 # ---------------------------------------------------------------- workload
 class LlamaLayer:
     """Inputs, quantised operands and outputs of every projection, all on the device."""
@@ -656,15 +709,20 @@ def main():
     timers = {"quant": [], "gemm": [], "quant_y": []}
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    nvml = NvmlClocks(local)
+    nvml.start()
+    win_pass = None
     if a.side_stream:
         # Per-kernel durations for the rooflines come from the same steps run on one
         # stream, where no kernel shares the SMs; the step time below overlaps them.
         for _ in range(a.warmup):
             layer.step(stream, None, allreduce, overlap=False)
         barrier()
+        tp0 = time.perf_counter()
         for _ in range(a.steps):
             layer.step(stream, timers, allreduce, overlap=False)
         barrier()
+        win_pass = (tp0, time.perf_counter())
         for _ in range(a.warmup):
             layer.step(stream, None, allreduce)
         barrier()
@@ -672,12 +730,20 @@ def main():
     clocks.start()
     time.sleep(0.3)
     barrier()
+    tt0 = time.perf_counter()
     e0.record(stream)
     for _ in range(a.steps):
         layer.step(stream, None if a.side_stream else timers, allreduce)
     e1.record(stream)
     barrier()
+    tt1 = time.perf_counter()
     clk = clocks.stop()
+    nvml.stop()
+    if win_pass is None:
+        win_pass = (tt0, tt1)
+    clk_fine = {"timed_region": nvml.window(tt0, tt1),
+                "kernel_timing_pass": nvml.window(*win_pass),
+                "source": "NVML every 5 ms (reads only)"} if nvml.ok else None
     ms = dp.max_over_ranks(e0.elapsed_time(e1), dev)
     status = fp4.fp4_check_status()
     if status != 0:
@@ -708,7 +774,14 @@ def main():
     traffic = (recorded_traffic("mxfp4" if fmt == 0 else "nvfp4")
                if a.workload == "llama" and a.hadamard == 16 and len(names) == len(all_names)
                else None)
+    # the GEMM rate referred to the maximum SM clock, from the clocks sampled while the
+    # per-launch times were taken (time x median MHz / max MHz)
+    at_max_clock = None
+    if clk_fine and clk_fine["kernel_timing_pass"] and clk.get("sm_max_mhz"):
+        at_max_clock = (gemm_tflops * clk["sm_max_mhz"]
+                        / clk_fine["kernel_timing_pass"]["sm_mhz_median"])
     roof = {"bound": "tensor", "achieved": gemm_tflops, "peak": peak_fp4, "unit": "TFLOP/s",
+            "achieved_at_max_sm_clock": at_max_clock,
             "frac": gemm_tflops / peak_fp4, "traffic": traffic,
             "frac_datasheet": gemm_tflops / sheet, "peak_datasheet": sheet,
             "frac_sustained": gemm_tflops / (pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
@@ -746,7 +819,7 @@ def main():
                       "l2": f"inputs larger than L2 ({(layer.bytes_in() + layer.bytes_out()) / 1e9:.1f} GB per step)",
                       "parallelism": f"dp{world}"},
            "gemm_tflops": gemm_tflops, "quantize_gbs": quant_gbs,
-           "roofline": roof, "roofline_quantize": qroof, "clocks": clk,
+           "roofline": roof, "roofline_quantize": qroof, "clocks": clk, "clocks_nvml": clk_fine,
            "gpu_launches": layer.launches_per_step() * a.steps}
     if a.next_layer_quant != "none":
         qy = [x.elapsed_time(y) for x, y in timers["quant_y"]]
