@@ -32,7 +32,8 @@ def _operands(orc, M, N, K, fmt, hn, seed):
 
 
 @pytest.mark.parametrize("shape", [(128, 256, 256), (256, 256, 256), (160, 96, 224),
-                                   (384, 512, 1024), (32, 32, 32), (256, 640, 4096)])
+                                   (384, 512, 1024), (32, 32, 32), (256, 640, 4096),
+                                   (416, 800, 512)])
 @pytest.mark.parametrize("fmt", [0, 1])
 def test_gemm_matches_oracle(orc, fmt, shape):
     M, N, K = shape
@@ -68,11 +69,13 @@ def test_gemm_integer_operands_exact(orc, fmt):
     assert np.array_equal(C.astype(np.float64), ref)
 
 
-def test_gemm_per_block_scales_exact(orc):
+@pytest.mark.parametrize("N", [256, 896])
+def test_gemm_per_block_scales_exact(orc, N):
     """Integer codes under varied power-of-two block scales (MXFP4): each 32-block
     product is exact, and scales are chosen so all partial sums stay exact, which
-    checks that every scale byte reaches the right rows and K blocks."""
-    M, N, K = 256, 256, 384  # 1.5 K-slabs: also covers the zero-filled K tail
+    checks that every scale byte reaches the right rows and K blocks. N = 896 takes
+    256 x 384 tiles (two full, one of 128 columns)."""
+    M, K = 256, 384  # 1.5 K-slabs: also covers the zero-filled K tail
     g = torch.Generator().manual_seed(6)
     a_codes = torch.randint(0, 256, (M, K // 2), generator=g, dtype=torch.uint8)
     b_codes = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8)
