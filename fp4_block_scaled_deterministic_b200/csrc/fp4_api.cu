@@ -405,7 +405,8 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtens
 // waits for a pair that is not resident.
 template <int FMT, int OUT, int QHN = -1>
 cudaError_t launch_gemm_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& sa,
-                             const CUtensorMap& sb, const GemmArgs& g, int dev, cudaStream_t s) {
+                             const CUtensorMap& sb, const CUtensorMap& c, const GemmArgs& g,
+                             int dev, cudaStream_t s) {
   static std::atomic<uint64_t> done{0};
   static int max_pairs[kMaxDevices];
   static std::once_flag once[kMaxDevices];
@@ -432,7 +433,7 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a, const CUtensorMap& b, const C
     max_pairs[dev] = n;
   });
   const int pairs = g.num_tiles < max_pairs[dev] ? g.num_tiles : max_pairs[dev];
-  k<<<2 * pairs, PairCfg<FMT>::kThreads, PairCfg<FMT>::kSmemBytes, s>>>(a, b, sa, sb, g);
+  k<<<2 * pairs, PairCfg<FMT>::kThreads, PairCfg<FMT>::kSmemBytes, s>>>(a, b, sa, sb, c, g);
   return cudaGetLastError();
 }
 
@@ -461,14 +462,17 @@ void choose_tile_order(GemmArgs& g, int64_t tile_rows, int64_t row_bytes_i) {
 // With q_hn >= 0 (fp4_gemm_quant) the output is bf16 and the epilogue also writes its
 // row-wise MXFP4 quantisation (rotation q_hn along N) to q_codes / q_scales; C may then
 // be null.
+// (This epilogue stores from registers; its instance ignores the output tensor map.)
 template <int FMT>
 cudaError_t launch_gemm_pair_quant(const CUtensorMap& a, const CUtensorMap& b,
                                    const CUtensorMap& sa, const CUtensorMap& sb,
                                    const GemmArgs& g, int q_hn, int dev, cudaStream_t s) {
+  CUtensorMap unused;
+  std::memset(&unused, 0, sizeof(unused));
   switch (q_hn) {
-    case 0: return launch_gemm_pair<FMT, 1, 0>(a, b, sa, sb, g, dev, s);
-    case 16: return launch_gemm_pair<FMT, 1, 16>(a, b, sa, sb, g, dev, s);
-    default: return launch_gemm_pair<FMT, 1, 32>(a, b, sa, sb, g, dev, s);
+    case 0: return launch_gemm_pair<FMT, 1, 0>(a, b, sa, sb, unused, g, dev, s);
+    case 16: return launch_gemm_pair<FMT, 1, 16>(a, b, sa, sb, unused, g, dev, s);
+    default: return launch_gemm_pair<FMT, 1, 32>(a, b, sa, sb, unused, g, dev, s);
   }
 }
 
@@ -553,15 +557,22 @@ fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void
             ? launch_gemm_pair_quant<kFmtMX>(ta, tb, tsa, tsb, g, q_hn, dev, stream)
             : launch_gemm_pair_quant<kFmtNV>(ta, tb, tsa, tsb, g, q_hn, dev, stream);
   } else if (pair) {
+    // The output as a tensor for the epilogue's TMA stores (fp32 outputs): boxes of 32
+    // rows x 32 bytes.
+    CUtensorMap tc;
+    const bool f32 = od == FP4_OUT_F32;
+    if (!make_map_2d(&tc, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                     f32 ? 4 : 2, C, N, M, f32 ? 8 : 16, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return FP4_ERR_CUDA;
     if (fmt == FP4_MXFP4)
-      e = od == FP4_OUT_F32 ? launch_gemm_pair<kFmtMX, 0>(ta, tb, tsa, tsb, g, dev, stream)
-                            : launch_gemm_pair<kFmtMX, 1>(ta, tb, tsa, tsb, g, dev, stream);
+      e = f32 ? launch_gemm_pair<kFmtMX, 0>(ta, tb, tsa, tsb, tc, g, dev, stream)
+              : launch_gemm_pair<kFmtMX, 1>(ta, tb, tsa, tsb, tc, g, dev, stream);
     else if (fmt == FP4_MXFP8)
-      e = od == FP4_OUT_F32 ? launch_gemm_pair<kFmtMX8, 0>(ta, tb, tsa, tsb, g, dev, stream)
-                            : launch_gemm_pair<kFmtMX8, 1>(ta, tb, tsa, tsb, g, dev, stream);
+      e = f32 ? launch_gemm_pair<kFmtMX8, 0>(ta, tb, tsa, tsb, tc, g, dev, stream)
+              : launch_gemm_pair<kFmtMX8, 1>(ta, tb, tsa, tsb, tc, g, dev, stream);
     else
-      e = od == FP4_OUT_F32 ? launch_gemm_pair<kFmtNV, 0>(ta, tb, tsa, tsb, g, dev, stream)
-                            : launch_gemm_pair<kFmtNV, 1>(ta, tb, tsa, tsb, g, dev, stream);
+      e = f32 ? launch_gemm_pair<kFmtNV, 0>(ta, tb, tsa, tsb, tc, g, dev, stream)
+              : launch_gemm_pair<kFmtNV, 1>(ta, tb, tsa, tsb, tc, g, dev, stream);
   } else if (fmt == FP4_MXFP4) {
     e = od == FP4_OUT_F32 ? launch_gemm<kFmtMX, 0>(ta, tb, tsa, tsb, g, grid, dev, stream)
                           : launch_gemm<kFmtMX, 1>(ta, tb, tsa, tsb, g, grid, dev, stream);

@@ -355,6 +355,12 @@ __device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[8]) {
                : "memory");
 }
 
+// Two fp32 values -> one word of two bf16 (RN), the first in the low half.
+__device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 // Scale (NVFP4) and store one thread's row segment of 128 accumulator columns:
 // output row m, columns [n0, n0 + 128), skipping rows >= M and 32-column chunks >= N.
 // Each store writes 32 bytes when the output is 32-byte aligned (g.c_v8; rows then are
@@ -415,6 +421,52 @@ __device__ __forceinline__ void store_row_segment(const uint32_t (&r)[128], int 
           }
         }
       }
+    }
+  }
+}
+
+// Epilogue of the pair kernel for fp32 outputs: one warp's 32-row x 128-column block
+// (rows row0 ... row0 + 31, lane i holding row row0 + i in r) leaves the SM through TMA
+// stores instead of per-thread global stores. Chunk by chunk (16 bf16 or 8 fp32 columns,
+// 32 bytes a row) the lanes write their rows into the warp's 1 KB staging buffer and
+// lane 0 issues one bulk tensor store of the 32 x 32-byte box; the TMA drops rows >= M
+// and columns >= N. Measured on the Llama layer's Wgrad GEMMs: +3 to +6% over 32-byte
+// global stores from registers; bf16 outputs (half the bytes) gained nothing and keep
+// store_row_segment.
+template <int FMT, int OUT_BF16>
+__device__ __forceinline__ void store_segment_tma(const uint32_t (&r)[128], uint8_t* stg,
+                                                  const CUtensorMap* tmC, int row0, int n0,
+                                                  const GemmArgs& g, float alpha, int lane) {
+  constexpr int kCols = OUT_BF16 ? 16 : 8;  // columns of one 32-byte row chunk
+  constexpr int kChunks = 128 / kCols;
+  if (row0 >= g.M) return;  // the warp's whole block lies beyond M
+  auto val = [&](int i) {
+    const float x = __uint_as_float(r[i]);
+    return FMT == kFmtNV ? __fmul_rn(x, alpha) : x;
+  };
+#pragma unroll
+  for (int ch = 0; ch < kChunks; ++ch) {
+    const int c0 = n0 + ch * kCols;
+    if (c0 >= g.N) break;  // the rest of the block lies beyond N
+    uint32_t w[8];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      if constexpr (OUT_BF16)
+        w[p] = pack2_bf16(val(ch * kCols + 2 * p), val(ch * kCols + 2 * p + 1));
+      else
+        w[p] = __float_as_uint(val(ch * kCols + p));
+    }
+    // the previous chunk's store has finished reading the buffer
+    if (lane == 0) bulk_wait_read<0>();
+    __syncwarp();
+    uint4* sp = reinterpret_cast<uint4*>(stg + lane * 32);
+    sp[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    sp[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tmC, stg, c0, row0);
+      bulk_commit();
     }
   }
 }
@@ -657,7 +709,10 @@ struct PairCfg {
   static constexpr int kSFBufs = kStages > 4 ? kStages : 4;
   static constexpr int kTmemSF = 256;
   static_assert(kTmemSF + kSFBufs * kSFCols <= 512, "TMEM columns");
-  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 256;
+  // 1 KB of output staging per epilogue warp (store_segment_tma, fp32 outputs) after the
+  // barriers.
+  static constexpr int kStagingBytes = 8 * 1024;
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 256 + kStagingBytes;
 };
 
 
@@ -668,7 +723,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<FMT>::kThrea
     gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmSFA,
-                         const __grid_constant__ CUtensorMap tmSFB, const GemmArgs g) {
+                         const __grid_constant__ CUtensorMap tmSFB,
+                         const __grid_constant__ CUtensorMap tmC, const GemmArgs g) {
   using Cfg = PairCfg<FMT>;
   constexpr int S = Cfg::kStages;
   using PairIssuer = Issuer<FMT, true, Cfg::kSlabK, S, Cfg::kABytes, Cfg::kBBytes,
@@ -690,6 +746,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<FMT>::kThrea
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cp_drained + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   static_assert((2 * S + 3 + Cfg::kSFBufs) * 8 + 8 <= 256, "barrier area");
+  uint8_t* s_stage_out = reinterpret_cast<uint8_t*>(bars) + 256;  // [8 warps][1 KB]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -700,6 +757,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<FMT>::kThrea
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmSFA);
     tma_prefetch_desc(&tmSFB);
+    if constexpr (QHN < 0) tma_prefetch_desc(&tmC);
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -804,11 +862,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<FMT>::kThrea
       // about a microsecond per tile.
       if (lane == 0) mbar_arrive_cluster_cta_release(leader_acc_empty);
       acc_phase ^= 1u;
-      const int m = tm * 256 + 128 * static_cast<int>(rank) + 32 * quarter + lane;
+      const int row0 = tm * 256 + 128 * static_cast<int>(rank) + 32 * quarter;
       if constexpr (QHN >= 0)
-        store_row_segment_quant<FMT, QHN>(r, m, tn * kGBN + 128 * half, g, alpha);
+        store_row_segment_quant<FMT, QHN>(r, row0 + lane, tn * kGBN + 128 * half, g, alpha);
+      else if constexpr (!OUT_BF16)  // fp32: through TMA stores (store_segment_tma)
+        store_segment_tma<FMT, OUT_BF16>(r, s_stage_out + 1024 * ew, &tmC, row0,
+                                         tn * kGBN + 128 * half, g, alpha, lane);
       else
-        store_row_segment<FMT, OUT_BF16>(r, m, tn * kGBN + 128 * half, g, alpha);
+        store_row_segment<FMT, OUT_BF16>(r, row0 + lane, tn * kGBN + 128 * half, g, alpha);
+    }
+    // every store of this warp has completed before the CTA (and its staging) goes away
+    if constexpr (QHN < 0 && !OUT_BF16) {
+      if (lane == 0) bulk_wait<0>();
+      __syncwarp();
     }
   }
   __syncwarp();
