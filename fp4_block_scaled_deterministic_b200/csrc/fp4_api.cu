@@ -396,7 +396,7 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtens
   auto k = gemm_fp4_kernel<FMT, OUT>;
   cudaError_t e = ensure_smem(k, GemmCfg<FMT>::kSmemBytes, dev, done);
   if (e != cudaSuccess) return e;
-  k<<<grid, kGThreads, GemmCfg<FMT>::kSmemBytes, s>>>(a, b, sa, sb, g);
+  k<<<grid, kGSingleThreads, GemmCfg<FMT>::kSmemBytes, s>>>(a, b, sa, sb, g);
   return cudaGetLastError();
 }
 

@@ -17,11 +17,13 @@
 // Design (one CTA per SM, persistent over 128x256 output tiles, K in slabs of 256):
 //   warp 0   : TMA producer. Per slab it loads A 128x128 B, B 256x128 B (128B swizzle)
 //              and the matching 512-byte scale atoms into a 4-stage ring.
-//   warp 1   : allocates 512 TMEM columns; one thread copies the slab's scale atoms
-//              smem -> TMEM (tcgen05.cp 32x128b.warpx4) and issues 4 MMAs of
-//              128x256x64 (tcgen05.mma kind::mxf4 / kind::mxf4nvf4), then commits
-//              the stage back to the producer; after the last slab it commits the
-//              accumulator to the epilogue.
+//   warp 1   : allocates 512 TMEM columns; one thread issues each slab's 4 MMAs of
+//              128x256x64 (tcgen05.mma kind::mxf4 / kind::mxf4nvf4) once its scales
+//              are in TMEM, then commits the stage back to the producer; after the
+//              last slab it commits the accumulator to the epilogue.
+//   warps 10, 11: one thread each copies half of the slab's scale atoms smem -> TMEM
+//              (tcgen05.cp 32x128b.warpx4) into the slab's ring slot and commits them
+//              to the MMA thread (Issuer::run_copies / run_split).
 //   warps 2-9: epilogue. Each warp owns one 32-lane quarter of TMEM and one half of
 //              the 256 columns: it pulls its 32x128 fp32 block into registers,
 //              releases the accumulator (so the next tile's MMAs start), then scales
@@ -229,6 +231,11 @@ struct Issuer {
     if constexpr (PAIR) tc_commit_pair_mc(bar, 0x3);
     else tc_commit(bar);
   }
+  // Commit to a barrier of the issuing CTA only (the leader's, for a pair).
+  __device__ __forceinline__ static void commit_local(uint64_t* bar) {
+    if constexpr (PAIR) tc_commit_pair_mc(bar, 0x1);
+    else tc_commit(bar);
+  }
 
   __device__ __forceinline__ static SlabCursor make_base(uint32_t tmem, uint8_t* sA, uint8_t* sB,
                                                          uint8_t* sSFA, uint8_t* sSFB) {
@@ -272,7 +279,7 @@ struct Issuer {
           break;
         }
         copies<LO, HI>(cur);
-        tc_commit_pair_mc(&sf_full[cur.slot], 0x1);
+        commit_local(&sf_full[cur.slot]);
         step(cur, base);
       }
       if (!ok) {
@@ -281,7 +288,7 @@ struct Issuer {
       }
     }
     // Every copy this thread issued has landed before TMEM can be released.
-    tc_commit_pair_mc(drained, 0x1);
+    commit_local(drained);
     if (!mbar_wait(drained, 0u, g.wait_limit_ns)) *abort_flag = 1;
   }
   __device__ static void run_split(uint32_t tmem, uint8_t* sA, uint8_t* sB, uint8_t* sSFA,
@@ -550,8 +557,12 @@ __device__ __forceinline__ void store_row_segment_quant(const uint32_t (&r)[128]
   *reinterpret_cast<uint32_t*>(g.q_scales + sc_off) = sbytes;
 }
 
+// Threads of the one-CTA kernel: as the pair kernel, warps 10 and 11 issue the scale
+// copies (Issuer::run_copies) while warp 1 issues the MMAs (Issuer::run_split).
+constexpr int kGSingleThreads = kGThreads + 32 * kGPairCopyThreads;
+
 template <int FMT, int OUT_BF16>
-__global__ void __launch_bounds__(kGThreads, 1)
+__global__ void __launch_bounds__(kGSingleThreads, 1)
     gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmSFA,
                     const __grid_constant__ CUtensorMap tmSFB, const GemmArgs g) {
@@ -568,8 +579,13 @@ __global__ void __launch_bounds__(kGThreads, 1)
   uint64_t* empty = bars + kGStages;
   uint64_t* acc_full = bars + 2 * kGStages;
   uint64_t* acc_empty = acc_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  uint64_t* sf_full = acc_empty + 1;  // one per scale ring slot
+  uint64_t* cp_drained = sf_full + Cfg::kSFBufs;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cp_drained + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  static_assert((2 * kGStages + 3 + Cfg::kSFBufs) * 8 + 8 <= 256, "barrier area");
+  using SingleIssuer = Issuer<FMT, false, kGBK, kGStages, kGABytes, kGBBytes, Cfg::kSFABytes,
+                              Cfg::kSFBBytes, Cfg::kSFCols, Cfg::kSFBufs>;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -584,6 +600,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 8);
+    for (int i = 0; i < Cfg::kSFBufs; ++i) mbar_init(&sf_full[i], kGPairCopyThreads);
+    mbar_init(cp_drained, kGPairCopyThreads);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -623,9 +641,21 @@ __global__ void __launch_bounds__(kGThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
-      Issuer<FMT, false, kGBK, kGStages, kGABytes, kGBBytes, Cfg::kSFABytes, Cfg::kSFBBytes,
-             Cfg::kSFCols, Cfg::kSFBufs>::run(tmem, sA, sB, sSFA, sSFB, full, empty, acc_full,
-                                              acc_empty, abort_flag, blockIdx.x, gridDim.x, g);
+      SingleIssuer::run_split(tmem, sA, sB, sSFA, sSFB, sf_full, empty, acc_full, acc_empty,
+                              abort_flag, blockIdx.x, gridDim.x, g);
+    }
+  } else if (warp >= kGThreads / 32) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ scale copies
+      constexpr int kC = SingleIssuer::kCopies, kN = kGPairCopyThreads;
+      if (warp == kGThreads / 32)
+        SingleIssuer::template run_copies<0, kC / kN>(tmem, sA, sB, sSFA, sSFB, full, sf_full,
+                                                      cp_drained, abort_flag, blockIdx.x,
+                                                      gridDim.x, g);
+      else
+        SingleIssuer::template run_copies<kC / kN, kC>(tmem, sA, sB, sSFA, sSFB, full, sf_full,
+                                                       cp_drained, abort_flag, blockIdx.x,
+                                                       gridDim.x, g);
     }
   } else {
     // -------------------------------------------------------------- epilogue
