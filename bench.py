@@ -102,6 +102,10 @@ def parse():
     ap.add_argument("--quant-batch", type=int, default=1, choices=[0, 1],
                     help="1: quantise each projection's X, W and dY in one batched launch "
                          "(fp4_quantize_dual_batch); 0: one launch per tensor")
+    ap.add_argument("--gemm-group", type=int, default=1, choices=[0, 1],
+                    help="1: a projection's Fprop, Dgrad and Wgrad GEMMs in one launch "
+                         "(fp4_gemm_group; Dgrad and Wgrad with --next-layer-quant fused); "
+                         "0: one launch per GEMM")
     ap.add_argument("--next-layer-quant", choices=["none", "standalone", "fused"], default="none",
                     help="also quantise each Fprop output Y row-wise (MXFP4, same rotation) for "
                          "the next layer: by a separate quantise launch after the GEMM, or in "
@@ -237,7 +241,7 @@ class LlamaLayer:
 
     def __init__(self, device, fmt, hn, tokens=8192, seed=0, names=None, variant="none",
                  side_stream=False, layers=None, outlier_mult=50.0, w_seed=0, next_quant="none",
-                 quant_batch=True):
+                 quant_batch=True, gemm_group=True):
         import fp4_block_scaled_deterministic_b200 as fp4
         from fp4_block_scaled_deterministic_b200 import synthetic
         self.fp4, self.fmt, self.hn, self.M = fp4, fmt, hn, tokens
@@ -245,6 +249,7 @@ class LlamaLayer:
         self.next_quant = next_quant
         # the plain quantiser takes a projection's three tensors in one batched launch
         self.quant_batch = quant_batch and variant == "none"
+        self.gemm_group = gemm_group
         self.qstream = torch.cuda.Stream(device) if side_stream else None
         self.projs = []
         g = torch.Generator(device=device)
@@ -286,6 +291,18 @@ class LlamaLayer:
                               p[key + "_col"][1].data_ptr(),
                               p[key + "_ts"].data_ptr() if fmt == 1 else None, r, c)
                 for key, (r, c) in self._operands(p)])
+            # the GEMMs of the projection in one fp4_gemm_group launch, built once:
+            # Fprop (unless its epilogue quantises Y), Dgrad, Wgrad
+            ts = (lambda k, i: p[k + "_ts"][i:i + 1].data_ptr()) if fmt == 1 else (lambda k, i: None)
+            M, N, K = tokens, p["N"], p["K"]
+            descs = [(p["dY_row"], p["W_col"], "dY", "W", 0, 1, p["dX"], M, K, N, 1),
+                     (p["dY_col"], p["X_col"], "dY", "X", 1, 1, p["dW"], N, K, M, 0)]
+            if next_quant != "fused":
+                descs.insert(0, (p["X_row"], p["W_row"], "X", "W", 0, 0, p["Y"], M, N, K, 1))
+            p["gdescs"] = (fp4.GemmDesc * len(descs))(*[
+                fp4.GemmDesc(a[0].data_ptr(), a[1].data_ptr(), ts(ka, ia), b[0].data_ptr(),
+                             b[1].data_ptr(), ts(kb, ib), out.data_ptr(), m, n, k, od)
+                for a, b, ka, kb, ia, ib, out, m, n, k, od in descs])
             for key, _ in self._operands(p):
                 o = None
                 if variant == "amax":
@@ -320,11 +337,18 @@ class LlamaLayer:
     def bytes_out(self):
         return sum(t.numel() * t.element_size() for p in self.projs for t in (p["Y"], p["dX"], p["dW"]))
 
+    def gemm_launches(self):
+        """GEMM launches of a projection: a group (plus the fused Fprop) or three."""
+        if self.gemm_group:
+            return 2 if self.next_quant == "fused" else 1
+        return 3
+
     def launches_per_step(self):
         # NVFP4 adds the amax pass (plus a memset) unless the amax is supplied
         per_q = 1 if self.fmt != 1 or self.variant == "amax" else 2
         q_launches = per_q if self.quant_batch else 3 * per_q
-        return len(self.projs) * (q_launches + 3 + (self.next_quant == "standalone"))
+        return len(self.projs) * (q_launches + self.gemm_launches() +
+                                  (self.next_quant == "standalone"))
 
     def step(self, stream, timers=None, allreduce=None, overlap=None, inputs_ready=None,
              outputs_free=None):
@@ -400,6 +424,25 @@ class LlamaLayer:
             tsx, tsw, tsy = p["X_ts"], p["W_ts"], p["dY_ts"]
             nv = fmt == 1
             M, N, K = self.M, p["N"], p["K"]
+            if self.gemm_group:
+                # Fprop, Dgrad and Wgrad (below) in one launch; with the fused epilogue the
+                # Fprop runs alone first and the group holds Dgrad and Wgrad
+                if self.next_quant == "fused":
+                    st = timed("gemm", lambda: f.fp4_gemm_quant(
+                        p["X_row"][0], p["X_row"][1], None, p["W_row"][0], p["W_row"][1], None,
+                        p["Y"], p["Yq"][0], p["Yq"][1], M, N, K, fmt, hn, s))
+                    assert st == 0
+                gd = p["gdescs"]
+                st = timed("gemm", lambda: f.lib().fp4_gemm_group(gd, len(gd), fmt, s))
+                assert st == 0, f.status_string(st)
+                if self.next_quant == "standalone":  # Q_row(Y) by a separate launch
+                    st = timed("quant_y", lambda: f.fp4_quantize(
+                        p["Y"], p["Yq"][0], p["Yq"][1], None, M, N, fmt, hn, 0, s))
+                    assert st == 0
+                self.gemms_done[i].record(stream)
+                if allreduce is not None:
+                    pending.append(allreduce(p["dW"]))
+                continue
             # Fprop: Y[M][N] = X_row . W_row^T
             if self.next_quant == "fused":  # and Q_row(Y) from the same epilogue
                 st = timed("gemm", lambda: f.fp4_gemm_quant(
@@ -432,9 +475,16 @@ class LlamaLayer:
 
 
 def gemm_flops_of(layer):
+    """Flops of each GEMM launch of one step, in launch order."""
     per = []
     for p in layer.projs:
-        per += [2.0 * layer.M * p["N"] * p["K"]] * 3
+        one = 2.0 * layer.M * p["N"] * p["K"]
+        if not layer.gemm_group:
+            per += [one] * 3
+        elif layer.next_quant == "fused":
+            per += [one, 2 * one]
+        else:
+            per += [3 * one]
     return per
 
 
@@ -691,7 +741,7 @@ def main():
     layer = LlamaLayer(dev, fmt, a.hadamard, tokens=tokens, seed=1000 * rank, names=names,
                        variant=a.variant, side_stream=bool(a.side_stream), layers=layers,
                        outlier_mult=omult, w_seed=0, next_quant=a.next_layer_quant,
-                       quant_batch=bool(a.quant_batch))
+                       quant_batch=bool(a.quant_batch), gemm_group=bool(a.gemm_group))
     stream = torch.cuda.current_stream(dev)
     from fp4_block_scaled_deterministic_b200 import dp
     allreduce = (lambda t: dp.allreduce_wgrad(t, async_op=True)) if world > 1 else None
@@ -771,7 +821,8 @@ def main():
     sheet = DATASHEET_TFLOPS["fp8" if fmt == 2 else "fp4"]
     avg_launch_ms = sum(gemm_ms) / len(gemm_ms)
     avg_flops = sum(per_launch_flops) / len(per_launch_flops)
-    traffic = (recorded_traffic("mxfp4" if fmt == 0 else "nvfp4")
+    traffic = (recorded_traffic(("mxfp4" if fmt == 0 else "nvfp4")
+                                + ("_group" if layer.gemm_launches() == 1 else ""))
                if a.workload == "llama" and a.hadamard == 16 and len(names) == len(all_names)
                else None)
     # the GEMM rate referred to the maximum SM clock, from the clocks sampled while the
@@ -787,7 +838,9 @@ def main():
             "frac_sustained": gemm_tflops / (pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
                                              * ratio),
             "kernel": "gemm_fp4_pair_kernel (tcgen05 block-scaled "
-                      f"{'MXFP8, kind::mxf8f6f4' if fmt == 2 else 'FP4'}, CTA pairs)",
+                      f"{'MXFP8, kind::mxf8f6f4' if fmt == 2 else 'FP4'}, CTA pairs"
+                      + ("; a projection's Fprop, Dgrad and Wgrad per launch)"
+                         if layer.gemm_launches() == 1 else ")"),
             "per_launch": {"avg_flops": avg_flops, "avg_ms": avg_launch_ms,
                            "launches": len(gemm_ms)},
             "timing": ("CUDA events around each launch over the timed steps" if not a.side_stream
@@ -814,6 +867,11 @@ def main():
                       "next_layer_quant": a.next_layer_quant,
                       "quant_launch": ("one batched launch per projection (X, W, dY)"
                                        if layer.quant_batch else "one launch per tensor"),
+                      "gemm_launch": (("one fp4_gemm_group launch per projection (Fprop, "
+                                       "Dgrad, Wgrad)" if layer.gemm_launches() == 1 else
+                                       "Fprop with the fused epilogue, then Dgrad and Wgrad "
+                                       "in one fp4_gemm_group launch")
+                                      if layer.gemm_group else "one launch per GEMM"),
                       "streams": 2 if a.side_stream else 1,
                       "tokens_per_rank": layer.M,
                       "l2": f"inputs larger than L2 ({(layer.bytes_in() + layer.bytes_out()) / 1e9:.1f} GB per step)",

@@ -52,6 +52,18 @@ class QuantItem(ctypes.Structure):
                 ("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
 
 
+class GemmDesc(ctypes.Structure):
+    """fp4_gemm_desc of include/fp4.h (one GEMM of fp4_gemm_group)."""
+    _fields_ = [("A_codes", ctypes.c_void_p), ("A_scales", ctypes.c_void_p),
+                ("A_tensor_scale", ctypes.c_void_p), ("B_codes", ctypes.c_void_p),
+                ("B_scales", ctypes.c_void_p), ("B_tensor_scale", ctypes.c_void_p),
+                ("C", ctypes.c_void_p), ("M", ctypes.c_int64), ("N", ctypes.c_int64),
+                ("K", ctypes.c_int64), ("out_dtype", ctypes.c_int)]
+
+
+GEMM_GROUP_MAX = 3
+
+
 class QuantOpts(ctypes.Structure):
     """fp4_quant_opts of include/fp4.h (host struct passed by pointer)."""
     _fields_ = [("amax", ctypes.c_void_p), ("stochastic", ctypes.c_int),
@@ -85,6 +97,7 @@ def lib() -> ctypes.CDLL:
             "fp4_quantize_dual_batch": (I32, [ctypes.POINTER(QuantItem), I32, I32, I32, P]),
             "fp4_gemm": (I32, [P, P, P, P, P, P, P, I64, I64, I64, I32, I32, P]),
             "fp4_gemm_quant": (I32, [P, P, P, P, P, P, P, P, P, I64, I64, I64, I32, I32, P]),
+            "fp4_gemm_group": (I32, [ctypes.POINTER(GemmDesc), I32, I32, P]),
             "fp4_linear_workspace_size": (SZ, [I32, I64, I64, I64, I32]),
             "fp4_linear_fprop": (I32, [P, P, P, I64, I64, I64, I32, I32, I32, P, SZ, P]),
             "fp4_linear_dgrad": (I32, [P, P, P, I64, I64, I64, I32, I32, I32, P, SZ, P]),
@@ -163,6 +176,14 @@ def fp4_quantize_dual_batch(items, fmt, hadamard_n, stream=None):
     arr = (QuantItem * len(items))(*[QuantItem(*[_ptr(v) for v in it[:6]], it[6], it[7])
                                      for it in items])
     return lib().fp4_quantize_dual_batch(arr, len(items), fmt, hadamard_n, _stream(stream))
+
+
+def fp4_gemm_group(descs, fmt, stream=None):
+    """descs: a sequence of (A_codes, A_scales, A_tensor_scale, B_codes, B_scales,
+    B_tensor_scale, C, M, N, K, out_dtype) -- tensors or pointers as for fp4_gemm."""
+    arr = (GemmDesc * max(1, len(descs)))(*[GemmDesc(*[_ptr(v) for v in d[:7]], *d[7:11])
+                                            for d in descs])
+    return lib().fp4_gemm_group(arr, len(descs), fmt, _stream(stream))
 
 
 def _opts(opts):
@@ -328,6 +349,27 @@ def gemm(a: QTensor, b: QTensor, out_dtype: int = OUT_F32, out: torch.Tensor | N
     _check(fp4_gemm(a.codes, a.scales, a.tensor_scale, b.codes, b.scales, b.tensor_scale, out, M,
                     N, K, a.fmt, out_dtype), "fp4_gemm")
     return out
+
+
+def gemm_group(problems, out_dtypes=None):
+    """Several GEMMs of one format in one launch: problems is a sequence of (a, b) QTensor
+    pairs (or (a, b, out) with out a preallocated output); returns the outputs, each equal
+    bit for bit to gemm(a, b, out_dtype)."""
+    assert 1 <= len(problems) <= GEMM_GROUP_MAX
+    fmt = problems[0][0].fmt
+    outs, descs = [], []
+    for i, pr in enumerate(problems):
+        a, b = pr[0], pr[1]
+        assert a.fmt == b.fmt == fmt and a.cols == b.cols
+        od = OUT_F32 if out_dtypes is None else out_dtypes[i]
+        out = pr[2] if len(pr) > 2 else torch.empty(
+            a.rows, b.rows, dtype=torch.float32 if od == OUT_F32 else torch.bfloat16,
+            device=a.codes.device)
+        outs.append(out)
+        descs.append((a.codes, a.scales, a.tensor_scale, b.codes, b.scales, b.tensor_scale,
+                      out, a.rows, b.rows, a.cols, od))
+    _check(fp4_gemm_group(descs, fmt), "fp4_gemm_group")
+    return outs
 
 
 def gemm_quant(a: QTensor, b: QTensor, q_hn: int = 16, with_output: bool = True):

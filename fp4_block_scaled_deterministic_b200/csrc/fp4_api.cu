@@ -403,14 +403,12 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtens
 // CTA-pair kernel: the grid is two CTAs per pair tile, capped at the number of CTA pairs
 // the device can hold at once (queried once per device), so the persistent loop never
 // waits for a pair that is not resident.
-template <int FMT, int OUT, int QHN = -1>
-cudaError_t launch_gemm_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& sa,
-                             const CUtensorMap& sb, const CUtensorMap& c, const GemmArgs& g,
-                             int dev, cudaStream_t s) {
+template <int FMT, int QHN = -1>
+cudaError_t launch_gemm_pair(const GemmGroup& grp, int dev, cudaStream_t s) {
   static std::atomic<uint64_t> done{0};
   static int max_pairs[kMaxDevices];
   static std::once_flag once[kMaxDevices];
-  auto k = gemm_fp4_pair_kernel<FMT, OUT, QHN>;
+  auto k = gemm_fp4_pair_kernel<FMT, QHN>;
   cudaError_t e = ensure_smem(k, PairCfg<FMT>::kSmemBytes, dev, done);
   if (e != cudaSuccess) return e;
   std::call_once(once[dev], [&] {
@@ -432,8 +430,8 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a, const CUtensorMap& b, const C
     }
     max_pairs[dev] = n;
   });
-  const int pairs = g.num_tiles < max_pairs[dev] ? g.num_tiles : max_pairs[dev];
-  k<<<2 * pairs, PairCfg<FMT>::kThreads, PairCfg<FMT>::kSmemBytes, s>>>(a, b, sa, sb, c, g);
+  const int pairs = grp.num_tiles < max_pairs[dev] ? grp.num_tiles : max_pairs[dev];
+  k<<<2 * pairs, PairCfg<FMT>::kThreads, PairCfg<FMT>::kSmemBytes, s>>>(grp);
   return cudaGetLastError();
 }
 
@@ -459,27 +457,13 @@ void choose_tile_order(GemmArgs& g, int64_t tile_rows, int64_t row_bytes_i) {
   g.band = g.band_n ? gb : ga;
 }
 
-// With q_hn >= 0 (fp4_gemm_quant) the output is bf16 and the epilogue also writes its
-// row-wise MXFP4 quantisation (rotation q_hn along N) to q_codes / q_scales; C may then
-// be null.
-// (This epilogue stores from registers; its instance ignores the output tensor map.)
-template <int FMT>
-cudaError_t launch_gemm_pair_quant(const CUtensorMap& a, const CUtensorMap& b,
-                                   const CUtensorMap& sa, const CUtensorMap& sb,
-                                   const GemmArgs& g, int q_hn, int dev, cudaStream_t s) {
-  CUtensorMap unused;
-  std::memset(&unused, 0, sizeof(unused));
-  switch (q_hn) {
-    case 0: return launch_gemm_pair<FMT, 1, 0>(a, b, sa, sb, unused, g, dev, s);
-    case 16: return launch_gemm_pair<FMT, 1, 16>(a, b, sa, sb, unused, g, dev, s);
-    default: return launch_gemm_pair<FMT, 1, 32>(a, b, sa, sb, unused, g, dev, s);
-  }
-}
-
-fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void* B,
-                     const void* Bs, const float* Bts, void* C, int64_t M, int64_t N, int64_t K,
-                     fp4_format fmt, fp4_out_dtype od, cudaStream_t stream,
-                     void* q_codes = nullptr, void* q_scales = nullptr, int q_hn = -1) {
+// Host checks of one GEMM (fp4_gemm, fp4_gemm_quant, a member of fp4_gemm_group); a
+// problem with M or N zero passes them and is then skipped (*empty).
+fp4_status check_gemm(const void* A, const void* As, const float* Ats, const void* B,
+                      const void* Bs, const float* Bts, const void* C, int64_t M, int64_t N,
+                      int64_t K, fp4_format fmt, fp4_out_dtype od, const void* q_codes,
+                      const void* q_scales, int q_hn, bool* empty) {
+  *empty = false;
   if (!valid_format(fmt)) return FP4_ERR_INVALID_ARG;
   if (od != FP4_OUT_F32 && od != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
   const bool quant = q_hn >= 0;
@@ -491,7 +475,10 @@ fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void
     return FP4_ERR_SHAPE;
   if (fmt != FP4_NVFP4 && (Ats || Bts)) return FP4_ERR_INVALID_ARG;
   if (fmt == FP4_NVFP4 && (!Ats || !Bts)) return FP4_ERR_INVALID_ARG;
-  if (M == 0 || N == 0) return FP4_OK;
+  if (M == 0 || N == 0) {
+    *empty = true;
+    return FP4_OK;
+  }
   if (!C && !quant) return FP4_ERR_INVALID_ARG;
   if (quant && (!q_codes || !q_scales)) return FP4_ERR_INVALID_ARG;
   if (K == 0) return FP4_ERR_SHAPE;  // an empty contraction is not a launch the tiles express
@@ -499,18 +486,18 @@ fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void
   if (!aligned16(A) || !aligned16(As) || !aligned16(B) || !aligned16(Bs) || (C && !aligned16(C)))
     return FP4_ERR_ALIGN;
   if (quant && (!aligned16(q_codes) || !aligned16(q_scales))) return FP4_ERR_ALIGN;
-  int dev;
-  const DeviceInfo* info;
-  fp4_status st = current_device(&dev, &info);
-  if (st != FP4_OK) return st;
+  return FP4_OK;
+}
 
+// Operand maps and arguments of one GEMM for either kernel: the pair kernel (256-row
+// tiles) or the one-CTA kernel (M <= 128, 128-row tiles). The output map (fp32 TMA-store
+// epilogue of the pair kernel) is made by the caller.
+fp4_status build_gemm(GemmProblem* P, bool pair, const void* A, const void* As,
+                      const float* Ats, const void* B, const void* Bs, const float* Bts,
+                      void* C, int64_t M, int64_t N, int64_t K, fp4_format fmt,
+                      fp4_out_dtype od, void* q_codes, void* q_scales) {
   const int bs = block_of(fmt);
   const int64_t kb4 = ceil_div(K / bs, 4);
-  // Rows of 256 (M > 128) go to the CTA-pair kernel; a single 128-row band of M to the
-  // one-CTA kernel. Each kernel has its own K per pipeline stage.
-  // (The MXFP8 comparator always takes the pair kernel; M <= 128 is then one zero-filled
-  // 256-row band.)
-  const bool pair = M > 128 || fmt == FP4_MXFP8 || quant;
   const int slab_k = !pair ? kGBK
                      : fmt == FP4_MXFP4 ? PairCfg<kFmtMX>::kSlabK
                      : fmt == FP4_NVFP4 ? PairCfg<kFmtNV>::kSlabK
@@ -518,18 +505,17 @@ fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void
   const int atoms = slab_k / (4 * bs);
   const uint32_t b_box_rows = pair ? 128 : kGBN;
   const int64_t kbytes = code_bytes(K, fmt);
-  CUtensorMap ta, tb, tsa, tsb;
-  if (!make_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, kbytes, M, 128, kGBM,
+  if (!make_map_2d(&P->a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, kbytes, M, 128, kGBM,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, kbytes, N, 128, b_box_rows,
+      !make_map_2d(&P->b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, kbytes, N, 128, b_box_rows,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tsa, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, As, kb4 * 64, ceil_div(M, 128),
+      !make_map_2d(&P->sa, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, As, kb4 * 64, ceil_div(M, 128),
                    atoms * 64, 1, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map_2d(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, Bs, kb4 * 64, ceil_div(N, 128),
+      !make_map_2d(&P->sb, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, Bs, kb4 * 64, ceil_div(N, 128),
                    atoms * 64, 2, CU_TENSOR_MAP_SWIZZLE_NONE))
     return FP4_ERR_CUDA;
-
-  GemmArgs g;
+  std::memset(&P->c, 0, sizeof(P->c));
+  GemmArgs& g = P->g;
   g.M = static_cast<int>(M);
   g.N = static_cast<int>(N);
   g.K = static_cast<int>(K);
@@ -549,38 +535,119 @@ fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void
   g.q_scales = static_cast<uint8_t*>(q_scales);
   g.q_kb4 = static_cast<int>(ceil_div(N / 32, 4));
   g.m_pad = static_cast<int>(ceil_div(M, 128) * 128);
-  const int grid = g.num_tiles < info->sm_count ? g.num_tiles : info->sm_count;
+  P->tile0 = 0;
+  P->out_bf16 = od == FP4_OUT_BF16 ? 1 : 0;
+  if (pair && !P->out_bf16 &&
+      !make_map_2d(&P->c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, C, N, M, 8, 32,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+    return FP4_ERR_CUDA;
+  return FP4_OK;
+}
 
+cudaError_t launch_group(const GemmGroup& grp, fp4_format fmt, int q_hn, int dev,
+                         cudaStream_t stream) {
+  if (q_hn >= 0) {
+    switch (q_hn) {
+      case 0:
+        return fmt == FP4_MXFP4 ? launch_gemm_pair<kFmtMX, 0>(grp, dev, stream)
+                                : launch_gemm_pair<kFmtNV, 0>(grp, dev, stream);
+      case 16:
+        return fmt == FP4_MXFP4 ? launch_gemm_pair<kFmtMX, 16>(grp, dev, stream)
+                                : launch_gemm_pair<kFmtNV, 16>(grp, dev, stream);
+      default:
+        return fmt == FP4_MXFP4 ? launch_gemm_pair<kFmtMX, 32>(grp, dev, stream)
+                                : launch_gemm_pair<kFmtNV, 32>(grp, dev, stream);
+    }
+  }
+  if (fmt == FP4_MXFP4) return launch_gemm_pair<kFmtMX>(grp, dev, stream);
+  if (fmt == FP4_MXFP8) return launch_gemm_pair<kFmtMX8>(grp, dev, stream);
+  return launch_gemm_pair<kFmtNV>(grp, dev, stream);
+}
+
+// thread_local: the group is ~2.4 KB and copied into the launch's parameters.
+thread_local GemmGroup t_group;
+
+fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void* B,
+                     const void* Bs, const float* Bts, void* C, int64_t M, int64_t N, int64_t K,
+                     fp4_format fmt, fp4_out_dtype od, cudaStream_t stream,
+                     void* q_codes = nullptr, void* q_scales = nullptr, int q_hn = -1) {
+  bool empty;
+  fp4_status st = check_gemm(A, As, Ats, B, Bs, Bts, C, M, N, K, fmt, od, q_codes, q_scales,
+                             q_hn, &empty);
+  if (st != FP4_OK || empty) return st;
+  int dev;
+  const DeviceInfo* info;
+  st = current_device(&dev, &info);
+  if (st != FP4_OK) return st;
+  // Rows of 256 (M > 128) go to the CTA-pair kernel; a single 128-row band of M to the
+  // one-CTA kernel. Each kernel has its own K per pipeline stage.
+  // (The MXFP8 comparator always takes the pair kernel; M <= 128 is then one zero-filled
+  // 256-row band.)
+  const bool quant = q_hn >= 0;
+  const bool pair = M > 128 || fmt == FP4_MXFP8 || quant;
+  GemmGroup& grp = t_group;
+  st = build_gemm(&grp.p[0], pair, A, As, Ats, B, Bs, Bts, C, M, N, K, fmt, od, q_codes,
+                  q_scales);
+  if (st != FP4_OK) return st;
   cudaError_t e;
-  if (quant) {
-    e = fmt == FP4_MXFP4
-            ? launch_gemm_pair_quant<kFmtMX>(ta, tb, tsa, tsb, g, q_hn, dev, stream)
-            : launch_gemm_pair_quant<kFmtNV>(ta, tb, tsa, tsb, g, q_hn, dev, stream);
-  } else if (pair) {
-    // The output as a tensor for the epilogue's TMA stores (fp32 outputs): boxes of 32
-    // rows x 32 bytes.
-    CUtensorMap tc;
-    const bool f32 = od == FP4_OUT_F32;
-    if (!make_map_2d(&tc, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                     f32 ? 4 : 2, C, N, M, f32 ? 8 : 16, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
-      return FP4_ERR_CUDA;
-    if (fmt == FP4_MXFP4)
-      e = f32 ? launch_gemm_pair<kFmtMX, 0>(ta, tb, tsa, tsb, tc, g, dev, stream)
-              : launch_gemm_pair<kFmtMX, 1>(ta, tb, tsa, tsb, tc, g, dev, stream);
-    else if (fmt == FP4_MXFP8)
-      e = f32 ? launch_gemm_pair<kFmtMX8, 0>(ta, tb, tsa, tsb, tc, g, dev, stream)
-              : launch_gemm_pair<kFmtMX8, 1>(ta, tb, tsa, tsb, tc, g, dev, stream);
-    else
-      e = f32 ? launch_gemm_pair<kFmtNV, 0>(ta, tb, tsa, tsb, tc, g, dev, stream)
-              : launch_gemm_pair<kFmtNV, 1>(ta, tb, tsa, tsb, tc, g, dev, stream);
-  } else if (fmt == FP4_MXFP4) {
-    e = od == FP4_OUT_F32 ? launch_gemm<kFmtMX, 0>(ta, tb, tsa, tsb, g, grid, dev, stream)
-                          : launch_gemm<kFmtMX, 1>(ta, tb, tsa, tsb, g, grid, dev, stream);
+  if (pair) {
+    grp.n = 1;
+    grp.num_tiles = grp.p[0].g.num_tiles;
+    e = launch_group(grp, fmt, q_hn, dev, stream);
   } else {
-    e = od == FP4_OUT_F32 ? launch_gemm<kFmtNV, 0>(ta, tb, tsa, tsb, g, grid, dev, stream)
-                          : launch_gemm<kFmtNV, 1>(ta, tb, tsa, tsb, g, grid, dev, stream);
+    const GemmProblem& P = grp.p[0];
+    const int grid = P.g.num_tiles < info->sm_count ? P.g.num_tiles : info->sm_count;
+    if (fmt == FP4_MXFP4)
+      e = od == FP4_OUT_F32 ? launch_gemm<kFmtMX, 0>(P.a, P.b, P.sa, P.sb, P.g, grid, dev, stream)
+                            : launch_gemm<kFmtMX, 1>(P.a, P.b, P.sa, P.sb, P.g, grid, dev, stream);
+    else
+      e = od == FP4_OUT_F32 ? launch_gemm<kFmtNV, 0>(P.a, P.b, P.sa, P.sb, P.g, grid, dev, stream)
+                            : launch_gemm<kFmtNV, 1>(P.a, P.b, P.sa, P.sb, P.g, grid, dev, stream);
   }
   return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+}
+
+// Up to kGMaxProblems GEMMs of one format in one launch of the pair kernel. Problems
+// with M or N zero are skipped; the rest run in order of decreasing K, so that the tiles
+// left for the last wave are the cheapest ones.
+fp4_status gemm_group_impl(const fp4_gemm_desc* d, int n, fp4_format fmt, cudaStream_t stream) {
+  if (n < 1 || n > FP4_GEMM_GROUP_MAX || !d) return FP4_ERR_INVALID_ARG;
+  int order[kGMaxProblems], used = 0;
+  for (int i = 0; i < n; ++i) {
+    bool empty;
+    const fp4_status st = check_gemm(d[i].A_codes, d[i].A_scales, d[i].A_tensor_scale,
+                                     d[i].B_codes, d[i].B_scales, d[i].B_tensor_scale, d[i].C,
+                                     d[i].M, d[i].N, d[i].K, fmt, d[i].out_dtype, nullptr,
+                                     nullptr, -1, &empty);
+    if (st != FP4_OK) return st;
+    if (!empty) order[used++] = i;
+  }
+  if (used == 0) return FP4_OK;
+  for (int i = 1; i < used; ++i)  // stable insertion sort by decreasing K
+    for (int j = i; j > 0 && d[order[j]].K > d[order[j - 1]].K; --j) {
+      const int t = order[j];
+      order[j] = order[j - 1];
+      order[j - 1] = t;
+    }
+  int dev;
+  const DeviceInfo* info;
+  fp4_status st = current_device(&dev, &info);
+  if (st != FP4_OK) return st;
+  GemmGroup& grp = t_group;
+  int64_t tiles = 0;
+  for (int q = 0; q < used; ++q) {
+    const fp4_gemm_desc& x = d[order[q]];
+    st = build_gemm(&grp.p[q], true, x.A_codes, x.A_scales, x.A_tensor_scale, x.B_codes,
+                    x.B_scales, x.B_tensor_scale, x.C, x.M, x.N, x.K, fmt, x.out_dtype, nullptr,
+                    nullptr);
+    if (st != FP4_OK) return st;
+    grp.p[q].tile0 = static_cast<int>(tiles);
+    tiles += grp.p[q].g.num_tiles;
+    if (tiles > INT32_MAX) return FP4_ERR_SHAPE;
+  }
+  grp.n = used;
+  grp.num_tiles = static_cast<int>(tiles);
+  return launch_group(grp, fmt, -1, dev, stream) == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------- linear-layer passes
@@ -834,6 +901,12 @@ fp4_status fp4_gemm(const void* A, const void* As, const float* Ats, const void*
   NvtxRange nvtx_range("fp4_gemm");
   return gemm_impl(A, As, Ats, B, Bs, Bts, C, M, N, K, fmt, od,
                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+fp4_status fp4_gemm_group(const fp4_gemm_desc* descs, int n, fp4_format fmt,
+                          fp4_stream_t stream) {
+  NvtxRange nvtx_range("fp4_gemm_group");
+  return gemm_group_impl(descs, n, fmt, reinterpret_cast<cudaStream_t>(stream));
 }
 
 fp4_status fp4_gemm_quant(const void* A, const void* As, const float* Ats, const void* B,

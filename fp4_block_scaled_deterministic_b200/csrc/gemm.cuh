@@ -99,6 +99,49 @@ __device__ __forceinline__ void tile_coords(int tile, const GemmArgs& g, int& tm
   }
 }
 
+// A group of GEMMs run by one launch of the pair kernel (fp4_gemm_group): their tiles
+// form one sequence, problem 0's first, that the persistent CTA pairs walk, so the last
+// wave of one GEMM is filled with tiles of the next. Each problem keeps its own tensor
+// maps, tile order, K and output type. A single GEMM is a group of one.
+constexpr int kGMaxProblems = 3;
+struct alignas(64) GemmProblem {
+  CUtensorMap a, b, sa, sb;  // operand codes and scales
+  CUtensorMap c;             // the output, for the fp32 epilogue's TMA stores
+  GemmArgs g;
+  int tile0;                 // index of the problem's first tile in the group
+  int out_bf16;              // epilogue output: bf16 (1) or fp32 (0)
+};
+struct GemmGroup {
+  GemmProblem p[kGMaxProblems];
+  int n;          // problems in use
+  int num_tiles;  // tiles of all problems
+};
+
+// Problem of a tile of the group (problems are few: a linear scan).
+__device__ __forceinline__ int group_problem(const GemmGroup& grp, int tile) {
+  int q = 0;
+#pragma unroll
+  for (int i = 1; i < kGMaxProblems; ++i)
+    if (i < grp.n && tile >= grp.p[i].tile0) q = i;
+  return q;
+}
+
+// Tile schedules the issue threads walk: how many tiles, and how many K slabs a tile has.
+struct ArgsSched {  // one GEMM (the one-CTA kernel)
+  const GemmArgs& g;
+  __device__ __forceinline__ int num_tiles() const { return g.num_tiles; }
+  __device__ __forceinline__ int k_tiles(int) const { return g.k_tiles; }
+  __device__ __forceinline__ uint64_t wait_ns() const { return g.wait_limit_ns; }
+};
+struct GroupSched {  // a group (the pair kernel)
+  const GemmGroup& grp;
+  __device__ __forceinline__ int num_tiles() const { return grp.num_tiles; }
+  __device__ __forceinline__ int k_tiles(int tile) const {
+    return grp.p[group_problem(grp, tile)].g.k_tiles;
+  }
+  __device__ __forceinline__ uint64_t wait_ns() const { return grp.p[0].g.wait_limit_ns; }
+};
+
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of 128 bytes,
 // 8-row groups 1024 bytes apart (SBO), sm_100 descriptor version 1.
 __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
@@ -263,18 +306,20 @@ struct Issuer {
   // later, whose load waited for the MMAs of the slab STAGES back; SF_BUFS >= STAGES makes
   // those the slot's previous readers (or later ones), so no slot is overwritten early.
   static_assert(SF_BUFS >= STAGES, "scale ring must cover the stage ring");
-  template <int LO, int HI>
+  template <int LO, int HI, class Sched>
   __device__ static void run_copies(uint32_t tmem, uint8_t* sA, uint8_t* sB, uint8_t* sSFA,
                                     uint8_t* sSFB, uint64_t* full, uint64_t* sf_full,
                                     uint64_t* drained, volatile int* abort_flag, int first,
-                                    int stride, const GemmArgs& g) {
+                                    int stride, const Sched& sc) {
     const SlabCursor base = make_base(tmem, sA, sB, sSFA, sSFB);
     SlabCursor cur = base;
-    const int my_tiles = first < g.num_tiles ? (g.num_tiles - first + stride - 1) / stride : 0;
+    const int nt = sc.num_tiles();
+    const int my_tiles = first < nt ? (nt - first + stride - 1) / stride : 0;
     for (int t = 0; t < my_tiles && !*abort_flag; ++t) {
       bool ok = true;
-      for (int kt = 0; kt < g.k_tiles; ++kt) {
-        if (!mbar_wait(&full[cur.stage], cur.phase, g.wait_limit_ns)) {
+      const int kts = sc.k_tiles(first + t * stride);
+      for (int kt = 0; kt < kts; ++kt) {
+        if (!mbar_wait(&full[cur.stage], cur.phase, sc.wait_ns())) {
           ok = false;
           break;
         }
@@ -289,25 +334,28 @@ struct Issuer {
     }
     // Every copy this thread issued has landed before TMEM can be released.
     commit_local(drained);
-    if (!mbar_wait(drained, 0u, g.wait_limit_ns)) *abort_flag = 1;
+    if (!mbar_wait(drained, 0u, sc.wait_ns())) *abort_flag = 1;
   }
+  template <class Sched>
   __device__ static void run_split(uint32_t tmem, uint8_t* sA, uint8_t* sB, uint8_t* sSFA,
                                    uint8_t* sSFB, uint64_t* sf_full, uint64_t* empty,
                                    uint64_t* acc_full, uint64_t* acc_empty,
                                    volatile int* abort_flag, int first, int stride,
-                                   const GemmArgs& g) {
+                                   const Sched& sc) {
     const SlabCursor base = make_base(tmem, sA, sB, sSFA, sSFB);
     SlabCursor cur = base;
-    const int my_tiles = first < g.num_tiles ? (g.num_tiles - first + stride - 1) / stride : 0;
+    const int nt = sc.num_tiles();
+    const int my_tiles = first < nt ? (nt - first + stride - 1) / stride : 0;
     uint32_t acc_phase = 0;
     for (int t = 0; t < my_tiles; ++t) {
-      if (!mbar_wait(acc_empty, acc_phase ^ 1u, g.wait_limit_ns) || *abort_flag) {
+      if (!mbar_wait(acc_empty, acc_phase ^ 1u, sc.wait_ns()) || *abort_flag) {
         *abort_flag = 1;
         return;
       }
       tc_fence_after();
-      for (int kt = 0; kt < g.k_tiles; ++kt) {
-        if (!mbar_wait(&sf_full[cur.slot], cur.sf_phase, g.wait_limit_ns)) {
+      const int kts = sc.k_tiles(first + t * stride);
+      for (int kt = 0; kt < kts; ++kt) {
+        if (!mbar_wait(&sf_full[cur.slot], cur.sf_phase, sc.wait_ns())) {
           *abort_flag = 1;
           return;
         }
@@ -322,25 +370,28 @@ struct Issuer {
   }
 
   // Runs all tiles of this CTA (or CTA pair): tiles first, first+stride, ... < num_tiles.
+  template <class Sched>
   __device__ static void run(uint32_t tmem, uint8_t* sA, uint8_t* sB, uint8_t* sSFA,
                              uint8_t* sSFB, uint64_t* full, uint64_t* empty, uint64_t* acc_full,
                              uint64_t* acc_empty, volatile int* abort_flag, int first,
-                             int stride, const GemmArgs& g) {
+                             int stride, const Sched& sc) {
     SlabCursor base = make_base(tmem, sA, sB, sSFA, sSFB);
     SlabCursor cur = base;
-    const int my_tiles = first < g.num_tiles ? (g.num_tiles - first + stride - 1) / stride : 0;
+    const int nt = sc.num_tiles();
+    const int my_tiles = first < nt ? (nt - first + stride - 1) / stride : 0;
     uint32_t acc_phase = 0;
     for (int t = 0; t < my_tiles; ++t) {
-      if (!mbar_wait(acc_empty, acc_phase ^ 1u, g.wait_limit_ns) || *abort_flag) {
+      if (!mbar_wait(acc_empty, acc_phase ^ 1u, sc.wait_ns()) || *abort_flag) {
         *abort_flag = 1;
         return;
       }
       tc_fence_after();
-      for (int kt = 0; kt < g.k_tiles; ++kt) {
+      const int kts = sc.k_tiles(first + t * stride);
+      for (int kt = 0; kt < kts; ++kt) {
         // Each slab: wait for its stage, copy its scales into its TMEM ring slot, issue its
         // MMAs back to back, then release the stage. (Spreading the next slab's copies
         // between this slab's MMAs was measured to be slower.)
-        if (!mbar_wait(&full[cur.stage], cur.phase, g.wait_limit_ns)) {
+        if (!mbar_wait(&full[cur.stage], cur.phase, sc.wait_ns())) {
           *abort_flag = 1;
           return;
         }
@@ -642,7 +693,7 @@ __global__ void __launch_bounds__(kGSingleThreads, 1)
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
       SingleIssuer::run_split(tmem, sA, sB, sSFA, sSFB, sf_full, empty, acc_full, acc_empty,
-                              abort_flag, blockIdx.x, gridDim.x, g);
+                              abort_flag, blockIdx.x, gridDim.x, ArgsSched{g});
     }
   } else if (warp >= kGThreads / 32) {
     if (lane == 0) {
@@ -651,11 +702,11 @@ __global__ void __launch_bounds__(kGSingleThreads, 1)
       if (warp == kGThreads / 32)
         SingleIssuer::template run_copies<0, kC / kN>(tmem, sA, sB, sSFA, sSFB, full, sf_full,
                                                       cp_drained, abort_flag, blockIdx.x,
-                                                      gridDim.x, g);
+                                                      gridDim.x, ArgsSched{g});
       else
         SingleIssuer::template run_copies<kC / kN, kC>(tmem, sA, sB, sSFA, sSFB, full, sf_full,
                                                        cp_drained, abort_flag, blockIdx.x,
-                                                       gridDim.x, g);
+                                                       gridDim.x, ArgsSched{g});
     }
   } else {
     // -------------------------------------------------------------- epilogue
@@ -746,15 +797,13 @@ struct PairCfg {
 };
 
 
+// The kernel runs a group of GEMMs (one problem for fp4_gemm); each tile's problem gives
+// its operand maps, coordinates, K, output type and (NVFP4) tensor scales.
 // QHN >= 0: the epilogue also quantises the output (store_row_segment_quant, rotation
-// QHN along N); OUT_BF16 is then 1.
-template <int FMT, int OUT_BF16, int QHN = -1>
+// QHN along N); the group then holds one problem with a bf16 output.
+template <int FMT, int QHN = -1>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<FMT>::kThreads, 1)
-    gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA,
-                         const __grid_constant__ CUtensorMap tmB,
-                         const __grid_constant__ CUtensorMap tmSFA,
-                         const __grid_constant__ CUtensorMap tmSFB,
-                         const __grid_constant__ CUtensorMap tmC, const GemmArgs g) {
+    gemm_fp4_pair_kernel(const __grid_constant__ GemmGroup grp) {
   using Cfg = PairCfg<FMT>;
   constexpr int S = Cfg::kStages;
   using PairIssuer = Issuer<FMT, true, Cfg::kSlabK, S, Cfg::kABytes, Cfg::kBBytes,
@@ -777,17 +826,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<FMT>::kThrea
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   static_assert((2 * S + 3 + Cfg::kSFBufs) * 8 + 8 <= 256, "barrier area");
   uint8_t* s_stage_out = reinterpret_cast<uint8_t*>(bars) + 256;  // [8 warps][1 KB]
+  const GroupSched sched{grp};
+  const uint64_t wait_ns = grp.p[0].g.wait_limit_ns;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-    tma_prefetch_desc(&tmSFA);
-    tma_prefetch_desc(&tmSFB);
-    if constexpr (QHN < 0) tma_prefetch_desc(&tmC);
+    for (int q = 0; q < grp.n; ++q) {
+      tma_prefetch_desc(&grp.p[q].a);
+      tma_prefetch_desc(&grp.p[q].b);
+      tma_prefetch_desc(&grp.p[q].sa);
+      tma_prefetch_desc(&grp.p[q].sb);
+      if (QHN < 0 && !grp.p[q].out_bf16) tma_prefetch_desc(&grp.p[q].c);
+    }
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -817,11 +870,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<FMT>::kThrea
       // ------------------------------------------------------------ TMA producer (both CTAs)
       int stage = 0;
       uint32_t phase = 0;
-      for (int tile = pair; tile < g.num_tiles && !*abort_flag; tile += npairs) {
+      for (int tile = pair; tile < grp.num_tiles && !*abort_flag; tile += npairs) {
+        const GemmProblem& P = grp.p[group_problem(grp, tile)];
         int tm, tn;
-        tile_coords(tile, g, tm, tn);
-        for (int kt = 0; kt < g.k_tiles; ++kt) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, g.wait_limit_ns)) {
+        tile_coords(tile - P.tile0, P.g, tm, tn);
+        for (int kt = 0; kt < P.g.k_tiles; ++kt) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, wait_ns)) {
             *abort_flag = 1;
             break;
           }
@@ -830,14 +884,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<FMT>::kThrea
 #pragma unroll
           for (int sub = 0; sub < Cfg::kSub; ++sub) {
             const int kx = kt * Cfg::kRowBytes + 128 * sub;
-            tma_load_2d_pair(sA + stage * Cfg::kABytes + sub * 16384, &tmA, bar, kx,
+            tma_load_2d_pair(sA + stage * Cfg::kABytes + sub * 16384, &P.a, bar, kx,
                              tm * 256 + 128 * static_cast<int>(rank));
-            tma_load_2d_pair(sB + stage * Cfg::kBBytes + sub * 16384, &tmB, bar, kx,
+            tma_load_2d_pair(sB + stage * Cfg::kBBytes + sub * 16384, &P.b, bar, kx,
                              tn * 256 + 128 * static_cast<int>(rank));
           }
-          tma_load_2d_pair(sSFA + stage * Cfg::kSFABytes, &tmSFA, bar, kt * Cfg::kAtoms * 64,
+          tma_load_2d_pair(sSFA + stage * Cfg::kSFABytes, &P.sa, bar, kt * Cfg::kAtoms * 64,
                            2 * tm + static_cast<int>(rank));
-          tma_load_2d_pair(sSFB + stage * Cfg::kSFBBytes, &tmSFB, bar, kt * Cfg::kAtoms * 64,
+          tma_load_2d_pair(sSFB + stage * Cfg::kSFBBytes, &P.sb, bar, kt * Cfg::kAtoms * 64,
                            2 * tn);
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
@@ -848,10 +902,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<FMT>::kThrea
       // ------------------------------------------------------------ MMA issuer (leader)
       if constexpr (Cfg::kCopyThreads > 0)
         PairIssuer::run_split(tmem, sA, sB, sSFA, sSFB, sf_full, empty, acc_full, acc_empty,
-                              abort_flag, pair, npairs, g);
+                              abort_flag, pair, npairs, sched);
       else
         PairIssuer::run(tmem, sA, sB, sSFA, sSFB, full, empty, acc_full, acc_empty,
-                        abort_flag, pair, npairs, g);
+                        abort_flag, pair, npairs, sched);
     }
   } else if (warp >= kGThreads / 32) {
     if (lane == 0 && rank == 0) {
@@ -861,23 +915,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<FMT>::kThrea
       const int ci = warp - kGThreads / 32;
       if (ci == 0)
         PairIssuer::template run_copies<0, kC / kN>(tmem, sA, sB, sSFA, sSFB, full, sf_full,
-                                                    cp_drained, abort_flag, pair, npairs, g);
+                                                    cp_drained, abort_flag, pair, npairs, sched);
       else
         PairIssuer::template run_copies<kC / kN, kC>(tmem, sA, sB, sSFA, sSFB, full, sf_full,
-                                                     cp_drained, abort_flag, pair, npairs, g);
+                                                     cp_drained, abort_flag, pair, npairs,
+                                                     sched);
     }
   } else {
     // -------------------------------------------------------------- epilogue (both CTAs)
     const int ew = warp - 2;
     const int quarter = warp & 3;
     const int half = ew >> 2;
-    float alpha = 1.0f;
-    if constexpr (FMT == kFmtNV) alpha = __fmul_rn(*g.sa, *g.sb);
     uint32_t acc_phase = 0;
-    for (int tile = pair; tile < g.num_tiles && !*abort_flag; tile += npairs) {
+    for (int tile = pair; tile < grp.num_tiles && !*abort_flag; tile += npairs) {
+      const GemmProblem& P = grp.p[group_problem(grp, tile)];
       int tm, tn;
-      tile_coords(tile, g, tm, tn);
-      if (!mbar_wait(acc_full, acc_phase, g.wait_limit_ns)) {
+      tile_coords(tile - P.tile0, P.g, tm, tn);
+      float alpha = 1.0f;
+      if constexpr (FMT == kFmtNV) alpha = __fmul_rn(*P.g.sa, *P.g.sb);
+      if (!mbar_wait(acc_full, acc_phase, wait_ns)) {
         *abort_flag = 1;
         break;
       }
@@ -893,16 +949,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<FMT>::kThrea
       if (lane == 0) mbar_arrive_cluster_cta_release(leader_acc_empty);
       acc_phase ^= 1u;
       const int row0 = tm * 256 + 128 * static_cast<int>(rank) + 32 * quarter;
+      const int n0 = tn * kGBN + 128 * half;
       if constexpr (QHN >= 0)
-        store_row_segment_quant<FMT, QHN>(r, row0 + lane, tn * kGBN + 128 * half, g, alpha);
-      else if constexpr (!OUT_BF16)  // fp32: through TMA stores (store_segment_tma)
-        store_segment_tma<FMT, OUT_BF16>(r, s_stage_out + 1024 * ew, &tmC, row0,
-                                         tn * kGBN + 128 * half, g, alpha, lane);
-      else
-        store_row_segment<FMT, OUT_BF16>(r, row0 + lane, tn * kGBN + 128 * half, g, alpha);
+        store_row_segment_quant<FMT, QHN>(r, row0 + lane, n0, P.g, alpha);
+      else if (P.out_bf16)
+        store_row_segment<FMT, 1>(r, row0 + lane, n0, P.g, alpha);
+      else  // fp32: through TMA stores (store_segment_tma)
+        store_segment_tma<FMT, 0>(r, s_stage_out + 1024 * ew, &P.c, row0, n0, P.g, alpha, lane);
     }
     // every store of this warp has completed before the CTA (and its staging) goes away
-    if constexpr (QHN < 0 && !OUT_BF16) {
+    if constexpr (QHN < 0) {
       if (lane == 0) bulk_wait<0>();
       __syncwarp();
     }

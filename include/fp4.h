@@ -238,6 +238,35 @@ FP4_API fp4_status fp4_gemm(const void *A_codes, const void *A_scales, const flo
                     fp4_out_dtype out_dtype, fp4_stream_t stream);
 
 /*
+ * fp4_gemm_group -- up to FP4_GEMM_GROUP_MAX independent fp4_gemm calls of one format in
+ * one launch: e.g. the Fprop, Dgrad and Wgrad GEMMs of one linear layer [MXFP4
+ * pre-training summary, Methodology item 2: all three passes in FP4]. The persistent
+ * CTA pairs walk the tiles of all problems as one sequence, so the last, partly filled
+ * wave of one GEMM is completed with tiles of the next. Each problem's output is
+ * bit-identical to the same fp4_gemm call.
+ *   descs[n]: host array (read during the call only), 1 <= n <= FP4_GEMM_GROUP_MAX; each
+ *     entry as the arguments of fp4_gemm. Problems with M or N zero are skipped.
+ *   The problems must not overlap one another's outputs; they run in order of
+ *   decreasing K, concurrently.
+ *   Errors: FP4_ERR_INVALID_ARG for n out of range or a NULL descs; otherwise the first
+ *   error of any entry as fp4_gemm reports it, and nothing is launched.
+ */
+#define FP4_GEMM_GROUP_MAX 3
+typedef struct fp4_gemm_desc {
+  const void *A_codes;
+  const void *A_scales;
+  const float *A_tensor_scale;
+  const void *B_codes;
+  const void *B_scales;
+  const float *B_tensor_scale;
+  void *C;
+  int64_t M, N, K;
+  fp4_out_dtype out_dtype;
+} fp4_gemm_desc;
+FP4_API fp4_status fp4_gemm_group(const fp4_gemm_desc *descs, int n, fp4_format fmt,
+                                  fp4_stream_t stream);
+
+/*
  * fp4_gemm_quant -- fp4_gemm with a bf16 output whose epilogue also quantises it for
  * the next layer: Q = the row-wise MXFP4 quantisation, with rotation q_hadamard_n
  * (0, 16, 32) along N, of Y = RN_bf16(C) -- bit-identical to

@@ -129,6 +129,21 @@ def test_gemm_quant_validation():
     assert gq(M=0) == OK
 
 
+def test_gemm_group_validation():
+    L = fp4.lib()
+    def d(M=128, N=128, K=128, C=A16, od=0, Ats=None):
+        return fp4.GemmDesc(A16, A16, Ats, A16, A16, None, C, M, N, K, od)
+    arr = lambda *ds: (fp4.GemmDesc * len(ds))(*ds)
+    assert L.fp4_gemm_group(None, 1, 0, None) == INVALID
+    assert L.fp4_gemm_group(arr(d()), 0, 0, None) == INVALID
+    assert L.fp4_gemm_group(arr(d(), d(), d(), d()), 4, 0, None) == INVALID  # above the maximum
+    assert L.fp4_gemm_group(arr(d(), d(N=100)), 2, 0, None) == SHAPE
+    assert L.fp4_gemm_group(arr(d(C=MIS), d()), 2, 0, None) == ALIGN
+    assert L.fp4_gemm_group(arr(d(od=3)), 1, 0, None) == INVALID
+    assert L.fp4_gemm_group(arr(d(Ats=A16)), 1, 0, None) == INVALID  # MXFP4 takes no scale
+    assert L.fp4_gemm_group(arr(d(M=0), d(N=0)), 2, 0, None) == OK   # nothing to launch
+
+
 def test_quantize_batch_validation():
     L = fp4.lib()
     item = fp4.QuantItem(A16, A16, A16, A16, A16, None, 64, 64)
