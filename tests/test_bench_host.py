@@ -55,9 +55,9 @@ def test_layer_tables():
 def test_traffic_record_is_tied_to_the_gemm_sources():
     rec = json.load(open(os.path.join(ROOT, "profiles", "gemm_llama_traffic.json")))
     assert bench.kernel_source_hash() == bench.kernel_source_hash()
-    got = bench.recorded_traffic("mxfp4")
+    got = bench.recorded_traffic("mxfp4_group")  # one grouped launch per projection
     if rec["source_sha1"] == bench.kernel_source_hash():
-        assert got == rec["per_launch_bytes"]["mxfp4"] and got > 0
+        assert got == rec["per_launch_bytes"]["mxfp4_group"] and got > 0
     else:
         assert got is None  # the kernel changed since the counters were taken
     assert bench.recorded_traffic("no-such-kernel") is None
