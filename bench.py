@@ -842,7 +842,10 @@ def main():
                       + ("; a projection's Fprop, Dgrad and Wgrad per launch)"
                          if layer.gemm_launches() == 1 else ")"),
             "per_launch": {"avg_flops": avg_flops, "avg_ms": avg_launch_ms,
+                           "median_ms": statistics.median(gemm_ms),
                            "launches": len(gemm_ms)},
+            "achieved_at_median_launch": (
+                statistics.median([f / (t * 1e-3) / 1e12 for f, t in zip(per_launch_flops, gemm_ms)])),
             "timing": ("CUDA events around each launch over the timed steps" if not a.side_stream
                        else "CUDA events around each launch over the same number of steps run "
                             "on one stream just before the overlapped timed region"),
@@ -854,7 +857,8 @@ def main():
              "kernel": ("quantize_kernel dual layout, "
                         + ("X, W, dY of a projection per launch" if layer.quant_batch
                            else "one tensor per launch")), "launches": len(quant_ms),
-             "avg_ms": sum(quant_ms) / len(quant_ms), "peak_source": f"{pk_kind}: hbm_gbs"}
+             "avg_ms": sum(quant_ms) / len(quant_ms), "median_ms": statistics.median(quant_ms),
+             "peak_source": f"{pk_kind}: hbm_gbs"}
 
     out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
            "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms / a.steps,

@@ -355,19 +355,19 @@ __device__ __forceinline__ Enc mx_encode_x2_h16fold(float2 (&p)[32], const Codes
   return mx_encode_x2(p, codes);
 }
 
-// True when q lies within 4 units in the last place of a number with at most two
-// fraction bits; every E2M1 rounding threshold (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5) is
-// such a number.
-__device__ __forceinline__ bool near_e2m1_threshold(float q) {
-  return ((__float_as_uint(q) + 4u) & 0x1FFFFFu) < 9u;
-}
-
 // NVFP4 block of 16 per lane under tensor scale S (six_s = 6*S, rounded once):
 // byte = UE4M3_RNE_satfinite(bmax / six_s), d = ue4m3(byte) * S, codes of the fp32
-// quotient v / d; a zero byte gives signed zeros.
-// The quotient is formed as v * y with y = RN(1/d): then |v*y - v/d| < 2 ulps, so v*y and
-// RN(v/d) fall on the same side of every E2M1 threshold unless v*y is within 4 ulps of
-// one; those (rare) blocks, and blocks whose 1/d overflows, are divided exactly.
+// quotient RN(v / d); a zero byte gives signed zeros.
+// The quotient comes from y = RN(1/d) by two FMA correction steps: q0 = RN(v*y), which
+// can be just over one ulp from v/d; q1 = RN(q0 + RN(v - q0*d)*y), which is faithful;
+// then, with the residual r = v - q1*d exact as one FMA, q = RN(q1 + r*y) is the
+// correctly rounded quotient RN(v/d) (the last step is Markstein's, "Computation of
+// elementary functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
+// 1990; Muller et al., Handbook of Floating-Point Arithmetic, the FMA-based division
+// section). That needs d and the reciprocal away from underflow and overflow: with
+// 2^-100 <= d <= 2^100 a residual can underflow only when |v/d| < 2^-3, whose code is a
+// signed zero either way, and the sign is taken from v (so -0 / d stays -0). Blocks
+// with a zero scale, a d outside that range or a non-finite element are divided exactly.
 template <int b, bool kExact = false, int L = 32>
 __device__ __forceinline__ void nv_block_x2(float2 (&p)[L], float S, float six_s,
                                             uint32_t& sbx, uint32_t& sby) {
@@ -375,32 +375,31 @@ __device__ __forceinline__ void nv_block_x2(float2 (&p)[L], float S, float six_s
   sbx = cvt_e4m3(__fdiv_rn(bm.x, six_s));
   sby = cvt_e4m3(__fdiv_rn(bm.y, six_s));
   const float dx = __fmul_rn(e4m3_to_f32(sbx), S), dy = __fmul_rn(e4m3_to_f32(sby), S);
-  const float yx = __frcp_rn(dx), yy = __frcp_rn(dy);
-  const float2 y2 = make_float2(yx, yy);
-  // Two passes (the quotients are not kept between them, which saves registers): find
-  // whether any reciprocal product lands near a threshold, then overwrite each value
-  // with its quotient, divided exactly when so.
-  bool exact = kExact || !(yx <= 3.0e38f) || !(yy <= 3.0e38f);
+  const bool fast = !kExact && dx >= 0x1p-100f && dy >= 0x1p-100f && dx <= 0x1p100f &&
+                    dy <= 0x1p100f && bm.x <= 3.0e38f && bm.y <= 3.0e38f;
+  if (fast) {
+    const float2 y2 = make_float2(__frcp_rn(dx), __frcp_rn(dy));
+    const float2 nd = make_float2(-dx, -dy);
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float2 q = mul2(p[b + i], y2);
-    exact |= near_e2m1_threshold(q.x) | near_e2m1_threshold(q.y);
+    for (int i = 0; i < 16; ++i) {
+      const float2 v = p[b + i];
+      const float2 q0 = mul2(v, y2);
+      const float2 q1 = __ffma2_rn(__ffma2_rn(q0, nd, v), y2, q0);  // faithful
+      const float2 q = __ffma2_rn(__ffma2_rn(q1, nd, v), y2, q1);   // RN(v/d)
+      p[b + i] = make_float2(copysignf(q.x, v.x), copysignf(q.y, v.y));
+    }
+    return;
   }
   // A zero block scale gives zeros that keep the sign of the element itself (the
   // quotient by d = 0 is an infinity, or a NaN for a zero element).
   const bool zx = sbx == 0u, zy = sby == 0u;
-  auto put = [&](int i, float2 q) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
     const float2 v = p[b + i];
-    p[b + i] = make_float2(zx ? __uint_as_float(__float_as_uint(v.x) & 0x80000000u) : q.x,
-                           zy ? __uint_as_float(__float_as_uint(v.y) & 0x80000000u) : q.y);
-  };
-  if (exact) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-      put(i, make_float2(__fdiv_rn(p[b + i].x, dx), __fdiv_rn(p[b + i].y, dy)));
-  } else {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) put(i, mul2(p[b + i], y2));
+    p[b + i] = make_float2(zx ? __uint_as_float(__float_as_uint(v.x) & 0x80000000u)
+                              : __fdiv_rn(v.x, dx),
+                           zy ? __uint_as_float(__float_as_uint(v.y) & 0x80000000u)
+                              : __fdiv_rn(v.y, dy));
   }
 }
 
@@ -1135,7 +1134,8 @@ __device__ __forceinline__ uint2 codes_col16y(const float2 (&p)[16]) {
 }
 
 // NVFP4 block of 16 values held as 8 pairs q2[B .. B+8) (ROW job): scale byte, and the
-// pairs replaced by their quotients (or signed zeros); the arithmetic of nv_block_x2.
+// pairs replaced by their quotients RN(v/d) (or signed zeros); the arithmetic of
+// nv_block_x2 (the correction step, else exact division).
 template <int B>
 __device__ __forceinline__ uint32_t nv_block_row_v(float2 (&q2)[16], float S, float six_s) {
   float a[16];
@@ -1147,25 +1147,25 @@ __device__ __forceinline__ uint32_t nv_block_row_v(float2 (&q2)[16], float S, fl
   const float bm = tree_max<16>(a);
   const uint32_t sb = cvt_e4m3(__fdiv_rn(bm, six_s));
   const float d = __fmul_rn(e4m3_to_f32(sb), S);
-  const float y = __frcp_rn(d);
-  const float2 y2 = make_float2(y, y);
-  bool exact = !(y <= 3.0e38f);  // two passes, as in nv_block_x2
+  if (d >= 0x1p-100f && d <= 0x1p100f && bm <= 3.0e38f) {  // the correction step
+    const float y = __frcp_rn(d);
+    const float2 y2 = make_float2(y, y), nd = make_float2(-d, -d);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float2 q = mul2(q2[B + i], y2);
-    exact |= near_e2m1_threshold(q.x) | near_e2m1_threshold(q.y);
-  }
-  if (sb == 0u) {  // a zero block scale: zeros that keep the sign of each element
+    for (int i = 0; i < 8; ++i) {
+      const float2 v = q2[B + i];
+      const float2 q0 = mul2(v, y2);
+      const float2 q1 = __ffma2_rn(__ffma2_rn(q0, nd, v), y2, q0);  // faithful
+      const float2 q = __ffma2_rn(__ffma2_rn(q1, nd, v), y2, q1);   // RN(v/d)
+      q2[B + i] = make_float2(copysignf(q.x, v.x), copysignf(q.y, v.y));
+    }
+  } else if (sb == 0u) {  // a zero block scale: zeros that keep the sign of each element
 #pragma unroll
     for (int i = 0; i < 8; ++i)
       q2[B + i] = make_float2(__uint_as_float(__float_as_uint(q2[B + i].x) & 0x80000000u),
                               __uint_as_float(__float_as_uint(q2[B + i].y) & 0x80000000u));
-  } else if (exact) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) q2[B + i] = make_float2(__fdiv_rn(q2[B + i].x, d), __fdiv_rn(q2[B + i].y, d));
   } else {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) q2[B + i] = mul2(q2[B + i], y2);
+    for (int i = 0; i < 8; ++i) q2[B + i] = make_float2(__fdiv_rn(q2[B + i].x, d), __fdiv_rn(q2[B + i].y, d));
   }
   return sb;
 }

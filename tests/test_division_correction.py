@@ -1,0 +1,85 @@
+"""The NVFP4 quantiser forms each quotient RN(v/d) from y = RN(1/d) by two correction
+steps: q0 = RN(v*y); q1 = RN(q0 + RN(v - q0*d)*y), which is faithful; then the step of
+Markstein (IBM J. Res. Dev. 34(1), 1990) with the exact residual r = v - q1*d:
+q = RN(q1 + r*y). One step from q0 is not enough: q0 can be just over one ulp from v/d
+(this test found such a case).
+
+Checked here in exact rational arithmetic, with fp32 round-to-nearest-even written out:
+the residual is representable and q is the correctly rounded quotient, over the
+kernel's operating range: d = RN(E4M3 value * S) with 2^-100 <= d <= 2^100 and
+quotients up to ~8: random, at the bottom of each binade (where v*y errs most) and
+within a few ulps of every E2M1 rounding threshold. (The kernels' own outputs are
+compared with the oracle's IEEE divisions in the GPU parity tests.)"""
+from fractions import Fraction
+
+import numpy as np
+
+THRESHOLDS = [Fraction(1, 4), Fraction(3, 4), Fraction(5, 4), Fraction(7, 4),
+              Fraction(5, 2), Fraction(7, 2), Fraction(5)]
+
+
+def rn32(x: Fraction) -> Fraction:
+    """x rounded to the nearest fp32 value, ties to even (no overflow in this range)."""
+    if x == 0:
+        return Fraction(0)
+    s = -1 if x < 0 else 1
+    a = abs(x)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    ulp = Fraction(2) ** (max(e, -126) - 23)
+    m = a / ulp
+    n = m.numerator // m.denominator
+    rem = m - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    return s * n * ulp
+
+
+def exact(v) -> Fraction:
+    return Fraction(float(np.float32(v)))
+
+
+def corrected_quotient(v: Fraction, d: Fraction):
+    y = rn32(1 / d)
+    q0 = rn32(v * y)                 # can be just over one ulp from v/d
+    q1 = rn32(q0 + rn32(v - q0 * d) * y)  # within about half an ulp: faithful
+    r = v - q1 * d
+    assert rn32(r) == r, "residual not representable"
+    return rn32(q1 + r * y)
+
+
+def e4m3_values():
+    vals = []
+    for e in range(-6, 9):
+        for m in range(8):
+            vals.append(Fraction(8 + m, 8) * Fraction(2) ** e)
+    vals += [Fraction(m, 8) * Fraction(2) ** -6 for m in range(1, 8)]  # subnormals
+    return [v for v in vals if v <= 448]
+
+
+def test_correction_step_is_correctly_rounded():
+    rng = np.random.default_rng(7)
+    scales = e4m3_values()
+    checked = 0
+    for _ in range(400):
+        S = exact(np.float32(2.0) ** rng.uniform(-60, 60) * rng.uniform(1, 2))
+        d = rn32(scales[rng.integers(len(scales))] * S)
+        if not (Fraction(2) ** -100 <= d <= Fraction(2) ** 100):
+            continue
+        cases = []
+        for _ in range(20):  # random quotients in [0, 8)
+            cases.append(rn32(Fraction(float(rng.uniform(-8, 8))) * d))
+        for e in range(-3, 3):  # the bottom 3% of each binade 2^-3 .. 2^3
+            for _ in range(4):
+                cases.append(rn32(Fraction(float(rng.uniform(1, 1.03))) * Fraction(2) ** e * d))
+        for t in THRESHOLDS:  # quotients within a few ulps of each threshold
+            base = rn32(t * d)
+            ulp = Fraction(2) ** ((base.numerator.bit_length() - base.denominator.bit_length()) - 24)
+            for k in range(-6, 7):
+                for sgn in (1, -1):
+                    cases.append(sgn * rn32(base + k * ulp))
+        for v in cases:
+            assert corrected_quotient(v, d) == rn32(v / d), (v, d)
+            checked += 1
+    assert checked > 30000
