@@ -626,10 +626,15 @@ def recorded_traffic(kernel_key: str):
 
 
 def kernel_source_hash():
+    """Hash of the GEMM sources' code: // comments, trailing blanks and empty lines are
+    left out, so that an edit of a comment does not void the recorded counters."""
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "fp4_block_scaled_deterministic_b200", "csrc")
     for f in ("common.cuh", "gemm.cuh"):
-        h.update(open(os.path.join(csrc, f), "rb").read())
+        for line in open(os.path.join(csrc, f), encoding="utf-8"):
+            code = line.split("//", 1)[0].rstrip()
+            if code:
+                h.update(code.encode() + b"\n")
     return h.hexdigest()
 
 

@@ -10,9 +10,9 @@
 // NVFP4/MaxText page, Key facts bullet 5 (FP4 tensor cores on Blackwell).]
 //
 // Two kernels share the MMA issue loop (Issuer) and the epilogue (store_row_segment):
-// gemm_fp4_pair_kernel (CTA pairs, cta_group::2, 256x256 tiles; every M > 128, and
-// all MXFP8) and gemm_fp4_kernel (one CTA, 128x256 tiles; FP4 with M <= 128), the
-// latter described here:
+// gemm_fp4_pair_kernel (CTA pairs, cta_group::2, 256x256 tiles; every M > 128, all
+// MXFP8, and groups of GEMMs run in one launch, GemmGroup) and gemm_fp4_kernel (one
+// CTA, 128x256 tiles; FP4 with M <= 128), the latter described here:
 //
 // Design (one CTA per SM, persistent over 128x256 output tiles, K in slabs of 256):
 //   warp 0   : TMA producer. Per slab it loads A 128x128 B, B 256x128 B (128B swizzle)
