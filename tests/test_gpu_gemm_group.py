@@ -1,8 +1,8 @@
 """fp4_gemm_group: several GEMMs in one launch of the pair kernel. Every output must equal
 the same fp4_gemm call bit for bit (same kernel, same per-tile K order), so the oracle
 parity of fp4_gemm carries over; a small group is also checked against the oracle
-directly. Shapes mix output types, ragged M and N, formats, an empty member and the
-full-size Llama-3.1-8B gate projection (the bench's launch)."""
+directly. Shapes mix output types, ragged M and N, formats, an empty member and every
+full-size Llama-3.1-8B projection (the bench's launches)."""
 import numpy as np
 import pytest
 import torch
@@ -84,14 +84,15 @@ def test_group_with_small_m_and_empty_member(orc):
     assert fp4.fp4_check_status() == 0
 
 
-def test_group_llama_gate_three_passes_full_size():
-    """Fprop, Dgrad and Wgrad of the Llama-3.1-8B gate projection (8192 tokens,
-    14336 x 4096, MXFP4 + H16) in one launch, as the bench runs them: each output equals
-    the separate fp4_gemm call (whose full-size parity against the oracle is tested
-    elsewhere) bit for bit."""
+@pytest.mark.parametrize("name", [n for n, _, _ in synthetic.LLAMA_LAYERS])
+def test_group_llama_three_passes_full_size(name):
+    """Fprop, Dgrad and Wgrad of each Llama-3.1-8B projection (8192 tokens, MXFP4 +
+    H16) in one launch, as the bench runs them: each output equals the separate
+    fp4_gemm call (whose full-size parity against the oracle is tested elsewhere) bit
+    for bit."""
     need_gpu()
     fmt = fp4.MXFP4
-    X, W, dY = synthetic.llama_layer("gate")
+    X, W, dY = synthetic.llama_layer(name)
     xr, xc = fp4.quantize_dual(X.cuda(), fmt, 16)
     wr, wc = fp4.quantize_dual(W.cuda(), fmt, 16)
     yr, yc = fp4.quantize_dual(dY.cuda(), fmt, 16)
