@@ -272,10 +272,11 @@ fp4_status prepare_item(QuantItem* item, bool* skip, float** amax_cells, size_t*
   // Bands of 32 tile columns once the column-layout codes are far larger than L2
   // (measured: a 2^30-element dual pass 0.57 -> 0.70 of HBM; at 2^27 and below plain
   // row-major order was 4% faster).
-  // Bands of 16 tile columns for the column layout alone, 32 for the dual pass (measured
-  // on 2^30-element tensors: the column layout 0.76 -> 0.84 of HBM with 16; the dual
-  // pass no better, and worse on 4096-column tensors, which it leaves unbanded).
-  const int band = do_row ? 32 : 16;
+  // Bands of 16 tile columns for the MXFP4 column layout alone, else 32 (measured on
+  // 2^30-element tensors: the MXFP4 column layout 0.76 -> 0.84 of HBM with 16; the dual
+  // pass and NVFP4 no better, and worse on 4096-column tensors, which 32 leaves
+  // unbanded).
+  const int band = (!do_row && fmt == FP4_MXFP4) ? 16 : 32;
   a.band_c = (do_col && !(opts && (opts->stochastic || opts->random_signs)) && a.tiles_c > band &&
               code_bytes(rows * cols, fmt) > (int64_t(256) << 20))
                  ? band : a.tiles_c;

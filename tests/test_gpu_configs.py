@@ -164,9 +164,9 @@ def test_sweep_2p30_banded_tile_order_sampled_rows(orc, fmt, row_len):
 
 @pytest.mark.parametrize("fmt,row_len", [(0, 4096), (0, 49152), (1, 14336)])
 def test_sweep_2p30_column_layout_banded_sampled_rows(orc, fmt, row_len):
-    """The column layout alone of a 2^30-element tensor takes the banded tile order with
-    bands of 16 tile columns (also for 4096-column tensors, which the dual pass leaves
-    unbanded): sampled rows of the transposed layout bit-exact."""
+    """The column layout alone of a 2^30-element tensor takes the banded tile order:
+    bands of 16 tile columns for MXFP4 (also for 4096-column tensors, which bands of 32
+    leave unbanded), 32 for NVFP4: sampled rows of the transposed layout bit-exact."""
     x = synthetic.sweep_tensor(30, row_len, seed=12, device="cuda")
     assert x.shape[1] // 128 > 16 and x.numel() // 2 > (256 << 20)
     cq = fp4.quantize(x, fmt, 16, COL)
