@@ -103,6 +103,8 @@ def lib() -> ctypes.CDLL:
             "fp4_linear_dgrad": (I32, [P, P, P, I64, I64, I64, I32, I32, I32, P, SZ, P]),
             "fp4_linear_wgrad": (I32, [P, P, P, I64, I64, I64, I32, I32, I32, P, SZ, P]),
             "fp4_linear_fprop_noalloc": (I32, [P, P, P, I64, I64, I64, I32, I32, I32, P]),
+            "fp4_linear_step_workspace_size": (SZ, [I64, I64, I64, I32]),
+            "fp4_linear_step": (I32, [P, P, P, P, P, P, I64, I64, I64, I32, I32, P, SZ, P]),
             "fp4_check_status": (I32, [P]),
             "fp4_selftest_timeout": (I32, [ctypes.c_uint64, P]),
             "fp4_status_string": (ctypes.c_char_p, [I32]),
@@ -349,6 +351,27 @@ def gemm(a: QTensor, b: QTensor, out_dtype: int = OUT_F32, out: torch.Tensor | N
     _check(fp4_gemm(a.codes, a.scales, a.tensor_scale, b.codes, b.scales, b.tensor_scale, out, M,
                     N, K, a.fmt, out_dtype), "fp4_gemm")
     return out
+
+
+def linear_step(X: torch.Tensor, W: torch.Tensor, dY: torch.Tensor, fmt: int = MXFP4,
+                hadamard_n: int = 16, ws: torch.Tensor | None = None):
+    """Fprop, Dgrad and Wgrad of one linear layer (fp4_linear_step): returns
+    (Y bf16 [M][N], dX bf16 [M][K], dW fp32 [N][K])."""
+    M, K = X.shape
+    N = W.shape[0]
+    assert W.shape == (N, K) and dY.shape == (M, N)
+    dev = X.device
+    need = lib().fp4_linear_step_workspace_size(M, N, K, fmt)
+    if ws is None:
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    dW = torch.empty(N, K, dtype=torch.float32, device=dev)
+    _check(lib().fp4_linear_step(_ptr(X.contiguous()), _ptr(W.contiguous()),
+                                 _ptr(dY.contiguous()), _ptr(Y), _ptr(dX), _ptr(dW), M, N, K,
+                                 fmt, hadamard_n, _ptr(ws), ws.numel(), _stream(None)),
+           "fp4_linear_step")
+    return Y, dX, dW
 
 
 def gemm_group(problems, out_dtypes=None):

@@ -957,6 +957,85 @@ fp4_status fp4_linear_wgrad(const void* dY, const void* X, void* dW, int64_t M, 
                      reinterpret_cast<cudaStream_t>(stream));
 }
 
+// Workspace of fp4_linear_step: for X [M][K], W [N][K] and dY [M][N] in turn, the row
+// codes and scales, the column codes and scales and 16 floats of NVFP4 tensor-scale
+// cells ({row S, column S, ...} as fp4_quantize_dual writes them), each 256-byte aligned.
+struct StepPlan {
+  size_t rc[3], rs[3], cc[3], cs[3], ts[3], total;
+};
+StepPlan plan_step(int64_t M, int64_t N, int64_t K, fp4_format fmt) {
+  const int64_t rows[3] = {M, N, M}, cols[3] = {K, K, N};
+  StepPlan p;
+  size_t off = 0;
+  for (int t = 0; t < 3; ++t) {
+    p.rc[t] = off; off += align256(fp4_codes_bytes_fmt(rows[t], cols[t], fmt));
+    p.rs[t] = off; off += align256(fp4_scales_bytes(rows[t], cols[t], fmt));
+    p.cc[t] = off; off += align256(fp4_codes_bytes_fmt(cols[t], rows[t], fmt));
+    p.cs[t] = off; off += align256(fp4_scales_bytes(cols[t], rows[t], fmt));
+    p.ts[t] = off; off += 256;
+  }
+  p.total = off;
+  return p;
+}
+
+size_t fp4_linear_step_workspace_size(int64_t M, int64_t N, int64_t K, fp4_format fmt) {
+  if (!valid_format(fmt) || M < 0 || N < 0 || K < 0) return 0;
+  return plan_step(M, N, K, fmt).total;
+}
+
+fp4_status fp4_linear_step(const void* X, const void* W, const void* dY, void* Y, void* dX,
+                           void* dW, int64_t M, int64_t N, int64_t K, fp4_format fmt, int hn,
+                           void* ws, size_t ws_bytes, fp4_stream_t stream) {
+  NvtxRange nvtx_range("fp4_linear_step");
+  if (!valid_format(fmt)) return FP4_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K < 0 || M % 32 || N % 32 || K % 32) return FP4_ERR_SHAPE;
+  if (M == 0 || N == 0 || K == 0) return FP4_OK;
+  const StepPlan p = plan_step(M, N, K, fmt);
+  if (!ws || ws_bytes < p.total) return FP4_ERR_WORKSPACE;
+  if (!aligned16(ws)) return FP4_ERR_ALIGN;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  const bool nv = fmt == FP4_NVFP4;
+  const void* src[3] = {X, W, dY};
+  const int64_t rows[3] = {M, N, M}, cols[3] = {K, K, N};
+  fp4_quant_item items[3];
+  float* ts[3];
+  for (int t = 0; t < 3; ++t) {
+    ts[t] = reinterpret_cast<float*>(w + p.ts[t]);
+    items[t] = fp4_quant_item{src[t], w + p.rc[t], w + p.rs[t], w + p.cc[t], w + p.cs[t],
+                              nv ? ts[t] : nullptr, rows[t], cols[t]};
+  }
+  enum { kX = 0, kW = 1, kDY = 2 };
+  auto S = [&](int t, int layout) -> const float* { return nv ? ts[t] + layout : nullptr; };
+  // Fprop: Q_row(X) . Q_row(W)^T; Dgrad: Q_row(dY) . Q_col(W)^T; Wgrad: Q_col(dY) . Q_col(X)^T
+  const fp4_gemm_desc descs[3] = {
+      {w + p.rc[kX], w + p.rs[kX], S(kX, 0), w + p.rc[kW], w + p.rs[kW], S(kW, 0), Y, M, N, K,
+       FP4_OUT_BF16},
+      {w + p.rc[kDY], w + p.rs[kDY], S(kDY, 0), w + p.cc[kW], w + p.cs[kW], S(kW, 1), dX, M, K, N,
+       FP4_OUT_BF16},
+      {w + p.cc[kDY], w + p.cs[kDY], S(kDY, 1), w + p.cc[kX], w + p.cs[kX], S(kX, 1), dW, N, K, M,
+       FP4_OUT_F32}};
+  // both calls' host checks before either launches
+  for (int i = 0; i < 3; ++i) {
+    bool empty;
+    const fp4_gemm_desc& d = descs[i];
+    const fp4_status st = check_gemm(d.A_codes, d.A_scales, d.A_tensor_scale, d.B_codes,
+                                     d.B_scales, d.B_tensor_scale, d.C, d.M, d.N, d.K, fmt,
+                                     d.out_dtype, nullptr, nullptr, -1, &empty);
+    if (st != FP4_OK) return st;
+  }
+  for (int t = 0; t < 3; ++t) {
+    bool skip;
+    const fp4_quant_item& q = items[t];
+    const fp4_status st = check_item(&skip, q.x_bf16, q.row_codes, q.row_scales, q.col_codes,
+                                     q.col_scales, q.tensor_scale, q.rows, q.cols, fmt, hn,
+                                     kModeDual, nullptr);
+    if (st != FP4_OK) return st;
+  }
+  fp4_status st = fp4_quantize_dual_batch(items, 3, fmt, hn, stream);
+  if (st != FP4_OK) return st;
+  return gemm_group_impl(descs, 3, fmt, reinterpret_cast<cudaStream_t>(stream));
+}
+
 fp4_status fp4_linear_fprop_noalloc(const void* X, const void* W, void* Y, int64_t M, int64_t N,
                                     int64_t K, fp4_format fmt, int hn, fp4_out_dtype od,
                                     fp4_stream_t stream) {

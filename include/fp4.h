@@ -313,6 +313,29 @@ FP4_API fp4_status fp4_linear_wgrad(const void *dY, const void *X, void *dW, int
                             void *ws, size_t ws_bytes, fp4_stream_t stream);
 
 /*
+ * fp4_linear_step -- the three passes above in two launches: the dual-layout
+ * quantisation of X, W and dY from one read of each (one batched launch, as
+ * fp4_quantize_dual_batch) and Fprop, Dgrad and Wgrad in one grouped launch (as
+ * fp4_gemm_group). [MXFP4 pre-training summary, Methodology item 2: all three passes
+ * in FP4.]
+ *   X bf16 [M][K], W bf16 [N][K], dY bf16 [M][N]: device inputs.
+ *   Y bf16 [M][N], dX bf16 [M][K], dW fp32 [N][K]: device outputs, equal bit for bit to
+ *   fp4_linear_fprop / _dgrad (bf16 out) and fp4_linear_wgrad (fp32 out).
+ *   ws / ws_bytes: caller-owned device scratch of at least
+ *   fp4_linear_step_workspace_size() bytes, 16-byte aligned; it receives both layouts
+ *   of the three quantised tensors (and NVFP4 tensor scales) in an unspecified layout.
+ *   Shape: M, N, K multiples of 32 and of the block and rotation sizes; M, N or K zero
+ *   launches nothing.
+ *   Errors: FP4_ERR_WORKSPACE for a NULL or small workspace; otherwise as the
+ *   quantisation and GEMM calls it makes, checked before anything is launched.
+ */
+FP4_API size_t fp4_linear_step_workspace_size(int64_t M, int64_t N, int64_t K, fp4_format fmt);
+FP4_API fp4_status fp4_linear_step(const void *X, const void *W, const void *dY, void *Y,
+                                   void *dX, void *dW, int64_t M, int64_t N, int64_t K,
+                                   fp4_format fmt, int hadamard_n, void *ws, size_t ws_bytes,
+                                   fp4_stream_t stream);
+
+/*
  * fp4_linear_fprop_noalloc -- fp4_linear_fprop with library-owned scratch instead
  * of a caller workspace. The pages have no counterpart to this call; it exists for
  * callers that cannot allocate device memory: code running inside a host framework

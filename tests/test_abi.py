@@ -144,6 +144,23 @@ def test_gemm_group_validation():
     assert L.fp4_gemm_group(arr(d(M=0), d(N=0)), 2, 0, None) == OK   # nothing to launch
 
 
+def test_linear_step_validation():
+    L = fp4.lib()
+    need = L.fp4_linear_step_workspace_size(64, 96, 128, 0)
+    per_pass = sum(fp4.fp4_linear_workspace_size(p, 64, 96, 128, 0) for p in range(3))
+    assert need >= per_pass // 2 > 0
+    assert L.fp4_linear_step_workspace_size(64, 96, 128, 7) == 0
+    args = lambda M=64, N=96, K=128, ws=A16, wsb=need, fmt=0, hn=16: (
+        A16, A16, A16, A16, A16, A16, M, N, K, fmt, hn, ws, wsb, None)
+    assert L.fp4_linear_step(*args(wsb=need - 1)) == WORKSPACE
+    assert L.fp4_linear_step(*args(ws=None)) == WORKSPACE
+    assert L.fp4_linear_step(*args(ws=MIS)) == ALIGN
+    assert L.fp4_linear_step(*args(N=100)) == SHAPE
+    assert L.fp4_linear_step(*args(fmt=9)) == INVALID
+    assert L.fp4_linear_step(*args(hn=12)) == INVALID
+    assert L.fp4_linear_step(*args(M=0)) == OK  # nothing to do
+
+
 def test_quantize_batch_validation():
     L = fp4.lib()
     item = fp4.QuantItem(A16, A16, A16, A16, A16, None, 64, 64)
