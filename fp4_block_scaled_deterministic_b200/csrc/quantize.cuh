@@ -760,15 +760,20 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
   const int col_c = 64 * col_b + 2 * col_w;
 
   float amax_r = 0.0f, amax_c = 0.0f;
+  // Every tensor of a batch has the same wait limit.
+  const uint64_t wait_ns = qb.item[0].a.wait_limit_ns;
   for (int it = 0; it < my_tiles; ++it) {
     const int tile = bid + it * nctas;
-    const int item = batch_item<NITEMS>(qb, tile);
-    const QuantItem& I = qb.item[item];
-    const QuantArgs& a = I.a;
-    int tr, tc;
-    qtile_coords<BANDED>(tile - I.tile0, a, tr, tc);
+    // The tile's tensor and coordinates are resolved where they are used: in the jobs
+    // only by the variants (always one tensor per launch, so item 0) and NVFP4 (its
+    // tensor scales), and after the tile's barrier by the threads that store or publish.
+    // Kept live through the jobs, they cost the batched instances registers and time.
+    const QuantArgs& a = qb.item[0].a;
+    int tr = 0, tc = 0;
+    if constexpr (EXT) qtile_coords<BANDED>(tile - qb.item[0].tile0, a, tr, tc);
     float S_r = 1.0f, S_c = 1.0f;  // NVFP4 tensor scales of this tile's tensor
     if constexpr (FMT == kFmtNV && !AMAX) {
+      const int item = batch_item<NITEMS>(qb, tile);
       S_r = s_S[2 * item];
       S_c = s_S[2 * item + 1];
     }
@@ -781,7 +786,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
     const uint32_t* s_rmask = s_cmask + 64;
     // A wait that runs out is acted on at the barrier below, together: the jobs then
     // read stale (never faulting) shared memory, and nothing of this tile is stored.
-    const bool ok = mbar_wait(&full[st], static_cast<uint32_t>((it / kQStages) & 1), a.wait_limit_ns);
+    const bool ok = mbar_wait(&full[st], static_cast<uint32_t>((it / kQStages) & 1), wait_ns);
     const uint8_t* in = s_in + st * kQInBytes;
     uint8_t* rcode = s_rcode + ob * kCodeBytes;
     uint8_t* ccode = s_ccode + ob * kCodeBytes;
@@ -915,6 +920,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
         amax_c = fmaxf(amax_c, __shfl_xor_sync(0xffffffffu, amax_c, o));
       }
       if (lane == 0) {
+        const int item = batch_item<NITEMS>(qb, tile);
         if constexpr (kRow) atomicMax(&s_amax[2 * item], __float_as_uint(amax_r));
         if constexpr (kCol) atomicMax(&s_amax[2 * item + 1], __float_as_uint(amax_c));
       }
@@ -924,6 +930,10 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSMOf(FMT, EXT))
     if (__syncthreads_or(!ok)) break;  // give up together; the status word says why
     if (tid == 0) {
       if constexpr (!AMAX) {
+        const int item = batch_item<NITEMS>(qb, tile);
+        const QuantItem& I = qb.item[item];
+        const QuantArgs& a = I.a;
+        qtile_coords<BANDED>(tile - I.tile0, a, tr, tc);
         constexpr int kAtomsPerTile = (FMT == kFmtNV) ? 2 : 1;
         constexpr int kTileCodeBytes = FMT == kFmtMX8 ? 128 : 64;  // code bytes per tile row
         const bool tile_ok = FP4_IN_BOUNDS(tr >= 0 && tr < a.tiles_r && tc >= 0 && tc < a.tiles_c);
