@@ -368,18 +368,32 @@ __device__ __forceinline__ Enc mx_encode_x2_h16fold(float2 (&p)[32], const Codes
 // 2^-100 <= d <= 2^100 a residual can underflow only when |v/d| < 2^-3, whose code is a
 // signed zero either way, and the sign is taken from v (so -0 / d stays -0). Blocks
 // with a zero scale, a d outside that range or a non-finite element are divided exactly.
-template <int b, bool kExact = false, int L = 32>
+//
+// kQuarter: p holds w = 4v, the H16 butterflies without their x0.25. Round-to-nearest
+// is monotonic and odd, so the block amax of v is RN(amax|w| / 4), one multiply per
+// block. Where v = w/4 exactly (|w| >= 2^-124), v/d = w/(4d) with 4d exact, so the
+// quotient is taken from w and d' = 4d, in the same range check: the same number
+// wherever the sequence is exact, and below 2^-3 a signed zero code either way.
+// Smaller elements have |v/d| and |w/d'| below 2^-22 (d' >= 2^-100): both encode as
+// the signed zero of w's sign. Blocks off the fast path scale by 0.25 first and go on
+// exactly as before.
+template <int b, bool kExact = false, int L = 32, bool kQuarter = false>
 __device__ __forceinline__ void nv_block_x2(float2 (&p)[L], float S, float six_s,
                                             uint32_t& sbx, uint32_t& sby) {
-  const float2 bm = amax_x2<b, 16>(p);
+  float2 bm = amax_x2<b, 16>(p);
+  if constexpr (kQuarter) bm = make_float2(__fmul_rn(bm.x, 0.25f), __fmul_rn(bm.y, 0.25f));
   sbx = cvt_e4m3(__fdiv_rn(bm.x, six_s));
   sby = cvt_e4m3(__fdiv_rn(bm.y, six_s));
   const float dx = __fmul_rn(e4m3_to_f32(sbx), S), dy = __fmul_rn(e4m3_to_f32(sby), S);
-  const bool fast = !kExact && dx >= 0x1p-100f && dy >= 0x1p-100f && dx <= 0x1p100f &&
-                    dy <= 0x1p100f && bm.x <= 3.0e38f && bm.y <= 3.0e38f;
+  // the divisor of the values held: d, or 4d for kQuarter (exact, or infinite and so
+  // off the fast path)
+  const float ex = kQuarter ? __fmul_rn(dx, 4.0f) : dx;
+  const float ey = kQuarter ? __fmul_rn(dy, 4.0f) : dy;
+  const bool fast = !kExact && ex >= 0x1p-100f && ey >= 0x1p-100f && ex <= 0x1p100f &&
+                    ey <= 0x1p100f && bm.x <= 3.0e38f && bm.y <= 3.0e38f;
   if (fast) {
-    const float2 y2 = make_float2(__frcp_rn(dx), __frcp_rn(dy));
-    const float2 nd = make_float2(-dx, -dy);
+    const float2 y2 = make_float2(__frcp_rn(ex), __frcp_rn(ey));
+    const float2 nd = make_float2(-ex, -ey);
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const float2 v = p[b + i];
@@ -395,7 +409,7 @@ __device__ __forceinline__ void nv_block_x2(float2 (&p)[L], float S, float six_s
   const bool zx = sbx == 0u, zy = sby == 0u;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const float2 v = p[b + i];
+    const float2 v = kQuarter ? mul2(p[b + i], make_float2(0.25f, 0.25f)) : p[b + i];
     p[b + i] = make_float2(zx ? __uint_as_float(__float_as_uint(v.x) & 0x80000000u)
                               : __fdiv_rn(v.x, dx),
                            zy ? __uint_as_float(__float_as_uint(v.y) & 0x80000000u)
@@ -1145,8 +1159,8 @@ __device__ __forceinline__ uint2 codes_col16y(const float2 (&p)[16]) {
 
 // NVFP4 block of 16 values held as 8 pairs q2[B .. B+8) (ROW job): scale byte, and the
 // pairs replaced by their quotients RN(v/d) (or signed zeros); the arithmetic of
-// nv_block_x2 (the correction step, else exact division).
-template <int B>
+// nv_block_x2 (the correction step, else exact division), kQuarter included.
+template <int B, bool kQuarter = false>
 __device__ __forceinline__ uint32_t nv_block_row_v(float2 (&q2)[16], float S, float six_s) {
   float a[16];
 #pragma unroll
@@ -1154,12 +1168,14 @@ __device__ __forceinline__ uint32_t nv_block_row_v(float2 (&q2)[16], float S, fl
     a[2 * i] = fabsf(q2[B + i].x);
     a[2 * i + 1] = fabsf(q2[B + i].y);
   }
-  const float bm = tree_max<16>(a);
+  float bm = tree_max<16>(a);
+  if constexpr (kQuarter) bm = __fmul_rn(bm, 0.25f);
   const uint32_t sb = cvt_e4m3(__fdiv_rn(bm, six_s));
   const float d = __fmul_rn(e4m3_to_f32(sb), S);
-  if (d >= 0x1p-100f && d <= 0x1p100f && bm <= 3.0e38f) {  // the correction step
-    const float y = __frcp_rn(d);
-    const float2 y2 = make_float2(y, y), nd = make_float2(-d, -d);
+  const float e = kQuarter ? __fmul_rn(d, 4.0f) : d;  // the divisor of the values held
+  if (e >= 0x1p-100f && e <= 0x1p100f && bm <= 3.0e38f) {  // the correction step
+    const float y = __frcp_rn(e);
+    const float2 y2 = make_float2(y, y), nd = make_float2(-e, -e);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const float2 v = q2[B + i];
@@ -1175,7 +1191,10 @@ __device__ __forceinline__ uint32_t nv_block_row_v(float2 (&q2)[16], float S, fl
                               __uint_as_float(__float_as_uint(q2[B + i].y) & 0x80000000u));
   } else {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) q2[B + i] = make_float2(__fdiv_rn(q2[B + i].x, d), __fdiv_rn(q2[B + i].y, d));
+    for (int i = 0; i < 8; ++i) {
+      const float2 v = kQuarter ? mul2(q2[B + i], make_float2(0.25f, 0.25f)) : q2[B + i];
+      q2[B + i] = make_float2(__fdiv_rn(v.x, d), __fdiv_rn(v.y, d));
+    }
   }
   return sb;
 }
@@ -1187,6 +1206,10 @@ __global__ void __launch_bounds__(kQWThreads, 2)
   constexpr bool kRow = (MODE & kModeRow) != 0;
   constexpr bool kCol = (MODE & kModeCol) != 0;
   constexpr bool kFold = FMT == kFmtMX && HN == 16 && !AMAX;
+  // NVFP4 + H16: the rotation's x0.25 is applied per block (to its amax and divisor),
+  // not per element; the amax pass applies it once to each published tile amax
+  constexpr bool kQuarter = FMT == kFmtNV && HN == 16;
+  constexpr bool kScale = !kFold && !kQuarter;
   constexpr bool kFuse1 = HN > 0;
   constexpr int kStages = 2;
   constexpr int kCodeBytes = kQCodeBytesOf(FMT);
@@ -1244,22 +1267,17 @@ __global__ void __launch_bounds__(kQWThreads, 2)
   const int col_c = 2 * col_cp;
 
   float amax_r = 0.0f, amax_c = 0.0f;
+  // Every tensor of a batch has the same wait limit.
+  const uint64_t wait_ns = qb.item[0].a.wait_limit_ns;
   for (int it = 0; it < my_tiles; ++it) {
     const int tile = bid + it * nctas;
-    const int item = batch_item<NITEMS>(qb, tile);
-    const QuantItem& I = qb.item[item];
-    const QuantArgs& a = I.a;
-    int tr, tc;
-    qtile_coords<BANDED>(tile - I.tile0, a, tr, tc);
-    float S_r = 1.0f, S_c = 1.0f;  // NVFP4 tensor scales of this tile's tensor
-    if constexpr (FMT == kFmtNV && !AMAX) {
-      S_r = s_S[2 * item];
-      S_c = s_S[2 * item + 1];
-    }
-    const float six_r = __fmul_rn(6.0f, S_r), six_c = __fmul_rn(6.0f, S_c);
+    // The jobs need only the NVFP4 tensor scales of the tile's tensor, read where each
+    // job uses them; its arguments and coordinates are resolved after the tile's
+    // barrier, by the threads that store or publish (kept live through the jobs they
+    // cost registers and spills).
+    const int item = (FMT == kFmtNV && !AMAX) ? batch_item<NITEMS>(qb, tile) : 0;
     const int st = it % kStages, ob = it & 1;
-    const bool ok =
-        mbar_wait(&full[st], static_cast<uint32_t>((it / kStages) & 1), a.wait_limit_ns);
+    const bool ok = mbar_wait(&full[st], static_cast<uint32_t>((it / kStages) & 1), wait_ns);
     const uint8_t* in = s_in + st * kQInBytes;
     uint8_t* rcode = s_rcode + ob * kCodeBytes;
     uint8_t* ccode = s_ccode + ob * kCodeBytes;
@@ -1269,7 +1287,7 @@ __global__ void __launch_bounds__(kQWThreads, 2)
     if constexpr (kRow) {
       float2 q2[16];
       load_row_v<kFuse1>(in, row_r, row_q, q2);
-      fwht_row_v<HN, !kFold>(q2);
+      fwht_row_v<HN, kScale>(q2);
       if constexpr (AMAX) {
         float v[32];
 #pragma unroll
@@ -1309,8 +1327,9 @@ __global__ void __launch_bounds__(kQWThreads, 2)
           *reinterpret_cast<uint4*>(code_chunk(rcode, row_r, row_q)) = codes_row16(q2);
         if (scale_ok(row_r, row_q, 1)) rsc[atom_off(row_r, row_q)] = static_cast<uint8_t>(byte);
       } else {  // NVFP4: blocks 2q and 2q+1
-        const uint32_t b0 = nv_block_row_v<0>(q2, S_r, six_r);
-        const uint32_t b1 = nv_block_row_v<8>(q2, S_r, six_r);
+        const float S_r = s_S[2 * item], six_r = __fmul_rn(6.0f, S_r);
+        const uint32_t b0 = nv_block_row_v<0, kQuarter>(q2, S_r, six_r);
+        const uint32_t b1 = nv_block_row_v<8, kQuarter>(q2, S_r, six_r);
         if (code_ok(row_r, row_q, 4))
           *reinterpret_cast<uint4*>(code_chunk(rcode, row_r, row_q)) = codes_row16(q2);
         if (scale_ok(row_r, 2 * row_q, 2))
@@ -1321,7 +1340,7 @@ __global__ void __launch_bounds__(kQWThreads, 2)
     if constexpr (kCol) {
       float2 p[16];
       load_col_v<kFuse1>(in, col_cp, col_r0, p);
-      fwht_col_v<HN, !kFold>(p, col_upper);
+      fwht_col_v<HN, kScale>(p, col_upper);
       if constexpr (AMAX) {
         const float2 m = amax_x2<0, 16>(p);
         amax_c = max3f(amax_c, m.x, m.y);
@@ -1361,8 +1380,9 @@ __global__ void __launch_bounds__(kQWThreads, 2)
           csc[atom_off(col_c + 1, col_s)] = static_cast<uint8_t>(by);
         }
       } else {  // NVFP4: the 16 rows are one block per column
+        const float S_c = s_S[2 * item + 1], six_c = __fmul_rn(6.0f, S_c);
         uint32_t sbx, sby;
-        nv_block_x2<0, false, 16>(p, S_c, six_c, sbx, sby);
+        nv_block_x2<0, false, 16, kQuarter>(p, S_c, six_c, sbx, sby);
         if (code_ok(col_c + 1, col_s, 4)) {
           *reinterpret_cast<uint2*>(code_chunk(ccode, col_c, col_s) + (col_upper ? 8 : 0)) =
               codes_col16x(p);
@@ -1387,8 +1407,14 @@ __global__ void __launch_bounds__(kQWThreads, 2)
         amax_c = fmaxf(amax_c, __shfl_xor_sync(0xffffffffu, amax_c, o));
       }
       if (lane == 0) {
-        if constexpr (kRow) atomicMax(&s_amax[2 * item], __float_as_uint(amax_r));
-        if constexpr (kCol) atomicMax(&s_amax[2 * item + 1], __float_as_uint(amax_c));
+        const int k = batch_item<NITEMS>(qb, tile);
+        // max |RN(w/4)| = RN(max |w| / 4): rounding is monotonic and odd
+        if constexpr (kQuarter) {
+          amax_r = __fmul_rn(amax_r, 0.25f);
+          amax_c = __fmul_rn(amax_c, 0.25f);
+        }
+        if constexpr (kRow) atomicMax(&s_amax[2 * k], __float_as_uint(amax_r));
+        if constexpr (kCol) atomicMax(&s_amax[2 * k + 1], __float_as_uint(amax_c));
       }
       amax_r = 0.0f;
       amax_c = 0.0f;
@@ -1396,6 +1422,10 @@ __global__ void __launch_bounds__(kQWThreads, 2)
     if (__syncthreads_or(!ok)) break;  // give up together; the status word says why
     if (tid == 0) {
       if constexpr (!AMAX) {
+        const QuantItem& I = qb.item[batch_item<NITEMS>(qb, tile)];
+        const QuantArgs& a = I.a;
+        int tr, tc;
+        qtile_coords<BANDED>(tile - I.tile0, a, tr, tc);
         constexpr int kAtomsPerTile = (FMT == kFmtNV) ? 2 : 1;
         const bool tile_ok = FP4_IN_BOUNDS(tr >= 0 && tr < a.tiles_r && tc >= 0 && tc < a.tiles_c);
         if constexpr (kRow) {

@@ -49,6 +49,14 @@ def corrected_quotient(v: Fraction, d: Fraction):
     return rn32(q1 + r * y)
 
 
+def fma_sequence(v: Fraction, d: Fraction) -> Fraction:
+    """The kernel's instructions as written, one rounding per FMA (no exactness assumed)."""
+    y = rn32(1 / d)
+    q0 = rn32(v * y)
+    q1 = rn32(q0 + rn32(v - q0 * d) * y)
+    return rn32(q1 + rn32(v - q1 * d) * y)
+
+
 def e4m3_values():
     vals = []
     for e in range(-6, 9):
@@ -83,3 +91,52 @@ def test_correction_step_is_correctly_rounded():
             assert corrected_quotient(v, d) == rn32(v / d), (v, d)
             checked += 1
     assert checked > 30000
+
+
+E2M1_GRID = [Fraction(0), Fraction(1, 2), Fraction(1), Fraction(3, 2), Fraction(2),
+             Fraction(3), Fraction(4), Fraction(6)]
+
+
+def e2m1_magnitude_code(m: Fraction) -> int:
+    """Index of the E2M1 magnitude that m >= 0 rounds to (nearest, ties to the even
+    code, saturating at 6)."""
+    for k in range(7):
+        lo, hi = E2M1_GRID[k], E2M1_GRID[k + 1]
+        mid = (lo + hi) / 2
+        if m < mid or (m == mid and k % 2 == 0):
+            return k
+    return 7
+
+
+def test_quarter_fold_gives_the_same_codes():
+    """NVFP4 + H16 quantiser: the quotient is taken from w = 4v (the butterflies without
+    their x0.25) and d' = 4d by the same FMA sequence. Where v = RN(w/4) is exactly w/4
+    (|w| >= 2^-124), v/d and w/d' are one number, and wherever the sequence is exact
+    (|v/d| >= 2^-3) both give RN(v/d). Every code, tiny quotients included, equals the
+    code of RN(v/d), with w's sign. The block amax of v is RN(amax|w| / 4) because
+    rounding is monotonic and odd."""
+    rng = np.random.default_rng(11)
+    scales = e4m3_values()
+    tiny = Fraction(2) ** -124
+    checked = 0
+    for _ in range(300):
+        S = exact(np.float32(2.0) ** rng.uniform(-60, 60) * rng.uniform(1, 2))
+        d = rn32(scales[rng.integers(len(scales))] * S)
+        e = 4 * d
+        if not (Fraction(2) ** -100 <= e <= Fraction(2) ** 100):
+            continue
+        ws = [rn32(Fraction(float(rng.uniform(-32, 32))) * d) for _ in range(10)]
+        ws += [Fraction(int(k)) * Fraction(2) ** -133 * 2 ** int(rng.integers(0, 12))
+               for k in rng.integers(-127, 128, size=6)]  # bf16-subnormal-sized sums
+        for w in ws:
+            v = rn32(w / 4)
+            folded = fma_sequence(w, e)
+            plain = rn32(v / d)
+            if abs(w) >= tiny and abs(plain) >= Fraction(1, 8):
+                assert folded == plain, (w, d)
+            assert e2m1_magnitude_code(abs(folded)) == e2m1_magnitude_code(abs(plain)), (w, d)
+            assert folded == 0 or (folded < 0) == (w < 0)
+            checked += 1
+        block = ws[:16]
+        assert rn32(max(abs(w) for w in block) / 4) == max(abs(rn32(w / 4)) for w in block)
+    assert checked > 3000

@@ -107,6 +107,39 @@ def test_quantize_edge_values(orc, fmt, hn):
         _check_same(orc.quantize(x, fmt, hn, axis), gpu_quantize_raw(x, fmt, hn, axis), fmt)
 
 
+def _cancellation_tensor(rows, cols, seed):
+    """Every 16x16 block holds one 2x2 corner of four equal values (+-2^k, k in
+    [-4, 4)) among bf16 subnormals. Along either axis the two equal leading inputs
+    cancel in the first butterfly, so under H16 a block's rotated values of normal size
+    sit beside sums of subnormals (some below 2^-124) while the tensor scale is set by
+    the normal values: the NVFP4 blocks take the fast quotient path with tiny elements
+    in it, and the blocks of subnormals alone get a zero scale."""
+    rng = np.random.default_rng(seed)
+    x = (rng.integers(-127, 128, size=(rows, cols)) * 2.0 ** -133).astype(np.float32)
+    big = (rng.choice([-1.0, 1.0], size=(rows // 16, cols // 16)) *
+           2.0 ** rng.integers(-4, 4, size=(rows // 16, cols // 16))).astype(np.float32)
+    for a in range(rows // 16):
+        for b in range(cols // 16):
+            x[16 * a:16 * a + 2, 16 * b:16 * b + 2] = big[a, b]
+    return torch.tensor(x).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_quantize_cancellation_blocks(orc, fmt):
+    x = _cancellation_tensor(256, 384, seed=5 + fmt)
+    assert torch.equal(x.float(), torch.tensor(x.float().numpy()))  # bf16-exact inputs
+    for axis in (0, 1):
+        _check_same(orc.quantize(x, fmt, 16, axis), gpu_quantize_raw(x, fmt, 16, axis), fmt)
+    rq, cq = fp4.quantize_dual(x.cuda(), fmt, 16)
+    bq = fp4.quantize_dual_batch([x.cuda(), x[:128].cuda().contiguous()], fmt, 16)
+    torch.cuda.synchronize()
+    for axis, q in ((orc.ROW, rq), (orc.COL, cq)):
+        o = orc.quantize(x, fmt, 16, axis)
+        assert np.array_equal(np_u8(q.codes), o[0]) and np.array_equal(np_u8(q.scales), o[1])
+    for got, ref in zip(bq[0], (rq, cq)):
+        assert torch.equal(got.codes, ref.codes) and torch.equal(got.scales, ref.scales)
+
+
 def test_quantize_is_deterministic():
     x = synthetic.normal(512, 1024, seed=3, outlier_frac=0.001, outlier_mult=50.0)
     a = gpu_quantize_raw(x, 1, 16, 0)
