@@ -23,6 +23,10 @@
 // stores) and written by bulk copies. Staging is double-buffered so stores overlap the
 // next tile.
 //
+// With H16 the rotation's x0.25 is a power of two and is applied per block, not per
+// element, wherever that is exact: MXFP4 folds it into the E8M0 exponent, and the
+// plain NVFP4 kernel into the block amax and the divisor (nv_block_x2, kQuarter).
+//
 // Also here: the MXFP8 comparator (E4M3 codes, one byte each, 128-byte code tiles,
 // one CTA per SM); the EXT instances with the quantiser variants (random Hadamard
 // signs, Philox-driven stochastic rounding); the BANDED instances, whose tile order
