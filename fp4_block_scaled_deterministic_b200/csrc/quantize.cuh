@@ -663,9 +663,10 @@ __device__ __forceinline__ void load_col_job_bfly1(const uint8_t* in, int b, int
 // flight long and sequential, which is best while the column-layout (transposed)
 // codes, written 64 bytes per output row per tile, can still be merged in L2. For
 // tensors whose column-layout codes far exceed L2 the host launches the BANDED kernels:
-// bands of a.band_c (32) tile columns with the tile column fastest inside a band. The
-// tiles in flight then cover about nine tile rows of one band, and each column-layout
-// row receives a 576-byte run instead of scattered 64-byte pieces.
+// bands of a.band_c tile columns (32; 16 for the MXFP4 column layout alone) with the
+// tile column fastest inside a band. With 32, the tiles in flight cover about nine tile
+// rows of one band, and each column-layout row receives a 576-byte run instead of
+// scattered 64-byte pieces.
 template <bool BANDED>
 __device__ __forceinline__ void qtile_coords(int tile, const QuantArgs& a, int& tr, int& tc) {
   if constexpr (!BANDED) {
