@@ -94,6 +94,10 @@ def parse():
     ap.add_argument("--workload", choices=["llama", "gpt3"], default="llama",
                     help="gpt3: the GPT-3 175B layer shapes on 4096 tokens (a parity config, "
                          "measured for the record; the headline line is the Llama layer)")
+    ap.add_argument("--library-compare", action="store_true",
+                    help="GEMM only: this library's block-scaled GEMM against the library kernel "
+                         "torch runs for the same format (torch.nn.functional.scaled_mm) on the "
+                         "layer's GEMM shapes, same operands; one JSON line per shape + totals")
     ap.add_argument("--sweep", action="store_true",
                     help="quantise-only bandwidth sweep (one JSON line per case) instead of the step")
     ap.add_argument("--side-stream", type=int, default=1, choices=[0, 1],
@@ -694,6 +698,144 @@ def run_sweep(a, dev):
     assert fp4.fp4_check_status() == 0
 
 
+def library_gemm(fmt, a, sa, ta, b, sb, tb):
+    """torch's library block-scaled GEMM for `fmt` on this library's buffers, C = A B^T in
+    bf16, as a callable; None where torch offers none. Codes [rows][K/2] (E2M1 pairs) or
+    [rows][K] (E4M3); scales in the 32x4x4 swizzled atoms this library writes: E8M0 per 32
+    (MX) or E4M3 per 16 under the fp32 tensor scales ta, tb (NVFP4)."""
+    F = torch.nn.functional
+    if not (hasattr(F, "scaled_mm") and hasattr(F, "ScalingType")
+            and hasattr(torch, "float4_e2m1fn_x2")):
+        return None
+    ST, SW = F.ScalingType, F.SwizzleType
+    if fmt == 1:
+        a4, b4 = a.view(torch.float4_e2m1fn_x2), b.view(torch.float4_e2m1fn_x2).t()
+        sa8, sb8 = sa.view(torch.float8_e4m3fn), sb.view(torch.float8_e4m3fn)
+        for sw in ([SW.SWIZZLE_32_4_4, SW.NO_SWIZZLE], [SW.SWIZZLE_32_4_4]):
+            def call(sw=sw):
+                return F.scaled_mm(a4, b4, [sa8, ta], [ST.BlockWise1x16, ST.TensorWise],
+                                   [sb8, tb], [ST.BlockWise1x16, ST.TensorWise],
+                                   swizzle_a=sw, swizzle_b=sw, output_dtype=torch.bfloat16)
+            try:
+                call()
+                return call
+            except (RuntimeError, TypeError, ValueError):
+                continue
+        return None
+    dt = torch.float8_e4m3fn if fmt == 2 else torch.float4_e2m1fn_x2
+    a_, b_ = a.view(dt), b.view(dt).t()
+    sa8, sb8 = sa.view(torch.float8_e8m0fnu), sb.view(torch.float8_e8m0fnu)
+
+    def call():
+        return F.scaled_mm(a_, b_, sa8, ST.BlockWise1x32, sb8, ST.BlockWise1x32,
+                           swizzle_a=SW.SWIZZLE_32_4_4, swizzle_b=SW.SWIZZLE_32_4_4,
+                           output_dtype=torch.bfloat16)
+    try:
+        call()
+        return call
+    except (RuntimeError, TypeError, ValueError):
+        return None
+
+
+def gemm_shapes(layers, tokens):
+    """(label, M, N, K) of the layer's Fprop, Dgrad and Wgrad GEMMs, as the step runs them."""
+    out = []
+    for name, n, k in layers:
+        out += [(f"{name}.fprop", tokens, n, k), (f"{name}.dgrad", tokens, k, n),
+                (f"{name}.wgrad", n, k, tokens)]
+    return out
+
+
+def run_library_compare(a, dev):
+    """This library's block-scaled GEMM against the kernel torch runs for the same format
+    (torch.nn.functional.scaled_mm) on the layer's GEMM shapes. Both get the same random
+    codes and scales (the scale layout is shared) and write bf16; each launch is timed
+    alone after a 256 MB L2 flush, CUDA events on the launching stream. One JSON line per
+    shape and one with the totals (flops over summed time) and whether every bf16 output
+    was bit-identical."""
+    import fp4_block_scaled_deterministic_b200 as fp4
+    fmt = FORMATS[a.format]
+    layers, tokens, _ = layer_table(a)
+    wanted = [p.strip() for p in a.proj.split(",")]
+    layers = [t for t in layers if t[0] in wanted] or layers
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(2)
+
+    def timed(fn, n=10, warm=3):
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize(dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n)]
+        for e0, e1 in ev:
+            flush.fill_(1)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return sum(x.elapsed_time(y) for x, y in ev) / n
+
+    def operand(rows, k):
+        codes = torch.randint(0, 256, (rows, k if fmt == 2 else k // 2), dtype=torch.uint8,
+                              device=dev, generator=gen)
+        if fmt == 2:  # no E4M3 NaN codes
+            codes[(codes & 0x7F) == 0x7F] -= 1
+        lo, hi = (0x30, 0x50) if fmt == 1 else (122, 131)  # E4M3 / E8M0 scale bytes
+        sc = torch.randint(lo, hi, (fp4.fp4_scales_bytes(rows, k, fmt),), dtype=torch.uint8,
+                           device=dev, generator=gen)
+        return codes, sc
+
+    ta = torch.tensor([0.75], dtype=torch.float32, device=dev)
+    tb = torch.tensor([1.3125], dtype=torch.float32, device=dev)
+    tot = {"ours": [0.0, 0.0], "library": [0.0, 0.0]}
+    all_equal, available = True, True
+    for label, m, n, k in gemm_shapes(layers, tokens):
+        A, As = operand(m, k)
+        B, Bs = operand(n, k)
+        C = torch.empty(m, n, dtype=torch.bfloat16, device=dev)
+        nv = fmt == 1
+
+        def ours():
+            st = fp4.fp4_gemm(A, As, ta if nv else None, B, Bs, tb if nv else None, C, m, n, k,
+                              fmt, fp4.OUT_BF16, stream.cuda_stream)
+            assert st == 0, fp4.status_string(st)
+        flops = 2.0 * m * n * k
+        ms = timed(ours)
+        rec = {"library_compare": a.format, "gemm": label, "mnk": [m, n, k],
+               "ours_tflops": flops / ms / 1e9}
+        tot["ours"][0] += flops
+        tot["ours"][1] += ms
+        lib = library_gemm(fmt, A, As, ta, B, Bs, tb)
+        if lib is None:
+            available = False
+        else:
+            ms2 = timed(lib)
+            rec["library_tflops"] = flops / ms2 / 1e9
+            tot["library"][0] += flops
+            tot["library"][1] += ms2
+            ours()
+            ref = lib()
+            torch.cuda.synchronize(dev)
+            rec["bf16_bit_identical"] = bool(torch.equal(C.view(torch.int16),
+                                                         ref.contiguous().view(torch.int16)))
+            all_equal = all_equal and rec["bf16_bit_identical"]
+            del ref
+        print(json.dumps(rec), flush=True)
+        del A, As, B, Bs, C
+        torch.cuda.empty_cache()
+    out = {"library_compare": a.format, "total": True, "gemms": len(gemm_shapes(layers, tokens)),
+           "ours_tflops": tot["ours"][0] / tot["ours"][1] / 1e9,
+           "library": "torch.nn.functional.scaled_mm" if available else None}
+    if available:
+        out["library_tflops"] = tot["library"][0] / tot["library"][1] / 1e9
+        out["ratio"] = out["ours_tflops"] / out["library_tflops"]
+        out["bf16_bit_identical_all"] = all_equal
+    print(json.dumps(out), flush=True)
+    assert fp4.fp4_check_status() == 0
+
+
 # ---------------------------------------------------------------- main
 def spawn_ranks(a) -> int:
     """`--gpus N` (N > 1) started as a plain process: re-launch this command as N ranks
@@ -739,6 +881,8 @@ def main():
     fmt = FORMATS[a.format]
     if a.sweep:
         return run_sweep(a, dev)
+    if a.library_compare:
+        return run_library_compare(a, dev)
     layers, tokens, omult = layer_table(a)
     all_names = [n for n, _, _ in layers]
     names = [n.strip() for n in a.proj.split(",") if n.strip() in all_names] or all_names

@@ -30,6 +30,22 @@ def test_defaults_follow_the_contract():
     assert _args("--warmup", "1").warmup == 3  # at least three warm-up steps
 
 
+def test_library_compare_shapes():
+    """--library-compare times the step's own GEMMs: per projection Fprop (M = tokens),
+    Dgrad (N and K swapped) and Wgrad (contraction over the tokens)."""
+    a = _args("--library-compare", "--format", "nvfp4")
+    assert a.library_compare and a.format == "nvfp4"
+    layers, tokens, _ = bench.layer_table(a)
+    shapes = bench.gemm_shapes(layers, tokens)
+    assert len(shapes) == 3 * len(layers) == 15
+    by = {lab: (m, n, k) for lab, m, n, k in shapes}
+    assert by["down.fprop"] == (8192, 4096, 14336)
+    assert by["down.dgrad"] == (8192, 14336, 4096)
+    assert by["down.wgrad"] == (4096, 14336, 8192)
+    flops = sum(2 * m * n * k for _, m, n, k in shapes)
+    assert abs(flops / 15 / 1e9 - 714.68) < 0.01  # 714.7 GFLOP per GEMM on average
+
+
 def test_workload_names():
     assert bench.workload_name(_args()) == bench.WORKLOAD
     assert "NVFP4 + H32" in bench.workload_name(_args("--format", "nvfp4", "--hadamard", "32"))
