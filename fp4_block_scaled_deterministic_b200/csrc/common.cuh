@@ -107,6 +107,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   }
 }
 
+// Warp-collective forms, for issuing roles run by a whole converged warp so that their
+// descriptors and loop state stay warp-uniform: every lane waits (one answer for all
+// lanes), and one elected lane issues each single-thread instruction (tcgen05.mma, .cp,
+// .commit, a TMA copy).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, limit_ns));
+}
+__device__ __forceinline__ bool elect_one_sync() {
+  uint32_t elected;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(elected));
+  return elected != 0;
+}
+__device__ __forceinline__ bool flag_set_warp(const volatile int* flag) {
+  return __any_sync(0xffffffffu, *flag != 0);
+}
+
 // Waits on barriers that the peer CTA of a pair completes (remote arrivals, remote
 // transaction bytes). kWaitCluster: try_wait with cluster-scope acquire. kWaitPoll:
 // non-suspending test_wait loop. Both bounded like mbar_wait.

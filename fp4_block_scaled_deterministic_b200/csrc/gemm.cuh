@@ -315,16 +315,19 @@ struct Issuer {
     SlabCursor cur = base;
     const int nt = sc.num_tiles();
     const int my_tiles = first < nt ? (nt - first + stride - 1) / stride : 0;
-    for (int t = 0; t < my_tiles && !*abort_flag; ++t) {
+    for (int t = 0; t < my_tiles && !flag_set_warp(abort_flag); ++t) {
       bool ok = true;
       const int kts = sc.k_tiles(first + t * stride);
       for (int kt = 0; kt < kts; ++kt) {
-        if (!mbar_wait(&full[cur.stage], cur.phase, sc.wait_ns())) {
+        if (!mbar_wait_warp(&full[cur.stage], cur.phase, sc.wait_ns())) {
           ok = false;
           break;
         }
-        copies<LO, HI>(cur);
-        commit_local(&sf_full[cur.slot]);
+        if (elect_one_sync()) {
+          copies<LO, HI>(cur);
+          commit_local(&sf_full[cur.slot]);
+        }
+        __syncwarp();
         step(cur, base);
       }
       if (!ok) {
@@ -332,9 +335,10 @@ struct Issuer {
         break;
       }
     }
-    // Every copy this thread issued has landed before TMEM can be released.
-    commit_local(drained);
-    if (!mbar_wait(drained, 0u, sc.wait_ns())) *abort_flag = 1;
+    // Every copy this warp issued has landed before TMEM can be released.
+    if (elect_one_sync()) commit_local(drained);
+    __syncwarp();
+    if (!mbar_wait_warp(drained, 0u, sc.wait_ns())) *abort_flag = 1;
   }
   template <class Sched>
   __device__ static void run_split(uint32_t tmem, uint8_t* sA, uint8_t* sB, uint8_t* sSFA,
@@ -348,23 +352,27 @@ struct Issuer {
     const int my_tiles = first < nt ? (nt - first + stride - 1) / stride : 0;
     uint32_t acc_phase = 0;
     for (int t = 0; t < my_tiles; ++t) {
-      if (!mbar_wait(acc_empty, acc_phase ^ 1u, sc.wait_ns()) || *abort_flag) {
+      if (!mbar_wait_warp(acc_empty, acc_phase ^ 1u, sc.wait_ns()) || flag_set_warp(abort_flag)) {
         *abort_flag = 1;
         return;
       }
       tc_fence_after();
       const int kts = sc.k_tiles(first + t * stride);
       for (int kt = 0; kt < kts; ++kt) {
-        if (!mbar_wait(&sf_full[cur.slot], cur.sf_phase, sc.wait_ns())) {
+        if (!mbar_wait_warp(&sf_full[cur.slot], cur.sf_phase, sc.wait_ns())) {
           *abort_flag = 1;
           return;
         }
         tc_fence_after();
-        slab_mmas<0>(cur, tmem, kt == 0);
-        commit(&empty[cur.stage]);
+        if (elect_one_sync()) {
+          slab_mmas<0>(cur, tmem, kt == 0);
+          commit(&empty[cur.stage]);
+        }
+        __syncwarp();
         step(cur, base);
       }
-      commit(acc_full);
+      if (elect_one_sync()) commit(acc_full);
+      __syncwarp();
       acc_phase ^= 1u;
     }
   }
@@ -381,7 +389,7 @@ struct Issuer {
     const int my_tiles = first < nt ? (nt - first + stride - 1) / stride : 0;
     uint32_t acc_phase = 0;
     for (int t = 0; t < my_tiles; ++t) {
-      if (!mbar_wait(acc_empty, acc_phase ^ 1u, sc.wait_ns()) || *abort_flag) {
+      if (!mbar_wait_warp(acc_empty, acc_phase ^ 1u, sc.wait_ns()) || flag_set_warp(abort_flag)) {
         *abort_flag = 1;
         return;
       }
@@ -391,16 +399,20 @@ struct Issuer {
         // Each slab: wait for its stage, copy its scales into its TMEM ring slot, issue its
         // MMAs back to back, then release the stage. (Spreading the next slab's copies
         // between this slab's MMAs was measured to be slower.)
-        if (!mbar_wait(&full[cur.stage], cur.phase, sc.wait_ns())) {
+        if (!mbar_wait_warp(&full[cur.stage], cur.phase, sc.wait_ns())) {
           *abort_flag = 1;
           return;
         }
-        copies<0, kCopies>(cur);
-        slab_mmas<0>(cur, tmem, kt == 0);
-        commit(&empty[cur.stage]);
+        if (elect_one_sync()) {
+          copies<0, kCopies>(cur);
+          slab_mmas<0>(cur, tmem, kt == 0);
+          commit(&empty[cur.stage]);
+        }
+        __syncwarp();
         step(cur, base);
       }
-      commit(acc_full);
+      if (elect_one_sync()) commit(acc_full);
+      __syncwarp();
       acc_phase ^= 1u;
     }
   }
@@ -666,37 +678,46 @@ __global__ void __launch_bounds__(kGSingleThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) {
+    {
       // ------------------------------------------------------------ TMA producer
       int stage = 0;
       uint32_t phase = 0;
-      for (int tile = blockIdx.x; tile < g.num_tiles && !*abort_flag; tile += gridDim.x) {
+      for (int tile = blockIdx.x; tile < g.num_tiles && !flag_set_warp(abort_flag);
+           tile += gridDim.x) {
         int tm, tn;
         tile_coords(tile, g, tm, tn);
+        bool ok = true;
         for (int kt = 0; kt < g.k_tiles; ++kt) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, g.wait_limit_ns)) {
-            *abort_flag = 1;
+          if (!mbar_wait_warp(&empty[stage], phase ^ 1u, g.wait_limit_ns)) {
+            ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], Cfg::kStageBytes);
-          tma_load_2d(sA + stage * kGABytes, &tmA, &full[stage], kt * (kGBK / 2), tm * kGBM);
-          tma_load_2d(sB + stage * kGBBytes, &tmB, &full[stage], kt * (kGBK / 2), tn * kGBN);
-          tma_load_2d(sSFA + stage * Cfg::kSFABytes, &tmSFA, &full[stage], kt * Cfg::kAtoms * 64,
-                      tm);
-          tma_load_2d(sSFB + stage * Cfg::kSFBBytes, &tmSFB, &full[stage], kt * Cfg::kAtoms * 64,
-                      tn * 2);
+          if (elect_one_sync()) {
+            mbar_arrive_expect_tx(&full[stage], Cfg::kStageBytes);
+            tma_load_2d(sA + stage * kGABytes, &tmA, &full[stage], kt * (kGBK / 2), tm * kGBM);
+            tma_load_2d(sB + stage * kGBBytes, &tmB, &full[stage], kt * (kGBK / 2), tn * kGBN);
+            tma_load_2d(sSFA + stage * Cfg::kSFABytes, &tmSFA, &full[stage],
+                        kt * Cfg::kAtoms * 64, tm);
+            tma_load_2d(sSFB + stage * Cfg::kSFBBytes, &tmSFB, &full[stage],
+                        kt * Cfg::kAtoms * 64, tn * 2);
+          }
+          __syncwarp();
           if (++stage == kGStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) {
+          *abort_flag = 1;
+          break;
         }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {
       // ------------------------------------------------------------ MMA issuer
       SingleIssuer::run_split(tmem, sA, sB, sSFA, sSFB, sf_full, empty, acc_full, acc_empty,
                               abort_flag, blockIdx.x, gridDim.x, ArgsSched{g});
     }
   } else if (warp >= kGThreads / 32) {
-    if (lane == 0) {
+    {
       // ------------------------------------------------------------ scale copies
       constexpr int kC = SingleIssuer::kCopies, kN = kGPairCopyThreads;
       if (warp == kGThreads / 32)
@@ -866,39 +887,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<FMT>::kThrea
   const uint32_t leader_acc_empty = mapa_shared(smem_u32(acc_empty), 0);
 
   if (warp == 0) {
-    if (lane == 0) {
+    {
       // ------------------------------------------------------------ TMA producer (both CTAs)
       int stage = 0;
       uint32_t phase = 0;
-      for (int tile = pair; tile < grp.num_tiles && !*abort_flag; tile += npairs) {
+      for (int tile = pair; tile < grp.num_tiles && !flag_set_warp(abort_flag); tile += npairs) {
         const GemmProblem& P = grp.p[group_problem(grp, tile)];
         int tm, tn;
         tile_coords(tile - P.tile0, P.g, tm, tn);
+        bool ok = true;
         for (int kt = 0; kt < P.g.k_tiles; ++kt) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, wait_ns)) {
-            *abort_flag = 1;
+          if (!mbar_wait_warp(&empty[stage], phase ^ 1u, wait_ns)) {
+            ok = false;
             break;
           }
-          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kStageBytes);
-          const uint32_t bar = leader_full + 8u * stage;
+          if (elect_one_sync()) {
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kStageBytes);
+            const uint32_t bar = leader_full + 8u * stage;
 #pragma unroll
-          for (int sub = 0; sub < Cfg::kSub; ++sub) {
-            const int kx = kt * Cfg::kRowBytes + 128 * sub;
-            tma_load_2d_pair(sA + stage * Cfg::kABytes + sub * 16384, &P.a, bar, kx,
-                             tm * 256 + 128 * static_cast<int>(rank));
-            tma_load_2d_pair(sB + stage * Cfg::kBBytes + sub * 16384, &P.b, bar, kx,
-                             tn * 256 + 128 * static_cast<int>(rank));
+            for (int sub = 0; sub < Cfg::kSub; ++sub) {
+              const int kx = kt * Cfg::kRowBytes + 128 * sub;
+              tma_load_2d_pair(sA + stage * Cfg::kABytes + sub * 16384, &P.a, bar, kx,
+                               tm * 256 + 128 * static_cast<int>(rank));
+              tma_load_2d_pair(sB + stage * Cfg::kBBytes + sub * 16384, &P.b, bar, kx,
+                               tn * 256 + 128 * static_cast<int>(rank));
+            }
+            tma_load_2d_pair(sSFA + stage * Cfg::kSFABytes, &P.sa, bar, kt * Cfg::kAtoms * 64,
+                             2 * tm + static_cast<int>(rank));
+            tma_load_2d_pair(sSFB + stage * Cfg::kSFBBytes, &P.sb, bar, kt * Cfg::kAtoms * 64,
+                             2 * tn);
           }
-          tma_load_2d_pair(sSFA + stage * Cfg::kSFABytes, &P.sa, bar, kt * Cfg::kAtoms * 64,
-                           2 * tm + static_cast<int>(rank));
-          tma_load_2d_pair(sSFB + stage * Cfg::kSFBBytes, &P.sb, bar, kt * Cfg::kAtoms * 64,
-                           2 * tn);
+          __syncwarp();
           if (++stage == S) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) {
+          *abort_flag = 1;
+          break;
         }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && rank == 0) {
+    if (rank == 0) {
       // ------------------------------------------------------------ MMA issuer (leader)
       if constexpr (Cfg::kCopyThreads > 0)
         PairIssuer::run_split(tmem, sA, sB, sSFA, sSFB, sf_full, empty, acc_full, acc_empty,
@@ -908,7 +937,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<FMT>::kThrea
                         abort_flag, pair, npairs, sched);
     }
   } else if (warp >= kGThreads / 32) {
-    if (lane == 0 && rank == 0) {
+    if (rank == 0) {
       // ------------------------------------------------------------ scale copies (leader)
       constexpr int kC = PairIssuer::kCopies;
       constexpr int kN = Cfg::kCopyThreads > 0 ? Cfg::kCopyThreads : 1;
