@@ -17,13 +17,16 @@
 // Design (one CTA per SM, persistent over 128x256 output tiles, K in slabs of 256):
 //   warp 0   : TMA producer. Per slab it loads A 128x128 B, B 256x128 B (128B swizzle)
 //              and the matching 512-byte scale atoms into a 4-stage ring.
-//   warp 1   : allocates 512 TMEM columns; one thread issues each slab's 4 MMAs of
+//   warp 1   : allocates 512 TMEM columns; issues each slab's 4 MMAs of
 //              128x256x64 (tcgen05.mma kind::mxf4 / kind::mxf4nvf4) once its scales
 //              are in TMEM, then commits the stage back to the producer; after the
 //              last slab it commits the accumulator to the epilogue.
-//   warps 10, 11: one thread each copies half of the slab's scale atoms smem -> TMEM
+//   warps 10, 11: each copies half of the slab's scale atoms smem -> TMEM
 //              (tcgen05.cp 32x128b.warpx4) into the slab's ring slot and commits them
-//              to the MMA thread (Issuer::run_copies / run_split).
+//              to the MMA warp (Issuer::run_copies / run_split).
+//   The producer, MMA and copy roles run their loops on all 32 lanes (waits and the
+//   abort flag combined by votes, so control flow and descriptors stay warp-uniform);
+//   one lane chosen by elect.sync issues each TMA copy and tcgen05 instruction.
 //   warps 2-9: epilogue. Each warp owns one 32-lane quarter of TMEM and one half of
 //              the 256 columns: it pulls its 32x128 fp32 block into registers,
 //              releases the accumulator (so the next tile's MMAs start), then scales
