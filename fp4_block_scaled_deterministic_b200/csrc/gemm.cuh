@@ -17,14 +17,13 @@
 // Design (one CTA per SM, persistent over 128x256 output tiles, K in slabs of 256):
 //   warp 0   : TMA producer. Per slab it loads A 128x128 B, B 256x128 B (128B swizzle)
 //              and the matching 512-byte scale atoms into a 4-stage ring.
-//   warp 1   : allocates 512 TMEM columns; issues each slab's 4 MMAs of
-//              128x256x64 (tcgen05.mma kind::mxf4 / kind::mxf4nvf4) once its scales
-//              are in TMEM, then commits the stage back to the producer; after the
-//              last slab it commits the accumulator to the epilogue.
-//   warps 10, 11: each copies half of the slab's scale atoms smem -> TMEM
-//              (tcgen05.cp 32x128b.warpx4) into the slab's ring slot and commits them
-//              to the MMA warp (Issuer::run_copies / run_split).
-//   The producer, MMA and copy roles run their loops on all 32 lanes (waits and the
+//   warp 1   : allocates 512 TMEM columns; per slab, once the stage has landed, copies
+//              its scale atoms smem -> TMEM (tcgen05.cp 32x128b.warpx4) into the slab's
+//              ring slot and issues its 4 MMAs of 128x256x64 (tcgen05.mma kind::mxf4 /
+//              kind::mxf4nvf4) behind them, in order, then commits the stage back to
+//              the producer; after the last slab it commits the accumulator to the
+//              epilogue (Issuer::run).
+//   The producer and MMA roles run their loops on all 32 lanes (waits and the
 //   abort flag combined by votes, so control flow and descriptors stay warp-uniform);
 //   one lane chosen by elect.sync issues each TMA copy and tcgen05 instruction.
 //   warps 2-9: epilogue. Each warp owns one 32-lane quarter of TMEM and one half of
@@ -44,9 +43,6 @@ namespace fp4k {
 constexpr int kGBM = 128, kGBN = 256, kGBK = 256;  // tile M, tile N, K elements per slab
 constexpr int kGStages = 4;
 constexpr int kGThreads = 320;
-// Scale-copy threads of the pair kernel (warps 10, 11, ...; see Issuer::run_copies).
-constexpr int kGPairCopyThreads = 2;
-static_assert(kGPairCopyThreads >= 1 && kGPairCopyThreads <= 2, "one or two copy threads");
 constexpr int kGABytes = kGBM * kGBK / 2;  // 16 KB
 constexpr int kGBBytes = kGBN * kGBK / 2;  // 32 KB
 
@@ -194,7 +190,7 @@ struct SlabCursor {
   int stage;
   uint32_t phase;
   uint64_t dA, dB, dSA, dSB;
-  uint32_t t_sf, slot, sf_phase;
+  uint32_t t_sf, slot;
 };
 
 template <int FMT, bool PAIR, int SLAB_K, int STAGES, int A_BYTES, int B_BYTES, int SFA_BYTES,
@@ -216,7 +212,6 @@ struct Issuer {
     if (++c.slot == SF_BUFS) {
       c.slot = 0;
       c.t_sf = base.t_sf;
-      c.sf_phase ^= 1u;
     } else {
       c.t_sf += SF_COLS;
     }
@@ -277,11 +272,6 @@ struct Issuer {
     if constexpr (PAIR) tc_commit_pair_mc(bar, 0x3);
     else tc_commit(bar);
   }
-  // Commit to a barrier of the issuing CTA only (the leader's, for a pair).
-  __device__ __forceinline__ static void commit_local(uint64_t* bar) {
-    if constexpr (PAIR) tc_commit_pair_mc(bar, 0x1);
-    else tc_commit(bar);
-  }
 
   __device__ __forceinline__ static SlabCursor make_base(uint32_t tmem, uint8_t* sA, uint8_t* sB,
                                                          uint8_t* sSFA, uint8_t* sSFB) {
@@ -294,91 +284,15 @@ struct Issuer {
     b.dSB = desc_sf_atom(smem_u32(sSFB));
     b.t_sf = tmem + 256;
     b.slot = 0;
-    b.sf_phase = 0;
     return b;
   }
 
-  // Split issue (pair kernel). Issuing a slab's scale copies and its MMAs from one thread
-  // takes that thread longer than the tensor cores take to run the MMAs, so the copies go
-  // to other threads (run_copies, each a share [LO, HI) of the slab's copies) that walk
-  // the same slabs: each waits for the stage, copies its scales into the slab's ring slot
-  // and commits them to sf_full[slot], which completes when every copy thread has
-  // arrived; the MMA thread (run_split) waits on sf_full instead of the stage barrier. The TMA
-  // data of the stage is complete before the copy thread sees full[stage], hence before
-  // sf_full[slot] completes. A slot is rewritten only after full[] of a slab SF_BUFS
-  // later, whose load waited for the MMAs of the slab STAGES back; SF_BUFS >= STAGES makes
-  // those the slot's previous readers (or later ones), so no slot is overwritten early.
+  // A slab's scale copies go to its TMEM ring slot, issued in order before its MMAs by
+  // the same warp. A slot is rewritten only once the slab SF_BUFS later has its stage,
+  // whose load waited for the MMAs of the slab STAGES back to complete; SF_BUFS >= STAGES
+  // makes those the slot's previous readers (or later ones), so no slot is overwritten
+  // while an MMA may still read it.
   static_assert(SF_BUFS >= STAGES, "scale ring must cover the stage ring");
-  template <int LO, int HI, class Sched>
-  __device__ static void run_copies(uint32_t tmem, uint8_t* sA, uint8_t* sB, uint8_t* sSFA,
-                                    uint8_t* sSFB, uint64_t* full, uint64_t* sf_full,
-                                    uint64_t* drained, volatile int* abort_flag, int first,
-                                    int stride, const Sched& sc) {
-    const SlabCursor base = make_base(tmem, sA, sB, sSFA, sSFB);
-    SlabCursor cur = base;
-    const int nt = sc.num_tiles();
-    const int my_tiles = first < nt ? (nt - first + stride - 1) / stride : 0;
-    for (int t = 0; t < my_tiles && !flag_set_warp(abort_flag); ++t) {
-      bool ok = true;
-      const int kts = sc.k_tiles(first + t * stride);
-      for (int kt = 0; kt < kts; ++kt) {
-        if (!mbar_wait_warp(&full[cur.stage], cur.phase, sc.wait_ns())) {
-          ok = false;
-          break;
-        }
-        if (elect_one_sync()) {
-          copies<LO, HI>(cur);
-          commit_local(&sf_full[cur.slot]);
-        }
-        __syncwarp();
-        step(cur, base);
-      }
-      if (!ok) {
-        *abort_flag = 1;
-        break;
-      }
-    }
-    // Every copy this warp issued has landed before TMEM can be released.
-    if (elect_one_sync()) commit_local(drained);
-    __syncwarp();
-    if (!mbar_wait_warp(drained, 0u, sc.wait_ns())) *abort_flag = 1;
-  }
-  template <class Sched>
-  __device__ static void run_split(uint32_t tmem, uint8_t* sA, uint8_t* sB, uint8_t* sSFA,
-                                   uint8_t* sSFB, uint64_t* sf_full, uint64_t* empty,
-                                   uint64_t* acc_full, uint64_t* acc_empty,
-                                   volatile int* abort_flag, int first, int stride,
-                                   const Sched& sc) {
-    const SlabCursor base = make_base(tmem, sA, sB, sSFA, sSFB);
-    SlabCursor cur = base;
-    const int nt = sc.num_tiles();
-    const int my_tiles = first < nt ? (nt - first + stride - 1) / stride : 0;
-    uint32_t acc_phase = 0;
-    for (int t = 0; t < my_tiles; ++t) {
-      if (!mbar_wait_warp(acc_empty, acc_phase ^ 1u, sc.wait_ns()) || flag_set_warp(abort_flag)) {
-        *abort_flag = 1;
-        return;
-      }
-      tc_fence_after();
-      const int kts = sc.k_tiles(first + t * stride);
-      for (int kt = 0; kt < kts; ++kt) {
-        if (!mbar_wait_warp(&sf_full[cur.slot], cur.sf_phase, sc.wait_ns())) {
-          *abort_flag = 1;
-          return;
-        }
-        tc_fence_after();
-        if (elect_one_sync()) {
-          slab_mmas<0>(cur, tmem, kt == 0);
-          commit(&empty[cur.stage]);
-        }
-        __syncwarp();
-        step(cur, base);
-      }
-      if (elect_one_sync()) commit(acc_full);
-      __syncwarp();
-      acc_phase ^= 1u;
-    }
-  }
 
   // Runs all tiles of this CTA (or CTA pair): tiles first, first+stride, ... < num_tiles.
   template <class Sched>
@@ -623,9 +537,9 @@ __device__ __forceinline__ void store_row_segment_quant(const uint32_t (&r)[128]
   *reinterpret_cast<uint32_t*>(g.q_scales + sc_off) = sbytes;
 }
 
-// Threads of the one-CTA kernel: as the pair kernel, warps 10 and 11 issue the scale
-// copies (Issuer::run_copies) while warp 1 issues the MMAs (Issuer::run_split).
-constexpr int kGSingleThreads = kGThreads + 32 * kGPairCopyThreads;
+// Threads of the one-CTA kernel: warp 0 loads, warp 1 issues each slab's scale copies
+// and MMAs (Issuer::run), warps 2-9 drain the accumulator.
+constexpr int kGSingleThreads = kGThreads;
 
 template <int FMT, int OUT_BF16>
 __global__ void __launch_bounds__(kGSingleThreads, 1)
@@ -645,11 +559,9 @@ __global__ void __launch_bounds__(kGSingleThreads, 1)
   uint64_t* empty = bars + kGStages;
   uint64_t* acc_full = bars + 2 * kGStages;
   uint64_t* acc_empty = acc_full + 1;
-  uint64_t* sf_full = acc_empty + 1;  // one per scale ring slot
-  uint64_t* cp_drained = sf_full + Cfg::kSFBufs;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cp_drained + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  static_assert((2 * kGStages + 3 + Cfg::kSFBufs) * 8 + 8 <= 256, "barrier area");
+  static_assert((2 * kGStages + 2) * 8 + 8 <= 256, "barrier area");
   using SingleIssuer = Issuer<FMT, false, kGBK, kGStages, kGABytes, kGBBytes, Cfg::kSFABytes,
                               Cfg::kSFBBytes, Cfg::kSFCols, Cfg::kSFBufs>;
 
@@ -666,8 +578,6 @@ __global__ void __launch_bounds__(kGSingleThreads, 1)
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 8);
-    for (int i = 0; i < Cfg::kSFBufs; ++i) mbar_init(&sf_full[i], kGPairCopyThreads);
-    mbar_init(cp_drained, kGPairCopyThreads);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -714,24 +624,9 @@ __global__ void __launch_bounds__(kGSingleThreads, 1)
       }
     }
   } else if (warp == 1) {
-    {
-      // ------------------------------------------------------------ MMA issuer
-      SingleIssuer::run_split(tmem, sA, sB, sSFA, sSFB, sf_full, empty, acc_full, acc_empty,
-                              abort_flag, blockIdx.x, gridDim.x, ArgsSched{g});
-    }
-  } else if (warp >= kGThreads / 32) {
-    {
-      // ------------------------------------------------------------ scale copies
-      constexpr int kC = SingleIssuer::kCopies, kN = kGPairCopyThreads;
-      if (warp == kGThreads / 32)
-        SingleIssuer::template run_copies<0, kC / kN>(tmem, sA, sB, sSFA, sSFB, full, sf_full,
-                                                      cp_drained, abort_flag, blockIdx.x,
-                                                      gridDim.x, ArgsSched{g});
-      else
-        SingleIssuer::template run_copies<kC / kN, kC>(tmem, sA, sB, sSFA, sSFB, full, sf_full,
-                                                       cp_drained, abort_flag, blockIdx.x,
-                                                       gridDim.x, ArgsSched{g});
-    }
+    // -------------------------------------------------------------- scale copies + MMAs
+    SingleIssuer::run(tmem, sA, sB, sSFA, sSFB, full, empty, acc_full, acc_empty, abort_flag,
+                      blockIdx.x, gridDim.x, ArgsSched{g});
   } else {
     // -------------------------------------------------------------- epilogue
     const int ew = warp - 2;
@@ -779,10 +674,8 @@ __global__ void __launch_bounds__(kGSingleThreads, 1)
 // pair-wide MMAs; both CTAs load through TMA into their own shared memory with the
 // transfers counted on the leader's barrier, and both drain their own half of the
 // accumulator (rows 128*rank ... +128, all 256 columns) from their own TMEM.
-// Roles: warp 0 of both CTAs loads; in the leader, warp 1 issues the MMAs and (MXFP4,
-// NVFP4) warps 10 and 11 issue the scale copies, half a slab each (Issuer::run_copies);
-// warps 2-9 of both CTAs run the epilogue. MXFP8 launches without warps 10-11 and
-// copies its scales from the MMA thread.
+// Roles: warp 0 of both CTAs loads; in the leader, warp 1 issues each slab's scale
+// copies and then its MMAs (Issuer::run); warps 2-9 of both CTAs run the epilogue.
 // The loads carry no multicast; only the tcgen05.commit arrivals are multicast to the
 // two CTAs of the pair.
 template <int FMT>
@@ -804,12 +697,13 @@ struct PairCfg {
   static constexpr int kSFBBytes = 2 * kAtoms * 512; // scales of all 256 B rows
   static constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
   static constexpr int kStages = FMT == kFmtNV ? 5 : (FMT == kFmtMX ? 6 : 3);
-  // MXFP8 (6 copies per 8 MMAs) keeps the copies in the MMA thread: there the extra wait
-  // of the split issue costs more than it saves.
-  static constexpr int kCopyThreads = FMT == kFmtMX8 ? 0 : kGPairCopyThreads;
-  static constexpr int kThreads = kGThreads + 32 * kCopyThreads;
+  // Every format issues a slab's scale copies from the MMA warp, in order before its MMAs
+  // (Issuer::run). With the issuing roles run as whole warps the issue is cheap; copy
+  // warps of their own, handing each slab to the MMA warp through a barrier, measured
+  // slower (the Llama layer's GEMMs: MXFP4 -2.0%, NVFP4 -5.4%).
+  static constexpr int kThreads = kGThreads;
   static constexpr int kSFCols = 12 * kAtoms;
-  // At least one ring slot per stage (the split issue's reuse rule): 5 x 48 columns for
+  // At least one ring slot per stage (the ring's reuse rule, Issuer): 5 x 48 columns for
   // NVFP4, 6 x 24 for MXFP4, 4 x 24 for MXFP8, after the 256 accumulator columns.
   static constexpr int kSFBufs = kStages > 4 ? kStages : 4;
   static constexpr int kTmemSF = 256;
@@ -844,11 +738,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<FMT>::kThrea
   uint64_t* empty = bars + S;
   uint64_t* acc_full = bars + 2 * S;
   uint64_t* acc_empty = acc_full + 1;
-  uint64_t* sf_full = acc_empty + 1;           // one per scale ring slot
-  uint64_t* cp_drained = sf_full + Cfg::kSFBufs;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cp_drained + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  static_assert((2 * S + 3 + Cfg::kSFBufs) * 8 + 8 <= 256, "barrier area");
+  static_assert((2 * S + 2) * 8 + 8 <= 256, "barrier area");
   uint8_t* s_stage_out = reinterpret_cast<uint8_t*>(bars) + 256;  // [8 warps][1 KB]
   const GroupSched sched{grp};
   const uint64_t wait_ns = grp.p[0].g.wait_limit_ns;
@@ -871,10 +763,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<FMT>::kThrea
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 16);  // 8 epilogue warps in each CTA of the pair
-    if constexpr (Cfg::kCopyThreads > 0) {
-      for (int i = 0; i < Cfg::kSFBufs; ++i) mbar_init(&sf_full[i], Cfg::kCopyThreads);
-      mbar_init(cp_drained, Cfg::kCopyThreads);
-    }
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -931,27 +819,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<FMT>::kThrea
     }
   } else if (warp == 1) {
     if (rank == 0) {
-      // ------------------------------------------------------------ MMA issuer (leader)
-      if constexpr (Cfg::kCopyThreads > 0)
-        PairIssuer::run_split(tmem, sA, sB, sSFA, sSFB, sf_full, empty, acc_full, acc_empty,
-                              abort_flag, pair, npairs, sched);
-      else
-        PairIssuer::run(tmem, sA, sB, sSFA, sSFB, full, empty, acc_full, acc_empty,
-                        abort_flag, pair, npairs, sched);
-    }
-  } else if (warp >= kGThreads / 32) {
-    if (rank == 0) {
-      // ------------------------------------------------------------ scale copies (leader)
-      constexpr int kC = PairIssuer::kCopies;
-      constexpr int kN = Cfg::kCopyThreads > 0 ? Cfg::kCopyThreads : 1;
-      const int ci = warp - kGThreads / 32;
-      if (ci == 0)
-        PairIssuer::template run_copies<0, kC / kN>(tmem, sA, sB, sSFA, sSFB, full, sf_full,
-                                                    cp_drained, abort_flag, pair, npairs, sched);
-      else
-        PairIssuer::template run_copies<kC / kN, kC>(tmem, sA, sB, sSFA, sSFB, full, sf_full,
-                                                     cp_drained, abort_flag, pair, npairs,
-                                                     sched);
+      // ------------------------------------------------------ scale copies + MMAs (leader)
+      PairIssuer::run(tmem, sA, sB, sSFA, sSFB, full, empty, acc_full, acc_empty, abort_flag,
+                      pair, npairs, sched);
     }
   } else {
     // -------------------------------------------------------------- epilogue (both CTAs)
