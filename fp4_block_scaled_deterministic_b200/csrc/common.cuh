@@ -114,13 +114,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, limit_ns));
 }
+// A tcgen05.commit tracks the operations of the thread that issues it, so the MMAs and
+// copies of a slab and the commits that follow must come from one lane. With the whole
+// warp active, elect.sync picks the same lane every time (lane 0); the debug build
+// checks that it does.
 __device__ __forceinline__ bool elect_one_sync() {
   uint32_t elected;
+#ifdef FP4_DEBUG_BOUNDS
+  uint32_t leader;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync %1|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(elected), "=r"(leader));
+  (void)FP4_IN_BOUNDS(leader == 0u);
+#else
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "elect.sync _|p, 0xffffffff;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(elected));
+#endif
   return elected != 0;
 }
 __device__ __forceinline__ bool flag_set_warp(const volatile int* flag) {
