@@ -108,12 +108,13 @@ def parse():
                          "(fp4_quantize_dual_batch); 0: one launch per tensor")
     ap.add_argument("--gemm-group", type=int, default=1, choices=[0, 1],
                     help="1: a projection's Fprop, Dgrad and Wgrad GEMMs in one launch "
-                         "(fp4_gemm_group; Dgrad and Wgrad with --next-layer-quant fused); "
-                         "0: one launch per GEMM")
+                         "(fp4_gemm_group; fp4_gemm_group_quant with --next-layer-quant "
+                         "fused); 0: one launch per GEMM")
     ap.add_argument("--next-layer-quant", choices=["none", "standalone", "fused"], default="none",
                     help="also quantise each Fprop output Y row-wise (MXFP4, same rotation) for "
                          "the next layer: by a separate quantise launch after the GEMM, or in "
-                         "the GEMM's epilogue (fp4_gemm_quant)")
+                         "the GEMM's epilogue (fp4_gemm_group_quant; fp4_gemm_quant with "
+                         "--gemm-group 0)")
     ap.add_argument("--variant", choices=["none", "sr", "rht", "sr+rht", "amax"], default="none",
                     help="quantiser variant: stochastic rounding, randomised Hadamard signs, "
                          "both, or (NVFP4) a supplied tensor amax instead of the amax pass")
@@ -296,13 +297,12 @@ class LlamaLayer:
                               p[key + "_ts"].data_ptr() if fmt == 1 else None, r, c)
                 for key, (r, c) in self._operands(p)])
             # the GEMMs of the projection in one fp4_gemm_group launch, built once:
-            # Fprop (unless its epilogue quantises Y), Dgrad, Wgrad
+            # Fprop (member 0; with the fused epilogue it also quantises Y), Dgrad, Wgrad
             ts = (lambda k, i: p[k + "_ts"][i:i + 1].data_ptr()) if fmt == 1 else (lambda k, i: None)
             M, N, K = tokens, p["N"], p["K"]
-            descs = [(p["dY_row"], p["W_col"], "dY", "W", 0, 1, p["dX"], M, K, N, 1),
+            descs = [(p["X_row"], p["W_row"], "X", "W", 0, 0, p["Y"], M, N, K, 1),
+                     (p["dY_row"], p["W_col"], "dY", "W", 0, 1, p["dX"], M, K, N, 1),
                      (p["dY_col"], p["X_col"], "dY", "X", 1, 1, p["dW"], N, K, M, 0)]
-            if next_quant != "fused":
-                descs.insert(0, (p["X_row"], p["W_row"], "X", "W", 0, 0, p["Y"], M, N, K, 1))
             p["gdescs"] = (fp4.GemmDesc * len(descs))(*[
                 fp4.GemmDesc(a[0].data_ptr(), a[1].data_ptr(), ts(ka, ia), b[0].data_ptr(),
                              b[1].data_ptr(), ts(kb, ib), out.data_ptr(), m, n, k, od)
@@ -342,10 +342,8 @@ class LlamaLayer:
         return sum(t.numel() * t.element_size() for p in self.projs for t in (p["Y"], p["dX"], p["dW"]))
 
     def gemm_launches(self):
-        """GEMM launches of a projection: a group (plus the fused Fprop) or three."""
-        if self.gemm_group:
-            return 2 if self.next_quant == "fused" else 1
-        return 3
+        """GEMM launches of a projection: one group or three."""
+        return 1 if self.gemm_group else 3
 
     def launches_per_step(self):
         # NVFP4 adds the amax pass (plus a memset) unless the amax is supplied
@@ -429,15 +427,15 @@ class LlamaLayer:
             nv = fmt == 1
             M, N, K = self.M, p["N"], p["K"]
             if self.gemm_group:
-                # Fprop, Dgrad and Wgrad (below) in one launch; with the fused epilogue the
-                # Fprop runs alone first and the group holds Dgrad and Wgrad
-                if self.next_quant == "fused":
-                    st = timed("gemm", lambda: f.fp4_gemm_quant(
-                        p["X_row"][0], p["X_row"][1], None, p["W_row"][0], p["W_row"][1], None,
-                        p["Y"], p["Yq"][0], p["Yq"][1], M, N, K, fmt, hn, s))
-                    assert st == 0
+                # Fprop, Dgrad and Wgrad in one launch; with the fused epilogue the Fprop's
+                # epilogue also quantises Y (member 0 of the group)
                 gd = p["gdescs"]
-                st = timed("gemm", lambda: f.lib().fp4_gemm_group(gd, len(gd), fmt, s))
+                if self.next_quant == "fused":
+                    yq = p["Yq"]
+                    st = timed("gemm", lambda: f.lib().fp4_gemm_group_quant(
+                        gd, len(gd), fmt, 0, yq[0].data_ptr(), yq[1].data_ptr(), hn, s))
+                else:
+                    st = timed("gemm", lambda: f.lib().fp4_gemm_group(gd, len(gd), fmt, s))
                 assert st == 0, f.status_string(st)
                 if self.next_quant == "standalone":  # Q_row(Y) by a separate launch
                     st = timed("quant_y", lambda: f.fp4_quantize(
@@ -483,12 +481,7 @@ def gemm_flops_of(layer):
     per = []
     for p in layer.projs:
         one = 2.0 * layer.M * p["N"] * p["K"]
-        if not layer.gemm_group:
-            per += [one] * 3
-        elif layer.next_quant == "fused":
-            per += [one, 2 * one]
-        else:
-            per += [3 * one]
+        per += [one] * 3 if not layer.gemm_group else [3 * one]
     return per
 
 
@@ -1020,10 +1013,11 @@ def main():
                       "next_layer_quant": a.next_layer_quant,
                       "quant_launch": ("one batched launch per projection (X, W, dY)"
                                        if layer.quant_batch else "one launch per tensor"),
-                      "gemm_launch": (("one fp4_gemm_group launch per projection (Fprop, "
-                                       "Dgrad, Wgrad)" if layer.gemm_launches() == 1 else
-                                       "Fprop with the fused epilogue, then Dgrad and Wgrad "
-                                       "in one fp4_gemm_group launch")
+                      "gemm_launch": (("one fp4_gemm_group_quant launch per projection (Fprop "
+                                       "with Y quantised in its epilogue, Dgrad, Wgrad)"
+                                       if layer.next_quant == "fused" else
+                                       "one fp4_gemm_group launch per projection (Fprop, "
+                                       "Dgrad, Wgrad)")
                                       if layer.gemm_group else "one launch per GEMM"),
                       "streams": 2 if a.side_stream else 1,
                       "tokens_per_rank": layer.M,

@@ -98,6 +98,7 @@ def lib() -> ctypes.CDLL:
             "fp4_gemm": (I32, [P, P, P, P, P, P, P, I64, I64, I64, I32, I32, P]),
             "fp4_gemm_quant": (I32, [P, P, P, P, P, P, P, P, P, I64, I64, I64, I32, I32, P]),
             "fp4_gemm_group": (I32, [ctypes.POINTER(GemmDesc), I32, I32, P]),
+            "fp4_gemm_group_quant": (I32, [ctypes.POINTER(GemmDesc), I32, I32, I32, P, P, I32, P]),
             "fp4_linear_workspace_size": (SZ, [I32, I64, I64, I64, I32]),
             "fp4_linear_fprop": (I32, [P, P, P, I64, I64, I64, I32, I32, I32, P, SZ, P]),
             "fp4_linear_dgrad": (I32, [P, P, P, I64, I64, I64, I32, I32, I32, P, SZ, P]),
@@ -186,6 +187,15 @@ def fp4_gemm_group(descs, fmt, stream=None):
     arr = (GemmDesc * max(1, len(descs)))(*[GemmDesc(*[_ptr(v) for v in d[:7]], *d[7:11])
                                             for d in descs])
     return lib().fp4_gemm_group(arr, len(descs), fmt, _stream(stream))
+
+
+def fp4_gemm_group_quant(descs, fmt, q_index, Q_codes, Q_scales, q_hadamard_n, stream=None):
+    """fp4_gemm_group whose member q_index also quantises its bf16 output (as
+    fp4_gemm_quant) into Q_codes / Q_scales."""
+    arr = (GemmDesc * max(1, len(descs)))(*[GemmDesc(*[_ptr(v) for v in d[:7]], *d[7:11])
+                                            for d in descs])
+    return lib().fp4_gemm_group_quant(arr, len(descs), fmt, q_index, _ptr(Q_codes),
+                                      _ptr(Q_scales), q_hadamard_n, _stream(stream))
 
 
 def _opts(opts):
@@ -393,6 +403,26 @@ def gemm_group(problems, out_dtypes=None):
                       out, a.rows, b.rows, a.cols, od))
     _check(fp4_gemm_group(descs, fmt), "fp4_gemm_group")
     return outs
+
+
+def gemm_group_quant(problems, out_dtypes, q_index, q_hn=16):
+    """gemm_group in one launch whose member q_index (a bf16 output) also has its output
+    quantised row-wise as gemm_quant does. Returns (outputs, QTensor of that output)."""
+    assert 1 <= len(problems) <= GEMM_GROUP_MAX and 0 <= q_index < len(problems)
+    fmt = problems[0][0].fmt
+    outs, descs = [], []
+    for i, (a, b) in enumerate(problems):
+        assert a.fmt == b.fmt == fmt and a.cols == b.cols
+        od = out_dtypes[i]
+        out = torch.empty(a.rows, b.rows, dtype=torch.float32 if od == OUT_F32 else torch.bfloat16,
+                          device=a.codes.device)
+        outs.append(out)
+        descs.append((a.codes, a.scales, a.tensor_scale, b.codes, b.scales, b.tensor_scale,
+                      out, a.rows, b.rows, a.cols, od))
+    M, N = problems[q_index][0].rows, problems[q_index][1].rows
+    codes, scales = _alloc_q(M, N, MXFP4, problems[q_index][0].codes.device)
+    _check(fp4_gemm_group_quant(descs, fmt, q_index, codes, scales, q_hn), "fp4_gemm_group_quant")
+    return outs, QTensor(codes, scales, None, MXFP4, M, N)
 
 
 def gemm_quant(a: QTensor, b: QTensor, q_hn: int = 16, with_output: bool = True):

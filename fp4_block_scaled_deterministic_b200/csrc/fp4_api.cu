@@ -615,17 +615,28 @@ fp4_status gemm_impl(const void* A, const void* As, const float* Ats, const void
 // Up to kGMaxProblems GEMMs of one format in one launch of the pair kernel. Problems
 // with M or N zero are skipped; the rest run in order of decreasing K, so that the tiles
 // left for the last wave are the cheapest ones.
-fp4_status gemm_group_impl(const fp4_gemm_desc* d, int n, fp4_format fmt, cudaStream_t stream) {
+// q_index >= 0: that member's epilogue also quantises its bf16 output (as fp4_gemm_quant,
+// rotation q_hn) into q_codes / q_scales.
+fp4_status gemm_group_impl(const fp4_gemm_desc* d, int n, fp4_format fmt, cudaStream_t stream,
+                           int q_index = -1, void* q_codes = nullptr, void* q_scales = nullptr,
+                           int q_hn = -1) {
   if (n < 1 || n > FP4_GEMM_GROUP_MAX || !d) return FP4_ERR_INVALID_ARG;
+  if (q_index >= n || (q_index >= 0) != (q_hn >= 0)) return FP4_ERR_INVALID_ARG;
   int order[kGMaxProblems], used = 0;
+  bool q_used = false;
   for (int i = 0; i < n; ++i) {
     bool empty;
+    const bool qi = i == q_index;
     const fp4_status st = check_gemm(d[i].A_codes, d[i].A_scales, d[i].A_tensor_scale,
                                      d[i].B_codes, d[i].B_scales, d[i].B_tensor_scale, d[i].C,
-                                     d[i].M, d[i].N, d[i].K, fmt, d[i].out_dtype, nullptr,
-                                     nullptr, -1, &empty);
+                                     d[i].M, d[i].N, d[i].K, fmt, d[i].out_dtype,
+                                     qi ? q_codes : nullptr, qi ? q_scales : nullptr,
+                                     qi ? q_hn : -1, &empty);
     if (st != FP4_OK) return st;
-    if (!empty) order[used++] = i;
+    if (!empty) {
+      order[used++] = i;
+      q_used = q_used || qi;
+    }
   }
   if (used == 0) return FP4_OK;
   for (int i = 1; i < used; ++i)  // stable insertion sort by decreasing K
@@ -642,9 +653,10 @@ fp4_status gemm_group_impl(const fp4_gemm_desc* d, int n, fp4_format fmt, cudaSt
   int64_t tiles = 0;
   for (int q = 0; q < used; ++q) {
     const fp4_gemm_desc& x = d[order[q]];
+    const bool qi = order[q] == q_index;
     st = build_gemm(&grp.p[q], true, x.A_codes, x.A_scales, x.A_tensor_scale, x.B_codes,
-                    x.B_scales, x.B_tensor_scale, x.C, x.M, x.N, x.K, fmt, x.out_dtype, nullptr,
-                    nullptr);
+                    x.B_scales, x.B_tensor_scale, x.C, x.M, x.N, x.K, fmt, x.out_dtype,
+                    qi ? q_codes : nullptr, qi ? q_scales : nullptr);
     if (st != FP4_OK) return st;
     grp.p[q].tile0 = static_cast<int>(tiles);
     tiles += grp.p[q].g.num_tiles;
@@ -652,7 +664,8 @@ fp4_status gemm_group_impl(const fp4_gemm_desc* d, int n, fp4_format fmt, cudaSt
   }
   grp.n = used;
   grp.num_tiles = static_cast<int>(tiles);
-  return launch_group(grp, fmt, -1, dev, stream) == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+  return launch_group(grp, fmt, q_used ? q_hn : -1, dev, stream) == cudaSuccess ? FP4_OK
+                                                                                 : FP4_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------- linear-layer passes
@@ -912,6 +925,16 @@ fp4_status fp4_gemm_group(const fp4_gemm_desc* descs, int n, fp4_format fmt,
                           fp4_stream_t stream) {
   NvtxRange nvtx_range("fp4_gemm_group");
   return gemm_group_impl(descs, n, fmt, reinterpret_cast<cudaStream_t>(stream));
+}
+
+fp4_status fp4_gemm_group_quant(const fp4_gemm_desc* descs, int n, fp4_format fmt, int q_index,
+                                void* Q_codes, void* Q_scales, int q_hadamard_n,
+                                fp4_stream_t stream) {
+  NvtxRange nvtx_range("fp4_gemm_group_quant");
+  if (q_hadamard_n != 0 && q_hadamard_n != 16 && q_hadamard_n != 32) return FP4_ERR_INVALID_ARG;
+  if (q_index < 0 || q_index >= n) return FP4_ERR_INVALID_ARG;
+  return gemm_group_impl(descs, n, fmt, reinterpret_cast<cudaStream_t>(stream), q_index, Q_codes,
+                         Q_scales, q_hadamard_n);
 }
 
 fp4_status fp4_gemm_quant(const void* A, const void* As, const float* Ats, const void* B,

@@ -717,8 +717,9 @@ struct PairCfg {
 
 // The kernel runs a group of GEMMs (one problem for fp4_gemm); each tile's problem gives
 // its operand maps, coordinates, K, output type and (NVFP4) tensor scales.
-// QHN >= 0: the epilogue also quantises the output (store_row_segment_quant, rotation
-// QHN along N); the group then holds one problem with a bf16 output.
+// QHN >= 0: the epilogue of the group's member with q_codes set also quantises its
+// output (store_row_segment_quant, rotation QHN along N); the other members store as
+// usual.
 template <int FMT, int QHN = -1>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<FMT>::kThreads, 1)
     gemm_fp4_pair_kernel(const __grid_constant__ GemmGroup grp) {
@@ -852,18 +853,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<FMT>::kThrea
       acc_phase ^= 1u;
       const int row0 = tm * 256 + 128 * static_cast<int>(rank) + 32 * quarter;
       const int n0 = tn * kGBN + 128 * half;
-      if constexpr (QHN >= 0)
-        store_row_segment_quant<FMT, QHN>(r, row0 + lane, n0, P.g, alpha);
-      else if (P.out_bf16)
+      if constexpr (QHN >= 0) {
+        if (P.g.q_codes != nullptr) {  // the group's member whose output is quantised too
+          store_row_segment_quant<FMT, QHN>(r, row0 + lane, n0, P.g, alpha);
+          continue;
+        }
+      }
+      if (P.out_bf16)
         store_row_segment<FMT, 1>(r, row0 + lane, n0, P.g, alpha);
       else  // fp32: through TMA stores (store_segment_tma)
         store_segment_tma<FMT, 0>(r, s_stage_out + 1024 * ew, &P.c, row0, n0, P.g, alpha, lane);
     }
     // every store of this warp has completed before the CTA (and its staging) goes away
-    if constexpr (QHN < 0) {
-      if (lane == 0) bulk_wait<0>();
-      __syncwarp();
-    }
+    if (lane == 0) bulk_wait<0>();
+    __syncwarp();
   }
   __syncwarp();
   tc_fence_before();

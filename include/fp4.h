@@ -290,6 +290,24 @@ FP4_API fp4_status fp4_gemm_quant(const void *A_codes, const void *A_scales,
                                   fp4_format fmt, int q_hadamard_n, fp4_stream_t stream);
 
 /*
+ * fp4_gemm_group_quant -- fp4_gemm_group in which member q_index also quantises its
+ * output in the epilogue, as fp4_gemm_quant does: Q = the row-wise MXFP4 quantisation,
+ * rotation q_hadamard_n (0, 16, 32) along N, of Y = RN_bf16(C). The other members
+ * store as in fp4_gemm_group; all run in one launch. [Producer-fused quantisation, as
+ * fp4_gemm_quant; the layer's three GEMMs in one launch, as fp4_gemm_group.]
+ *   descs, n, fmt: as fp4_gemm_group; member q_index has out_dtype FP4_OUT_BF16 and C a
+ *   bf16 [M][N] output or NULL (only Q is written).
+ *   Q_codes [M][N/2], Q_scales (fp4_scales_bytes(M, N, FP4_MXFP4) bytes): as
+ *   fp4_gemm_quant.
+ *   Errors: FP4_ERR_INVALID_ARG for q_index outside [0, n), FP4_ERR_INVALID_ARG as
+ *   fp4_gemm_quant for the quantised member; otherwise as fp4_gemm_group. A quantised
+ *   member with M or N zero is skipped like any other.
+ */
+FP4_API fp4_status fp4_gemm_group_quant(const fp4_gemm_desc *descs, int n, fp4_format fmt,
+                                        int q_index, void *Q_codes, void *Q_scales,
+                                        int q_hadamard_n, fp4_stream_t stream);
+
+/*
  * The three passes of a linear layer Y = X W^T with X [M][K], W [N][K], dY [M][N],
  * each quantising its operands along its own contraction axis and multiplying them.
  * [MXFP4 pre-training summary, Methodology item 2: Fprop, Dgrad, Wgrad.]

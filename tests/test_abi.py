@@ -144,6 +144,26 @@ def test_gemm_group_validation():
     assert L.fp4_gemm_group(arr(d(M=0), d(N=0)), 2, 0, None) == OK   # nothing to launch
 
 
+def test_gemm_group_quant_validation():
+    """The quantised member is checked as fp4_gemm_quant checks its call; the rest as
+    fp4_gemm_group. Every case returns before anything is launched."""
+    L = fp4.lib()
+    def d(M=128, N=128, K=128, C=A16, od=1):
+        return fp4.GemmDesc(A16, A16, None, A16, A16, None, C, M, N, K, od)
+    arr = lambda *ds: (fp4.GemmDesc * len(ds))(*ds)
+    g = lambda ds, qi=0, Qc=A16, Qs=A16, qhn=16, fmt=0: L.fp4_gemm_group_quant(
+        arr(*ds), len(ds), fmt, qi, Qc, Qs, qhn, None)
+    assert g([d()], qi=1) == INVALID and g([d()], qi=-1) == INVALID  # no such member
+    assert g([d()], qhn=8) == INVALID
+    assert g([d()], fmt=2) == INVALID                  # MXFP8 has no fused output
+    assert g([d(od=0)]) == INVALID                     # the quantised member writes bf16
+    assert g([d(), d(od=0)], qi=0, Qc=None) == INVALID
+    assert g([d(), d(od=0)], qi=0, Qc=MIS) == ALIGN
+    assert g([d(), d(N=100)], qi=0) == SHAPE           # another member's shape
+    assert L.fp4_gemm_group_quant(None, 1, 0, 0, A16, A16, 16, None) == INVALID
+    assert g([d(M=0), d(N=0, od=0)], qi=0) == OK       # nothing to launch
+
+
 def test_linear_step_validation():
     L = fp4.lib()
     need = L.fp4_linear_step_workspace_size(64, 96, 128, 0)

@@ -68,3 +68,41 @@ def test_fused_output_rejects_bad_arguments():
     assert fp4.fp4_gemm_quant(*args, Y, codes, scales, 128, 128, 128, 2, 16) == 1
     assert fp4.fp4_gemm_quant(*args, Y, codes, scales, 128, 128, 128, 0, 16) == 0
     torch.cuda.synchronize()
+
+
+def _same_bits(a, b):
+    if a.dtype == torch.bfloat16:
+        return torch.equal(a.view(torch.int16), b.view(torch.int16))
+    return torch.equal(a.view(torch.int32), b.view(torch.int32))
+
+
+@pytest.mark.parametrize("fmt", [fp4.MXFP4, fp4.NVFP4])
+@pytest.mark.parametrize("shape,q_index", [((256, 512, 1024), 0), ((160, 288, 640), 1),
+                                           ((8192, 6144, 4096), 0)])
+def test_group_with_fused_output_quantisation(orc, fmt, shape, q_index):
+    """fp4_gemm_group_quant: a layer's Fprop, Dgrad and Wgrad in one launch, the member
+    q_index (a bf16 output) also quantised in its epilogue. Its output and codes equal
+    fp4_gemm_quant's bit for bit, the other members equal fp4_gemm's, and the codes
+    equal the oracle's row-wise quantisation of that bf16 output."""
+    M, N, K = shape
+    X = synthetic.normal(M, K, 1.0, seed=M + 3, outlier_frac=0.01, outlier_mult=30.0).cuda()
+    W = synthetic.normal(N, K, 0.02, seed=N + 5).cuda()
+    dY = synthetic.heavy_tailed_grad(M, N, 1e-3, seed=K + 7).cuda()
+    xr, xc = fp4.quantize_dual(X, fmt, 16)
+    wr, wc = fp4.quantize_dual(W, fmt, 16)
+    yr, yc = fp4.quantize_dual(dY, fmt, 16)
+    probs = [(xr, wr), (yr, wc), (yc, xc)]              # Fprop, Dgrad, Wgrad
+    ods = [fp4.OUT_BF16, fp4.OUT_BF16, fp4.OUT_F32]
+    outs, Q = fp4.gemm_group_quant(probs, ods, q_index, 16)
+    a, b = probs[q_index]
+    Y_ref, Q_ref = fp4.gemm_quant(a, b, 16)
+    refs = [fp4.gemm(pa, pb, od) for (pa, pb), od in zip(probs, ods)]
+    torch.cuda.synchronize()
+    assert fp4.fp4_check_status() == 0
+    for out, ref in zip(outs, refs):
+        assert _same_bits(out, ref)
+    assert _same_bits(outs[q_index], Y_ref)
+    assert torch.equal(Q.codes, Q_ref.codes) and torch.equal(Q.scales, Q_ref.scales)
+    if M * N <= 1 << 20:  # the oracle on the smaller shapes (the full one equals gemm_quant)
+        oc, os_, _, _ = orc.quantize(outs[q_index].cpu(), orc.MXFP4, 16, orc.ROW)
+        assert np.array_equal(np_u8(Q.codes), oc) and np.array_equal(np_u8(Q.scales), os_)
