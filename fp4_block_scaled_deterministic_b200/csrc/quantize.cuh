@@ -140,6 +140,7 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
   return __fadd2_rn(a, make_float2(-b.x, -b.y));  // a - b == a + (-b), same rounding
 }
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 neg2(float2 a) { return make_float2(-a.x, -a.y); }
 
 // Normalised block FWHT of both lanes: groups of HN along the 32 elements, butterfly
 // strides 1, 2, 4, ... in that order, then x RN(1/sqrt(HN)).
@@ -370,7 +371,9 @@ __device__ __forceinline__ Enc mx_encode_x2_h16fold(float2 (&p)[32], const Codes
 // 1990; Muller et al., Handbook of Floating-Point Arithmetic, the FMA-based division
 // section). That needs d and the reciprocal away from underflow and overflow: with
 // 2^-100 <= d <= 2^100 a residual can underflow only when |v/d| < 2^-3, whose code is a
-// signed zero either way, and the sign is taken from v (so -0 / d stays -0). Blocks
+// signed zero either way. The residual is formed negated, n = RN(q*d - v), and each step
+// adds (-n)*y: round-to-nearest is odd, so every nonzero value is the one above, and the
+// zero sums that can arise keep v's sign (-0 / d stays -0) with no sign copy. Blocks
 // with a zero scale, a d outside that range or a non-finite element are divided exactly.
 //
 // kQuarter: p holds w = 4v, the H16 butterflies without their x0.25. Round-to-nearest
@@ -397,14 +400,13 @@ __device__ __forceinline__ void nv_block_x2(float2 (&p)[L], float S, float six_s
                     ey <= 0x1p100f && bm.x <= 3.0e38f && bm.y <= 3.0e38f;
   if (fast) {
     const float2 y2 = make_float2(__frcp_rn(ex), __frcp_rn(ey));
-    const float2 nd = make_float2(-ex, -ey);
+    const float2 e2 = make_float2(ex, ey);
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const float2 v = p[b + i];
       const float2 q0 = mul2(v, y2);
-      const float2 q1 = __ffma2_rn(__ffma2_rn(q0, nd, v), y2, q0);  // faithful
-      const float2 q = __ffma2_rn(__ffma2_rn(q1, nd, v), y2, q1);   // RN(v/d)
-      p[b + i] = make_float2(copysignf(q.x, v.x), copysignf(q.y, v.y));
+      const float2 q1 = __ffma2_rn(neg2(__ffma2_rn(q0, e2, neg2(v))), y2, q0);  // faithful
+      p[b + i] = __ffma2_rn(neg2(__ffma2_rn(q1, e2, neg2(v))), y2, q1);           // RN(v/d)
     }
     return;
   }
@@ -1180,14 +1182,13 @@ __device__ __forceinline__ uint32_t nv_block_row_v(float2 (&q2)[16], float S, fl
   const float e = kQuarter ? __fmul_rn(d, 4.0f) : d;  // the divisor of the values held
   if (e >= 0x1p-100f && e <= 0x1p100f && bm <= 3.0e38f) {  // the correction step
     const float y = __frcp_rn(e);
-    const float2 y2 = make_float2(y, y), nd = make_float2(-e, -e);
+    const float2 y2 = make_float2(y, y), e2 = make_float2(e, e);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const float2 v = q2[B + i];
       const float2 q0 = mul2(v, y2);
-      const float2 q1 = __ffma2_rn(__ffma2_rn(q0, nd, v), y2, q0);  // faithful
-      const float2 q = __ffma2_rn(__ffma2_rn(q1, nd, v), y2, q1);   // RN(v/d)
-      q2[B + i] = make_float2(copysignf(q.x, v.x), copysignf(q.y, v.y));
+      const float2 q1 = __ffma2_rn(neg2(__ffma2_rn(q0, e2, neg2(v))), y2, q0);  // faithful
+      q2[B + i] = __ffma2_rn(neg2(__ffma2_rn(q1, e2, neg2(v))), y2, q1);          // RN(v/d)
     }
   } else if (sb == 0u) {  // a zero block scale: zeros that keep the sign of each element
 #pragma unroll

@@ -140,3 +140,78 @@ def test_quarter_fold_gives_the_same_codes():
         block = ws[:16]
         assert rn32(max(abs(w) for w in block) / 4) == max(abs(rn32(w / 4)) for w in block)
     assert checked > 3000
+
+
+# ---- IEEE signed zeros, for the sign-preserving form of the sequence ------------------
+# A value is (x, neg): x a Fraction; neg is its sign bit (which matters only for x == 0).
+def _val(x: Fraction, neg_zero: bool = False):
+    return (x, (x < 0) if x != 0 else neg_zero)
+
+
+def _neg(a):
+    return (-a[0], not a[1])
+
+
+def fma_rn(a, b, c):
+    """RN(a*b + c) with IEEE zero signs: an exact zero sum is +0 unless both addends are
+    -0; a nonzero result that rounds to zero keeps its sign."""
+    prod = a[0] * b[0]
+    prod_neg = (prod < 0) if prod != 0 else (a[1] != b[1])
+    exact = prod + c[0]
+    if exact != 0:
+        r = rn32(exact)
+        return (r, exact < 0) if r != 0 else (Fraction(0), exact < 0)
+    if prod == 0 and c[0] == 0:
+        return (Fraction(0), prod_neg and c[1])
+    return (Fraction(0), False)  # cancellation of nonzero terms: +0
+
+
+def mul_rn(a, b):
+    """RN(a*b) with IEEE zero signs (a zero product's sign is the XOR of the operands')."""
+    prod = a[0] * b[0]
+    if prod != 0:
+        r = rn32(prod)
+        return (r, prod < 0)
+    return (Fraction(0), a[1] != b[1])
+
+
+def signed_sequence(v, e):
+    """The quantiser's sign-preserving form: n = RN(q*e - v) (the negated residual), and
+    each step q + (-n)*y, so that no sign copy is needed."""
+    y = _val(rn32(1 / e[0]))
+    nv = _neg(v)
+    q0 = mul_rn(v, y)
+    q1 = fma_rn(_neg(fma_rn(q0, e, nv)), y, q0)
+    return fma_rn(_neg(fma_rn(q1, e, nv)), y, q1)
+
+
+def test_signed_sequence_keeps_the_sign_and_the_code():
+    """Without a sign copy, the sequence gives the quotient of v's sign (also for v = +-0
+    and for quotients that underflow) and the same E2M1 code as RN(v/d); where the
+    sequence is exact (|v/d| >= 2^-3) it gives RN(v/d) itself."""
+    rng = np.random.default_rng(13)
+    scales = e4m3_values()
+    checked = 0
+    for _ in range(300):
+        S = exact(np.float32(2.0) ** rng.uniform(-60, 60) * rng.uniform(1, 2))
+        d = rn32(scales[rng.integers(len(scales))] * S)
+        e = 4 * d
+        if not (Fraction(2) ** -100 <= e <= Fraction(2) ** 100):
+            continue
+        mags = [rn32(Fraction(float(rng.uniform(0, 32))) * d) for _ in range(8)]
+        mags += [Fraction(int(k)) * Fraction(2) ** -133 * 2 ** int(rng.integers(0, 12))
+                 for k in rng.integers(1, 128, size=6)]
+        for m in mags:
+            for neg in (False, True):
+                w = -m if neg else m
+                q, q_neg = signed_sequence(_val(w), _val(e))
+                assert q_neg == neg, (w, e)
+                plain = rn32(w / e)
+                assert e2m1_magnitude_code(abs(q)) == e2m1_magnitude_code(abs(plain)), (w, e)
+                if abs(plain) >= Fraction(1, 8):
+                    assert q == plain, (w, e)
+                checked += 1
+        for neg in (False, True):  # signed zeros
+            q, q_neg = signed_sequence(_val(Fraction(0), neg), _val(e))
+            assert q == 0 and q_neg == neg
+    assert checked > 5000
